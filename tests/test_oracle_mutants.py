@@ -1,0 +1,71 @@
+"""Mutation check of the oracle's pins: each plausible mistake, planted in a
+copy of the oracle's C source on the CPU, must make at least one pin fail."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = open(os.path.join(os.path.dirname(oracle.__file__), "q4_oracle.c")).read()
+
+MUTANTS = {
+    "nibble_halves_swapped": ("(blk[2 + j] & 0x0F) : (blk[2 + j - 16] >> 4)",
+                              "(blk[2 + j] >> 4) : (blk[2 + j - 16] & 0x0F)"),
+    "offset_7": ("(double)(q - 8) * d", "(double)(q - 7) * d"),
+    "sign_dropped": ("(double)(q - 8) * d", "(double)(8 - q) * d"),
+    "scale_big_endian": ("(uint16_t)(blk[0] | (blk[1] << 8))", "(uint16_t)(blk[1] | (blk[0] << 8))"),
+    "block_stride_16": ("row + (k / 32) * 18", "row + (k / 32) * 16"),
+    "code_index_off_by_one": ("blk[2 + j - 16] >> 4", "blk[2 + j - 15] >> 4"),
+    "x_transposed": ("oracle_f16_to_f64(x[m * K + k])", "oracle_f16_to_f64(x[k * M + m])"),
+    "f16_bias_16": ("ldexp((double)(1024 + f), e - 25)", "ldexp((double)(1024 + f), e - 26)"),
+    "f16_subnormal_unit": ("ldexp((double)f, -24)", "ldexp((double)f, -25)"),
+    "acc_dropped_term": ("for (int64_t k = 0; k < K; ++k)\n                acc +=",
+                         "for (int64_t k = 1; k < K; ++k)\n                acc +="),
+    "repack_g_i_swapped": ("16 * (4 * g + c) + 4 * i + e", "16 * (4 * i + c) + 4 * g + e"),
+    "repack_scale_slot": ("64 * s + 8 * g + 2 * i + h", "64 * s + 8 * i + 2 * g + h"),
+    "repack_pad_code": ("(h < 2 ? 0x00 : 0x88)", "(h < 2 ? 0x00 : 0x00)"),
+    "renorm_no_len": ("sqrt(s / (double)len)", "sqrt(s)"),
+    "rne_ties_up": ("(frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0))", "(frac >= 0.5)"),
+}
+
+PIN_TESTS = [
+    pins.test_f16_decoder_table,
+    pins.test_f16_decoder_all_patterns_match_numpy,
+    lambda: pins.test_f16_encoders("oracle"),
+    pins.test_all_codes_eight_give_zero,
+    pins.test_unit_vectors_pin_nibble_order_offset_and_scale,
+    pins.test_single_nonzero_block,
+    pins.test_linearity_in_scales,
+    pins.test_brute_force_exact_rationals,
+    pins.test_dense_matvec_equivalence_32x32_and_larger,
+    pins.test_golden_hand_cases,
+    lambda: pins.test_repack_round_trip_and_padding(40, 64),
+    pins.test_renorm_invariants,
+    pins.test_stack_chain_closed_form,
+]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    assert old in SRC, f"mutation anchor for {name} no longer in the oracle"
+    src = tmp_path / "mut.c"
+    src.write_text(SRC.replace(old, new, 1))
+    so = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+                           str(src), "-o", str(so), "-lm"])
+    prev = oracle._swap_library(str(so))
+    failed = []
+    try:
+        for t in PIN_TESTS:
+            try:
+                t()
+            except AssertionError:
+                failed.append(getattr(t, "__name__", "lambda"))
+            except Exception:                      # a crash also counts as caught
+                failed.append(getattr(t, "__name__", "lambda"))
+    finally:
+        oracle._restore_library(prev)
+    assert failed, f"mutant {name} survived every pin"
