@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Benchmark of the Q4_0 GEMV decode step on B200.
+
+One step = one synthetic 27B-shaped decode step (M = 1): 64 layers x
+(QKV 5120->7168, O 5120->5120, gate+up 5120->34816, down 17408->5120) Q4_0
+GEMVs with the renorm chain, issued as one CUDA graph through the C-ABI
+(q4gemv_run_stack).  11.9 GB of weights per step, far larger than L2, so no
+flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs an independent replica (same weights,
+its own activation stream); there is no data-path collective, only a barrier
+and a max-reduction of the timings.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "achieved HBM GB/s (% of B200 peak) for Q4_0 GEMV; 27B-shaped decode steps/s"
+L, HIDDEN, QKV_N, FFN = 64, 5120, 7168, 17408
+DIMS = [(QKV_N, HIDDEN), (HIDDEN, HIDDEN), (2 * FFN, HIDDEN), (HIDDEN, FFN)]
+SHAPE_NAMES = ["qkv_5120x7168", "o_5120x5120", "gate_up_5120x34816", "down_17408x5120"]
+CONFIG_SEED = synth.config_seed(4)
+NOMINAL_HBM_GBS = 8000.0
+
+
+def gemv_bytes(N: int, K: int) -> int:
+    """Algorithmic bytes of one M=1 GEMV: Q4_0 weights (18 B per 32) + x + y."""
+    return N * (K // 32) * 18 + 2 * K + 2 * N
+
+
+STEP_GEMV_BYTES = L * sum(gemv_bytes(N, K) for N, K in DIMS)
+STEP_WEIGHT_BYTES = L * sum(N * (K // 32) * 18 for N, K in DIMS)
+WORKLOAD = ("27B-shaped decode step, M=1: 64 layers x (QKV 5120->7168, O 5120->5120, "
+            "gate+up 5120->34816, down 17408->5120) Q4_0 GEMVs with unit-RMS renorm between "
+            "matrices, one CUDA graph per step")
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "200"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = list(csv.reader(io.StringIO(self.tmp.read())))
+        self.tmp.close()
+        os.unlink(self.tmp.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def oracle_sample(min_seconds: float, threads: int):
+    """Times the fp64 oracle on whole layers of the workload (all four
+    matrices) until at least `min_seconds` have elapsed; returns GB/s of
+    Q4_0 bytes (+x,y) and a description of the sample."""
+    import oracle
+    x = synth.normal_f16(CONFIG_SEED, synth.act_id(0), max(HIDDEN, FFN))
+    done_bytes, elapsed, layers = 0, 0.0, 0
+    while elapsed < min_seconds and layers < L:
+        for t, (N, K) in enumerate(DIMS):
+            rows = synth.q4_0_matrix(CONFIG_SEED, synth.weight_id(4 * layers + t), N, K)
+            t0 = time.perf_counter()
+            oracle.q4_gemv(rows, K, x[None, :K], threads=threads)
+            elapsed += time.perf_counter() - t0
+            done_bytes += gemv_bytes(N, K)
+        layers += 1
+    return done_bytes / elapsed / 1e9, f"{layers} full layer(s) of the step ({done_bytes / 1e6:.0f} MB), fp64 oracle", elapsed
+
+
+def oracle_rows_step(i: int, threads: int, frac: int = 64):
+    """One bounded reference step: GEMV (i mod 4) of layer (i/4 mod 64) on
+    every `frac`-th row."""
+    import oracle
+    l, t = (i // 4) % L, i % 4
+    N, K = DIMS[t]
+    sel = np.arange(0, N, frac)
+    rows = synth.q4_0_row_list(CONFIG_SEED, synth.weight_id(4 * l + t), K, sel) if len(sel) < 64 else \
+        synth.q4_0_matrix(CONFIG_SEED, synth.weight_id(4 * l + t), N, K)[sel]
+    x = synth.normal_f16(CONFIG_SEED, synth.act_id(0), K)
+    t0 = time.perf_counter()
+    oracle.q4_gemv(rows, K, x[None, :], threads=threads)
+    dt = time.perf_counter() - t0
+    return rows.size + 2 * K + 2 * len(sel), dt
+
+
+def run_reference(args, rank: int):
+    """Reference arm: the fp64 CPU oracle as it stands, on the host cores."""
+    if rank != 0:
+        return 0
+    threads = os.cpu_count() or 1
+    for i in range(args.warmup):
+        oracle_rows_step(i, threads)
+    tot_b, tot_t = 0, 0.0
+    for i in range(args.steps):
+        b, dt = oracle_rows_step(args.warmup + i, threads)
+        tot_b += b
+        tot_t += dt
+    gbs = tot_b / tot_t / 1e9
+    sample = "each step: one GEMV of the 27B-shaped step (cycling QKV, O, gate+up, down over the 64 layers) on every 64th row"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "parallelism": "replicas"},
+        "decode_steps_per_s": gbs * 1e9 / STEP_GEMV_BYTES,
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def build_weights(eng, torch, rank: int):
+    """Packed weights of the 64-layer step: generated on the host (seeded),
+    copied to the device, repacked by the library's repack kernel."""
+    layers = []
+    host = {t: np.empty((N, (K // 32) * 18), dtype=np.uint8) for t, (N, K) in enumerate(DIMS)}
+    staging = torch.empty(max(h.size for h in host.values()), dtype=torch.uint8, device="cuda")
+    t_repack = 0.0
+    for l in range(L):
+        mats = []
+        for t, (N, K) in enumerate(DIMS):
+            synth.q4_0_matrix(CONFIG_SEED, synth.weight_id(4 * l + t), N, K, out=host[t])
+            g = staging[: host[t].size]
+            g.copy_(torch.from_numpy(host[t].reshape(-1)))
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            mats.append(eng.repack(g, N, K))
+            torch.cuda.synchronize()
+            t_repack += time.perf_counter() - t0
+        layers.append(tuple(mats))
+    del staging
+    return layers, t_repack
+
+
+def time_shapes(eng, torch, layers, reps: int = 5):
+    """Per-shape M=1 GEMV timing: a CUDA graph of 64 launches, one per
+    layer's matrix of that shape (64 distinct matrices, larger than L2)."""
+    out = {}
+    for t, (N, K) in enumerate(DIMS):
+        x = torch.randn(K, device="cuda").half()
+        y = torch.empty(N, device="cuda", dtype=torch.float16)
+        s = torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        eng.run(layers[0][t], x, N, K, out=y)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            for l in range(L):
+                eng.run(layers[l][t], x, N, K, out=y)
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (reps * L)
+        out[SHAPE_NAMES[t]] = {"us_per_launch": us, "GB/s": gemv_bytes(N, K) / us / 1e3,
+                               "rows_per_s": N / us * 1e6}
+        del g
+    return out
+
+
+def run_ours(args, rank: int, world: int, dist):
+    import torch
+    import q4_quantized_decode_b200 as q4
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    eng = q4.Q4Gemv(local)
+    layers, t_repack = build_weights(eng, torch, rank)
+    x_host = torch.from_numpy(synth.normal_f16(CONFIG_SEED, synth.act_id(rank), HIDDEN).view(np.float16)).pin_memory()
+    out_host = torch.empty(HIDDEN, dtype=torch.float16).pin_memory()
+    x_in = x_host.to(dev)
+    x_out = torch.empty(HIDDEN, dtype=torch.float16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        eng.run_stack(layers, x_in, HIDDEN, QKV_N, FFN, x_out=x_out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = eng.sync_status()
+    if st != q4.Q4_OK:
+        raise RuntimeError(f"device status {st}")
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(local).uuid)
+        if uuid and not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    # ---- device-timed region: K steps, inputs resident in HBM
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier()
+    ms = e0.elapsed_time(e1)
+
+    # ---- end-to-end: host x -> device, step, device x_out -> host, every step
+    barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        x_in.copy_(x_host, non_blocking=True)
+        step()
+        out_host.copy_(x_out, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = f0.elapsed_time(f1)
+
+    per_shape = time_shapes(eng, torch, layers) if (rank == 0 and not args.no_per_shape) else None
+    if eng.sync_status() != q4.Q4_OK:
+        raise RuntimeError("device status after timing")
+
+    t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, ms_e2e = float(t[0]), float(t[1])
+    if rank != 0:
+        return 0
+
+    ms_step = ms / args.steps
+    value = world * STEP_GEMV_BYTES * args.steps / (ms * 1e-3) / 1e9
+    e2e_value = world * STEP_GEMV_BYTES * args.steps / (ms_e2e * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    per_rank_gbs = STEP_GEMV_BYTES / (ms_step * 1e-3) / 1e9
+    roofline = {
+        "bound": "hbm", "achieved": per_rank_gbs, "peak": peak, "unit": "GB/s",
+        "frac": per_rank_gbs / peak, "traffic": None,
+        "kernel": "q4::gemv_dp2a_kernel<1,16,8> (256 launches per step; duration = step time, "
+                  "which also holds one small renorm kernel)",
+        "peak_source": f"{peak_kind} hbm_gbs (copy) in MEASURED_PEAKS.json",
+        "frac_of_nominal_8TBps": per_rank_gbs / NOMINAL_HBM_GBS,
+    }
+    traffic = os.path.join(ROOT, "profiles", "traffic_per_launch.json")
+    if os.path.exists(traffic):
+        with open(traffic) as f:
+            tr = json.load(f)
+        roofline["traffic"] = tr.get("bytes_per_step_equivalent")
+        roofline["traffic_note"] = tr.get("note")
+    cpu = None
+    if not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        cgbs, sample, secs = oracle_sample(args.cpu_seconds, threads)
+        cpu = {"value": cgbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"{sample}, {secs:.1f} s on {threads} host threads"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "q4_0 x f16 (s32 block sums, f32 accumulate)", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "bytes_per_step": STEP_GEMV_BYTES,
+                   "weight_bytes_per_step": STEP_WEIGHT_BYTES,
+                   "l2": "inputs larger than L2 (11.9 GB of weights per step)",
+                   "parallelism": f"replicas x{world}", "seed": CONFIG_SEED},
+        "decode_steps_per_s": world * args.steps / (ms * 1e-3),
+        "pct_of_8TBps_nominal": 100.0 * per_rank_gbs / NOMINAL_HBM_GBS,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": 2 * HIDDEN,
+                "d2h_bytes_per_step": 2 * HIDDEN,
+                "steps_per_s": world * args.steps / (ms_e2e * 1e-3)},
+        "gpu_launches": args.steps * (4 * L + 1),
+        "clocks": clocks,
+        "repack_s_per_step_weights": t_repack,
+        "per_shape_m1": per_shape,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-shape", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist_mod
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = dist_mod
+    try:
+        return run_ours(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

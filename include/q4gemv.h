@@ -1,0 +1,203 @@
+/*
+ * q4gemv -- Q4_0 dequantise-and-multiply matrix-vector products on NVIDIA
+ * B200 (sm_100a), the memory-bound core of quantised LLM decode.
+ *
+ * The operation (SwarmLLM coverage, originshq.com page, section "The Engine:
+ * ~50 WGSL Kernels Written From Scratch"): decode reads every weight once per
+ * token, dequantises the 4-bit values and accumulates the matrix-vector
+ * product; speculative verification and prefill apply the same weights to a
+ * handful of activation vectors (aipolix en-US page, section "Speculation is
+ * used to amortize network round trips"; originshq.com page, section
+ * "Multi-Device Performance and the Network Penalty", 16 tokens per round
+ * trip).
+ *
+ *   y[m][n] = sum_k W[n][k] * x[m][k],   0 <= m < M, 0 <= n < N, 0 <= k < K
+ *
+ * W is Q4_0: the pages name the format (taozi.news page, section
+ * "支持模型与限制") without laying it out; the GGUF block is used.  Each row
+ * holds K/32 blocks of 18 bytes: an f16 scale d (little-endian) and 16 bytes
+ * qs; weight j of a block has code q_j = qs[j] & 15 (j < 16) or
+ * qs[j-16] >> 4 (j >= 16) and value (q_j - 8) * d.  x and y are row-major
+ * IEEE binary16.
+ *
+ * Conventions for every entry point
+ *  - All buffers are caller-owned device memory (except where a parameter
+ *    says "host"); the library never frees them.  Pointers to device data
+ *    must be 16-byte aligned.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream) and perform no implicit device synchronisation, except
+ *    q4gemv_create, q4gemv_destroy and q4gemv_sync_status.
+ *  - Every call returns a q4gemv_status.  Arguments are validated on the host
+ *    before anything is launched; an invalid call launches nothing.  The
+ *    library throws no C++ exception across this interface and never traps
+ *    on the device.  The text of the last error of a handle is available from
+ *    q4gemv_last_error.
+ *  - A handle owns a small device workspace (split-K partial sums, per-tile
+ *    arrival counters, an error word) and the cached CUDA graph of
+ *    q4gemv_run_stack.  Calls on one handle must not overlap on the GPU: keep
+ *    them on one stream, or order them with events.  Use one handle per
+ *    concurrent stream.  Overlap that the kernels detect is reported as
+ *    Q4_ECONCURRENT by the next q4gemv_sync_status.
+ */
+#ifndef Q4GEMV_H
+#define Q4GEMV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define Q4GEMV_API __attribute__((visibility("default")))
+#else
+#define Q4GEMV_API
+#endif
+
+typedef struct q4gemv_ctx* q4gemv_t;   /* opaque, library-owned */
+typedef void* q4gemv_stream_t;         /* a cudaStream_t */
+
+typedef enum {
+    Q4_OK = 0,
+    Q4_EINVAL = -1,        /* null handle or pointer, bad enum value */
+    Q4_ESHAPE = -2,        /* K % 32 != 0, N or K <= 0, sizes beyond the limits */
+    Q4_EALIGN = -3,        /* a device pointer is not 16-byte aligned */
+    Q4_ENOMEM = -4,        /* device or host allocation failed */
+    Q4_ECUDA = -5,         /* a CUDA runtime call failed (see q4gemv_last_error) */
+    Q4_EUNSUPPORTED = -6,  /* M outside [1, 16], or the device is not sm_100 */
+    Q4_ETIMEOUT = -7,      /* a bounded device-side wait gave up */
+    Q4_EFAULTINJ = -8,     /* a host step failed on purpose (fault injection) */
+    Q4_ECONCURRENT = -9    /* kernels saw overlapping calls on one handle */
+} q4gemv_status;
+
+/* Limits checked by validation. */
+#define Q4GEMV_MAX_M 16
+#define Q4GEMV_MAX_N (1 << 22)     /* rows */
+#define Q4GEMV_MAX_K (1 << 20)     /* columns */
+
+/* Library version, (major << 16) | minor. */
+Q4GEMV_API int q4gemv_version(void);
+
+/* Creates a handle bound to CUDA device `device` (made current for the
+ * call).  Queries the SM count and allocates the workspace.  Returns
+ * Q4_EUNSUPPORTED on a device that is not compute capability 10.x. */
+Q4GEMV_API int q4gemv_create(q4gemv_t* out, int device);
+
+/* Synchronises the device, releases the workspace and cached graphs, frees
+ * the handle.  Null is accepted (no-op). */
+Q4GEMV_API int q4gemv_destroy(q4gemv_t h);
+
+/* Bytes of a GGUF Q4_0 matrix: N * (K/32) * 18; 0 if the shape is invalid. */
+Q4GEMV_API size_t q4gemv_gguf_bytes(int64_t N, int64_t K);
+
+/* Bytes of the packed (repacked) matrix: Np * (K/32) * 18 with
+ * Np = ceil(N/32)*32; 0 if the shape is invalid.
+ *
+ * Packed layout (the input of q4gemv_run).  Rows are padded to Np (padding
+ * rows hold qs bytes 0x88 and d = +0, i.e. zero weights) and grouped into
+ * tiles of 32 rows.  With KB = K/32, segment s = t*KB + b holds block b of
+ * the rows of tile t; row n = 32t + g + 8i (g in [0,8), i in [0,4)).
+ *   nibble plane, bytes [0, Np*K/2): segment s occupies 512 bytes from
+ *     512*s; its byte 16*(4g + c) + 4i + e is qs[4c + e] of that block of
+ *     row n (c, e in [0,4)).  A lane (g, c) of a warp thus loads, with one
+ *     16-byte load, qs word c of rows g, g+8, g+16, g+24.
+ *   scale plane, bytes [Np*K/2, Np*K/2 + Np*K/16): segment s occupies 64
+ *     bytes from Np*K/2 + 64*s; bytes 8g + 2i, 8g + 2i + 1 hold d of row n.
+ * Every weight byte is read with 16-byte, fully coalesced loads. */
+Q4GEMV_API size_t q4gemv_packed_bytes(int64_t N, int64_t K);
+
+/* Host-only check of q4gemv_run's arguments (no device access, no handle).
+ * Returns the status q4gemv_run would return for these arguments before
+ * launching anything. */
+Q4GEMV_API int q4gemv_validate(int M, int64_t N, int64_t K, const void* W_packed,
+                    const void* x, const void* y);
+
+/* One-time repack of a GGUF Q4_0 matrix into the packed layout.
+ *   gguf   : device, q4gemv_gguf_bytes(N, K) bytes (any alignment >= 2)
+ *   packed : device, q4gemv_packed_bytes(N, K) bytes, 16-byte aligned,
+ *            must not overlap gguf
+ * Bit-exact: the packed bytes are a permutation of the GGUF bytes plus the
+ * padding rows. */
+Q4GEMV_API int q4gemv_repack(q4gemv_t h, const void* gguf, void* packed,
+                  int64_t N, int64_t K, q4gemv_stream_t stream);
+
+/* y[M][N] = W x[M][K]^T for a packed W.
+ *   W_packed : device, q4gemv_packed_bytes(N, K) bytes
+ *   x        : device, M*K binary16, row-major
+ *   y        : device, M*N binary16, row-major (written, never read)
+ * 1 <= M <= 16, K % 32 == 0.  Accumulation is fp32 or exact integer; y is
+ * rounded to nearest even once.  Results beyond the binary16 range become
+ * +-Inf; a non-finite x element makes the affected outputs NaN.  For M <= 2
+ * the activations of each 32-column block are converted to 16-bit integers
+ * with a power-of-two scale chosen so the block's largest magnitude is held
+ * exactly (elements within a factor 16 of it are exact; others are rounded
+ * to 2^-15 of the block maximum) and the per-block dot products are exact
+ * integers.  Deterministic: the same inputs on the same device give the
+ * same bits. */
+Q4GEMV_API int q4gemv_run(q4gemv_t h, const void* W_packed, const void* x, void* y,
+               int M, int64_t N, int64_t K, q4gemv_stream_t stream);
+
+/* One layer's packed matrices for q4gemv_run_stack. */
+typedef struct {
+    const void* qkv;      /* qkv_n  x hidden */
+    const void* o;        /* hidden x hidden */
+    const void* gate_up;  /* 2*ffn  x hidden (rows [0,ffn) gate, [ffn,2ffn) up) */
+    const void* down;     /* hidden x ffn */
+} q4gemv_layer;
+
+/* One synthetic decode step (M = 1) through n_layers layers of four Q4_0
+ * GEMVs each, the 27B-shaped workload of the pages (hidden 5120: taozi.news
+ * page, section "技术架构"; 64 layers: originshq.com page, section "The
+ * Architecture: Layers Distributed, Activations in Flight"):
+ *     a = renorm(f16(QKV x)[0:hidden])
+ *     b = renorm(f16(O a))
+ *     u = renorm(f16(gate_up b)[0:ffn])
+ *     x = renorm(f16(down u))
+ * renorm(v) scales v to unit RMS: s = sum v_i^2 in fp32, v_i * (1/sqrt(s/len))
+ * in fp32 rounded to binary16; an all-zero v stays zero.  The pages give no
+ * layer math beyond the GEMVs, so this chain (Q slice in place of attention,
+ * gate half without an activation) is the reading adopted.
+ *   layers  : HOST array of n_layers entries (device pointers inside)
+ *   x_in    : device, hidden binary16 (not modified)
+ *   x_out   : device, hidden binary16 (may alias x_in)
+ *   trace_x : device or NULL; [4*n_layers][max(hidden, ffn)] binary16: the
+ *             input vector of GEMV i = 4l + t (t = 0 QKV, 1 O, 2 gate_up,
+ *             3 down) in its first K_i entries
+ *   trace_y : device or NULL; [4*n_layers][max(qkv_n, hidden, 2*ffn)]
+ *             binary16: the raw output of GEMV i in its first N_i entries
+ * Requires qkv_n >= hidden, qkv_n % 8 == 0, 1 <= n_layers <= 4096.  The first call with a
+ * given set of arguments captures the whole step (4*n_layers GEMVs, each
+ * with the renorm of its input fused in, plus one final renorm) as a CUDA
+ * graph on an internal stream; later calls with the same arguments replay it
+ * with one cudaGraphLaunch on `stream`.  If `stream` is capturing, the
+ * kernels are launched directly into the caller's capture instead. */
+Q4GEMV_API int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers,
+                     int64_t hidden, int64_t qkv_n, int64_t ffn,
+                     const void* x_in, void* x_out, void* trace_x,
+                     void* trace_y, q4gemv_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the handle's device error
+ * word: Q4_OK, Q4_ETIMEOUT, Q4_ECONCURRENT, or Q4_ECUDA if an earlier
+ * asynchronous error is pending on the device. */
+Q4GEMV_API int q4gemv_sync_status(q4gemv_t h, q4gemv_stream_t stream);
+
+/* Static text for a status code. */
+Q4GEMV_API const char* q4gemv_strerror(int status);
+
+/* Text of the handle's last error (empty if none).  Valid until the next
+ * call on the handle. */
+Q4GEMV_API const char* q4gemv_last_error(q4gemv_t h);
+
+/* Host fault injection for tests: makes the named host step of later calls
+ * fail with Q4_EFAULTINJ.  which: "none", "alloc" (workspace or buffer
+ * allocation), "launch" (kernel launch), "graph" (graph capture or
+ * instantiation).  The environment variable Q4GEMV_FAULT sets the initial
+ * value at q4gemv_create. */
+Q4GEMV_API int q4gemv_set_fault(q4gemv_t h, const char* which);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4GEMV_H */

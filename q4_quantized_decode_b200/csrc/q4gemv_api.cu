@@ -1,0 +1,484 @@
+// Host side of the q4gemv C ABI (see include/q4gemv.h): argument validation,
+// workspace ownership, kernel selection and launch, and the CUDA-graph
+// decode-step runner.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/q4gemv.h"
+#include "gemv_dp2a.cuh"
+
+namespace {
+
+constexpr int kWarps = 16;                 // warps per CTA of the GEMV kernels
+constexpr int kThreads = kWarps * 32;
+constexpr int kPrefetch = 8;               // segments in flight per warp
+constexpr int kMinSegsPerWarp = 4;         // small problems use fewer warps
+constexpr int kMaxTiles = Q4GEMV_MAX_N / 32;
+constexpr size_t kMaxDynSmem = 200 * 1024;   // opt-in dynamic shared memory per CTA
+
+enum Fault { kFaultNone = 0, kFaultAlloc, kFaultLaunch, kFaultGraph };
+
+struct StackKey {
+    std::vector<q4gemv_layer> layers;
+    int64_t hidden = 0, qkv_n = 0, ffn = 0;
+    const void* x_in = nullptr;
+    void* x_out = nullptr;
+    void* trace_x = nullptr;
+    void* trace_y = nullptr;
+    bool operator==(const StackKey& o) const {
+        if (layers.size() != o.layers.size()) return false;
+        for (size_t i = 0; i < layers.size(); ++i) {
+            const q4gemv_layer& a = layers[i];
+            const q4gemv_layer& b = o.layers[i];
+            if (a.qkv != b.qkv || a.o != b.o || a.gate_up != b.gate_up || a.down != b.down)
+                return false;
+        }
+        return hidden == o.hidden && qkv_n == o.qkv_n && ffn == o.ffn && x_in == o.x_in &&
+               x_out == o.x_out && trace_x == o.trace_x && trace_y == o.trace_y;
+    }
+};
+
+}  // namespace
+
+struct q4gemv_ctx {
+    int device = 0;
+    int sms = 0;
+    int fault = kFaultNone;
+    float* ws = nullptr;          // [max warps][2][MAX_M][32] fp32
+    int max_warps = 0;
+    int* cnt = nullptr;           // [kMaxTiles]
+    int* err = nullptr;           // device error word
+    __half* act = nullptr;        // stack intermediates
+    size_t act_elems = 0;
+    cudaStream_t cap = nullptr;   // private capture stream
+    cudaGraphExec_t exec = nullptr;
+    StackKey key;
+    std::string last_error;
+};
+
+namespace {
+
+int fail(q4gemv_ctx* h, int status, const char* fmt, ...) {
+    if (h) {
+        char buf[512];
+        va_list ap;
+        va_start(ap, fmt);
+        vsnprintf(buf, sizeof buf, fmt, ap);
+        va_end(ap);
+        h->last_error = buf;
+    }
+    return status;
+}
+
+int cuda_fail(q4gemv_ctx* h, cudaError_t e, const char* what) {
+    return fail(h, Q4_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define Q4_CUDA(h, call)                                          \
+    do {                                                          \
+        cudaError_t e_ = (call);                                  \
+        if (e_ != cudaSuccess) return cuda_fail((h), e_, #call);  \
+    } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int64_t N, int64_t K) {
+    if (N <= 0 || K <= 0 || K % 32 != 0) return Q4_ESHAPE;
+    if (N > Q4GEMV_MAX_N || K > Q4GEMV_MAX_K) return Q4_ESHAPE;
+    const int64_t T = (N + 31) / 32;
+    if (T * (K / 32) >= (int64_t(1) << 31)) return Q4_ESHAPE;
+    return Q4_OK;
+}
+
+int parse_fault(const char* s) {
+    if (!s || !*s || !strcmp(s, "none")) return kFaultNone;
+    if (!strcmp(s, "alloc")) return kFaultAlloc;
+    if (!strcmp(s, "launch")) return kFaultLaunch;
+    if (!strcmp(s, "graph")) return kFaultGraph;
+    return -1;
+}
+
+template <int M>
+int set_gemv_attrs() {
+    const cudaError_t e = cudaFuncSetAttribute(q4::gemv_dp2a_kernel<M, kWarps, kPrefetch>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)kMaxDynSmem);
+    return e == cudaSuccess ? 0 : -1;
+}
+
+// Launch one GEMV (M <= 2 path).  `pdl` adds the programmatic-dependent-
+// launch attribute (only used between the library's own kernels).
+int launch_gemv(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M, int64_t N,
+                int64_t K, int renorm, __half* trace_x, cudaStream_t st, bool pdl) {
+    if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
+    const int KB = (int)(K / 32);
+    const int T = (int)((N + 31) / 32);
+    const int64_t Np = (int64_t)T * 32;
+    const int S = T * KB;
+    int ctas = h->sms;
+    const int want_warps = (S + kMinSegsPerWarp - 1) / kMinSegsPerWarp;
+    if (want_warps < ctas * kWarps) ctas = (want_warps + kWarps - 1) / kWarps;
+    if (ctas < 1) ctas = 1;
+    q4::GemvArgs a;
+    a.nib = static_cast<const uint8_t*>(W);
+    a.scl = static_cast<const uint8_t*>(W) + Np * K / 2;
+    a.x = x;
+    a.y = y;
+    a.ws = h->ws;
+    a.cnt = h->cnt;
+    a.err = h->err;
+    a.trace_x = trace_x;
+    a.N = N;
+    a.K = (int)K;
+    a.KB = KB;
+    a.T = T;
+    a.S = S;
+    a.G = ctas * kWarps;
+    a.renorm = renorm;
+    const size_t smem = q4::gemv_dp2a_smem_bytes(M, (int)K);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ctas);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cudaError_t e;
+    if (M == 1)
+        e = cudaLaunchKernelEx(&cfg, q4::gemv_dp2a_kernel<1, kWarps, kPrefetch>, a);
+    else
+        e = cudaLaunchKernelEx(&cfg, q4::gemv_dp2a_kernel<2, kWarps, kPrefetch>, a);
+    if (e != cudaSuccess) return cuda_fail(h, e, "gemv launch");
+    return Q4_OK;
+}
+
+int launch_renorm(q4gemv_ctx* h, const __half* in, __half* out, int len, cudaStream_t st,
+                  bool pdl) {
+    if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)len * 2;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, q4::renorm_kernel<kWarps>, in, out, len, h->err);
+    if (e != cudaSuccess) return cuda_fail(h, e, "renorm launch");
+    return Q4_OK;
+}
+
+bool dp2a_fits(int M, int64_t K) {
+    return M <= 2 && q4::gemv_dp2a_smem_bytes(M, (int)K) <= kMaxDynSmem;
+}
+
+}  // namespace
+
+extern "C" {
+
+int q4gemv_version(void) { return (0 << 16) | 1; }
+
+const char* q4gemv_strerror(int status) {
+    switch (status) {
+        case Q4_OK: return "ok";
+        case Q4_EINVAL: return "invalid argument";
+        case Q4_ESHAPE: return "invalid shape (N, K > 0, K % 32 == 0, within limits)";
+        case Q4_EALIGN: return "device pointer not 16-byte aligned";
+        case Q4_ENOMEM: return "out of memory";
+        case Q4_ECUDA: return "CUDA runtime error";
+        case Q4_EUNSUPPORTED: return "unsupported configuration";
+        case Q4_ETIMEOUT: return "bounded device wait timed out";
+        case Q4_EFAULTINJ: return "injected fault";
+        case Q4_ECONCURRENT: return "overlapping calls on one handle";
+        default: return "unknown status";
+    }
+}
+
+const char* q4gemv_last_error(q4gemv_t h) { return h ? h->last_error.c_str() : ""; }
+
+size_t q4gemv_gguf_bytes(int64_t N, int64_t K) {
+    if (check_shape(N, K) != Q4_OK) return 0;
+    return (size_t)N * (size_t)(K / 32) * 18;
+}
+
+size_t q4gemv_packed_bytes(int64_t N, int64_t K) {
+    if (check_shape(N, K) != Q4_OK) return 0;
+    return (size_t)((N + 31) / 32 * 32) * (size_t)(K / 32) * 18;
+}
+
+int q4gemv_validate(int M, int64_t N, int64_t K, const void* W, const void* x, const void* y) {
+    if (M < 1 || M > Q4GEMV_MAX_M) return Q4_EUNSUPPORTED;
+    const int sh = check_shape(N, K);
+    if (sh != Q4_OK) return sh;
+    if (!W || !x || !y) return Q4_EINVAL;
+    if (!aligned16(W) || !aligned16(x) || !aligned16(y)) return Q4_EALIGN;
+    if (!dp2a_fits(M, K)) return Q4_EUNSUPPORTED;
+    return Q4_OK;
+}
+
+int q4gemv_set_fault(q4gemv_t h, const char* which) {
+    if (!h) return Q4_EINVAL;
+    const int f = parse_fault(which);
+    if (f < 0) return fail(h, Q4_EINVAL, "unknown fault name");
+    h->fault = f;
+    return Q4_OK;
+}
+
+int q4gemv_create(q4gemv_t* out, int device) {
+    if (!out) return Q4_EINVAL;
+    *out = nullptr;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev)
+        return Q4_EINVAL;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return Q4_ECUDA;
+    if (prop.major != 10) return Q4_EUNSUPPORTED;
+    q4gemv_ctx* h = new (std::nothrow) q4gemv_ctx;
+    if (!h) return Q4_ENOMEM;
+    h->device = device;
+    h->sms = prop.multiProcessorCount;
+    const int f = parse_fault(getenv("Q4GEMV_FAULT"));
+    h->fault = f < 0 ? kFaultNone : f;
+    int rc = Q4_OK;
+    cudaError_t e = cudaSetDevice(device);
+    if (e != cudaSuccess) rc = cuda_fail(h, e, "cudaSetDevice");
+    if (rc == Q4_OK && h->fault == kFaultAlloc) rc = fail(h, Q4_EFAULTINJ, "injected allocation failure");
+    if (rc == Q4_OK) {
+        h->max_warps = h->sms * kWarps;
+        const size_t ws_bytes = (size_t)h->max_warps * 2 * Q4GEMV_MAX_M * 32 * sizeof(float);
+        if (cudaMalloc(&h->ws, ws_bytes) != cudaSuccess ||
+            cudaMalloc(&h->cnt, (size_t)kMaxTiles * sizeof(int)) != cudaSuccess ||
+            cudaMalloc(&h->err, sizeof(int)) != cudaSuccess)
+            rc = fail(h, Q4_ENOMEM, "workspace allocation failed");
+    }
+    if (rc == Q4_OK) {
+        if (cudaMemset(h->cnt, 0, (size_t)kMaxTiles * sizeof(int)) != cudaSuccess ||
+            cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess)
+            rc = fail(h, Q4_ECUDA, "workspace initialisation failed");
+    }
+    if (rc == Q4_OK) {
+        if (set_gemv_attrs<1>() || set_gemv_attrs<2>() ||
+            cudaFuncSetAttribute(q4::renorm_kernel<kWarps>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kMaxDynSmem) != cudaSuccess)
+            rc = fail(h, Q4_ECUDA, "cudaFuncSetAttribute failed");
+    }
+    if (rc == Q4_OK) {
+        e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
+        if (e != cudaSuccess) rc = cuda_fail(h, e, "cudaStreamCreate");
+    }
+    if (rc == Q4_OK) {
+        e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) rc = cuda_fail(h, e, "cudaDeviceSynchronize");
+    }
+    if (rc != Q4_OK) {
+        cudaFree(h->ws);
+        cudaFree(h->cnt);
+        cudaFree(h->err);
+        if (h->cap) cudaStreamDestroy(h->cap);
+        delete h;
+        return rc;
+    }
+    *out = h;
+    return Q4_OK;
+}
+
+int q4gemv_destroy(q4gemv_t h) {
+    if (!h) return Q4_OK;
+    cudaSetDevice(h->device);
+    cudaDeviceSynchronize();
+    if (h->exec) cudaGraphExecDestroy(h->exec);
+    if (h->cap) cudaStreamDestroy(h->cap);
+    cudaFree(h->ws);
+    cudaFree(h->cnt);
+    cudaFree(h->err);
+    cudaFree(h->act);
+    delete h;
+    return Q4_OK;
+}
+
+int q4gemv_repack(q4gemv_t h, const void* gguf, void* packed, int64_t N, int64_t K,
+                  q4gemv_stream_t stream) {
+    if (!h) return Q4_EINVAL;
+    const int sh = check_shape(N, K);
+    if (sh != Q4_OK) return fail(h, sh, "repack: invalid shape N=%lld K=%lld", (long long)N, (long long)K);
+    if (!gguf || !packed) return fail(h, Q4_EINVAL, "repack: null pointer");
+    if ((reinterpret_cast<uintptr_t>(gguf) & 1u) || !aligned16(packed))
+        return fail(h, Q4_EALIGN, "repack: misaligned pointer");
+    const uintptr_t g0 = reinterpret_cast<uintptr_t>(gguf), g1 = g0 + q4gemv_gguf_bytes(N, K);
+    const uintptr_t p0 = reinterpret_cast<uintptr_t>(packed), p1 = p0 + q4gemv_packed_bytes(N, K);
+    if (g0 < p1 && p0 < g1) return fail(h, Q4_EINVAL, "repack: gguf and packed overlap");
+    if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
+    Q4_CUDA(h, cudaSetDevice(h->device));
+    const int KB = (int)(K / 32);
+    const int64_t T = (N + 31) / 32;
+    const int64_t S = T * KB;
+    int64_t blocks = (S + 7) / 8;
+    if (blocks > (int64_t)h->sms * 32) blocks = (int64_t)h->sms * 32;
+    q4::repack_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint8_t*>(gguf), static_cast<uint8_t*>(packed), N, KB, S, T * 32);
+    Q4_CUDA(h, cudaGetLastError());
+    return Q4_OK;
+}
+
+int q4gemv_run(q4gemv_t h, const void* W, const void* x, void* y, int M, int64_t N, int64_t K,
+               q4gemv_stream_t stream) {
+    if (!h) return Q4_EINVAL;
+    const int v = q4gemv_validate(M, N, K, W, x, y);
+    if (v != Q4_OK)
+        return fail(h, v, "run: %s (M=%d N=%lld K=%lld)", q4gemv_strerror(v), M, (long long)N,
+                    (long long)K);
+    Q4_CUDA(h, cudaSetDevice(h->device));
+    return launch_gemv(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K, 0,
+                       nullptr, static_cast<cudaStream_t>(stream), false);
+}
+
+namespace {
+
+// Enqueue the whole decode step on `st`.
+int enqueue_stack(q4gemv_ctx* h, const StackKey& k, cudaStream_t st) {
+    const int64_t hidden = k.hidden, qkv_n = k.qkv_n, ffn = k.ffn;
+    const int64_t kmax = hidden > ffn ? hidden : ffn;
+    int64_t nmax = qkv_n > hidden ? qkv_n : hidden;
+    if (2 * ffn > nmax) nmax = 2 * ffn;
+    // Intermediate outputs: QKV, O, gate_up, down (rounded up to 16 bytes).
+    const int64_t n_of[4] = {qkv_n, hidden, 2 * ffn, hidden};
+    const int64_t k_of[4] = {hidden, hidden, hidden, ffn};
+    __half* buf[4];
+    size_t off = 0;
+    for (int t = 0; t < 4; ++t) {
+        buf[t] = h->act + off;
+        off += (size_t)((n_of[t] + 7) / 8 * 8);
+    }
+    const int n_gemv = 4 * (int)k.layers.size();
+    const __half* prev = nullptr;
+    for (int i = 0; i < n_gemv; ++i) {
+        const int l = i / 4, t = i % 4;
+        const q4gemv_layer& L = k.layers[l];
+        const void* W = t == 0 ? L.qkv : t == 1 ? L.o : t == 2 ? L.gate_up : L.down;
+        __half* yout = k.trace_y ? static_cast<__half*>(k.trace_y) + (size_t)i * nmax : buf[t];
+        __half* tx = k.trace_x ? static_cast<__half*>(k.trace_x) + (size_t)i * kmax : nullptr;
+        const __half* xin = (i == 0) ? static_cast<const __half*>(k.x_in) : prev;
+        const int rc = launch_gemv(h, W, xin, yout, 1, n_of[t], k_of[t], i == 0 ? 0 : 1, tx, st,
+                                   i != 0);
+        if (rc != Q4_OK) return rc;
+        prev = yout;
+    }
+    return launch_renorm(h, prev, static_cast<__half*>(k.x_out), (int)hidden, st, true);
+}
+
+}  // namespace
+
+int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64_t hidden,
+                     int64_t qkv_n, int64_t ffn, const void* x_in, void* x_out, void* trace_x,
+                     void* trace_y, q4gemv_stream_t stream) {
+    if (!h) return Q4_EINVAL;
+    if (!layers || !x_in || !x_out) return fail(h, Q4_EINVAL, "run_stack: null pointer");
+    if (n_layers < 1 || n_layers > 4096) return fail(h, Q4_ESHAPE, "run_stack: n_layers out of range");
+    if (qkv_n < hidden) return fail(h, Q4_ESHAPE, "run_stack: qkv_n < hidden");
+    if (qkv_n % 8 != 0)   // trace_y rows must start on 16-byte boundaries
+        return fail(h, Q4_ESHAPE, "run_stack: qkv_n must be a multiple of 8");
+    const int64_t dims[4][2] = {{qkv_n, hidden}, {hidden, hidden}, {2 * ffn, hidden}, {hidden, ffn}};
+    for (auto& d : dims) {
+        const int s = check_shape(d[0], d[1]);
+        if (s != Q4_OK) return fail(h, s, "run_stack: invalid matrix shape");
+        if (!dp2a_fits(1, d[1])) return fail(h, Q4_EUNSUPPORTED, "run_stack: K too large");
+    }
+    if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(trace_x) || !aligned16(trace_y))
+        return fail(h, Q4_EALIGN, "run_stack: misaligned pointer");
+    for (int l = 0; l < n_layers; ++l) {
+        const q4gemv_layer& L = layers[l];
+        if (!L.qkv || !L.o || !L.gate_up || !L.down)
+            return fail(h, Q4_EINVAL, "run_stack: null matrix in layer %d", l);
+        if (!aligned16(L.qkv) || !aligned16(L.o) || !aligned16(L.gate_up) || !aligned16(L.down))
+            return fail(h, Q4_EALIGN, "run_stack: misaligned matrix in layer %d", l);
+    }
+    Q4_CUDA(h, cudaSetDevice(h->device));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    StackKey k;
+    k.layers.assign(layers, layers + n_layers);
+    k.hidden = hidden;
+    k.qkv_n = qkv_n;
+    k.ffn = ffn;
+    k.x_in = x_in;
+    k.x_out = x_out;
+    k.trace_x = trace_x;
+    k.trace_y = trace_y;
+
+    // Intermediate buffers (outside any capture: allocation is not captured).
+    const size_t need = (size_t)((qkv_n + 7) / 8 * 8 + (hidden + 7) / 8 * 8 +
+                                 (2 * ffn + 7) / 8 * 8 + (hidden + 7) / 8 * 8);
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    Q4_CUDA(h, cudaStreamIsCapturing(st, &cs));
+    if (need > h->act_elems) {
+        if (cs != cudaStreamCaptureStatusNone)
+            return fail(h, Q4_EUNSUPPORTED,
+                        "run_stack: first call with these sizes must happen outside stream capture");
+        if (h->fault == kFaultAlloc) return fail(h, Q4_EFAULTINJ, "injected allocation failure");
+        Q4_CUDA(h, cudaStreamSynchronize(st));
+        cudaFree(h->act);
+        h->act = nullptr;
+        h->act_elems = 0;
+        if (cudaMalloc(&h->act, need * sizeof(__half)) != cudaSuccess)
+            return fail(h, Q4_ENOMEM, "run_stack: activation buffer allocation failed");
+        h->act_elems = need;
+    }
+
+    if (cs != cudaStreamCaptureStatusNone) return enqueue_stack(h, k, st);
+
+    if (!h->exec || !(h->key == k)) {
+        if (h->fault == kFaultGraph) return fail(h, Q4_EFAULTINJ, "injected graph failure");
+        if (h->exec) {
+            cudaGraphExecDestroy(h->exec);
+            h->exec = nullptr;
+        }
+        Q4_CUDA(h, cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
+        const int rc = enqueue_stack(h, k, h->cap);
+        cudaGraph_t graph = nullptr;
+        const cudaError_t ee = cudaStreamEndCapture(h->cap, &graph);
+        if (rc != Q4_OK) {
+            if (graph) cudaGraphDestroy(graph);
+            return rc;
+        }
+        if (ee != cudaSuccess) return cuda_fail(h, ee, "cudaStreamEndCapture");
+        const cudaError_t ei = cudaGraphInstantiate(&h->exec, graph, 0);
+        cudaGraphDestroy(graph);
+        if (ei != cudaSuccess) {
+            h->exec = nullptr;
+            return cuda_fail(h, ei, "cudaGraphInstantiate");
+        }
+        h->key = k;
+    }
+    Q4_CUDA(h, cudaGraphLaunch(h->exec, st));
+    return Q4_OK;
+}
+
+int q4gemv_sync_status(q4gemv_t h, q4gemv_stream_t stream) {
+    if (!h) return Q4_EINVAL;
+    Q4_CUDA(h, cudaSetDevice(h->device));
+    Q4_CUDA(h, cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    int word = 0;
+    Q4_CUDA(h, cudaMemcpy(&word, h->err, sizeof(int), cudaMemcpyDeviceToHost));
+    if (word != 0) {
+        Q4_CUDA(h, cudaMemset(h->err, 0, sizeof(int)));
+        if (word == q4::kDevTimeout) return fail(h, Q4_ETIMEOUT, "device wait timed out");
+        if (word == q4::kDevConcurrent) return fail(h, Q4_ECONCURRENT, "overlapping calls detected");
+        return fail(h, Q4_ECUDA, "device error word %d", word);
+    }
+    return Q4_OK;
+}
+
+}  // extern "C"
