@@ -40,7 +40,7 @@ struct GemvArgs {
     int64_t N;
     int K, KB, T;
     int S;                  // segments = T * KB
-    int G;                  // warps in the grid
+    int G;                  // warps that own segments (G <= S)
     int renorm;             // 1: the input is renorm(x[0:K]) (M == 1 only)
 };
 
@@ -53,17 +53,17 @@ __host__ __device__ constexpr size_t gemv_dp2a_smem_bytes(int M, int K) {
 
 // First segment of warp g under the flat balanced split of S segments over
 // G warps, and the warp that owns segment s.
-__device__ __forceinline__ int seg_begin(int g, int S, int G) {
+__host__ __device__ __forceinline__ int seg_begin(int g, int S, int G) {
     return (int)(((int64_t)g * S) / G);
 }
-__device__ __forceinline__ int warp_of_seg(int s, int S, int G) {
+__host__ __device__ __forceinline__ int warp_of_seg(int s, int S, int G) {
     return (int)((((int64_t)s + 1) * G - 1) / S);
 }
 
 // Position of element j of a 32-column block in the permuted X layout: the
 // eight entries lane group c needs ([4c..4c+3] and [4c+16..4c+19]) are
 // contiguous.
-__device__ __forceinline__ int xperm_pos(int j) {
+__host__ __device__ __forceinline__ int xperm_pos(int j) {
     return ((j & 15) >> 2) * 8 + ((j >> 4) << 2) + (j & 3);
 }
 
@@ -156,7 +156,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, c = lane & 3;
     const int gw = blockIdx.x * WARPS + warp;
-    const int s0 = seg_begin(gw, a.S, a.G), s1 = seg_begin(gw + 1, a.S, a.G);
+    // G <= S, so every warp below G owns at least one segment; warps of the
+    // last CTA beyond G only help stage the activations.
+    const int s0 = gw < a.G ? seg_begin(gw, a.S, a.G) : a.S;
+    const int s1 = gw < a.G ? seg_begin(gw + 1, a.S, a.G) : a.S;
 
     if (threadIdx.x == 0) {
         mbar_init(&bar, 1);

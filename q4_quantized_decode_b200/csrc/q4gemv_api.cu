@@ -139,7 +139,7 @@ int launch_gemv(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M,
     a.KB = KB;
     a.T = T;
     a.S = S;
-    a.G = ctas * kWarps;
+    a.G = ctas * kWarps < S ? ctas * kWarps : S;   // every owning warp gets >= 1 segment
     a.renorm = renorm;
     const size_t smem = q4::gemv_dp2a_smem_bytes(M, (int)K);
 

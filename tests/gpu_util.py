@@ -16,6 +16,8 @@ def rel_err(y_gpu_bits: np.ndarray, y_ref: np.ndarray) -> float:
     yg = np.asarray(y_gpu_bits, dtype=np.uint16).view(np.float16).astype(np.float64)
     yr = np.atleast_2d(np.asarray(y_ref, dtype=np.float64))
     yg = yg.reshape(yr.shape)
+    if not np.array_equal(np.isfinite(yg), np.isfinite(yr)):
+        return float("inf")
     worst = 0.0
     for m in range(yr.shape[0]):
         rms = np.sqrt(np.mean(yr[m] ** 2))

@@ -214,7 +214,10 @@ def check_teacher_forced(ggufs, x_in, tx, ty, L, hidden, qkv_n, ffn, rows=None, 
             # rms(y) from the GPU output itself for the error denominator
             rms = np.sqrt(np.mean(ty[i, :N].view(np.float16).astype(np.float64) ** 2))
             den = np.maximum(np.abs(ref), rms)
-            e = float(np.max(np.abs(got.view(np.float16).astype(np.float64) - ref) / den))
+            gv = got.view(np.float16).astype(np.float64)
+            if not np.all(np.isfinite(gv)):
+                return float("inf")
+            e = float(np.max(np.abs(gv - ref) / den))
             worst = max(worst, e)
             continue
         worst = max(worst, rel_err(got, ref))

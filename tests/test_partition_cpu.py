@@ -1,0 +1,80 @@
+"""Host checks of the GEMV kernel's work partition (compiled from the
+kernel's own header, run on the CPU): every segment has exactly one owning
+warp, the tile contributor ranges contain only owning warps, and the arrival
+bookkeeping (slots, counts) is consistent."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+from q4_quantized_decode_b200 import build_ext
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+@pytest.fixture(scope="module")
+def probe(tmp_path_factory):
+    out = tmp_path_factory.mktemp("probe") / "libprobe.so"
+    subprocess.check_call([build_ext.nvcc(), "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
+                           os.path.join(HERE, "partition_probe.cu"), "-o", str(out)])
+    lib = ctypes.CDLL(str(out))
+    for f in ("probe_seg_begin", "probe_warp_of_seg"):
+        getattr(lib, f).argtypes = [ctypes.c_int] * 3
+    lib.probe_xperm_pos.argtypes = [ctypes.c_int]
+    return lib
+
+
+CASES = [(1, 1), (4, 4), (4, 2), (17, 5), (1024, 256), (25600, 2368), (87040, 2368),
+         (174080, 2368), (160, 148), (1088 * 160, 2368), (7, 7), (100, 99)]
+
+
+@pytest.mark.parametrize("S,G", CASES)
+def test_partition_is_exact_cover(probe, S, G):
+    begins = [probe.probe_seg_begin(g, S, G) for g in range(G + 1)]
+    assert begins[0] == 0 and begins[G] == S
+    for g in range(G):
+        assert begins[g + 1] - begins[g] >= 1          # G <= S: no empty warp
+    for s in range(0, S, max(1, S // 5000)):
+        g = probe.probe_warp_of_seg(s, S, G)
+        assert begins[g] <= s < begins[g + 1]
+
+
+@pytest.mark.parametrize("S,G,KB", [(4, 4, 2), (25600, 2368, 160), (87040, 2368, 544),
+                                    (174080, 2368, 160), (1024, 256, 32), (8192, 2048, 1),
+                                    (12, 12, 3), (99, 50, 9)])
+def test_arrival_bookkeeping(probe, S, G, KB):
+    begins = [probe.probe_seg_begin(g, S, G) for g in range(G + 1)]
+    T = S // KB
+    arrivals = [0] * T
+    slots_used = set()
+    for g in range(G):
+        s0, s1 = begins[g], begins[g + 1]
+        t_first, t_last = s0 // KB, (s1 - 1) // KB
+        for t in range(t_first, t_last + 1):
+            gf = probe.probe_warp_of_seg(t * KB, S, G)
+            gl = probe.probe_warp_of_seg(t * KB + KB - 1, S, G)
+            whole = gf == gl
+            if t not in (t_first, t_last):
+                assert whole                        # middle tiles are owned whole
+            if not whole:
+                slot = 0 if t == t_first else 1
+                assert (g, slot) not in slots_used
+                slots_used.add((g, slot))
+                arrivals[t] += 1
+    for t in range(T):
+        gf = probe.probe_warp_of_seg(t * KB, S, G)
+        gl = probe.probe_warp_of_seg(t * KB + KB - 1, S, G)
+        assert arrivals[t] == (0 if gf == gl else gl - gf + 1)
+        for gg in range(gf, gl + 1):                # the reducer's slot choice
+            if gf != gl:
+                sl = 0 if begins[gg] // KB == t else 1
+                assert (gg, sl) in slots_used
+
+
+def test_xperm_is_a_permutation_grouping_lane_words(probe):
+    pos = [probe.probe_xperm_pos(j) for j in range(32)]
+    assert sorted(pos) == list(range(32))
+    for c in range(4):
+        group = {pos[j] for j in list(range(4 * c, 4 * c + 4)) + list(range(16 + 4 * c, 20 + 4 * c))}
+        assert group == set(range(8 * c, 8 * c + 8))
