@@ -230,8 +230,13 @@ def test_stack_small_end_to_end_and_teacher_forced(eng):
     x = synth.normal_f16(4321, synth.act_id(0), hidden)
     out, tx, ty = run_stack_traced(eng, layers, x, hidden, qkv_n, ffn)
     assert check_teacher_forced(ggufs, x, tx, ty, L, hidden, qkv_n, ffn) <= TOL
+    # End to end the chain only drifts as f16 rounding differences compound
+    # (an fp32 emulation drifts as much: tests/test_chain_drift_cpu.py), so
+    # this is a sanity bound, not the parity gate.
     want = oracle.stack_step(lambda l, t: ggufs[(l, t)], x, L, hidden, qkv_n, ffn)
-    assert rel_err(out, oracle.f16_to_f64(want)) <= TOL
+    drift = rel_err(out, oracle.f16_to_f64(want))
+    print(f"end-to-end drift after {L} layers: {drift:.2e}")
+    assert drift <= 10 * TOL
     # final renorm of the GPU's own last output
     assert np.abs(oracle.renorm(ty[4 * L - 1, :hidden]).astype(np.int32) - out.astype(np.int32)).max() <= 1
     # without traces the same bits come out
@@ -266,8 +271,9 @@ def test_stack_graph_replay_follows_input(eng):
     ob = bits_of(xout)
     wa = oracle.stack_step(lambda l, t: ggufs[(l, t)], xa, L, hidden, qkv_n, ffn)
     wb = oracle.stack_step(lambda l, t: ggufs[(l, t)], xb, L, hidden, qkv_n, ffn)
-    assert rel_err(oa, oracle.f16_to_f64(wa)) <= TOL
-    assert rel_err(ob, oracle.f16_to_f64(wb)) <= TOL
+    assert rel_err(oa, oracle.f16_to_f64(wa)) <= 10 * TOL
+    assert rel_err(ob, oracle.f16_to_f64(wb)) <= 10 * TOL
+    assert not np.array_equal(oa, ob)
     # x_out aliasing x_in is allowed
     eng.run_stack(layers, xin, hidden, qkv_n, ffn, x_out=xin)
     assert np.array_equal(bits_of(xin), ob)
