@@ -362,6 +362,53 @@ def run_ours(args, rank: int, world: int, dist):
     return 0
 
 
+def run_case(args):
+    """Standalone GEMV timing on one shape (configs 0-3 and profiling): R
+    copies of one packed matrix (R * size > 4 x L2 unless --rotate is given)
+    launched in rotation inside a CUDA graph; prints one JSON line."""
+    import torch
+    import q4_quantized_decode_b200 as q4
+    N, K = (int(v) for v in args.shape.lower().split("x"))
+    M = args.M
+    eng = q4.Q4Gemv(0)
+    seed = synth.config_seed(args.config_seed)
+    gguf = synth.q4_0_matrix(seed, synth.weight_id(0), N, K)
+    W0 = eng.repack(torch.from_numpy(gguf.reshape(-1)).cuda(), N, K)
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    R = args.rotate or max(2, -(-4 * l2 // W0.numel()))
+    mats = [W0] + [W0.clone() for _ in range(R - 1)]
+    x = torch.from_numpy(synth.activations(seed, M, K).view(np.float16)).cuda()
+    y = torch.empty(M, N, dtype=torch.float16, device="cuda")
+    eng.run(mats[0], x, N, K, out=y)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for W in mats:
+            eng.run(W, x, N, K, out=y)
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    if eng.sync_status() != q4.Q4_OK:
+        raise RuntimeError("device status")
+    us = e0.elapsed_time(e1) * 1e3 / (args.steps * R)
+    nbytes = N * (K // 32) * 18 + 2 * M * (K + N)
+    peak, kind = measured_peaks()
+    print(json.dumps({"case": f"gemv M={M} {N}x{K}", "N": N, "K": K, "M": M, "rotate": R,
+                      "us_per_launch": us, "GB/s": nbytes / us / 1e3,
+                      "frac_of_peak": nbytes / us / 1e3 / peak, "peak": peak, "peak_kind": kind,
+                      "rows_per_s": N / us * 1e6, "tflops": 2 * M * N * K / us / 1e6,
+                      "launches": args.steps * R}), flush=True)
+    eng.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -371,6 +418,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-shape", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--case", choices=["step", "gemv"], default="step",
+                    help="step: the decode step (default); gemv: one shape, see --shape/--M")
+    ap.add_argument("--shape", default="34816x5120", help="NxK for --case gemv")
+    ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--rotate", type=int, default=0, help="matrix copies in rotation (0: > 4x L2)")
+    ap.add_argument("--config-seed", type=int, default=2)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -378,6 +431,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank)
+    if args.case == "gemv":
+        return run_case(args)
     dist = None
     if world > 1:
         import datetime
