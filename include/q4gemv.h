@@ -97,14 +97,15 @@ Q4GEMV_API size_t q4gemv_gguf_bytes(int64_t N, int64_t K);
  * Packed layout (the input of q4gemv_run).  Rows are padded to Np (padding
  * rows hold qs bytes 0x88 and d = +0, i.e. zero weights) and grouped into
  * tiles of 32 rows.  With KB = K/32, segment s = t*KB + b holds block b of
- * the rows of tile t; row n = 32t + g + 8i (g in [0,8), i in [0,4)).
- *   nibble plane, bytes [0, Np*K/2): segment s occupies 512 bytes from
- *     512*s; its byte 16*(4g + c) + 4i + e is qs[4c + e] of that block of
- *     row n (c, e in [0,4)).  A lane (g, c) of a warp thus loads, with one
- *     16-byte load, qs word c of rows g, g+8, g+16, g+24.
- *   scale plane, bytes [Np*K/2, Np*K/2 + Np*K/16): segment s occupies 64
- *     bytes from Np*K/2 + 64*s; bytes 8g + 2i, 8g + 2i + 1 hold d of row n.
- * Every weight byte is read with 16-byte, fully coalesced loads. */
+ * the rows of tile t and occupies the 576 bytes from 576*s; row
+ * n = 32t + g + 8i (g in [0,8), i in [0,4)):
+ *   segment bytes 16*(4g + c) + 4i + e  = qs[4c + e] of that block of row n
+ *                                          (c, e in [0,4)), bytes [0, 512);
+ *   segment bytes 512 + 8g + 2i, +1      = d of that block of row n
+ *                                          (little-endian), bytes [512, 576).
+ * A lane (g, c) of a warp thus finds qs word c of rows g, g+8, g+16, g+24 in
+ * one 16-byte word and their four scales in one 8-byte word, and a run of
+ * segments is one contiguous byte range (one bulk copy). */
 Q4GEMV_API size_t q4gemv_packed_bytes(int64_t N, int64_t K);
 
 /* Host-only check of q4gemv_run's arguments (no device access, no handle).

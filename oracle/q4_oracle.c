@@ -101,30 +101,27 @@ void oracle_q4_gemv(const uint8_t* rows, int64_t nrows, int64_t K,
  * documented contract.  Rows are padded to Np = ceil(N/32)*32 (padding rows
  * hold qs bytes 0x88, i.e. q = 8, and d = +0) and grouped into tiles of 32.
  * With KB = K/32, segment s = t*KB + b holds block b of the 32 rows of tile
- * t.  Row n = 32t + r is written as r = g + 8i (g in [0,8), i in [0,4)).
- *   nibble plane, bytes [0, Np*K/2):
- *     byte 512*s + 16*(4g + c) + 4i + e  <-  qs[4c + e]     (c, e in [0,4))
- *   scale plane, bytes [Np*K/2, Np*K/2 + Np*K/16):
- *     bytes Np*K/2 + 64*s + 8g + 2i + {0,1}  <-  d (little-endian f16)   */
+ * t in the 576 bytes from 576*s.  Row n = 32t + r is written as r = g + 8i
+ * (g in [0,8), i in [0,4)).
+ *   byte 576*s + 16*(4g + c) + 4i + e      <-  qs[4c + e]     (c, e in [0,4))
+ *   bytes 576*s + 512 + 8g + 2i + {0,1}    <-  d (little-endian f16)        */
 void oracle_repack(const uint8_t* gguf, int64_t N, int64_t K, uint8_t* packed) {
     const int64_t KB = K / 32;
     const int64_t Np = (N + 31) / 32 * 32;
-    uint8_t* nib = packed;
-    uint8_t* scl = packed + Np * K / 2;
     for (int64_t n = 0; n < Np; ++n) {
         const int64_t t = n / 32, r = n % 32;
         const int64_t g = r % 8, i = r / 8;
         for (int64_t b = 0; b < KB; ++b) {
-            const int64_t s = t * KB + b;
+            uint8_t* seg = packed + 576 * (t * KB + b);
             uint8_t blk[18];
             for (int h = 0; h < 18; ++h)
                 blk[h] = (n < N) ? gguf[(n * KB + b) * 18 + h] : (h < 2 ? 0x00 : 0x88);
             for (int64_t j = 0; j < 16; ++j) {
                 const int64_t c = j / 4, e = j % 4;
-                nib[512 * s + 16 * (4 * g + c) + 4 * i + e] = blk[2 + j];
+                seg[16 * (4 * g + c) + 4 * i + e] = blk[2 + j];
             }
             for (int64_t h = 0; h < 2; ++h)
-                scl[64 * s + 8 * g + 2 * i + h] = blk[h];
+                seg[512 + 8 * g + 2 * i + h] = blk[h];
         }
     }
 }

@@ -5,15 +5,19 @@
 // section "The Engine: ~50 WGSL Kernels Written From Scratch").  On sm_100a
 // the row sweep is replaced by a flat, perfectly balanced split of all
 // (tile of 32 rows, 32-column block) segments over every warp of the grid:
-//   * lane (g, c) of a warp loads, with one 16-byte streaming load, qs word c
-//     of rows g, g+8, g+16, g+24 of a segment, so a warp reads 512 contiguous
-//     bytes per segment, and the 64-byte scale chunk alongside;
-//   * the activations of a 32-column block are converted once per CTA to
-//     16-bit integers with a power-of-two scale (the block maximum held
-//     exactly), staged in shared memory in the lane order of the weight
-//     words; each weight word is split into two byte vectors of codes with
-//     one shift and two masks and multiplied with dp2a (16-bit x 8-bit dot
-//     products), so the block sum of (q - 8) * X is an exact integer;
+//   * each warp streams its contiguous run of 576-byte segments (512 bytes of
+//     codes, 64 of scales) through a private ring of shared-memory stages,
+//     each filled by one bulk asynchronous copy (TMA); a few warps per SM
+//     keep ~150 KB per SM in flight, which register-staged loads cannot;
+//   * lane (g, c) reads qs word c of rows g, g+8, g+16, g+24 (16 bytes) and
+//     the four row scales (8 bytes) of a segment from the stage;
+//   * the activations are loaded once per CTA with plain 16-byte loads and
+//     converted in registers, per 32-column block, to 16-bit integers with a
+//     power-of-two scale (the block maximum held exactly); they are stored in
+//     shared memory in the lane order of the weight words.  Each weight word
+//     is split into two byte vectors of codes with one shift and two masks and
+//     multiplied with dp2a (16-bit x 8-bit dot products), so the block sum of
+//     (q - 8) * X is an exact integer;
 //   * the block sum is scaled by d * 2^e in fp32 and accumulated per row;
 //   * a warp's accumulators are combined across its four column lanes with
 //     two shuffles; tiles split between warps are combined by the last warp
@@ -22,15 +26,16 @@
 #pragma once
 
 #include "device_common.cuh"
+#include "partition.cuh"
 
 namespace q4 {
 
-constexpr int kSegNibBytes = 512;   // 32 rows x 16 bytes of codes
-constexpr int kSegSclBytes = 64;    // 32 rows x f16 scale
+constexpr int kSegBytes = 576;       // one segment: 512 bytes of codes, then 64 of scales
+constexpr int kSegSclOff = 512;
+constexpr int kXChunksPerThread = 9; // activation staging: M*K <= 9 * 8 * threads
 
 struct GemvArgs {
-    const uint8_t* nib;     // packed nibble plane
-    const uint8_t* scl;     // packed scale plane
+    const uint8_t* W;       // packed matrix (segments of 576 bytes)
     const __half* x;        // [M][K] activations, or the renorm source (M == 1)
     __half* y;              // [M][N]
     float* ws;              // split-tile partials [G][2][M][32]
@@ -44,20 +49,16 @@ struct GemvArgs {
     int renorm;             // 1: the input is renorm(x[0:K]) (M == 1 only)
 };
 
-// Shared-memory footprint of the kernel for M vectors of K columns.
-__host__ __device__ constexpr size_t gemv_dp2a_smem_bytes(int M, int K) {
-    // raw f16 x | int16 X (permuted) | -8*sum X per lane group | block scale
-    return (size_t)M * K * 2 + (size_t)M * K * 2 + (size_t)M * (K / 32) * 16 +
-           (size_t)M * (K / 32) * 4;
+// Per-warp ring of R stages of C segments.
+__host__ __device__ constexpr size_t ring_bytes(int warps, int R, int C) {
+    return (size_t)warps * R * C * kSegBytes;
 }
 
-// First segment of warp g under the flat balanced split of S segments over
-// G warps, and the warp that owns segment s.
-__host__ __device__ __forceinline__ int seg_begin(int g, int S, int G) {
-    return (int)(((int64_t)g * S) / G);
-}
-__host__ __device__ __forceinline__ int warp_of_seg(int s, int S, int G) {
-    return (int)((((int64_t)s + 1) * G - 1) / S);
+// Shared-memory footprint of the M <= 2 kernel: the ring, the int16
+// activations (2 bytes per element) and, per block and lane group, the pair
+// {-8 * sum X, block scale} (8 bytes, 32 per block).
+__host__ __device__ constexpr size_t gemv_dp2a_smem_bytes(int M, int K, int warps, int R, int C) {
+    return ring_bytes(warps, R, C) + (size_t)M * K * 2 + (size_t)M * (K / 32) * 32;
 }
 
 // Position of element j of a 32-column block in the permuted X layout: the
@@ -67,122 +68,174 @@ __host__ __device__ __forceinline__ int xperm_pos(int j) {
     return ((j & 15) >> 2) * 8 + ((j >> 4) << 2) + (j & 3);
 }
 
-// Renormalise buf[0:len) (f16, shared memory) in place to unit RMS:
-// s = sum v^2 in fp32 (fixed order: thread-strided partials, warp xor tree,
-// then warps in order), scale = 1/sqrt(s/len), v <- f16(v * scale); an
-// all-zero vector stays zero.  Must be called by all NT threads of the CTA.
-template <int NT>
-__device__ __forceinline__ void block_renorm_inplace(__half* buf, int len, float* red) {
-    const int tid = threadIdx.x;
-    float part = 0.f;
-    for (int i = tid; i < len; i += NT) {
-        const float v = __half2float(buf[i]);
-        part = fmaf(v, v, part);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    if ((tid & 31) == 0) red[tid >> 5] = part;
-    __syncthreads();
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < NT / 32; ++w) s += red[w];
-    const float scale = (s > 0.f) ? __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(s, (float)len))) : 0.f;
-    for (int i = tid; i < len; i += NT)
-        buf[i] = __float2half_rn(__half2float(buf[i]) * scale);
-    __syncthreads();
-}
+// A warp's private ring: stage k holds C consecutive segments of the warp's
+// run [s0, s1), filled by one elected lane with one bulk copy.
+template <int R, int C>
+struct WarpRing {
+    uint32_t stage0;        // shared address of this warp's first stage
+    uint64_t* bars;         // R full-barriers
+    const uint8_t* src;     // segment s0 in global memory
+    int nseg;               // s1 - s0
+    int nch;                // ceil(nseg / C)
 
-// Stage x: bulk copy into shared memory (after the dependency wait),
-// optional renorm, conversion to per-block 16-bit integers.
-template <int M, int WARPS>
-__device__ __forceinline__ bool stage_activations(const GemvArgs& a, __half* raw, int16_t* Xs,
-                                                  int* negC, float* sb, uint64_t* bar,
+    __device__ void init(uint32_t ring_base, uint64_t* bar_base, int warp, const uint8_t* W, int s0,
+                         int s1) {
+        stage0 = ring_base + (uint32_t)warp * R * C * kSegBytes;
+        bars = bar_base + warp * R;
+        src = W + (size_t)s0 * kSegBytes;
+        nseg = s1 - s0;
+        nch = (nseg + C - 1) / C;
+    }
+    __device__ uint32_t stage(int k) const { return stage0 + (uint32_t)k * C * kSegBytes; }
+    // Lane 0 only.
+    __device__ void issue(int ch) const {
+        const int k = ch % R;
+        const uint32_t bytes = (uint32_t)min(C, nseg - ch * C) * kSegBytes;
+        mbar_arrive_expect_tx(bars + k, bytes);
+        bulk_g2s_addr(stage(k), src + (size_t)ch * C * kSegBytes, bytes, bars + k);
+    }
+    __device__ bool wait(int ch) const {
+        return mbar_wait_bounded(bars + (ch % R), (uint32_t)((ch / R) & 1), 1u << 22);
+    }
+};
+
+// Activation staging for the M <= 2 kernel, all threads of the CTA.  Thread
+// t holds the 16-byte chunks q = t, t + NT, ... of x (8 elements each; four
+// chunks make a 32-column block, held by four consecutive lanes).  For M = 1
+// with `renorm`, the vector is first scaled to unit RMS: s = sum v^2 in fp32
+// (fixed order: per thread, then warp xor tree, then warps in order), each v
+// becomes f16(v * 1/sqrt(s/K)), an all-zero vector stays zero.  Each block is
+// then converted to X = rint(v * 2^(14-E)) (E: exponent of the block maximum,
+// so |X| <= 32752 and the maximum is exact) and written in lane order; lane
+// group c of the block gets {-8 * sum of its eight X, 2^(E-14)}.
+template <int M, int NT>
+__device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs, uint32_t rec,
                                                   float* red) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const uint32_t bytes = (uint32_t)M * a.K * 2;
-    if (tid == 0) {
-        mbar_arrive_expect_tx(bar, bytes);
-        bulk_g2s(raw, a.x, bytes, bar);
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int nq = M * a.K / 8;
+    uint4 xr[kXChunksPerThread];
+#pragma unroll
+    for (int i = 0; i < kXChunksPerThread; ++i) {
+        const int q = tid + NT * i;
+        xr[i] = q < nq ? *reinterpret_cast<const uint4*>(a.x + (size_t)q * 8) : make_uint4(0, 0, 0, 0);
     }
-    // ~1e6 polls: far beyond any real completion time, short of a hang.  The
-    // CTA agrees on the outcome so that every thread leaves together.
-    const bool arrived = mbar_wait_bounded(bar, 0, 1u << 20);
-    if (!__syncthreads_and(arrived)) {
-        if (tid == 0) set_device_error(a.err, kDevTimeout);
-        return false;
-    }
-    if (M == 1 && a.renorm) block_renorm_inplace<WARPS * 32>(raw, a.K, red);
-    if (a.trace_x != nullptr && blockIdx.x == 0) {
-        for (int i = tid; i < a.K; i += WARPS * 32) a.trace_x[i] = raw[i];
-    }
-    const int nblk = M * a.KB;
-    for (int bb = warp; bb < nblk; bb += WARPS) {
-        const int m = bb / a.KB, b = bb - m * a.KB;
-        const float v = __half2float(raw[(size_t)m * a.K + b * 32 + lane]);
-        const uint32_t mx = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v)));
-        int X = 0;
+    if (M == 1 && a.renorm) {
+        float part = 0.f;
+#pragma unroll
+        for (int i = 0; i < kXChunksPerThread; ++i) {
+            const __half2* h = reinterpret_cast<const __half2*>(&xr[i]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(h[e]);
+                part = fmaf(f.x, f.x, part);
+                part = fmaf(f.y, f.y, part);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (lane == 0) red[tid >> 5] = part;
+        __syncthreads();
         float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < NT / 32; ++w) s += red[w];
+        const float scale = (s > 0.f) ? __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(s, (float)a.K))) : 0.f;
+#pragma unroll
+        for (int i = 0; i < kXChunksPerThread; ++i) {
+            __half2* h = reinterpret_cast<__half2*>(&xr[i]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(h[e]);
+                h[e] = __floats2half2_rn(f.x * scale, f.y * scale);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kXChunksPerThread; ++i) {
+        const int q = tid + NT * i;
+        if (M == 1 && a.trace_x != nullptr && blockIdx.x == 0 && q < nq)
+            *reinterpret_cast<uint4*>(a.trace_x + (size_t)q * 8) = xr[i];
+        // The four chunks of a block sit in lanes 4j..4j+3 (NT*i is a multiple
+        // of 4), so every lane takes part in the shuffles below.
+        const __half2* h = reinterpret_cast<const __half2*>(&xr[i]);
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(h[e]);
+            v[2 * e] = f.x;
+            v[2 * e + 1] = f.y;
+        }
+        uint32_t mx = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx = max(mx, __float_as_uint(fabsf(v[e])));
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        int X[8];
+        float sc = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) X[e] = 0;
         if (mx >= 0x7F800000u) {
-            s = __uint_as_float(0x7FC00000u);          // non-finite block -> NaN outputs
+            sc = __uint_as_float(0x7FC00000u);          // non-finite block -> NaN outputs
         } else if (mx != 0u) {
             const int E = (int)(mx >> 23) - 127;        // block max in [2^E, 2^(E+1))
             const float inv = __uint_as_float((uint32_t)(141 - E) << 23);   // 2^(14-E)
-            X = __float2int_rn(v * inv);                // |X| <= 32752, exact for the max
-            s = __uint_as_float((uint32_t)(113 + E) << 23);                 // 2^(E-14)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) X[e] = __float2int_rn(v[e] * inv);
+            sc = __uint_as_float((uint32_t)(113 + E) << 23);                 // 2^(E-14)
         }
-        Xs[(size_t)m * a.K + b * 32 + xperm_pos(lane)] = (int16_t)X;
-        int gs = X;
-        gs += __shfl_xor_sync(0xffffffffu, gs, 1);
-        gs += __shfl_xor_sync(0xffffffffu, gs, 2);
-        gs += __shfl_xor_sync(0xffffffffu, gs, 16);
-        if (lane < 16 && (lane & 3) == 0) negC[((size_t)m * a.KB + b) * 4 + (lane >> 2)] = -8 * gs;
-        if (lane == 0) sb[(size_t)m * a.KB + b] = s;
+        int h0 = X[0] + X[1] + X[2] + X[3], h1 = X[4] + X[5] + X[6] + X[7];
+        h0 += __shfl_xor_sync(0xffffffffu, h0, 2);      // quarters u and u^2 share lane groups
+        h1 += __shfl_xor_sync(0xffffffffu, h1, 2);
+        if (q < nq) {
+            const int bb = q >> 2, u = q & 3;
+            const int pos0 = (u & 1) * 16 + (u >> 1) * 4;   // elements 8u..8u+3 (then +8 for 8u+4..8u+7)
+            const uint32_t xb = xs + (uint32_t)bb * 64;
+            sts64(xb + pos0 * 2, pack_s16x4(X[0], X[1], X[2], X[3]));
+            sts64(xb + pos0 * 2 + 16, pack_s16x4(X[4], X[5], X[6], X[7]));
+            if (u < 2) {
+                const int c0 = (u & 1) * 2;
+                const uint32_t rb = rec + (uint32_t)bb * 32 + c0 * 8;
+                sts64(rb, make_uint2((uint32_t)(-8 * h0), __float_as_uint(sc)));
+                sts64(rb + 8, make_uint2((uint32_t)(-8 * h1), __float_as_uint(sc)));
+            }
+        }
     }
     __syncthreads();
-    return true;
 }
 
-template <int M, int WARPS, int U>
+template <int M, int WARPS, int R, int C>
 __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ __align__(8) uint64_t bar;
+    __shared__ __align__(8) uint64_t bars[WARPS * R];
     __shared__ float red[WARPS];
 
-    __half* raw = reinterpret_cast<__half*>(smem);
-    int16_t* Xs = reinterpret_cast<int16_t*>(smem + (size_t)M * a.K * 2);
-    int* negC = reinterpret_cast<int*>(smem + (size_t)M * a.K * 4);
-    float* sb = reinterpret_cast<float*>(smem + (size_t)M * a.K * 4 + (size_t)M * a.KB * 16);
+    const uint32_t smem_base = smem_addr(smem);
+    const uint32_t xs = smem_base + (uint32_t)ring_bytes(WARPS, R, C);   // int16 X, lane order
+    const uint32_t rec = xs + (uint32_t)(M * a.K * 2);                  // {-8 sum X, scale}
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, c = lane & 3;
     const int gw = blockIdx.x * WARPS + warp;
     // G <= S, so every warp below G owns at least one segment; warps of the
     // last CTA beyond G only help stage the activations.
-    const int s0 = gw < a.G ? seg_begin(gw, a.S, a.G) : a.S;
-    const int s1 = gw < a.G ? seg_begin(gw + 1, a.S, a.G) : a.S;
+    WarpSplit sp;
+    sp.init(gw, a.S, a.G, a.KB);
+    const int s0 = sp.s0, s1 = sp.s1;
 
-    if (threadIdx.x == 0) {
-        mbar_init(&bar, 1);
+    WarpRing<R, C> ring;
+    ring.init(smem_base, bars, warp, a.W, s0, s1);
+    if (lane == 0) {
+        for (int k = 0; k < R; ++k) mbar_init(bars + warp * R + k, 1);
         fence_barrier_init();
     }
-
-    // Weight prefetch: independent of the previous kernel, so it is issued
-    // before the dependency wait.
-    uint4 wq[U];
-    uint2 wd[U];
-#pragma unroll
-    for (int j = 0; j < U; ++j) {
-        const int s = s0 + j;
-        if (s < s1) {
-            wq[j] = ldg_stream_v4(a.nib + (size_t)s * kSegNibBytes + lane * 16);
-            wd[j] = ldg_stream_v2(a.scl + (size_t)s * kSegSclBytes + g * 8);
-        }
-    }
+    __syncwarp();
+    // Weights do not depend on the previous kernel: start the stream before
+    // the dependency wait.
+    if (lane == 0)
+        for (int ch = 0; ch < R && ch < ring.nch; ++ch) ring.issue(ch);
     pdl_launch_dependents();
-    __syncthreads();   // barrier init visible to all threads
     pdl_wait();
 
-    if (!stage_activations<M, WARPS>(a, raw, Xs, negC, sb, &bar, red)) return;
+    stage_activations<M, WARPS * 32>(a, xs, rec, red);
 
     float acc[M][4];
 #pragma unroll
@@ -191,10 +244,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
         for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
 
     const int KB = a.KB;
-    const int t_first = s0 / KB;
+    const int t_first = sp.t_first;
     int t_cur = t_first;
-    int tile_end = (t_cur + 1) * KB;
-    const int r = g + 8 * c;                  // row of the tile this lane emits
+    int b = s0 - t_first * KB;                 // block of the next segment
+    const int r = g + 8 * c;                   // row of the tile this lane emits
+    // Running shared addresses of block b's X words and records for this lane.
+    const uint32_t x_lane0 = xs + (uint32_t)c * 16, r_lane0 = rec + (uint32_t)c * 8;
+    uint32_t xp = x_lane0 + (uint32_t)b * 64, rp = r_lane0 + (uint32_t)b * 32;
 
     // Combine a finished tile: reduce over the four column lanes, then either
     // write y (this warp owns the whole tile) or park the partial.
@@ -208,7 +264,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
                 v += __shfl_xor_sync(0xffffffffu, v, 2);
                 acc[m][i] = v;
             }
-        const bool whole = warp_of_seg(t * KB, a.S, a.G) == warp_of_seg(t * KB + KB - 1, a.S, a.G);
+        const bool whole = sp.whole(t);
         const int64_t row = (int64_t)t * 32 + r;
 #pragma unroll
         for (int m = 0; m < M; ++m) {
@@ -216,135 +272,188 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
             if (whole) {
                 if (row < a.N) a.y[(size_t)m * a.N + row] = __float2half_rn(val);
             } else {
-                const int slot = (t == t_first) ? 0 : 1;
-                a.ws[(((size_t)gw * 2 + slot) * M + m) * 32 + r] = val;
+                a.ws[(((size_t)gw * 2 + sp.slot(t)) * M + m) * 32 + r] = val;
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
         }
     };
 
-    for (int base = s0; base < s1; base += U) {
+    // One segment at shared address `seg`: codes and scales from the ring
+    // stage, X and the block record from the staged activations.
+    auto segment = [&](uint32_t seg) {
+        const uint4 w = lds128(seg + lane * 16);
+        const uint2 dd = lds64(seg + kSegSclOff + g * 8);
+        const float2 d01 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
+        const float2 d23 = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
+        const float d[4] = {d01.x, d01.y, d23.x, d23.y};
+        const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+        uint4 xq[M];
+        uint2 rc[M];
 #pragma unroll
-        for (int j = 0; j < U; ++j) {
-            const int s = base + j;
-            if (s < s1) {
-                if (s == tile_end) {
-                    flush(t_cur);
-                    ++t_cur;
-                    tile_end += KB;
-                }
-                const int b = s - t_cur * KB;
-                const uint4 w = wq[j];
-                const uint2 dd = wd[j];
-                const int sn = s + U;
-                if (sn < s1) {
-                    wq[j] = ldg_stream_v4(a.nib + (size_t)sn * kSegNibBytes + lane * 16);
-                    wd[j] = ldg_stream_v2(a.scl + (size_t)sn * kSegSclBytes + g * 8);
-                }
-                const float2 d01 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
-                const float2 d23 = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
-                const float d[4] = {d01.x, d01.y, d23.x, d23.y};
-                const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-                uint4 xq[M];
-                int nc[M];
-                float sbm[M];
+        for (int m = 0; m < M; ++m) {
+            xq[m] = lds128(xp + (uint32_t)m * a.K * 2);
+            rc[m] = lds64(rp + (uint32_t)m * KB * 32);
+        }
 #pragma unroll
-                for (int m = 0; m < M; ++m) {
-                    xq[m] = *reinterpret_cast<const uint4*>(Xs + (size_t)m * a.K + b * 32 + c * 8);
-                    nc[m] = negC[((size_t)m * KB + b) * 4 + c];
-                    sbm[m] = sb[(size_t)m * KB + b];
-                }
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = words[i] & 0x0F0F0F0Fu;          // codes 4c..4c+3
+            const uint32_t hi = (words[i] >> 4) & 0x0F0F0F0Fu;   // codes 4c+16..4c+19
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t lo = words[i] & 0x0F0F0F0Fu;          // codes 4c..4c+3
-                    const uint32_t hi = (words[i] >> 4) & 0x0F0F0F0Fu;   // codes 4c+16..4c+19
-#pragma unroll
-                    for (int m = 0; m < M; ++m) {
-                        int v = dp2a_lo(xq[m].x, lo, nc[m]);
-                        v = dp2a_hi(xq[m].y, lo, v);
-                        v = dp2a_lo(xq[m].z, hi, v);
-                        v = dp2a_hi(xq[m].w, hi, v);
-                        acc[m][i] = fmaf((float)v, d[i] * sbm[m], acc[m][i]);
-                    }
-                }
+            for (int m = 0; m < M; ++m) {
+                int v = dp2a_lo(xq[m].x, lo, (int)rc[m].x);
+                v = dp2a_hi(xq[m].y, lo, v);
+                v = dp2a_lo(xq[m].z, hi, v);
+                v = dp2a_hi(xq[m].w, hi, v);
+                acc[m][i] = fmaf((float)v, d[i] * __uint_as_float(rc[m].y), acc[m][i]);
             }
         }
+    };
+    auto advance = [&]() {
+        ++b;
+        xp += 64;
+        rp += 32;
+    };
+    auto maybe_flush = [&]() {
+        if (b == KB) {
+            flush(t_cur);
+            ++t_cur;
+            b = 0;
+            xp = x_lane0;
+            rp = r_lane0;
+        }
+    };
+
+    for (int ch = 0; ch < ring.nch; ++ch) {
+        if (!ring.wait(ch)) set_device_error(a.err, kDevTimeout);   // data then unreliable
+        const uint32_t st = ring.stage(ch % R);
+        const int n = min(C, ring.nseg - ch * C);
+        if (n == C) {
+#pragma unroll
+            for (int j = 0; j < C; ++j) {
+                maybe_flush();
+                segment(st + j * kSegBytes);
+                advance();
+            }
+        } else {
+            for (int j = 0; j < n; ++j) {
+                maybe_flush();
+                segment(st + j * kSegBytes);
+                advance();
+            }
+        }
+        // Stage fully read: hand it back to the async proxy for the refill.
+        __syncwarp();
+        fence_proxy_async_smem();
+        if (lane == 0 && ch + R < ring.nch) ring.issue(ch + R);
     }
     if (s1 > s0) flush(t_cur);
 
     // Tiles shared with other warps (at most the first and the last one of
     // this warp's range): count arrivals; the last warp to arrive sums the
     // partials in warp order, writes y and re-arms the counter.
-    auto arrive = [&](int t) {
-        const int gf = warp_of_seg(t * KB, a.S, a.G), gl = warp_of_seg(t * KB + KB - 1, a.S, a.G);
+    auto arrive = [&](int t, int gf, int gl) {
         if (gf == gl) return;
-        __threadfence();
         __syncwarp();
         int old = 0;
-        if (lane == 0) old = atomicAdd(a.cnt + t, 1);
+        if (lane == 0) old = atom_add_acq_rel_gpu(a.cnt + t, 1);
         old = __shfl_sync(0xffffffffu, old, 0);
+        __syncwarp();                       // order the lanes' reads after lane 0's acquire
         const int need = gl - gf + 1;
         if (old == need - 1) {
-            __threadfence();
             const int64_t row = (int64_t)t * 32 + r;
+            float sum[M];
 #pragma unroll
-            for (int m = 0; m < M; ++m) {
-                float sum = 0.f;
-                for (int gg = gf; gg <= gl; ++gg) {
-                    const int sl = (seg_begin(gg, a.S, a.G) / KB == t) ? 0 : 1;
-                    sum += __ldcg(a.ws + (((size_t)gg * 2 + sl) * M + m) * 32 + r);
+            for (int m = 0; m < M; ++m) sum[m] = 0.f;
+            SegWalker wk;
+            wk.init(gf, a.S, a.G);
+            // Eight contributors per round: their loads are issued together,
+            // the sum is still taken in warp order.
+            for (int g0 = gf; g0 <= gl; g0 += 8) {
+                float pv[8][M];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int gg = g0 + u;
+                    const int sl = (wk.sb >= t * KB) ? 0 : 1;   // t is where gg's run starts
+#pragma unroll
+                    for (int m = 0; m < M; ++m)
+                        pv[u][m] = gg <= gl ? ld_relaxed_gpu(a.ws + (((size_t)gg * 2 + sl) * M + m) * 32 + r)
+                                            : 0.f;
+                    wk.next();
                 }
-                if (row < a.N) a.y[(size_t)m * a.N + row] = __float2half_rn(sum);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+#pragma unroll
+                    for (int m = 0; m < M; ++m) sum[m] += pv[u][m];
             }
+#pragma unroll
+            for (int m = 0; m < M; ++m)
+                if (row < a.N) a.y[(size_t)m * a.N + row] = __float2half_rn(sum[m]);
             if (lane == 0) a.cnt[t] = 0;
         } else if (old >= need) {
             if (lane == 0) set_device_error(a.err, kDevConcurrent);
         }
     };
     if (s1 > s0) {
-        const int t_last = (s1 - 1) / KB;
-        arrive(t_first);
-        if (t_last != t_first) arrive(t_last);
+        arrive(sp.t_first, sp.gf0, sp.gl0);
+        if (sp.t_last != sp.t_first) arrive(sp.t_last, sp.gf1, sp.gl1);
     }
 }
 
-// Final renorm of the decode step: out = renorm(in[0:len)).
+// Final renorm of the decode step: out = renorm(in[0:len)), with the same
+// arithmetic (and order) as the renorm fused into the GEMV prologue.
 template <int WARPS>
-__global__ void __launch_bounds__(WARPS * 32, 1) renorm_kernel(const __half* in, __half* out, int len,
-                                                             int* err) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ __align__(8) uint64_t bar;
+__global__ void __launch_bounds__(WARPS * 32, 1) renorm_kernel(const __half* in, __half* out, int len) {
     __shared__ float red[WARPS];
-    __half* buf = reinterpret_cast<__half*>(smem);
-    if (threadIdx.x == 0) {
-        mbar_init(&bar, 1);
-        fence_barrier_init();
-    }
-    __syncthreads();
+    constexpr int NT = WARPS * 32;
+    const int tid = threadIdx.x, lane = tid & 31;
     pdl_wait();
-    if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(&bar, (uint32_t)len * 2);
-        bulk_g2s(buf, in, (uint32_t)len * 2, &bar);
+    const int nq = len / 8;
+    uint4 xr[kXChunksPerThread];
+#pragma unroll
+    for (int i = 0; i < kXChunksPerThread; ++i) {
+        const int q = tid + NT * i;
+        xr[i] = q < nq ? *reinterpret_cast<const uint4*>(in + (size_t)q * 8) : make_uint4(0, 0, 0, 0);
     }
-    const bool arrived = mbar_wait_bounded(&bar, 0, 1u << 20);
-    if (!__syncthreads_and(arrived)) {
-        if (threadIdx.x == 0) set_device_error(err, kDevTimeout);
-        return;
+    float part = 0.f;
+#pragma unroll
+    for (int i = 0; i < kXChunksPerThread; ++i) {
+        const __half2* h = reinterpret_cast<const __half2*>(&xr[i]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(h[e]);
+            part = fmaf(f.x, f.x, part);
+            part = fmaf(f.y, f.y, part);
+        }
     }
-    block_renorm_inplace<WARPS * 32>(buf, len, red);
-    for (int i = threadIdx.x; i < len; i += WARPS * 32) out[i] = buf[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) red[tid >> 5] = part;
+    __syncthreads();
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) s += red[w];
+    const float scale = (s > 0.f) ? __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(s, (float)len))) : 0.f;
+#pragma unroll
+    for (int i = 0; i < kXChunksPerThread; ++i) {
+        const int q = tid + NT * i;
+        __half2* h = reinterpret_cast<__half2*>(&xr[i]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(h[e]);
+            h[e] = __floats2half2_rn(f.x * scale, f.y * scale);
+        }
+        if (q < nq) *reinterpret_cast<uint4*>(out + (size_t)q * 8) = xr[i];
+    }
 }
 
 // GGUF Q4_0 -> packed layout, one warp per segment (grid-stride).
 __global__ void __launch_bounds__(256) repack_kernel(const uint8_t* __restrict__ gguf,
                                                      uint8_t* __restrict__ packed, int64_t N,
-                                                     int KB, int64_t S, int64_t Np) {
+                                                     int KB, int64_t S) {
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    uint8_t* nib = packed;
-    uint8_t* scl = packed + Np * KB * 16;
     for (int64_t s = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); s < S; s += nwarps) {
         const int64_t t = s / KB, b = s - t * KB;
         uint32_t words[4];
@@ -361,10 +470,10 @@ __global__ void __launch_bounds__(256) repack_kernel(const uint8_t* __restrict__
                 dv[i] = 0;
             }
         }
-        *reinterpret_cast<uint4*>(nib + s * kSegNibBytes + lane * 16) =
-            make_uint4(words[0], words[1], words[2], words[3]);
+        uint8_t* seg = packed + s * kSegBytes;
+        *reinterpret_cast<uint4*>(seg + lane * 16) = make_uint4(words[0], words[1], words[2], words[3]);
         if (c == 0) {
-            *reinterpret_cast<uint2*>(scl + s * kSegSclBytes + g * 8) =
+            *reinterpret_cast<uint2*>(seg + kSegSclOff + g * 8) =
                 make_uint2((uint32_t)dv[0] | ((uint32_t)dv[1] << 16),
                            (uint32_t)dv[2] | ((uint32_t)dv[3] << 16));
         }

@@ -1,0 +1,307 @@
+// Q4_0 GEMV for M = 3..16 activation vectors (speculative verify, prefill
+// chunks): each dequantised weight tile is applied to all M vectors with
+// tensor-core mma.sync.m16n8k16 (f16 inputs, f32 accumulate).
+//
+// Speculative verification runs a batch of draft tokens through the trunk in
+// one pass and prefill batches 16 tokens per round trip (aipolix en-US page,
+// section "Speculation is used to amortize network round trips";
+// originshq.com page, section "Multi-Device Performance and the Network
+// Penalty"); the weight stream is the same as decode, the arithmetic grows
+// with M.  With M >= 4 the CUDA-core dp2a path needs more issue slots per
+// weight than the HBM rate allows on B200, so the block products move to the
+// tensor cores while the rest of the design is shared with the M <= 2 kernel
+// (segment-tiled layout, per-warp TMA ring, flat warp split, deterministic
+// split-tile combine).
+//
+// Per segment (32 rows x one 32-column block) and lane (g, c): the four
+// 32-bit code words of rows g, g+8, g+16, g+24 give, with one shift and four
+// masks, exact (q - 8) as f16 pairs (magic exponent 2^10 in the mantissa,
+// then one subtract or fused multiply-add); they are the A fragments of two
+// 16-row MMA tiles in the fragment order of m16n8k16 after a fixed
+// permutation of k inside the block, matched by the order in which the
+// activations are staged in shared memory.  Two MMAs (low and high nibbles)
+// give the exact block dot products in fp32; the per-row scale d is applied
+// with one FFMA per output, so no rounding of d * (q - 8) is ever made.
+#pragma once
+
+#include "gemv_dp2a.cuh"
+
+namespace q4 {
+
+struct MmaArgs {
+    const uint8_t* W;    // packed matrix (segments of 576 bytes)
+    const __half* x;     // [M][K]
+    __half* y;           // [M][N]
+    float* ws;           // [G][2][16][32] split-tile partials
+    int* cnt;            // [T] arrival counters, zero between calls
+    int* err;
+    int64_t N;
+    int K, KB, T, S, G;
+    int M;               // 1..16 (columns >= M are zero-padded)
+};
+
+// Bytes per staged activation vector for `nblk` blocks: 64 per block, padded
+// so consecutive vectors start 64 bytes apart modulo 128 (conflict-free
+// 16-byte loads by the eight lane groups).
+__host__ __device__ constexpr int mma_vstride(int nblk) {
+    return nblk * 64 + ((nblk & 1) ? 0 : 64);
+}
+__host__ __device__ constexpr size_t gemv_mma_smem_bytes(int nt8, int nblk) {
+    return (size_t)8 * nt8 * mma_vstride(nblk);
+}
+
+// Position of element e of a 32-column block in the staged order: lane group
+// c reads [x4c, x4c+2, x4c+1, x4c+3 | x4c+16, x4c+18, x4c+17, x4c+19].
+__host__ __device__ __forceinline__ int mma_xpos(int e) {
+    const int r = e & 3;
+    return ((e & 15) >> 2) * 8 + (e >> 4) * 4 + (((r & 1) << 1) | (r >> 1));
+}
+
+__device__ __forceinline__ uint32_t lop_mask_or(uint32_t w, uint32_t mask, uint32_t magic) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "r"(mask), "r"(magic));  // (a & b) | c
+    return d;
+}
+
+__device__ __forceinline__ void mma_16816(float& d0, float& d1, float& d2, float& d3, uint32_t a0,
+                                          uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                          uint32_t b1, float c0, float c1, float c2, float c3) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%11,%12,%13};"
+        : "=f"(d0), "=f"(d1), "=f"(d2), "=f"(d3)
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(c2),
+          "f"(c3));
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// Exact (q - 8) f16 pairs from one code word: lo/hi nibbles of bytes (0, 2)
+// and (1, 3).
+struct CodePairs {
+    uint32_t p, q, r, s;   // p: k(4c, 4c+2)  q: k(4c+1, 4c+3)  r: k(4c+16, 4c+18)  s: k(4c+17, 4c+19)
+};
+__device__ __forceinline__ CodePairs unpack_pairs(uint32_t w) {
+    const uint32_t magic = 0x64006400u;     // f16 1024.0 in both halves
+    const uint32_t w8 = w >> 8;
+    const __half2 off_lo = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));  // 1032
+    const __half2 sixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));  // 1/16
+    const __half2 m72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));  // -72
+    CodePairs o;
+    o.p = h2_bits(__hsub2(bits_h2(lop_mask_or(w, 0x000F000Fu, magic)), off_lo));
+    o.q = h2_bits(__hsub2(bits_h2(lop_mask_or(w8, 0x000F000Fu, magic)), off_lo));
+    o.r = h2_bits(__hfma2(bits_h2(lop_mask_or(w, 0x00F000F0u, magic)), sixteenth, m72));
+    o.s = h2_bits(__hfma2(bits_h2(lop_mask_or(w8, 0x00F000F0u, magic)), sixteenth, m72));
+    return o;
+}
+
+template <int NT8, int WARPS, int R, int C>
+__global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ __align__(8) uint64_t bars[WARPS * R];
+    constexpr int NT = WARPS * 32;
+    const uint32_t smem_base = smem_addr(smem);
+    const uint32_t xsm = smem_base + (uint32_t)ring_bytes(WARPS, R, C);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, c = lane & 3;
+    const int gw = blockIdx.x * WARPS + warp;
+    WarpSplit sp;
+    sp.init(gw, a.S, a.G, a.KB);
+    const int s0 = sp.s0, s1 = sp.s1;
+    const int KB = a.KB;
+
+    // The CTA's blocks: its warps own one contiguous run of segments.
+    const int w_lo = blockIdx.x * WARPS;
+    const int w_hi = min(w_lo + WARPS, a.G);
+    const int cs0 = w_lo < a.G ? seg_begin(w_lo, a.S, a.G) : a.S;
+    const int cs1 = w_hi > w_lo ? (w_hi < a.G ? seg_begin(w_hi, a.S, a.G) : a.S) : cs0;
+    const int nblk = (cs1 - cs0 >= KB) ? KB : (cs1 - cs0);
+    const int b0 = (cs1 - cs0 >= KB) ? 0 : (cs0 % KB);
+    const int vstride = mma_vstride(nblk);
+
+    WarpRing<R, C> ring;
+    ring.init(smem_base, bars, warp, a.W, s0, s1);
+    if (lane == 0) {
+        for (int k = 0; k < R; ++k) mbar_init(bars + warp * R + k, 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    if (lane == 0)
+        for (int ch = 0; ch < R && ch < ring.nch; ++ch) ring.issue(ch);
+    pdl_launch_dependents();
+    pdl_wait();
+
+    // Stage the CTA's activation blocks with plain 16-byte loads (four per
+    // round per thread), reordered into lane order; zero vectors pad M up to
+    // 8*NT8.
+    {
+        const int nchunk = a.M * nblk * 4;
+        for (int p0 = threadIdx.x; p0 < nchunk; p0 += 4 * NT) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int p = p0 + u * NT;
+                if (p < nchunk) {
+                    const int vv = p / (nblk * 4), rem = p - vv * nblk * 4;
+                    int b = b0 + (rem >> 2);
+                    if (b >= KB) b -= KB;
+                    v[u] = *reinterpret_cast<const uint4*>(a.x + (size_t)vv * a.K + b * 32 + (rem & 3) * 8);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int p = p0 + u * NT;
+                if (p < nchunk) {
+                    const int vv = p / (nblk * 4), rem = p - vv * nblk * 4;
+                    const int jb = rem >> 2, qt = rem & 3;
+                    const int pos0 = (qt & 1) * 16 + (qt >> 1) * 4;
+                    const uint32_t dst = xsm + (uint32_t)vv * vstride + (uint32_t)jb * 64 + pos0 * 2;
+                    sts64(dst, make_uint2(__byte_perm(v[u].x, v[u].y, 0x5410),
+                                          __byte_perm(v[u].x, v[u].y, 0x7632)));
+                    sts64(dst + 16, make_uint2(__byte_perm(v[u].z, v[u].w, 0x5410),
+                                               __byte_perm(v[u].z, v[u].w, 0x7632)));
+                }
+            }
+        }
+        const int zwords = (8 * NT8 - a.M) * vstride / 8;
+        for (int i = threadIdx.x; i < zwords; i += NT)
+            sts64(xsm + (uint32_t)a.M * vstride + (uint32_t)i * 8, make_uint2(0u, 0u));
+        __syncthreads();
+    }
+
+    float acc[2][NT8][4];
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+        for (int nt = 0; nt < NT8; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[tt][nt][i] = 0.f;
+
+    const int t_first = sp.t_first;
+    int t_cur = t_first;
+
+    // Output (row, column) held by acc[tt][nt][i]:
+    //   row = 16*tt + g + 8*(i >> 1), column = 8*nt + 2c + (i & 1).
+    auto flush = [&](int t) {
+        const bool whole = sp.whole(t);
+        const int slot = sp.slot(t);
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+            for (int nt = 0; nt < NT8; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = 16 * tt + g + 8 * (i >> 1);
+                    const int col = 8 * nt + 2 * c + (i & 1);
+                    const int64_t row = (int64_t)t * 32 + r;
+                    if (whole) {
+                        if (col < a.M && row < a.N)
+                            a.y[(size_t)col * a.N + row] = __float2half_rn(acc[tt][nt][i]);
+                    } else {
+                        a.ws[(((size_t)gw * 2 + slot) * 16 + col) * 32 + r] = acc[tt][nt][i];
+                    }
+                    acc[tt][nt][i] = 0.f;
+                }
+    };
+
+    int b = s0 - t_first * KB;                 // block of the next segment
+    int jb = b - b0;                           // its staged slot
+    if (jb < 0) jb += KB;
+    const uint32_t x_lane = xsm + (uint32_t)g * vstride + (uint32_t)c * 16;
+
+    auto segment = [&](uint32_t seg) {
+        const uint4 w = lds128(seg + lane * 16);
+        const uint2 dd = lds64(seg + kSegSclOff + g * 8);
+        uint4 xv[NT8];
+#pragma unroll
+        for (int nt = 0; nt < NT8; ++nt)
+            xv[nt] = lds128(x_lane + (uint32_t)(8 * nt) * vstride + (uint32_t)jb * 64);
+        const float2 d01 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
+        const float2 d23 = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
+        const float dA[2] = {d01.x, d23.x};   // rows g, g+16
+        const float dB[2] = {d01.y, d23.y};   // rows g+8, g+24
+        const uint32_t w0s[2] = {w.x, w.z};
+        const uint32_t w1s[2] = {w.y, w.w};
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+            const CodePairs u0 = unpack_pairs(w0s[tt]);   // row g (+16)
+            const CodePairs u1 = unpack_pairs(w1s[tt]);   // row g+8 (+16)
+#pragma unroll
+            for (int nt = 0; nt < NT8; ++nt) {
+                float e0, e1, e2, e3;
+                mma_16816(e0, e1, e2, e3, u0.p, u1.p, u0.q, u1.q, xv[nt].x, xv[nt].y, 0.f, 0.f,
+                          0.f, 0.f);
+                mma_16816(e0, e1, e2, e3, u0.r, u1.r, u0.s, u1.s, xv[nt].z, xv[nt].w, e0, e1, e2,
+                          e3);
+                acc[tt][nt][0] = fmaf(e0, dA[tt], acc[tt][nt][0]);
+                acc[tt][nt][1] = fmaf(e1, dA[tt], acc[tt][nt][1]);
+                acc[tt][nt][2] = fmaf(e2, dB[tt], acc[tt][nt][2]);
+                acc[tt][nt][3] = fmaf(e3, dB[tt], acc[tt][nt][3]);
+            }
+        }
+    };
+
+    for (int ch = 0; ch < ring.nch; ++ch) {
+        if (!ring.wait(ch)) set_device_error(a.err, kDevTimeout);   // data then unreliable
+        const uint32_t st = ring.stage(ch % R);
+        const int n = min(C, ring.nseg - ch * C);
+        for (int j = 0; j < n; ++j) {
+            if (b == KB) {
+                flush(t_cur);
+                ++t_cur;
+                b = 0;
+                jb = KB - b0;
+                if (jb >= KB) jb -= KB;
+            }
+            segment(st + j * kSegBytes);
+            ++b;
+            if (++jb == KB) jb = 0;
+        }
+        __syncwarp();
+        fence_proxy_async_smem();
+        if (lane == 0 && ch + R < ring.nch) ring.issue(ch + R);
+    }
+    if (s1 > s0) flush(t_cur);
+
+    auto arrive = [&](int t, int gf, int gl) {
+        if (gf == gl) return;
+        __syncwarp();
+        int old = 0;
+        if (lane == 0) old = atom_add_acq_rel_gpu(a.cnt + t, 1);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        __syncwarp();                       // order the lanes' reads after lane 0's acquire
+        const int need = gl - gf + 1;
+        if (old == need - 1) {
+            const int64_t row = (int64_t)t * 32 + lane;
+            for (int col = 0; col < a.M; ++col) {
+                float sum = 0.f;
+                SegWalker wk;
+                wk.init(gf, a.S, a.G);
+                for (int g0 = gf; g0 <= gl; g0 += 8) {
+                    float pv[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int gg = g0 + u;
+                        const int sl = (wk.sb >= t * KB) ? 0 : 1;
+                        pv[u] = gg <= gl ? ld_relaxed_gpu(a.ws + (((size_t)gg * 2 + sl) * 16 + col) * 32 + lane)
+                                         : 0.f;
+                        wk.next();
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) sum += pv[u];
+                }
+                if (row < a.N) a.y[(size_t)col * a.N + row] = __float2half_rn(sum);
+            }
+            if (lane == 0) a.cnt[t] = 0;
+        } else if (old >= need) {
+            if (lane == 0) set_device_error(a.err, kDevConcurrent);
+        }
+    };
+    if (s1 > s0) {
+        arrive(sp.t_first, sp.gf0, sp.gl0);
+        if (sp.t_last != sp.t_first) arrive(sp.t_last, sp.gf1, sp.gl1);
+    }
+}
+
+}  // namespace q4

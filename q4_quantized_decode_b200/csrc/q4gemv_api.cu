@@ -12,15 +12,28 @@
 
 #include "../../include/q4gemv.h"
 #include "gemv_dp2a.cuh"
+#include "gemv_mma.cuh"
 
 namespace {
 
 constexpr int kWarps = 16;                 // warps per CTA of the GEMV kernels
 constexpr int kThreads = kWarps * 32;
-constexpr int kPrefetch = 8;               // segments in flight per warp
+// Per-warp TMA ring (stages x segments per stage) of each kernel.
+constexpr int kR1 = 4, kC1 = 4;            // M = 1
+constexpr int kR2 = 2, kC2 = 4;            // M = 2 and the tensor-core kernel
 constexpr int kMinSegsPerWarp = 4;         // small problems use fewer warps
 constexpr int kMaxTiles = Q4GEMV_MAX_N / 32;
-constexpr size_t kMaxDynSmem = 200 * 1024;   // opt-in dynamic shared memory per CTA
+constexpr size_t kMaxDynSmem = 224 * 1024;   // opt-in dynamic shared memory per CTA
+
+#define Q4_DP2A_KERNEL_1 q4::gemv_dp2a_kernel<1, kWarps, kR1, kC1>
+#define Q4_DP2A_KERNEL_2 q4::gemv_dp2a_kernel<2, kWarps, kR2, kC2>
+#define Q4_MMA_KERNEL_1 q4::gemv_mma_kernel<1, kWarps, kR2, kC2>
+#define Q4_MMA_KERNEL_2 q4::gemv_mma_kernel<2, kWarps, kR2, kC2>
+
+size_t dp2a_smem(int M, int64_t K) {
+    return M == 1 ? q4::gemv_dp2a_smem_bytes(1, (int)K, kWarps, kR1, kC1)
+                  : q4::gemv_dp2a_smem_bytes(2, (int)K, kWarps, kR2, kC2);
+}
 
 enum Fault { kFaultNone = 0, kFaultAlloc, kFaultLaunch, kFaultGraph };
 
@@ -50,8 +63,8 @@ struct q4gemv_ctx {
     int device = 0;
     int sms = 0;
     int fault = kFaultNone;
-    float* ws = nullptr;          // [max warps][2][MAX_M][32] fp32
-    int max_warps = 0;
+    float* ws = nullptr;          // [ws_warps][2][MAX_M][32] fp32
+    int ws_warps = 0;
     int* cnt = nullptr;           // [kMaxTiles]
     int* err = nullptr;           // device error word
     __half* act = nullptr;        // stack intermediates
@@ -104,10 +117,9 @@ int parse_fault(const char* s) {
     return -1;
 }
 
-template <int M>
-int set_gemv_attrs() {
-    const cudaError_t e = cudaFuncSetAttribute(q4::gemv_dp2a_kernel<M, kWarps, kPrefetch>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <typename F>
+int set_smem_attr(F* kernel) {
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (int)kMaxDynSmem);
     return e == cudaSuccess ? 0 : -1;
 }
@@ -119,15 +131,13 @@ int launch_gemv(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M,
     if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
     const int KB = (int)(K / 32);
     const int T = (int)((N + 31) / 32);
-    const int64_t Np = (int64_t)T * 32;
     const int S = T * KB;
     int ctas = h->sms;
     const int want_warps = (S + kMinSegsPerWarp - 1) / kMinSegsPerWarp;
     if (want_warps < ctas * kWarps) ctas = (want_warps + kWarps - 1) / kWarps;
     if (ctas < 1) ctas = 1;
     q4::GemvArgs a;
-    a.nib = static_cast<const uint8_t*>(W);
-    a.scl = static_cast<const uint8_t*>(W) + Np * K / 2;
+    a.W = static_cast<const uint8_t*>(W);
     a.x = x;
     a.y = y;
     a.ws = h->ws;
@@ -141,7 +151,7 @@ int launch_gemv(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M,
     a.S = S;
     a.G = ctas * kWarps < S ? ctas * kWarps : S;   // every owning warp gets >= 1 segment
     a.renorm = renorm;
-    const size_t smem = q4::gemv_dp2a_smem_bytes(M, (int)K);
+    const size_t smem = dp2a_smem(M, K);
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ctas);
@@ -155,10 +165,89 @@ int launch_gemv(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M,
     cfg.numAttrs = pdl ? 1 : 0;
     cudaError_t e;
     if (M == 1)
-        e = cudaLaunchKernelEx(&cfg, q4::gemv_dp2a_kernel<1, kWarps, kPrefetch>, a);
+        e = cudaLaunchKernelEx(&cfg, Q4_DP2A_KERNEL_1, a);
     else
-        e = cudaLaunchKernelEx(&cfg, q4::gemv_dp2a_kernel<2, kWarps, kPrefetch>, a);
+        e = cudaLaunchKernelEx(&cfg, Q4_DP2A_KERNEL_2, a);
     if (e != cudaSuccess) return cuda_fail(h, e, "gemv launch");
+    return Q4_OK;
+}
+
+// Grows the split-tile workspace to hold `warps` warps (never during capture).
+int ensure_ws(q4gemv_ctx* h, int warps, cudaStream_t st) {
+    if (warps <= h->ws_warps) return Q4_OK;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    Q4_CUDA(h, cudaStreamIsCapturing(st, &cs));
+    if (cs != cudaStreamCaptureStatusNone)
+        return fail(h, Q4_EUNSUPPORTED,
+                    "the first call with this shape must come outside stream capture (workspace growth)");
+    if (h->fault == kFaultAlloc) return fail(h, Q4_EFAULTINJ, "injected allocation failure");
+    Q4_CUDA(h, cudaDeviceSynchronize());
+    cudaFree(h->ws);
+    h->ws = nullptr;
+    h->ws_warps = 0;
+    if (cudaMalloc(&h->ws, (size_t)warps * 2 * Q4GEMV_MAX_M * 32 * sizeof(float)) != cudaSuccess)
+        return fail(h, Q4_ENOMEM, "workspace growth to %d warps failed", warps);
+    h->ws_warps = warps;
+    return Q4_OK;
+}
+
+// Launch one GEMV on the tensor-core path (any M in 1..16, any K).
+int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M, int64_t N,
+                    int64_t K, cudaStream_t st) {
+    if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
+    const int nt8 = M <= 8 ? 1 : 2;
+    const int KB = (int)(K / 32);
+    const int T = (int)((N + 31) / 32);
+    const int S = T * KB;
+    // Largest block count one CTA may stage; a CTA whose run of segments is
+    // at least KB stages all KB blocks, so KB must fit or runs stay shorter.
+    const size_t ring = q4::ring_bytes(kWarps, kR2, kC2);
+    int xcap = 1;
+    while (ring + q4::gemv_mma_smem_bytes(nt8, xcap + 1) <= kMaxDynSmem) ++xcap;
+    const int wave = h->sms;                   // resident CTAs (one per SM)
+    int64_t ctas;
+    if (KB <= xcap) {
+        // Any run length fits: one wave, fewer for small problems.
+        ctas = wave;
+        const int64_t cap = S / (kWarps * kMinSegsPerWarp);
+        if (ctas > cap) ctas = cap < 1 ? 1 : cap;
+    } else {
+        // Runs must stay within xcap blocks: whole waves of short runs.
+        ctas = (S + xcap - 1) / xcap;
+        ctas = (ctas + wave - 1) / wave * wave;
+    }
+    int64_t G = ctas * kWarps;
+    if (G > S) G = S;
+    if (G > q4::kMaxSplitWarps) G = q4::kMaxSplitWarps;
+    const int rc = ensure_ws(h, (int)G, st);
+    if (rc != Q4_OK) return rc;
+    const int nblk_max = (KB <= xcap) ? KB : xcap;
+    q4::MmaArgs a;
+    a.W = static_cast<const uint8_t*>(W);
+    a.x = x;
+    a.y = y;
+    a.ws = h->ws;
+    a.cnt = h->cnt;
+    a.err = h->err;
+    a.N = N;
+    a.K = (int)K;
+    a.KB = KB;
+    a.T = T;
+    a.S = S;
+    a.G = (int)G;
+    a.M = M;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ctas);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = ring + q4::gemv_mma_smem_bytes(nt8, nblk_max);
+    cfg.stream = st;
+    cfg.numAttrs = 0;
+    cudaError_t e;
+    if (nt8 == 1)
+        e = cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_1, a);
+    else
+        e = cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_2, a);
+    if (e != cudaSuccess) return cuda_fail(h, e, "gemv (mma) launch");
     return Q4_OK;
 }
 
@@ -168,20 +257,24 @@ int launch_renorm(q4gemv_ctx* h, const __half* in, __half* out, int len, cudaStr
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = (size_t)len * 2;
+    cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, q4::renorm_kernel<kWarps>, in, out, len, h->err);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, q4::renorm_kernel<kWarps>, in, out, len);
     if (e != cudaSuccess) return cuda_fail(h, e, "renorm launch");
     return Q4_OK;
 }
 
+// The M <= 2 kernel holds the staged activations in registers (up to
+// kXChunksPerThread 16-byte chunks per thread) and its ring plus the int16
+// activations in shared memory.
 bool dp2a_fits(int M, int64_t K) {
-    return M <= 2 && q4::gemv_dp2a_smem_bytes(M, (int)K) <= kMaxDynSmem;
+    return M <= 2 && M * K <= (int64_t)q4::kXChunksPerThread * 8 * kThreads &&
+           dp2a_smem(M, K) <= kMaxDynSmem;
 }
 
 }  // namespace
@@ -224,7 +317,6 @@ int q4gemv_validate(int M, int64_t N, int64_t K, const void* W, const void* x, c
     if (sh != Q4_OK) return sh;
     if (!W || !x || !y) return Q4_EINVAL;
     if (!aligned16(W) || !aligned16(x) || !aligned16(y)) return Q4_EALIGN;
-    if (!dp2a_fits(M, K)) return Q4_EUNSUPPORTED;
     return Q4_OK;
 }
 
@@ -256,8 +348,8 @@ int q4gemv_create(q4gemv_t* out, int device) {
     if (e != cudaSuccess) rc = cuda_fail(h, e, "cudaSetDevice");
     if (rc == Q4_OK && h->fault == kFaultAlloc) rc = fail(h, Q4_EFAULTINJ, "injected allocation failure");
     if (rc == Q4_OK) {
-        h->max_warps = h->sms * kWarps;
-        const size_t ws_bytes = (size_t)h->max_warps * 2 * Q4GEMV_MAX_M * 32 * sizeof(float);
+        h->ws_warps = h->sms * kWarps;
+        const size_t ws_bytes = (size_t)h->ws_warps * 2 * Q4GEMV_MAX_M * 32 * sizeof(float);
         if (cudaMalloc(&h->ws, ws_bytes) != cudaSuccess ||
             cudaMalloc(&h->cnt, (size_t)kMaxTiles * sizeof(int)) != cudaSuccess ||
             cudaMalloc(&h->err, sizeof(int)) != cudaSuccess)
@@ -269,10 +361,9 @@ int q4gemv_create(q4gemv_t* out, int device) {
             rc = fail(h, Q4_ECUDA, "workspace initialisation failed");
     }
     if (rc == Q4_OK) {
-        if (set_gemv_attrs<1>() || set_gemv_attrs<2>() ||
-            cudaFuncSetAttribute(q4::renorm_kernel<kWarps>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kMaxDynSmem) != cudaSuccess)
+        if (set_smem_attr(Q4_DP2A_KERNEL_1) || set_smem_attr(Q4_DP2A_KERNEL_2) ||
+            set_smem_attr(Q4_MMA_KERNEL_1) || set_smem_attr(Q4_MMA_KERNEL_2) ||
+            0)
             rc = fail(h, Q4_ECUDA, "cudaFuncSetAttribute failed");
     }
     if (rc == Q4_OK) {
@@ -328,7 +419,7 @@ int q4gemv_repack(q4gemv_t h, const void* gguf, void* packed, int64_t N, int64_t
     int64_t blocks = (S + 7) / 8;
     if (blocks > (int64_t)h->sms * 32) blocks = (int64_t)h->sms * 32;
     q4::repack_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint8_t*>(gguf), static_cast<uint8_t*>(packed), N, KB, S, T * 32);
+        static_cast<const uint8_t*>(gguf), static_cast<uint8_t*>(packed), N, KB, S);
     Q4_CUDA(h, cudaGetLastError());
     return Q4_OK;
 }
@@ -341,8 +432,12 @@ int q4gemv_run(q4gemv_t h, const void* W, const void* x, void* y, int M, int64_t
         return fail(h, v, "run: %s (M=%d N=%lld K=%lld)", q4gemv_strerror(v), M, (long long)N,
                     (long long)K);
     Q4_CUDA(h, cudaSetDevice(h->device));
-    return launch_gemv(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K, 0,
-                       nullptr, static_cast<cudaStream_t>(stream), false);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dp2a_fits(M, K))
+        return launch_gemv(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K,
+                           0, nullptr, st, false);
+    return launch_gemv_mma(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K,
+                           st);
 }
 
 namespace {

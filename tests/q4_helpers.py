@@ -30,16 +30,18 @@ def f16_values(bits) -> np.ndarray:
     return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
 
 
-def unrepack(packed: np.ndarray, N: int, K: int) -> np.ndarray:
+def unrepack(packed: np.ndarray, N: int, K: int):
     """Inverse of the packed tile layout written with reshapes: returns GGUF
-    bytes (N, K/32*18).  The nibble plane is [T][KB][g=8][c=4][i=4][e=4]
-    (row 32t+8i+g, qs byte 4c+e); the scale plane is [T][KB][g=8][i=4][2]."""
+    bytes (N, K/32*18) and the padding rows.  Segment (t, b) is 576 bytes:
+    codes [g=8][c=4][i=4][e=4] (row 32t+8i+g, qs byte 4c+e), then scales
+    [g=8][i=4][2]."""
     KB = K // 32
     Np = (N + 31) // 32 * 32
     T = Np // 32
-    nib = packed[: Np * K // 2].reshape(T, KB, 8, 4, 4, 4)
+    seg = packed.reshape(T, KB, 576)
+    nib = seg[:, :, :512].reshape(T, KB, 8, 4, 4, 4)
     nib = nib.transpose(0, 4, 2, 1, 3, 5).reshape(Np, KB, 16)   # (t,i,g,b,c,e)
-    scl = packed[Np * K // 2:].reshape(T, KB, 8, 4, 2)
+    scl = seg[:, :, 512:].reshape(T, KB, 8, 4, 2)
     scl = scl.transpose(0, 3, 2, 1, 4).reshape(Np, KB, 2)        # (t,i,g,b,h)
     out = np.concatenate([scl, nib], axis=2)
     return out[:N].reshape(N, KB * 18), out[N:].reshape(Np - N, KB * 18)

@@ -73,6 +73,34 @@ def test_gemv_m2(eng, N, K):
     assert rel_err(y, ref) <= TOL
 
 
+@pytest.mark.parametrize("M", [4, 16])
+@pytest.mark.parametrize("N,K", [(34816, 5120), (5120, 17408)])
+def test_gemv_small_m_configs(eng, M, N, K):
+    """Config 3: speculative-verify batch (M=4) and prefill chunk (M=16)."""
+    gguf, x, y = gemv_case(eng, N, K, M, synth.config_seed(3) + M, tid=0 if K == 5120 else 1)
+    ref = oracle.q4_gemv(gguf, K, x, threads=THREADS)
+    err = rel_err(y, ref)
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("M", [3, 5, 8, 9, 13, 16])
+@pytest.mark.parametrize("N,K", [(1, 32), (33, 64), (100, 96), (257, 160), (4096, 64), (40, 6400),
+                                 (64, 40960)])
+def test_gemv_small_m_edge_shapes(eng, M, N, K):
+    gguf, x, y = gemv_case(eng, N, K, M, 500 + 7 * M + N + K)
+    ref = oracle.q4_gemv(gguf, K, x, threads=THREADS)
+    assert rel_err(y, ref) <= TOL
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_gemv_wide_k_uses_tensor_core_path(eng, M):
+    """K beyond the shared-memory limit of the M <= 2 kernel."""
+    N, K = 96, 65536
+    gguf, x, y = gemv_case(eng, N, K, M, 4242)
+    ref = oracle.q4_gemv(gguf, K, x, threads=THREADS)
+    assert rel_err(y, ref) <= TOL
+
+
 @pytest.mark.parametrize("N,K", [(1, 32), (31, 32), (33, 64), (100, 96), (7, 1056), (257, 160),
                                  (8192, 32), (4096, 64), (2, 17408), (40, 40960)])
 def test_gemv_edge_shapes(eng, N, K):

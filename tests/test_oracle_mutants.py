@@ -24,7 +24,8 @@ MUTANTS = {
     "acc_dropped_term": ("for (int64_t k = 0; k < K; ++k)\n                acc +=",
                          "for (int64_t k = 1; k < K; ++k)\n                acc +="),
     "repack_g_i_swapped": ("16 * (4 * g + c) + 4 * i + e", "16 * (4 * i + c) + 4 * g + e"),
-    "repack_scale_slot": ("64 * s + 8 * g + 2 * i + h", "64 * s + 8 * i + 2 * g + h"),
+    "repack_segment_stride": ("packed + 576 * (t * KB + b)", "packed + 512 * (t * KB + b)"),
+    "repack_scale_slot": ("seg[512 + 8 * g + 2 * i + h]", "seg[512 + 8 * i + 2 * g + h]"),
     "repack_pad_code": ("(h < 2 ? 0x00 : 0x88)", "(h < 2 ? 0x00 : 0x00)"),
     "renorm_no_len": ("sqrt(s / (double)len)", "sqrt(s)"),
     "rne_ties_up": ("(frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0))", "(frac >= 0.5)"),
