@@ -178,6 +178,39 @@ Q4GEMV_API int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_la
                      const void* x_in, void* x_out, void* trace_x,
                      void* trace_y, q4gemv_stream_t stream);
 
+/* Fixed limits of q4gemv_run_noalloc. */
+#define Q4GEMV_NOALLOC_MAX_N (1 << 22)                 /* rows */
+#define Q4GEMV_NOALLOC_SCRATCH_BYTES (2u << 20)        /* static device scratch */
+
+/* q4gemv_run for M <= 2 without a handle and without allocating anything.
+ * The paper has no counterpart; this is a library convenience.
+ *
+ * Who needs it: q4gemv_create obtains its workspace with cudaMalloc, which
+ * some callers cannot do -- code that runs while a stream is captured in
+ * global capture mode (cudaMalloc is then an error), threads that must not
+ * take the implicit device synchronisation of cudaMalloc/cudaFree, and
+ * plug-ins whose host application owns all device memory.  This entry point
+ * runs the same kernel as q4gemv_run with its scratch (split-tile partial
+ * sums, per-tile arrival counters, an error word) in one file-scope device
+ * array of Q4GEMV_NOALLOC_SCRATCH_BYTES (2 MiB) that every GPU which loads
+ * the library holds until the process exits.  It calls no cudaMalloc,
+ * cudaFree or allocating library routine.
+ *
+ * Arguments as q4gemv_run (device pointers, 16-byte aligned, packed W), on
+ * the current CUDA device, asynchronous on `stream`.  Limits: 1 <= M <= 2
+ * (else Q4_EUNSUPPORTED); K % 32 == 0, N <= Q4GEMV_NOALLOC_MAX_N, M*K <=
+ * 36864 (else Q4_ESHAPE); at most 2560 warps are used.  Device-side error
+ * reports are not surfaced.
+ *
+ * The first call on a device sets that device up (resolves the array's
+ * device address with cudaGetSymbolAddress, queries the SM count, sets the
+ * kernels' shared-memory limit); make that first call before any stream
+ * capture.  Every call shares the one array and clears its counters before
+ * launching: calls that overlap on the GPU race and give wrong results, so
+ * order them on one stream. */
+Q4GEMV_API int q4gemv_run_noalloc(const void* W_packed, const void* x, void* y, int M,
+                                  int64_t N, int64_t K, q4gemv_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the handle's device error
  * word: Q4_OK, Q4_ETIMEOUT, Q4_ECONCURRENT, or Q4_ECUDA if an earlier
  * asynchronous error is pending on the device. */

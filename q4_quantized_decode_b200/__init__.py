@@ -61,6 +61,7 @@ def _load_library():
         "q4gemv_strerror": ([ci], ctypes.c_char_p),
         "q4gemv_last_error": ([vp], ctypes.c_char_p),
         "q4gemv_set_fault": ([vp, ctypes.c_char_p], ci),
+        "q4gemv_run_noalloc": ([vp, vp, vp, ci, i64, i64, vp], ci),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
@@ -127,6 +128,11 @@ def q4gemv_sync_status(h, stream) -> int:
 
 def q4gemv_set_fault(h, which: str) -> int:
     return _lib.q4gemv_set_fault(h, which.encode())
+
+
+def q4gemv_run_noalloc(W, x, y, M, N, K, stream) -> int:
+    """The M <= 2 GEMV without a handle or any allocation (see the header)."""
+    return _lib.q4gemv_run_noalloc(W, x, y, M, N, K, stream)
 
 
 def _ptr(t) -> int | None:

@@ -10,7 +10,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libq4gemv.so")
-SOURCES = ["q4gemv_api.cu"]
+SOURCES = ["q4gemv_api.cu", "q4gemv_noalloc.cu"]
 HEADERS = ["device_common.cuh", "partition.cuh", "gemv_dp2a.cuh", "gemv_mma.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -41,6 +41,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
+           "-rdc=false",
            "-Xcompiler", "-fvisibility=hidden", "-cudart", "static",
            "-o", tmp, *[os.path.join(CSRC, f) for f in SOURCES]]
     if verbose:

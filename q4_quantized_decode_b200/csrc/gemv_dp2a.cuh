@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) renorm_kernel(const __half* in,
 }
 
 // GGUF Q4_0 -> packed layout, one warp per segment (grid-stride).
-__global__ void __launch_bounds__(256) repack_kernel(const uint8_t* __restrict__ gguf,
+static __global__ void __launch_bounds__(256) repack_kernel(const uint8_t* __restrict__ gguf,
                                                      uint8_t* __restrict__ packed, int64_t N,
                                                      int KB, int64_t S) {
     const int lane = threadIdx.x & 31;
