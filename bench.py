@@ -62,6 +62,26 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+# ------------------------------------------------------------------ multi-rank helpers
+
+def max_over_ranks(dist, values, device=None):
+    """Element-wise max of `values` over all ranks (device times are taken as
+    the slowest rank's).  Works with gloo (CPU tensors) and nccl (CUDA)."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def step_throughput(world: int, steps: int, ms_max: float, bytes_per_step: int = None):
+    """Whole-job GB/s and steps/s of `world` replicas that each ran `steps`
+    steps, from the slowest rank's time in ms."""
+    b = STEP_GEMV_BYTES if bytes_per_step is None else bytes_per_step
+    secs = ms_max * 1e-3
+    return world * b * steps / secs / 1e9, world * steps / secs
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -305,16 +325,13 @@ def run_ours(args, rank: int, world: int, dist):
     if eng.sync_status() != q4.Q4_OK:
         raise RuntimeError("device status after timing")
 
-    t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, ms_e2e = float(t[0]), float(t[1])
+    ms, ms_e2e = max_over_ranks(dist, [ms, ms_e2e], device=dev)
     if rank != 0:
         return 0
 
     ms_step = ms / args.steps
-    value = world * STEP_GEMV_BYTES * args.steps / (ms * 1e-3) / 1e9
-    e2e_value = world * STEP_GEMV_BYTES * args.steps / (ms_e2e * 1e-3) / 1e9
+    value, steps_per_s = step_throughput(world, args.steps, ms)
+    e2e_value, e2e_steps_per_s = step_throughput(world, args.steps, ms_e2e)
     peak, peak_kind = measured_peaks()
     per_rank_gbs = STEP_GEMV_BYTES / (ms_step * 1e-3) / 1e9
     roofline = {
@@ -346,13 +363,13 @@ def run_ours(args, rank: int, world: int, dist):
                    "weight_bytes_per_step": STEP_WEIGHT_BYTES,
                    "l2": "inputs larger than L2 (11.9 GB of weights per step)",
                    "parallelism": f"replicas x{world}", "seed": CONFIG_SEED},
-        "decode_steps_per_s": world * args.steps / (ms * 1e-3),
+        "decode_steps_per_s": steps_per_s,
         "pct_of_8TBps_nominal": 100.0 * per_rank_gbs / NOMINAL_HBM_GBS,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": 2 * HIDDEN,
                 "d2h_bytes_per_step": 2 * HIDDEN,
-                "steps_per_s": world * args.steps / (ms_e2e * 1e-3)},
+                "steps_per_s": e2e_steps_per_s},
         "gpu_launches": args.steps * (4 * L + 1),
         "clocks": clocks,
         "repack_s_per_step_weights": t_repack,

@@ -71,7 +71,12 @@ typedef enum {
     Q4_ECONCURRENT = -9    /* kernels saw overlapping calls on one handle */
 } q4gemv_status;
 
-/* Limits checked by validation. */
+/* Limits checked by validation.  Besides these, ceil(N/32) * (K/32) must be
+ * below 2^31, and on the tensor-core path (M >= 3, or M <= 2 with K beyond
+ * the CUDA-core kernel's staging) a matrix wider than the activations one
+ * CTA can stage (about 9700 columns for M <= 8, 4800 for M <= 16) is
+ * accepted up to about 3839 * that many columns' worth of 32-row tiles
+ * (Q4_ESHAPE beyond). */
 #define Q4GEMV_MAX_M 16
 #define Q4GEMV_MAX_N (1 << 22)     /* rows */
 #define Q4GEMV_MAX_K (1 << 20)     /* columns */

@@ -47,6 +47,7 @@ struct GemvArgs {
     int S;                  // segments = T * KB
     int G;                  // warps that own segments (G <= S)
     int renorm;             // 1: the input is renorm(x[0:K]) (M == 1 only)
+    SplitConsts sc;         // make_split(S, G)
 };
 
 // Per-warp ring of R stages of C segments.
@@ -108,21 +109,25 @@ struct WarpRing {
 // then converted to X = rint(v * 2^(14-E)) (E: exponent of the block maximum,
 // so |X| <= 32752 and the maximum is exact) and written in lane order; lane
 // group c of the block gets {-8 * sum of its eight X, 2^(E-14)}.
-template <int M, int NT>
+// kCoherent: load x through L2 only (it was written by other CTAs of the
+// same running kernel, so an L1 copy could be stale).
+// QN: 16-byte chunks held per thread (M * K <= QN * 8 * NT).
+template <int M, int NT, bool kCoherent = false, int QN = kXChunksPerThread>
 __device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs, uint32_t rec,
                                                   float* red) {
     const int tid = threadIdx.x, lane = tid & 31;
     const int nq = M * a.K / 8;
-    uint4 xr[kXChunksPerThread];
+    uint4 xr[QN];
 #pragma unroll
-    for (int i = 0; i < kXChunksPerThread; ++i) {
+    for (int i = 0; i < QN; ++i) {
         const int q = tid + NT * i;
-        xr[i] = q < nq ? *reinterpret_cast<const uint4*>(a.x + (size_t)q * 8) : make_uint4(0, 0, 0, 0);
+        const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)q * 8);
+        xr[i] = q < nq ? (kCoherent ? __ldcg(src) : *src) : make_uint4(0, 0, 0, 0);
     }
     if (M == 1 && a.renorm) {
         float part = 0.f;
 #pragma unroll
-        for (int i = 0; i < kXChunksPerThread; ++i) {
+        for (int i = 0; i < QN; ++i) {
             const __half2* h = reinterpret_cast<const __half2*>(&xr[i]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -140,7 +145,7 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs
         for (int w = 0; w < NT / 32; ++w) s += red[w];
         const float scale = (s > 0.f) ? __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(s, (float)a.K))) : 0.f;
 #pragma unroll
-        for (int i = 0; i < kXChunksPerThread; ++i) {
+        for (int i = 0; i < QN; ++i) {
             __half2* h = reinterpret_cast<__half2*>(&xr[i]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -150,7 +155,7 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs
         }
     }
 #pragma unroll
-    for (int i = 0; i < kXChunksPerThread; ++i) {
+    for (int i = 0; i < QN; ++i) {
         const int q = tid + NT * i;
         if (M == 1 && a.trace_x != nullptr && blockIdx.x == 0 && q < nq)
             *reinterpret_cast<uint4*>(a.trace_x + (size_t)q * 8) = xr[i];
@@ -202,59 +207,42 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs
     __syncthreads();
 }
 
-template <int M, int WARPS, int R, int C>
-__global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ __align__(8) uint64_t bars[WARPS * R];
-    __shared__ float red[WARPS];
-
-    const uint32_t smem_base = smem_addr(smem);
-    const uint32_t xs = smem_base + (uint32_t)ring_bytes(WARPS, R, C);   // int16 X, lane order
-    const uint32_t rec = xs + (uint32_t)(M * a.K * 2);                  // {-8 sum X, scale}
-
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, c = lane & 3;
-    const int gw = blockIdx.x * WARPS + warp;
-    // G <= S, so every warp below G owns at least one segment; warps of the
-    // last CTA beyond G only help stage the activations.
-    WarpSplit sp;
-    sp.init(gw, a.S, a.G, a.KB);
-    const int s0 = sp.s0, s1 = sp.s1;
-
-    WarpRing<R, C> ring;
-    ring.init(smem_base, bars, warp, a.W, s0, s1);
-    if (lane == 0) {
-        for (int k = 0; k < R; ++k) mbar_init(bars + warp * R + k, 1);
-        fence_barrier_init();
-    }
-    __syncwarp();
-    // Weights do not depend on the previous kernel: start the stream before
-    // the dependency wait.
-    if (lane == 0)
-        for (int ch = 0; ch < R && ch < ring.nch; ++ch) ring.issue(ch);
-    pdl_launch_dependents();
-    pdl_wait();
-
-    stage_activations<M, WARPS * 32>(a, xs, rec, red);
-
+// One warp's share of one GEMV on the dp2a path: accumulators, position in
+// its run of segments, and the split-tile bookkeeping.
+template <int M>
+struct Dp2aConsumer {
     float acc[M][4];
-#pragma unroll
-    for (int m = 0; m < M; ++m)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
+    WarpSplit sp;
+    int gw, lane, g, c, r;   // r: the tile row this lane emits
+    int KB, t_cur, b;        // b: block of the next segment
+    uint32_t x_lane0, r_lane0, xp, rp;   // running shared addresses of block b's X words and record
+    uint32_t xstride, rstride;           // per activation vector
 
-    const int KB = a.KB;
-    const int t_first = sp.t_first;
-    int t_cur = t_first;
-    int b = s0 - t_first * KB;                 // block of the next segment
-    const int r = g + 8 * c;                   // row of the tile this lane emits
-    // Running shared addresses of block b's X words and records for this lane.
-    const uint32_t x_lane0 = xs + (uint32_t)c * 16, r_lane0 = rec + (uint32_t)c * 8;
-    uint32_t xp = x_lane0 + (uint32_t)b * 64, rp = r_lane0 + (uint32_t)b * 32;
+    __device__ __forceinline__ void init(const GemvArgs& a, int gw_, uint32_t xs, uint32_t rec) {
+        gw = gw_;
+        lane = threadIdx.x & 31;
+        g = lane >> 2;
+        c = lane & 3;
+        r = g + 8 * c;
+        KB = a.KB;
+        sp.init(gw, a.sc, KB);
+        t_cur = sp.t_first;
+        b = sp.s0 - sp.t_first * KB;
+        x_lane0 = xs + (uint32_t)c * 16;
+        r_lane0 = rec + (uint32_t)c * 8;
+        xp = x_lane0 + (uint32_t)b * 64;
+        rp = r_lane0 + (uint32_t)b * 32;
+        xstride = (uint32_t)a.K * 2;
+        rstride = (uint32_t)KB * 32;
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
+    }
 
     // Combine a finished tile: reduce over the four column lanes, then either
     // write y (this warp owns the whole tile) or park the partial.
-    auto flush = [&](int t) {
+    __device__ __forceinline__ void flush(const GemvArgs& a, int t) {
 #pragma unroll
         for (int m = 0; m < M; ++m)
 #pragma unroll
@@ -277,82 +265,88 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
         }
-    };
+    }
 
-    // One segment at shared address `seg`: codes and scales from the ring
-    // stage, X and the block record from the staged activations.
-    auto segment = [&](uint32_t seg) {
+    // One segment at shared address `seg`, whose block's X words and record
+    // are at xb and rb: codes and scales from a ring stage, X from the staged
+    // activations.  Rows are handled in pairs on the packed fp32x2 pipes.
+    __device__ __forceinline__ void segment(uint32_t seg, uint32_t xb, uint32_t rb) {
         const uint4 w = lds128(seg + lane * 16);
         const uint2 dd = lds64(seg + kSegSclOff + g * 8);
         const float2 d01 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
         const float2 d23 = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
-        const float d[4] = {d01.x, d01.y, d23.x, d23.y};
         const uint32_t words[4] = {w.x, w.y, w.z, w.w};
         uint4 xq[M];
         uint2 rc[M];
 #pragma unroll
         for (int m = 0; m < M; ++m) {
-            xq[m] = lds128(xp + (uint32_t)m * a.K * 2);
-            rc[m] = lds64(rp + (uint32_t)m * KB * 32);
+            xq[m] = lds128(xb + (uint32_t)m * xstride);
+            rc[m] = lds64(rb + (uint32_t)m * rstride);
         }
+        int v[M][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint32_t lo = words[i] & 0x0F0F0F0Fu;          // codes 4c..4c+3
             const uint32_t hi = (words[i] >> 4) & 0x0F0F0F0Fu;   // codes 4c+16..4c+19
 #pragma unroll
             for (int m = 0; m < M; ++m) {
-                int v = dp2a_lo(xq[m].x, lo, (int)rc[m].x);
-                v = dp2a_hi(xq[m].y, lo, v);
-                v = dp2a_lo(xq[m].z, hi, v);
-                v = dp2a_hi(xq[m].w, hi, v);
-                acc[m][i] = fmaf((float)v, d[i] * __uint_as_float(rc[m].y), acc[m][i]);
+                int t = dp2a_lo(xq[m].x, lo, (int)rc[m].x);
+                t = dp2a_hi(xq[m].y, lo, t);
+                t = dp2a_lo(xq[m].z, hi, t);
+                v[m][i] = dp2a_hi(xq[m].w, hi, t);
             }
         }
-    };
-    auto advance = [&]() {
-        ++b;
-        xp += 64;
-        rp += 32;
-    };
-    auto maybe_flush = [&]() {
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const float sbm = __uint_as_float(rc[m].y);
+            const float2 s2 = make_float2(sbm, sbm);
+            const float2 ds01 = fmul2(d01, s2), ds23 = fmul2(d23, s2);
+            float2 a01 = make_float2(acc[m][0], acc[m][1]), a23 = make_float2(acc[m][2], acc[m][3]);
+            a01 = ffma2(make_float2((float)v[m][0], (float)v[m][1]), ds01, a01);
+            a23 = ffma2(make_float2((float)v[m][2], (float)v[m][3]), ds23, a23);
+            acc[m][0] = a01.x;
+            acc[m][1] = a01.y;
+            acc[m][2] = a23.x;
+            acc[m][3] = a23.y;
+        }
+    }
+
+    // Next segment of the run (flushing a finished tile first).
+    __device__ __forceinline__ void step(const GemvArgs& a, uint32_t seg) {
         if (b == KB) {
-            flush(t_cur);
+            flush(a, t_cur);
             ++t_cur;
             b = 0;
             xp = x_lane0;
             rp = r_lane0;
         }
-    };
-
-    for (int ch = 0; ch < ring.nch; ++ch) {
-        if (!ring.wait(ch)) set_device_error(a.err, kDevTimeout);   // data then unreliable
-        const uint32_t st = ring.stage(ch % R);
-        const int n = min(C, ring.nseg - ch * C);
-        if (n == C) {
-#pragma unroll
-            for (int j = 0; j < C; ++j) {
-                maybe_flush();
-                segment(st + j * kSegBytes);
-                advance();
-            }
-        } else {
-            for (int j = 0; j < n; ++j) {
-                maybe_flush();
-                segment(st + j * kSegBytes);
-                advance();
-            }
-        }
-        // Stage fully read: hand it back to the async proxy for the refill.
-        __syncwarp();
-        fence_proxy_async_smem();
-        if (lane == 0 && ch + R < ring.nch) ring.issue(ch + R);
+        segment(seg, xp, rp);
+        ++b;
+        xp += 64;
+        rp += 32;
     }
-    if (s1 > s0) flush(t_cur);
+
+    // A whole ring stage of C segments.  When no tile ends inside it the
+    // segments are addressed with constant offsets and no per-segment checks.
+    template <int C>
+    __device__ __forceinline__ void stage_full(const GemvArgs& a, uint32_t st) {
+        if (b + C <= KB) {
+#pragma unroll
+            for (int j = 0; j < C; ++j)
+                segment(st + j * kSegBytes, xp + j * 64, rp + j * 32);
+            b += C;
+            xp += C * 64;
+            rp += C * 32;
+        } else {
+#pragma unroll
+            for (int j = 0; j < C; ++j) step(a, st + j * kSegBytes);
+        }
+    }
 
     // Tiles shared with other warps (at most the first and the last one of
-    // this warp's range): count arrivals; the last warp to arrive sums the
+    // this warp's run): count arrivals; the last warp to arrive sums the
     // partials in warp order, writes y and re-arms the counter.
-    auto arrive = [&](int t, int gf, int gl) {
+    __device__ __forceinline__ void arrive(const GemvArgs& a, int t, int gf, int gl) {
         if (gf == gl) return;
         __syncwarp();
         int old = 0;
@@ -366,13 +360,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
 #pragma unroll
             for (int m = 0; m < M; ++m) sum[m] = 0.f;
             SegWalker wk;
-            wk.init(gf, a.S, a.G);
-            // Eight contributors per round: their loads are issued together,
+            wk.init(gf, a.sc);
+            // Sixteen contributors per round: their loads are issued together,
             // the sum is still taken in warp order.
-            for (int g0 = gf; g0 <= gl; g0 += 8) {
-                float pv[8][M];
+            for (int g0 = gf; g0 <= gl; g0 += 16) {
+                float pv[16][M];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < 16; ++u) {
                     const int gg = g0 + u;
                     const int sl = (wk.sb >= t * KB) ? 0 : 1;   // t is where gg's run starts
 #pragma unroll
@@ -382,7 +376,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
                     wk.next();
                 }
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
+                for (int u = 0; u < 16; ++u)
 #pragma unroll
                     for (int m = 0; m < M; ++m) sum[m] += pv[u][m];
             }
@@ -393,11 +387,69 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
         } else if (old >= need) {
             if (lane == 0) set_device_error(a.err, kDevConcurrent);
         }
-    };
-    if (s1 > s0) {
-        arrive(sp.t_first, sp.gf0, sp.gl0);
-        if (sp.t_last != sp.t_first) arrive(sp.t_last, sp.gf1, sp.gl1);
     }
+
+    // End of the run: last tile, then the arrivals.
+    __device__ __forceinline__ void finish(const GemvArgs& a) {
+        if (sp.s1 > sp.s0) {
+            flush(a, t_cur);
+            arrive(a, sp.t_first, sp.gf0, sp.gl0);
+            if (sp.t_last != sp.t_first) arrive(a, sp.t_last, sp.gf1, sp.gl1);
+        }
+    }
+};
+
+template <int M, int WARPS, int R, int C>
+__global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ __align__(8) uint64_t bars[WARPS * R];
+    __shared__ float red[WARPS];
+
+    const uint32_t smem_base = smem_addr(smem);
+    const uint32_t xs = smem_base + (uint32_t)ring_bytes(WARPS, R, C);   // int16 X, lane order
+    const uint32_t rec = xs + (uint32_t)(M * a.K * 2);                  // {-8 sum X, scale}
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gw = blockIdx.x * WARPS + warp;
+    // G <= S, so every warp below G owns at least one segment; warps of the
+    // last CTA beyond G only help stage the activations.
+    Dp2aConsumer<M> cons;
+    WarpRing<R, C> ring;
+    {
+        WarpSplit sp;
+        sp.init(gw, a.sc, a.KB);
+        ring.init(smem_base, bars, warp, a.W, sp.s0, sp.s1);
+    }
+    if (lane == 0) {
+        for (int k = 0; k < R; ++k) mbar_init(bars + warp * R + k, 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    // Weights do not depend on the previous kernel: start the stream before
+    // the dependency wait.
+    if (lane == 0)
+        for (int ch = 0; ch < R && ch < ring.nch; ++ch) ring.issue(ch);
+    pdl_launch_dependents();
+    pdl_wait();
+
+    stage_activations<M, WARPS * 32>(a, xs, rec, red);
+    cons.init(a, gw, xs, rec);
+
+    for (int ch = 0; ch < ring.nch; ++ch) {
+        if (!ring.wait(ch)) set_device_error(a.err, kDevTimeout);   // data then unreliable
+        const uint32_t st = ring.stage(ch % R);
+        const int n = min(C, ring.nseg - ch * C);
+        if (n == C) {
+            cons.template stage_full<C>(a, st);
+        } else {
+            for (int j = 0; j < n; ++j) cons.step(a, st + j * kSegBytes);
+        }
+        // Stage fully read: hand it back to the async proxy for the refill.
+        __syncwarp();
+        fence_proxy_async_smem();
+        if (lane == 0 && ch + R < ring.nch) ring.issue(ch + R);
+    }
+    cons.finish(a);
 }
 
 // Final renorm of the decode step: out = renorm(in[0:len)), with the same

@@ -38,6 +38,7 @@ struct MmaArgs {
     int64_t N;
     int K, KB, T, S, G;
     int M;               // 1..16 (columns >= M are zero-padded)
+    SplitConsts sc;      // make_split(S, G)
 };
 
 // Bytes per staged activation vector for `nblk` blocks: 64 per block, padded
@@ -107,15 +108,15 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
     const int g = lane >> 2, c = lane & 3;
     const int gw = blockIdx.x * WARPS + warp;
     WarpSplit sp;
-    sp.init(gw, a.S, a.G, a.KB);
+    sp.init(gw, a.sc, a.KB);
     const int s0 = sp.s0, s1 = sp.s1;
     const int KB = a.KB;
 
     // The CTA's blocks: its warps own one contiguous run of segments.
     const int w_lo = blockIdx.x * WARPS;
     const int w_hi = min(w_lo + WARPS, a.G);
-    const int cs0 = w_lo < a.G ? seg_begin(w_lo, a.S, a.G) : a.S;
-    const int cs1 = w_hi > w_lo ? (w_hi < a.G ? seg_begin(w_hi, a.S, a.G) : a.S) : cs0;
+    const int cs0 = w_lo < a.G ? seg_begin(w_lo, a.sc) : a.S;
+    const int cs1 = w_hi > w_lo ? (w_hi < a.G ? seg_begin(w_hi, a.sc) : a.S) : cs0;
     const int nblk = (cs1 - cs0 >= KB) ? KB : (cs1 - cs0);
     const int b0 = (cs1 - cs0 >= KB) ? 0 : (cs0 % KB);
     const int vstride = mma_vstride(nblk);
@@ -277,7 +278,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
             for (int col = 0; col < a.M; ++col) {
                 float sum = 0.f;
                 SegWalker wk;
-                wk.init(gf, a.S, a.G);
+                wk.init(gf, a.sc);
                 for (int g0 = gf; g0 <= gl; g0 += 8) {
                     float pv[8];
 #pragma unroll

@@ -9,8 +9,10 @@
 // the tile is where its run starts, else slot 1) and the last to arrive sums
 // them in warp order.
 //
-// All arithmetic is 32-bit: with S = Q*G + Rm, floor(g*S/G) = g*Q +
-// floor(g*Rm/G) and g*Rm < G^2 < 2^32 for G < 65536.
+// The divisions by G and S are done by multiplication with host-computed
+// reciprocals (SplitConsts): for n < 2^32 and M = ceil(2^64 / d),
+// floor(n * M / 2^64) == floor(n / d) exactly, because the error n*(M/2^64 -
+// 1/d) < 2^-32 is smaller than the gap 1/d between n/d and the next integer.
 #pragma once
 
 #include <cstdint>
@@ -19,38 +21,68 @@ namespace q4 {
 
 constexpr int kMaxSplitWarps = 65535;
 
-__host__ __device__ __forceinline__ int seg_begin(int g, int S, int G) {
-    const uint32_t Q = (uint32_t)S / (uint32_t)G, Rm = (uint32_t)S - Q * (uint32_t)G;
-    return (int)((uint32_t)g * Q + ((uint32_t)g * Rm) / (uint32_t)G);
+struct SplitConsts {
+    int S, G;             // segments, warps (1 <= G <= S, G <= kMaxSplitWarps)
+    uint32_t Q, Rm;       // S = Q*G + Rm
+    uint64_t MG;          // ceil(2^64 / G) (0 when G == 1: then Rm == 0)
+    uint64_t MS;          // ceil(2^64 / S) (0 when S == 1)
+    int fast;             // S * G < 2^32: warp_of_seg numerators fit 32 bits
+};
+
+__host__ __device__ inline uint64_t recip64(uint32_t d) {
+    return d <= 1 ? 0 : (~(uint64_t)0) / d + 1;   // ceil(2^64 / d) for d >= 2
 }
 
-// Largest g < G with seg_begin(g) <= s, for 0 <= s < S: a single-precision
-// estimate of floor((s+1)*G/S) corrected against seg_begin.
-__host__ __device__ __forceinline__ int warp_of_seg(int s, int S, int G) {
-    int g = (int)((float)(s + 1) * ((float)G / (float)S));
-    if (g > G - 1) g = G - 1;
-    if (g < 0) g = 0;
-    while (g > 0 && seg_begin(g, S, G) > s) --g;
-    while (g + 1 < G && seg_begin(g + 1, S, G) <= s) ++g;
-    return g;
+__host__ __device__ inline SplitConsts make_split(int S, int G) {
+    SplitConsts k;
+    k.S = S;
+    k.G = G;
+    k.Q = (uint32_t)S / (uint32_t)G;
+    k.Rm = (uint32_t)S - k.Q * (uint32_t)G;
+    k.MG = recip64((uint32_t)G);
+    k.MS = recip64((uint32_t)S);
+    k.fast = ((uint64_t)S * (uint64_t)G < ((uint64_t)1 << 32)) ? 1 : 0;
+    return k;
 }
 
-// Per-warp view of the split, computed once at kernel start.
+__host__ __device__ __forceinline__ uint32_t mulhi64(uint32_t n, uint64_t m) {
+#ifdef __CUDA_ARCH__
+    return (uint32_t)__umul64hi((uint64_t)n, m);
+#else
+    return (uint32_t)(((unsigned __int128)n * m) >> 64);
+#endif
+}
+
+// floor(g * S / G)
+__host__ __device__ __forceinline__ int seg_begin(int g, const SplitConsts& k) {
+    const uint32_t n = (uint32_t)g * k.Rm;        // < G^2 < 2^32
+    const uint32_t f = k.G == 1 ? 0u : mulhi64(n, k.MG);
+    return (int)((uint32_t)g * k.Q + f);
+}
+
+// Largest g < G with seg_begin(g) <= s (0 <= s < S): floor(((s+1)*G - 1) / S).
+__host__ __device__ __forceinline__ int warp_of_seg(int s, const SplitConsts& k) {
+    if (k.S == 1) return k.G - 1;
+    if (k.fast) return (int)mulhi64((uint32_t)(s + 1) * (uint32_t)k.G - 1u, k.MS);
+    return (int)((((uint64_t)s + 1) * (uint64_t)k.G - 1) / (uint64_t)k.S);
+}
+
+// Per-warp view of the split, computed once per GEMV.
 struct WarpSplit {
     int s0, s1;             // owned segments
     int t_first, t_last;    // first and last tile touched (t_last < t_first if none)
     int gf0, gl0, gf1, gl1; // contributors of t_first and t_last
 
-    __host__ __device__ __forceinline__ void init(int gw, int S, int G, int KB) {
-        s0 = gw < G ? seg_begin(gw, S, G) : S;
-        s1 = gw < G ? seg_begin(gw + 1, S, G) : S;
+    __host__ __device__ __forceinline__ void init(int gw, const SplitConsts& k, int KB) {
+        s0 = gw < k.G ? seg_begin(gw, k) : k.S;
+        s1 = gw < k.G ? seg_begin(gw + 1, k) : k.S;
         t_first = s0 / KB;
         t_last = (s1 > s0) ? (s1 - 1) / KB : t_first - 1;
         if (s1 > s0) {
-            gf0 = warp_of_seg(t_first * KB, S, G);
-            gl0 = warp_of_seg(t_first * KB + KB - 1, S, G);
-            gf1 = warp_of_seg(t_last * KB, S, G);
-            gl1 = warp_of_seg(t_last * KB + KB - 1, S, G);
+            gf0 = warp_of_seg(t_first * KB, k);
+            gl0 = warp_of_seg(t_first * KB + KB - 1, k);
+            gf1 = warp_of_seg(t_last * KB, k);
+            gl1 = warp_of_seg(t_last * KB + KB - 1, k);
         } else {
             gf0 = gl0 = gf1 = gl1 = 0;
         }
@@ -67,12 +99,12 @@ struct WarpSplit {
 // Walks seg_begin(g) for g = g_start, g_start + 1, ... with additions only.
 struct SegWalker {
     int sb, r, Q, Rm, G;
-    __host__ __device__ __forceinline__ void init(int g_start, int S, int G_) {
-        G = G_;
-        Q = S / G;
-        Rm = S - Q * G;
-        sb = seg_begin(g_start, S, G);
-        r = (int)(((uint32_t)g_start * (uint32_t)Rm) % (uint32_t)G);
+    __host__ __device__ __forceinline__ void init(int g_start, const SplitConsts& k) {
+        G = k.G;
+        Q = (int)k.Q;
+        Rm = (int)k.Rm;
+        sb = seg_begin(g_start, k);
+        r = (int)(((uint32_t)g_start * k.Rm) - (uint32_t)(sb - g_start * Q) * (uint32_t)G);
     }
     __host__ __device__ __forceinline__ void next() {
         sb += Q;

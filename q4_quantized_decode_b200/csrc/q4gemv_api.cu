@@ -13,13 +13,14 @@
 #include "../../include/q4gemv.h"
 #include "gemv_dp2a.cuh"
 #include "gemv_mma.cuh"
+#include "stack.cuh"
 
 namespace {
 
 constexpr int kWarps = 16;                 // warps per CTA of the GEMV kernels
 constexpr int kThreads = kWarps * 32;
 // Per-warp TMA ring (stages x segments per stage) of each kernel.
-constexpr int kR1 = 4, kC1 = 4;            // M = 1
+constexpr int kR1 = 3, kC1 = 6;            // M = 1 and the decode step
 constexpr int kR2 = 2, kC2 = 4;            // M = 2 and the tensor-core kernel
 constexpr int kMinSegsPerWarp = 4;         // small problems use fewer warps
 constexpr int kMaxTiles = Q4GEMV_MAX_N / 32;
@@ -29,6 +30,9 @@ constexpr size_t kMaxDynSmem = 224 * 1024;   // opt-in dynamic shared memory per
 #define Q4_DP2A_KERNEL_2 q4::gemv_dp2a_kernel<2, kWarps, kR2, kC2>
 #define Q4_MMA_KERNEL_1 q4::gemv_mma_kernel<1, kWarps, kR2, kC2>
 #define Q4_MMA_KERNEL_2 q4::gemv_mma_kernel<2, kWarps, kR2, kC2>
+#define Q4_STACK_KERNEL q4::stack_kernel<kWarps, kR1, kC1>
+
+enum StackMode { kStackPersistent = 0, kStackKernels = 1 };
 
 size_t dp2a_smem(int M, int64_t K) {
     return M == 1 ? q4::gemv_dp2a_smem_bytes(1, (int)K, kWarps, kR1, kC1)
@@ -72,6 +76,12 @@ struct q4gemv_ctx {
     cudaStream_t cap = nullptr;   // private capture stream
     cudaGraphExec_t exec = nullptr;
     StackKey key;
+    int stack_mode = kStackPersistent;
+    q4::StackGemv* desc = nullptr;   // device descriptors of the persistent step
+    int desc_cap = 0;
+    StackKey desc_key;
+    bool desc_valid = false;
+    int* sync = nullptr;             // grid barrier words of the persistent step
     std::string last_error;
 };
 
@@ -151,6 +161,7 @@ int launch_gemv(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M,
     a.S = S;
     a.G = ctas * kWarps < S ? ctas * kWarps : S;   // every owning warp gets >= 1 segment
     a.renorm = renorm;
+    a.sc = q4::make_split(a.S, a.G);
     const size_t smem = dp2a_smem(M, K);
 
     cudaLaunchConfig_t cfg = {};
@@ -191,6 +202,26 @@ int ensure_ws(q4gemv_ctx* h, int warps, cudaStream_t st) {
     return Q4_OK;
 }
 
+// Largest block count one CTA of the tensor-core kernel may stage (nt8 = 1:
+// up to 8 vectors, 2: up to 16).
+int mma_xcap(int nt8) {
+    const size_t ring = q4::ring_bytes(kWarps, kR2, kC2);
+    int xcap = 1;
+    while (ring + q4::gemv_mma_smem_bytes(nt8, xcap + 1) <= kMaxDynSmem) ++xcap;
+    return xcap;
+}
+
+// Wide-K problems on the tensor-core path launch ceil(S / xcap) CTAs rounded
+// up to whole waves; the warp count must stay within the split's limit for
+// any wave of up to 256 SMs.
+constexpr int64_t kMmaMaxRunCtas = q4::kMaxSplitWarps / kWarps - 256;
+
+bool mma_split_fits(int M, int64_t N, int64_t K) {
+    const int64_t KB = K / 32, S = (N + 31) / 32 * KB;
+    const int xcap = mma_xcap(M <= 8 ? 1 : 2);
+    return KB <= xcap || (S + xcap - 1) / xcap <= kMmaMaxRunCtas;
+}
+
 // Launch one GEMV on the tensor-core path (any M in 1..16, any K).
 int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M, int64_t N,
                     int64_t K, cudaStream_t st) {
@@ -201,9 +232,7 @@ int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, in
     const int S = T * KB;
     // Largest block count one CTA may stage; a CTA whose run of segments is
     // at least KB stages all KB blocks, so KB must fit or runs stay shorter.
-    const size_t ring = q4::ring_bytes(kWarps, kR2, kC2);
-    int xcap = 1;
-    while (ring + q4::gemv_mma_smem_bytes(nt8, xcap + 1) <= kMaxDynSmem) ++xcap;
+    const int xcap = mma_xcap(nt8);
     const int wave = h->sms;                   // resident CTAs (one per SM)
     int64_t ctas;
     if (KB <= xcap) {
@@ -218,7 +247,10 @@ int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, in
     }
     int64_t G = ctas * kWarps;
     if (G > S) G = S;
-    if (G > q4::kMaxSplitWarps) G = q4::kMaxSplitWarps;
+    // Capping G would lengthen the CTAs' runs past xcap blocks of staged
+    // activations: refuse such (very large, very wide) problems instead.
+    if (G > q4::kMaxSplitWarps)
+        return fail(h, Q4_ESHAPE, "run: N * K too large for the M >= 3 / wide-K path");
     const int rc = ensure_ws(h, (int)G, st);
     if (rc != Q4_OK) return rc;
     const int nblk_max = (KB <= xcap) ? KB : xcap;
@@ -236,10 +268,11 @@ int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, in
     a.S = S;
     a.G = (int)G;
     a.M = M;
+    a.sc = q4::make_split(a.S, a.G);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)ctas);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = ring + q4::gemv_mma_smem_bytes(nt8, nblk_max);
+    cfg.dynamicSmemBytes = q4::ring_bytes(kWarps, kR2, kC2) + q4::gemv_mma_smem_bytes(nt8, nblk_max);
     cfg.stream = st;
     cfg.numAttrs = 0;
     cudaError_t e;
@@ -315,6 +348,7 @@ int q4gemv_validate(int M, int64_t N, int64_t K, const void* W, const void* x, c
     if (M < 1 || M > Q4GEMV_MAX_M) return Q4_EUNSUPPORTED;
     const int sh = check_shape(N, K);
     if (sh != Q4_OK) return sh;
+    if (!dp2a_fits(M, K) && !mma_split_fits(M, N, K)) return Q4_ESHAPE;
     if (!W || !x || !y) return Q4_EINVAL;
     if (!aligned16(W) || !aligned16(x) || !aligned16(y)) return Q4_EALIGN;
     return Q4_OK;
@@ -352,8 +386,11 @@ int q4gemv_create(q4gemv_t* out, int device) {
         const size_t ws_bytes = (size_t)h->ws_warps * 2 * Q4GEMV_MAX_M * 32 * sizeof(float);
         if (cudaMalloc(&h->ws, ws_bytes) != cudaSuccess ||
             cudaMalloc(&h->cnt, (size_t)kMaxTiles * sizeof(int)) != cudaSuccess ||
-            cudaMalloc(&h->err, sizeof(int)) != cudaSuccess)
+            cudaMalloc(&h->err, sizeof(int)) != cudaSuccess ||
+            cudaMalloc(&h->sync, 4 * sizeof(int)) != cudaSuccess)
             rc = fail(h, Q4_ENOMEM, "workspace allocation failed");
+        const char* mode = getenv("Q4GEMV_STACK_MODE");
+        if (mode && !strcmp(mode, "kernels")) h->stack_mode = kStackKernels;
     }
     if (rc == Q4_OK) {
         if (cudaMemset(h->cnt, 0, (size_t)kMaxTiles * sizeof(int)) != cudaSuccess ||
@@ -363,6 +400,7 @@ int q4gemv_create(q4gemv_t* out, int device) {
     if (rc == Q4_OK) {
         if (set_smem_attr(Q4_DP2A_KERNEL_1) || set_smem_attr(Q4_DP2A_KERNEL_2) ||
             set_smem_attr(Q4_MMA_KERNEL_1) || set_smem_attr(Q4_MMA_KERNEL_2) ||
+            set_smem_attr(Q4_STACK_KERNEL) ||
             0)
             rc = fail(h, Q4_ECUDA, "cudaFuncSetAttribute failed");
     }
@@ -378,6 +416,7 @@ int q4gemv_create(q4gemv_t* out, int device) {
         cudaFree(h->ws);
         cudaFree(h->cnt);
         cudaFree(h->err);
+        cudaFree(h->sync);
         if (h->cap) cudaStreamDestroy(h->cap);
         delete h;
         return rc;
@@ -396,6 +435,8 @@ int q4gemv_destroy(q4gemv_t h) {
     cudaFree(h->cnt);
     cudaFree(h->err);
     cudaFree(h->act);
+    cudaFree(h->desc);
+    cudaFree(h->sync);
     delete h;
     return Q4_OK;
 }
@@ -474,6 +515,69 @@ int enqueue_stack(q4gemv_ctx* h, const StackKey& k, cudaStream_t st) {
     return launch_renorm(h, prev, static_cast<__half*>(k.x_out), (int)hidden, st, true);
 }
 
+// Descriptors of the persistent step for key k (host side).
+void build_descriptors(q4gemv_ctx* h, const StackKey& k, std::vector<q4::StackGemv>& out) {
+    const int64_t hidden = k.hidden, qkv_n = k.qkv_n, ffn = k.ffn;
+    const int64_t kmax = hidden > ffn ? hidden : ffn;
+    int64_t nmax = qkv_n > hidden ? qkv_n : hidden;
+    if (2 * ffn > nmax) nmax = 2 * ffn;
+    const int64_t n_of[4] = {qkv_n, hidden, 2 * ffn, hidden};
+    const int64_t k_of[4] = {hidden, hidden, hidden, ffn};
+    __half* buf[4];
+    size_t off = 0;
+    for (int t = 0; t < 4; ++t) {
+        buf[t] = h->act + off;
+        off += (size_t)((n_of[t] + 7) / 8 * 8);
+    }
+    const int n_gemv = 4 * (int)k.layers.size();
+    out.resize(n_gemv);
+    for (int i = 0; i < n_gemv; ++i) {
+        const int l = i / 4, t = i % 4;
+        const q4gemv_layer& L = k.layers[l];
+        q4::StackGemv& d = out[i];
+        d.W = static_cast<const uint8_t*>(t == 0 ? L.qkv : t == 1 ? L.o : t == 2 ? L.gate_up : L.down);
+        d.y = k.trace_y ? static_cast<__half*>(k.trace_y) + (size_t)i * nmax : buf[t];
+        d.trace_x = k.trace_x ? static_cast<__half*>(k.trace_x) + (size_t)i * kmax : nullptr;
+        d.N = (int)n_of[t];
+        d.K = (int)k_of[t];
+        d.renorm = i == 0 ? 0 : 1;
+        d.pad = 0;
+        const int S = (int)((n_of[t] + 31) / 32 * (k_of[t] / 32));
+        const int gmax = h->sms * kWarps;
+        d.sc = q4::make_split(S, gmax < S ? gmax : S);
+    }
+}
+
+// The whole step as one cooperative launch (plus the barrier reset).
+int enqueue_stack_persistent(q4gemv_ctx* h, const StackKey& k, cudaStream_t st) {
+    if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
+    const int64_t kmax = k.hidden > k.ffn ? k.hidden : k.ffn;
+    Q4_CUDA(h, cudaMemsetAsync(h->sync, 0, 4 * sizeof(int), st));
+    q4::StackArgs sa;
+    sa.gemv = h->desc;
+    sa.n_gemv = 4 * (int)k.layers.size();
+    sa.x_in = static_cast<const __half*>(k.x_in);
+    sa.x_out = static_cast<__half*>(k.x_out);
+    sa.hidden = (int)k.hidden;
+    sa.ws = h->ws;
+    sa.cnt = h->cnt;
+    sa.err = h->err;
+    sa.sync = h->sync;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(h->sms);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = q4::ring_bytes(kWarps, kR1, kC1) + (size_t)kmax * 3;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, Q4_STACK_KERNEL, sa, (int)kmax);
+    if (e != cudaSuccess) return cuda_fail(h, e, "decode-step launch");
+    return Q4_OK;
+}
+
 }  // namespace
 
 int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64_t hidden,
@@ -532,6 +636,33 @@ int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64
         h->act_elems = need;
     }
 
+    const int64_t kmax_step = hidden > ffn ? hidden : ffn;
+    if (h->stack_mode == kStackPersistent && kmax_step <= (int64_t)q4::kStackXChunks * 8 * kThreads &&
+        q4::ring_bytes(kWarps, kR1, kC1) + (size_t)kmax_step * 3 <= kMaxDynSmem) {
+        if (!h->desc_valid || !(h->desc_key == k)) {
+            if (cs != cudaStreamCaptureStatusNone)
+                return fail(h, Q4_EUNSUPPORTED,
+                            "run_stack: first call with these arguments must happen outside stream capture");
+            std::vector<q4::StackGemv> desc;
+            build_descriptors(h, k, desc);
+            if ((int)desc.size() > h->desc_cap) {
+                if (h->fault == kFaultAlloc) return fail(h, Q4_EFAULTINJ, "injected allocation failure");
+                Q4_CUDA(h, cudaStreamSynchronize(st));
+                cudaFree(h->desc);
+                h->desc = nullptr;
+                h->desc_cap = 0;
+                if (cudaMalloc(&h->desc, desc.size() * sizeof(q4::StackGemv)) != cudaSuccess)
+                    return fail(h, Q4_ENOMEM, "run_stack: descriptor allocation failed");
+                h->desc_cap = (int)desc.size();
+            }
+            Q4_CUDA(h, cudaStreamSynchronize(st));
+            Q4_CUDA(h, cudaMemcpy(h->desc, desc.data(), desc.size() * sizeof(q4::StackGemv),
+                                  cudaMemcpyHostToDevice));
+            h->desc_key = k;
+            h->desc_valid = true;
+        }
+        return enqueue_stack_persistent(h, k, st);
+    }
     if (cs != cudaStreamCaptureStatusNone) return enqueue_stack(h, k, st);
 
     if (!h->exec || !(h->key == k)) {

@@ -130,6 +130,7 @@ extern "C" int q4gemv_run_noalloc(const void* W, const void* x, void* y, int M, 
     a.S = S;
     a.G = ctas * kNaWarps < S ? ctas * kNaWarps : S;
     a.renorm = 0;
+    a.sc = q4::make_split(a.S, a.G);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ctas);
     cfg.blockDim = dim3(kNaThreads);

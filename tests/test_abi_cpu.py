@@ -73,6 +73,18 @@ def test_validate_paths():
     assert v(1, 32, 32, A, A, A + 4) == q4.Q4_EALIGN
 
 
+def test_validate_wide_k_split_limit():
+    """Very wide matrices on the tensor-core path are accepted while the warp
+    split stays within its limit, refused (not truncated) beyond it."""
+    v = q4.q4gemv_validate
+    assert v(1, 32, 1 << 17, A, A, A) == q4.Q4_OK          # one tile, 4096 blocks
+    assert v(4, 4096, 1 << 17, A, A, A) == q4.Q4_OK        # 131072 segments
+    assert v(1, 1 << 20, 1 << 17, A, A, A) == q4.Q4_ESHAPE  # 2^27 segments
+    assert v(16, 1 << 16, 1 << 16, A, A, A) == q4.Q4_ESHAPE
+    assert v(4, 5120, 5120, A, A, A) == q4.Q4_OK           # KB fits one CTA: no limit
+    assert v(4, 1 << 22, 4096, A, A, A) == q4.Q4_OK
+
+
 def test_null_handle_is_rejected():
     assert q4.q4gemv_run(None, A, A, A, 1, 32, 32, None) == q4.Q4_EINVAL
     assert q4.q4gemv_repack(None, A, A, 32, 32, None) == q4.Q4_EINVAL

@@ -307,6 +307,24 @@ def test_stack_graph_replay_follows_input(eng):
     assert np.array_equal(bits_of(xin), ob)
 
 
+def test_stack_persistent_matches_per_gemv_kernels(monkeypatch):
+    """The one-launch step and the graph of per-GEMV kernels run the same
+    per-warp arithmetic over the same split: identical bits at full width."""
+    L, hidden, qkv_n, ffn = 2, 5120, 7168, 17408
+    outs = {}
+    for mode in ("persistent", "kernels"):
+        monkeypatch.setenv("Q4GEMV_STACK_MODE", mode)
+        e = q4.Q4Gemv(0)
+        if mode == "persistent":
+            layers, _ = build_stack(e, L, hidden, qkv_n, ffn, 77)
+        x = synth.normal_f16(77, synth.act_id(0), hidden)
+        o1, tx, ty = run_stack_traced(e, layers, x, hidden, qkv_n, ffn)
+        outs[mode] = (o1, tx, ty)
+        e.close()
+    for a, b in zip(outs["persistent"], outs["kernels"]):
+        assert np.array_equal(a, b)
+
+
 @pytest.mark.slow
 def test_stack_full_27b_teacher_forced_sampled():
     """The full 64-layer, 27B-shaped step (11.9 GB of Q4_0), checked per GEMV
@@ -362,7 +380,7 @@ def test_fault_injection_and_invalid_calls(eng):
     with pytest.raises(q4.Q4Error) as e:
         fresh.run_stack(layers, xs, hidden, qkv_n, ffn)
     assert e.value.status == q4.Q4_EFAULTINJ
-    fresh.set_fault("graph")
+    fresh.set_fault("launch")
     with pytest.raises(q4.Q4Error) as e:
         fresh.run_stack(layers, xs, hidden, qkv_n, ffn)
     assert e.value.status == q4.Q4_EFAULTINJ
@@ -372,6 +390,22 @@ def test_fault_injection_and_invalid_calls(eng):
     fresh.close()
     eng.run(W, x, N, K)
     assert eng.sync_status() == q4.Q4_OK
+
+
+def test_graph_fault_in_per_gemv_mode(monkeypatch):
+    monkeypatch.setenv("Q4GEMV_STACK_MODE", "kernels")
+    eng = q4.Q4Gemv(0)
+    L, hidden, qkv_n, ffn = 1, 64, 96, 128
+    layers, _ = build_stack(eng, L, hidden, qkv_n, ffn, 3)
+    xs = f16_dev(synth.normal_f16(3, synth.act_id(0), hidden))
+    eng.set_fault("graph")
+    with pytest.raises(q4.Q4Error) as e:
+        eng.run_stack(layers, xs, hidden, qkv_n, ffn)
+    assert e.value.status == q4.Q4_EFAULTINJ
+    eng.set_fault("none")
+    eng.run_stack(layers, xs, hidden, qkv_n, ffn)
+    assert eng.sync_status() == q4.Q4_OK
+    eng.close()
 
 
 def test_create_fault_from_environment(monkeypatch):

@@ -21,6 +21,7 @@ def probe(tmp_path_factory):
     lib = ctypes.CDLL(str(out))
     for f in ("probe_seg_begin", "probe_warp_of_seg"):
         getattr(lib, f).argtypes = [ctypes.c_int] * 3
+    lib.probe_walk.argtypes = [ctypes.c_int] * 4
     lib.probe_xperm_pos.argtypes = [ctypes.c_int]
     return lib
 
@@ -70,6 +71,32 @@ def test_arrival_bookkeeping(probe, S, G, KB):
             if gf != gl:
                 sl = 0 if begins[gg] // KB == t else 1
                 assert (gg, sl) in slots_used
+
+
+BIG = [(2**31 - 1, 2368), (2**31 - 1, 65535), (123456789, 40000), (2**30 + 7, 3),
+       (5 * 2**20 + 3, 65535), (2**24, 2**16 - 1), (65535, 65535), (2, 2), (3, 2)]
+
+
+@pytest.mark.parametrize("S,G", BIG)
+def test_reciprocal_division_is_exact(probe, S, G):
+    """seg_begin / warp_of_seg divide by multiplying with a 64-bit reciprocal;
+    check them against exact integer division, including splits whose
+    numerators need 64 bits."""
+    import random
+    rng = random.Random(S * 7919 + G)
+    gs = [0, 1, G - 1, G] + [rng.randrange(G + 1) for _ in range(300)]
+    for g in gs:
+        assert probe.probe_seg_begin(g, S, G) == g * S // G
+    ss = [0, 1, S - 1, S - 2 if S > 1 else 0] + [rng.randrange(S) for _ in range(300)]
+    for s in ss:
+        assert probe.probe_warp_of_seg(s, S, G) == ((s + 1) * G - 1) // S
+
+
+@pytest.mark.parametrize("S,G", [(25600, 2368), (87040, 2368), (17, 5), (100, 99), (9, 1)])
+def test_walker_matches_seg_begin(probe, S, G):
+    for g0 in (0, 1, G // 3, G - 1):
+        for steps in range(0, min(G - g0, 40) + 1):
+            assert probe.probe_walk(g0, steps, S, G) == (g0 + steps) * S // G
 
 
 def test_xperm_is_a_permutation_grouping_lane_words(probe):
