@@ -3,11 +3,15 @@
 
 One step = one synthetic 27B-shaped decode step (M = 1): 64 layers x
 (QKV 5120->7168, O 5120->5120, gate+up 5120->34816, down 17408->5120) Q4_0
-GEMVs with the renorm chain, issued as one CUDA graph through the C-ABI
-(q4gemv_run_stack).  11.9 GB of weights per step, far larger than L2, so no
-flush is needed between steps.
+GEMVs with the renorm chain, run through the C-ABI (q4gemv_run_stack) as one
+persistent kernel launch (plus a 16-byte reset of its barrier words).
+11.9 GB of weights per step, far larger than L2, so no flush is needed
+between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--layers L runs an L-layer step instead (profiling captures only; the
+reported workload then says so).
 
 Under torchrun (N > 1) every rank runs an independent replica (same weights,
 its own activation stream); there is no data-path collective, only a barrier
@@ -34,7 +38,7 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "achieved HBM GB/s (% of B200 peak) for Q4_0 GEMV; 27B-shaped decode steps/s"
-L, HIDDEN, QKV_N, FFN = 64, 5120, 7168, 17408
+L, HIDDEN, QKV_N, FFN = 64, 5120, 7168, 17408   # L: layers of the step (--layers)
 DIMS = [(QKV_N, HIDDEN), (HIDDEN, HIDDEN), (2 * FFN, HIDDEN), (HIDDEN, FFN)]
 SHAPE_NAMES = ["qkv_5120x7168", "o_5120x5120", "gate_up_5120x34816", "down_17408x5120"]
 CONFIG_SEED = synth.config_seed(4)
@@ -50,7 +54,7 @@ STEP_GEMV_BYTES = L * sum(gemv_bytes(N, K) for N, K in DIMS)
 STEP_WEIGHT_BYTES = L * sum(N * (K // 32) * 18 for N, K in DIMS)
 WORKLOAD = ("27B-shaped decode step, M=1: 64 layers x (QKV 5120->7168, O 5120->5120, "
             "gate+up 5120->34816, down 17408->5120) Q4_0 GEMVs with unit-RMS renorm between "
-            "matrices, one CUDA graph per step")
+            "matrices, one persistent kernel launch per step")
 
 
 def measured_peaks():
@@ -337,8 +341,9 @@ def run_ours(args, rank: int, world: int, dist):
     roofline = {
         "bound": "hbm", "achieved": per_rank_gbs, "peak": peak, "unit": "GB/s",
         "frac": per_rank_gbs / peak, "traffic": None,
-        "kernel": "q4::gemv_dp2a_kernel<1,16,8> (256 launches per step; duration = step time, "
-                  "which also holds one small renorm kernel)",
+        "kernel": "q4::stack_kernel<16,3,6> (one persistent launch per step, all 4L GEMVs and "
+                  "the final renorm; duration = step time, which also holds the 16-byte "
+                  "barrier-word reset before each launch)",
         "peak_source": f"{peak_kind} hbm_gbs (copy) in MEASURED_PEAKS.json",
         "frac_of_nominal_8TBps": per_rank_gbs / NOMINAL_HBM_GBS,
     }
@@ -370,7 +375,7 @@ def run_ours(args, rank: int, world: int, dist):
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": 2 * HIDDEN,
                 "d2h_bytes_per_step": 2 * HIDDEN,
                 "steps_per_s": e2e_steps_per_s},
-        "gpu_launches": args.steps * (4 * L + 1),
+        "gpu_launches": args.steps,      # one stack_kernel per step (and one 16-byte memset)
         "clocks": clocks,
         "repack_s_per_step_weights": t_repack,
         "per_shape_m1": per_shape,
@@ -426,6 +431,16 @@ def run_case(args):
     return 0
 
 
+def set_layers(n: int):
+    """Switch the step to n layers (profiling captures of a smaller case)."""
+    global L, STEP_GEMV_BYTES, STEP_WEIGHT_BYTES, WORKLOAD
+    L = n
+    STEP_GEMV_BYTES = L * sum(gemv_bytes(N, K) for N, K in DIMS)
+    STEP_WEIGHT_BYTES = L * sum(N * (K // 32) * 18 for N, K in DIMS)
+    if n != 64:
+        WORKLOAD = WORKLOAD.replace("64 layers", f"{n} layers (profiling case, not the benchmark)")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -441,7 +456,10 @@ def main():
     ap.add_argument("--M", type=int, default=1)
     ap.add_argument("--rotate", type=int, default=0, help="matrix copies in rotation (0: > 4x L2)")
     ap.add_argument("--config-seed", type=int, default=2)
+    ap.add_argument("--layers", type=int, default=64, help="layers of the step (profiling only)")
     args = ap.parse_args()
+    if args.layers != 64:
+        set_layers(args.layers)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))

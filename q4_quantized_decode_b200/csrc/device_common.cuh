@@ -110,6 +110,11 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     return false;
 }
 
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
 __device__ __forceinline__ void sts64(uint32_t addr, uint2 v) {
     asm volatile("st.shared.v2.u32 [%0], {%1,%2};" :: "r"(addr), "r"(v.x), "r"(v.y) : "memory");
 }
@@ -146,6 +151,18 @@ __device__ __forceinline__ float ld_relaxed_gpu(const float* p) {
     float v;
     asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
     return v;
+}
+
+// Unit-RMS scale of a vector of `len` entries with sum of squares s (fp32):
+// 1/sqrt(s/len) from the hardware's approximate quotient and reciprocal
+// square root (a few ulp, the same on every call); 0 for s <= 0 or NaN.
+__device__ __forceinline__ float renorm_scale(float s, int len) {
+    return (s > 0.f) ? rsqrtf(__fdividef(s, (float)len)) : 0.f;
+}
+
+// One-line prefetch into L1.
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
 
 // global -> shared bulk copy to a shared-window address.

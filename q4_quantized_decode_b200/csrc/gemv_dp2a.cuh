@@ -20,9 +20,12 @@
 //     (q - 8) * X is an exact integer;
 //   * the block sum is scaled by d * 2^e in fp32 and accumulated per row;
 //   * a warp's accumulators are combined across its four column lanes with
-//     two shuffles; tiles split between warps are combined by the last warp
-//     to arrive (per-tile counter), summing the partials in warp order, so
-//     results are deterministic.
+//     two shuffles.  A tile split between warps is combined in two levels,
+//     each a sum in a fixed order, so results are deterministic: the warps of
+//     one CTA park their partials in shared memory and the CTA's first
+//     contributing warp sums them in warp order; a tile shared by several
+//     CTAs then leaves one partial per CTA in global memory, summed in CTA
+//     order by the last CTA to arrive (per-tile counter).
 #pragma once
 
 #include "device_common.cuh"
@@ -38,7 +41,7 @@ struct GemvArgs {
     const uint8_t* W;       // packed matrix (segments of 576 bytes)
     const __half* x;        // [M][K] activations, or the renorm source (M == 1)
     __half* y;              // [M][N]
-    float* ws;              // split-tile partials [G][2][M][32]
+    float* ws;              // CTA partials of tiles shared by CTAs [CTAs][2][M][32]
     int* cnt;               // per-tile arrival counters [T], zero between calls
     int* err;               // device error word
     __half* trace_x;        // nullable: CTA 0 writes the f16 input vector it used
@@ -55,11 +58,18 @@ __host__ __device__ constexpr size_t ring_bytes(int warps, int R, int C) {
     return (size_t)warps * R * C * kSegBytes;
 }
 
+// Per warp, two parked tile partials (the first and the last tile of its
+// run), M vectors of 32 fp32 each.
+__host__ __device__ constexpr size_t warp_partial_bytes(int M, int warps) {
+    return (size_t)warps * 2 * M * 32 * sizeof(float);
+}
+
 // Shared-memory footprint of the M <= 2 kernel: the ring, the int16
-// activations (2 bytes per element) and, per block and lane group, the pair
-// {-8 * sum X, block scale} (8 bytes, 32 per block).
+// activations (2 bytes per element), per block and lane group the pair
+// {-8 * sum X, block scale} (8 bytes, 32 per block), then the warp partials.
 __host__ __device__ constexpr size_t gemv_dp2a_smem_bytes(int M, int K, int warps, int R, int C) {
-    return ring_bytes(warps, R, C) + (size_t)M * K * 2 + (size_t)M * (K / 32) * 32;
+    return ring_bytes(warps, R, C) + (size_t)M * K * 2 + (size_t)M * (K / 32) * 32 +
+           warp_partial_bytes(M, warps);
 }
 
 // Position of element j of a 32-column block in the permuted X layout: the
@@ -111,10 +121,23 @@ struct WarpRing {
 // group c of the block gets {-8 * sum of its eight X, 2^(E-14)}.
 // kCoherent: load x through L2 only (it was written by other CTAs of the
 // same running kernel, so an L1 copy could be stale).
-// QN: 16-byte chunks held per thread (M * K <= QN * 8 * NT).
-template <int M, int NT, bool kCoherent = false, int QN = kXChunksPerThread>
+// QN: 16-byte chunks held per thread (M * K <= QN * 8 * NT); all QN rounds
+// run (chunks past the end are zeros), so callers pick the smallest QN that
+// covers the vector: the rounds then overlap instead of running one by one.
+// Fix: completes the loaded input where it exists only as partial sums (the
+// persistent step); NoFix keeps what was loaded.  A Fix with kActive runs
+// prepare() with all threads (it may use the X area of shared memory as
+// scratch), then, after a CTA barrier, apply() per chunk.
+struct NoFix {
+    static constexpr bool kActive = false;
+    template <int NT>
+    __device__ __forceinline__ void prepare(int, uint32_t) const {}
+    __device__ __forceinline__ uint4 apply(int, uint4 v, uint32_t) const { return v; }
+};
+
+template <int M, int NT, bool kCoherent = false, int QN = kXChunksPerThread, class Fix = NoFix>
 __device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs, uint32_t rec,
-                                                  float* red) {
+                                                  float* red, const Fix& fix = Fix()) {
     const int tid = threadIdx.x, lane = tid & 31;
     const int nq = M * a.K / 8;
     uint4 xr[QN];
@@ -123,6 +146,15 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs
         const int q = tid + NT * i;
         const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)q * 8);
         xr[i] = q < nq ? (kCoherent ? __ldcg(src) : *src) : make_uint4(0, 0, 0, 0);
+    }
+    if constexpr (Fix::kActive) {
+        fix.template prepare<NT>(nq, xs);
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < QN; ++i) {
+            const int q = tid + NT * i;
+            if (q < nq) xr[i] = fix.apply(q, xr[i], xs);
+        }
     }
     if (M == 1 && a.renorm) {
         float part = 0.f;
@@ -143,7 +175,7 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs
         float s = 0.f;
 #pragma unroll
         for (int w = 0; w < NT / 32; ++w) s += red[w];
-        const float scale = (s > 0.f) ? __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(s, (float)a.K))) : 0.f;
+        const float scale = renorm_scale(s, a.K);
 #pragma unroll
         for (int i = 0; i < QN; ++i) {
             __half2* h = reinterpret_cast<__half2*>(&xr[i]);
@@ -174,28 +206,32 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs
         for (int e = 0; e < 8; ++e) mx = max(mx, __float_as_uint(fabsf(v[e])));
         mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
         mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        int X[8];
-        float sc = 0.f;
+        // X = rint(v * 2^(14-E)) (E: exponent of the block maximum), read from
+        // the low mantissa bits of v * 2^(14-E) + 1.5 * 2^23: the product is
+        // exact and |X| <= 32752, so the one rounding of the addition is the
+        // round-to-nearest-even to an integer and the bits hold 0x4B400000 + X.
+        // All-zero block: X = 0, scale 0.  Non-finite block: scale NaN (the
+        // outputs become NaN whatever X holds).
+        const int E = (int)(mx >> 23) - 127;                                   // max in [2^E, 2^(E+1))
+        const bool live = mx != 0u && mx < 0x7F800000u;
+        const float inv = live ? __uint_as_float((uint32_t)(141 - E) << 23) : 0.f;   // 2^(14-E)
+        const float sc = live ? __uint_as_float((uint32_t)(113 + E) << 23)            // 2^(E-14)
+                              : (mx == 0u ? 0.f : __uint_as_float(0x7FC00000u));
+        uint32_t xb[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) X[e] = 0;
-        if (mx >= 0x7F800000u) {
-            sc = __uint_as_float(0x7FC00000u);          // non-finite block -> NaN outputs
-        } else if (mx != 0u) {
-            const int E = (int)(mx >> 23) - 127;        // block max in [2^E, 2^(E+1))
-            const float inv = __uint_as_float((uint32_t)(141 - E) << 23);   // 2^(14-E)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) X[e] = __float2int_rn(v[e] * inv);
-            sc = __uint_as_float((uint32_t)(113 + E) << 23);                 // 2^(E-14)
-        }
-        int h0 = X[0] + X[1] + X[2] + X[3], h1 = X[4] + X[5] + X[6] + X[7];
+        for (int e = 0; e < 8; ++e) xb[e] = __float_as_uint(fmaf(v[e], inv, 12582912.0f));
+        int h0 = (int)(xb[0] + xb[1] + xb[2] + xb[3] - 4u * 0x4B400000u);
+        int h1 = (int)(xb[4] + xb[5] + xb[6] + xb[7] - 4u * 0x4B400000u);
         h0 += __shfl_xor_sync(0xffffffffu, h0, 2);      // quarters u and u^2 share lane groups
         h1 += __shfl_xor_sync(0xffffffffu, h1, 2);
         if (q < nq) {
             const int bb = q >> 2, u = q & 3;
             const int pos0 = (u & 1) * 16 + (u >> 1) * 4;   // elements 8u..8u+3 (then +8 for 8u+4..8u+7)
-            const uint32_t xb = xs + (uint32_t)bb * 64;
-            sts64(xb + pos0 * 2, pack_s16x4(X[0], X[1], X[2], X[3]));
-            sts64(xb + pos0 * 2 + 16, pack_s16x4(X[4], X[5], X[6], X[7]));
+            const uint32_t xsb = xs + (uint32_t)bb * 64;
+            // The low 16 bits of xb[e] are X[e] in two's complement.
+            sts64(xsb + pos0 * 2, make_uint2(__byte_perm(xb[0], xb[1], 0x5410), __byte_perm(xb[2], xb[3], 0x5410)));
+            sts64(xsb + pos0 * 2 + 16,
+                  make_uint2(__byte_perm(xb[4], xb[5], 0x5410), __byte_perm(xb[6], xb[7], 0x5410)));
             if (u < 2) {
                 const int c0 = (u & 1) * 2;
                 const uint32_t rb = rec + (uint32_t)bb * 32 + c0 * 8;
@@ -217,9 +253,12 @@ struct Dp2aConsumer {
     int KB, t_cur, b;        // b: block of the next segment
     uint32_t x_lane0, r_lane0, xp, rp;   // running shared addresses of block b's X words and record
     uint32_t xstride, rstride;           // per activation vector
+    float* park;             // this warp's two parked partials [2][M][32] (shared memory)
 
-    __device__ __forceinline__ void init(const GemvArgs& a, int gw_, uint32_t xs, uint32_t rec) {
+    __device__ __forceinline__ void init(const GemvArgs& a, int gw_, uint32_t xs, uint32_t rec,
+                                         float* park_) {
         gw = gw_;
+        park = park_;
         lane = threadIdx.x & 31;
         g = lane >> 2;
         c = lane & 3;
@@ -260,7 +299,7 @@ struct Dp2aConsumer {
             if (whole) {
                 if (row < a.N) a.y[(size_t)m * a.N + row] = __float2half_rn(val);
             } else {
-                a.ws[(((size_t)gw * 2 + sp.slot(t)) * M + m) * 32 + r] = val;
+                park[(sp.slot(t) * M + m) * 32 + r] = val;
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
@@ -343,61 +382,102 @@ struct Dp2aConsumer {
         }
     }
 
-    // Tiles shared with other warps (at most the first and the last one of
-    // this warp's run): count arrivals; the last warp to arrive sums the
-    // partials in warp order, writes y and re-arms the counter.
-    __device__ __forceinline__ void arrive(const GemvArgs& a, int t, int gf, int gl) {
-        if (gf == gl) return;
-        __syncwarp();
-        int old = 0;
-        if (lane == 0) old = atom_add_acq_rel_gpu(a.cnt + t, 1);
-        old = __shfl_sync(0xffffffffu, old, 0);
-        __syncwarp();                       // order the lanes' reads after lane 0's acquire
-        const int need = gl - gf + 1;
-        if (old == need - 1) {
-            const int64_t row = (int64_t)t * 32 + r;
+    // End of the run: the last tile.
+    __device__ __forceinline__ void flush_last(const GemvArgs& a) {
+        if (sp.s1 > sp.s0) flush(a, t_cur);
+    }
+
+    // First level of the split-tile combine, after a CTA-wide barrier that
+    // follows every warp's flush_last.  Of each tile split between warps, the
+    // CTA's first contributing warp sums the parked partials of the CTA's
+    // contributors in warp order (lane = row).  A tile inside the CTA is then
+    // finished (y written); for a tile shared with other CTAs the CTA's
+    // partial goes to ws[cta][slot], slot 0 if the CTA's run starts in the
+    // tile, else 1, and the tile is returned in xt[] (at most two, -1: none)
+    // with its contributing CTAs [xcf, xcl].
+    template <int WARPS>
+    __device__ __forceinline__ void combine_cta(const GemvArgs& a, const float* park_base, float* ws,
+                                                int xt[2], int xcf[2], int xcl[2]) {
+        xt[0] = xt[1] = -1;
+        if (sp.s1 <= sp.s0) return;
+        const int cta_lo = blockIdx.x * WARPS, cta_hi = cta_lo + WARPS - 1;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int t = e == 0 ? sp.t_first : sp.t_last;
+            const int gf = e == 0 ? sp.gf0 : sp.gf1, gl = e == 0 ? sp.gl0 : sp.gl1;
+            if (!cta_combiner(sp, e, gw, cta_lo)) continue;
+            const int w_to = min(gl, cta_hi);
             float sum[M];
 #pragma unroll
             for (int m = 0; m < M; ++m) sum[m] = 0.f;
-            SegWalker wk;
-            wk.init(gf, a.sc);
-            // Sixteen contributors per round: their loads are issued together,
-            // the sum is still taken in warp order.
-            for (int g0 = gf; g0 <= gl; g0 += 16) {
-                float pv[16][M];
+            for (int w = gw; w <= w_to; ++w) {
+                const int sl = park_slot_read(sp, gw, w, t);
+                const float* p = park_base + ((size_t)(w - cta_lo) * 2 + sl) * M * 32;
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int gg = g0 + u;
-                    const int sl = (wk.sb >= t * KB) ? 0 : 1;   // t is where gg's run starts
-#pragma unroll
-                    for (int m = 0; m < M; ++m)
-                        pv[u][m] = gg <= gl ? ld_relaxed_gpu(a.ws + (((size_t)gg * 2 + sl) * M + m) * 32 + r)
-                                            : 0.f;
-                    wk.next();
-                }
-#pragma unroll
-                for (int u = 0; u < 16; ++u)
-#pragma unroll
-                    for (int m = 0; m < M; ++m) sum[m] += pv[u][m];
+                for (int m = 0; m < M; ++m) sum[m] += p[m * 32 + lane];
             }
+            if (gf >= cta_lo && gl <= cta_hi) {
+                const int64_t row = (int64_t)t * 32 + lane;
 #pragma unroll
-            for (int m = 0; m < M; ++m)
-                if (row < a.N) a.y[(size_t)m * a.N + row] = __float2half_rn(sum[m]);
-            if (lane == 0) a.cnt[t] = 0;
-        } else if (old >= need) {
-            if (lane == 0) set_device_error(a.err, kDevConcurrent);
-        }
-    }
-
-    // End of the run: last tile, then the arrivals.
-    __device__ __forceinline__ void finish(const GemvArgs& a) {
-        if (sp.s1 > sp.s0) {
-            flush(a, t_cur);
-            arrive(a, sp.t_first, sp.gf0, sp.gl0);
-            if (sp.t_last != sp.t_first) arrive(a, sp.t_last, sp.gf1, sp.gl1);
+                for (int m = 0; m < M; ++m)
+                    if (row < a.N) a.y[(size_t)m * a.N + row] = __float2half_rn(sum[m]);
+            } else {
+                const int slc = cta_slot_write(blockIdx.x, t, KB, a.sc, WARPS);
+#pragma unroll
+                for (int m = 0; m < M; ++m)
+                    ws[(((size_t)blockIdx.x * 2 + slc) * M + m) * 32 + lane] = sum[m];
+                xt[e] = t;
+                xcf[e] = gf / WARPS;
+                xcl[e] = gl / WARPS;
+            }
         }
     }
 };
+
+// Second level, q4gemv_run's kernel: CTAs that left a partial of tile t count
+// their arrival; the last to arrive sums the CTA partials in CTA order,
+// writes y and re-arms the counter.  One warp, lane = row.
+template <int M, int WARPS>
+__device__ __forceinline__ void combine_ctas_arrive(const GemvArgs& a, int t, int cf, int cl) {
+    const int lane = threadIdx.x & 31;
+    __syncwarp();
+    int old = 0;
+    if (lane == 0) old = atom_add_acq_rel_gpu(a.cnt + t, 1);
+    old = __shfl_sync(0xffffffffu, old, 0);
+    __syncwarp();                       // order the lanes' reads after lane 0's acquire
+    const int need = cl - cf + 1;
+    if (old == need - 1) {
+        float sum[M];
+#pragma unroll
+        for (int m = 0; m < M; ++m) sum[m] = 0.f;
+        // Eight contributors per round: their loads are issued together, the
+        // sum is still taken in CTA order.
+        for (int c0 = cf; c0 <= cl; c0 += 8) {
+            float pv[8][M];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int c = c0 + u;
+                const int sl = cta_slot_read(c, cf, t, a.KB, a.sc, WARPS);
+#pragma unroll
+                for (int m = 0; m < M; ++m)
+                    pv[u][m] = c <= cl ? ld_relaxed_gpu(a.ws + (((size_t)c * 2 + sl) * M + m) * 32 + lane)
+                                       : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (c0 + u <= cl)
+#pragma unroll
+                    for (int m = 0; m < M; ++m) sum[m] += pv[u][m];
+        }
+        const int64_t row = (int64_t)t * 32 + lane;
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+            if (row < a.N) a.y[(size_t)m * a.N + row] = __float2half_rn(sum[m]);
+        if (lane == 0) a.cnt[t] = 0;
+    } else if (old >= need) {
+        if (lane == 0) set_device_error(a.err, kDevConcurrent);
+    }
+}
 
 template <int M, int WARPS, int R, int C>
 __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs a) {
@@ -408,6 +488,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
     const uint32_t smem_base = smem_addr(smem);
     const uint32_t xs = smem_base + (uint32_t)ring_bytes(WARPS, R, C);   // int16 X, lane order
     const uint32_t rec = xs + (uint32_t)(M * a.K * 2);                  // {-8 sum X, scale}
+    float* park = reinterpret_cast<float*>(smem + ring_bytes(WARPS, R, C) + (size_t)M * a.K * 2 +
+                                           (size_t)M * a.KB * 32);      // [WARPS][2][M][32]
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gw = blockIdx.x * WARPS + warp;
@@ -429,11 +511,17 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
     // the dependency wait.
     if (lane == 0)
         for (int ch = 0; ch < R && ch < ring.nch; ++ch) ring.issue(ch);
+    cons.init(a, gw, xs, rec, park + (size_t)warp * 2 * M * 32);
     pdl_launch_dependents();
     pdl_wait();
 
-    stage_activations<M, WARPS * 32>(a, xs, rec, red);
-    cons.init(a, gw, xs, rec);
+    {
+        constexpr int NT = WARPS * 32;
+        const int nq = M * a.K / 8;
+        if (nq <= 2 * NT) stage_activations<M, NT, false, 2>(a, xs, rec, red);
+        else if (nq <= 5 * NT) stage_activations<M, NT, false, 5>(a, xs, rec, red);
+        else stage_activations<M, NT, false, kXChunksPerThread>(a, xs, rec, red);
+    }
 
     for (int ch = 0; ch < ring.nch; ++ch) {
         if (!ring.wait(ch)) set_device_error(a.err, kDevTimeout);   // data then unreliable
@@ -449,7 +537,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
         fence_proxy_async_smem();
         if (lane == 0 && ch + R < ring.nch) ring.issue(ch + R);
     }
-    cons.finish(a);
+    cons.flush_last(a);
+    __syncthreads();
+    int xt[2], xcf[2], xcl[2];
+    cons.template combine_cta<WARPS>(a, park, a.ws, xt, xcf, xcl);
+    if (xt[0] >= 0) combine_ctas_arrive<M, WARPS>(a, xt[0], xcf[0], xcl[0]);
+    if (xt[1] >= 0) combine_ctas_arrive<M, WARPS>(a, xt[1], xcf[1], xcl[1]);
 }
 
 // Final renorm of the decode step: out = renorm(in[0:len)), with the same
@@ -485,7 +578,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) renorm_kernel(const __half* in,
     float s = 0.f;
 #pragma unroll
     for (int w = 0; w < WARPS; ++w) s += red[w];
-    const float scale = (s > 0.f) ? __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(s, (float)len))) : 0.f;
+    const float scale = renorm_scale(s, len);
 #pragma unroll
     for (int i = 0; i < kXChunksPerThread; ++i) {
         const int q = tid + NT * i;

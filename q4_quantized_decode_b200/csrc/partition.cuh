@@ -96,6 +96,48 @@ struct WarpSplit {
     __host__ __device__ __forceinline__ int slot(int t) const { return t == t_first ? 0 : 1; }
 };
 
+// Two-level combine of split tiles, CTAs of `warps` consecutive warps.
+//
+// Level 1 (inside a CTA): every warp parks its partial of a split tile in
+// its slot sp.slot(t); of each split tile the CTA's first contributing warp
+// sums the parked partials of the CTA's contributors.  Warp gw is that warp
+// for end e of its run (0: t_first, 1: t_last) when:
+__host__ __device__ __forceinline__ bool cta_combiner(const WarpSplit& sp, int e, int gw,
+                                                      int cta_lo) {
+    if (e == 0) return sp.gf0 != sp.gl0 && (sp.gf0 == gw || gw == cta_lo);
+    return sp.t_last != sp.t_first && sp.gf1 != sp.gl1;
+}
+// ... and the parked slot it reads of contributor w (gw <= w) for tile t:
+// only its own run may end in t; every later warp's run starts in t.
+__host__ __device__ __forceinline__ int park_slot_read(const WarpSplit& sp, int gw, int w, int t) {
+    return (w == gw && t != sp.t_first) ? 1 : 0;
+}
+// Level 2 (tiles shared by CTAs): CTA c leaves its partial in slot
+// cta_slot_write(c) = 0 if its run starts in t, else 1; the reader finds it
+// from the tile's first contributing CTA cf alone.
+__host__ __device__ __forceinline__ int cta_slot_write(int c, int t, int KB, const SplitConsts& k,
+                                                       int warps) {
+    return seg_begin(c * warps, k) >= t * KB ? 0 : 1;
+}
+__host__ __device__ __forceinline__ int cta_slot_read(int c, int cf, int t, int KB,
+                                                      const SplitConsts& k, int warps) {
+    return (c == cf && seg_begin(c * warps, k) < t * KB) ? 1 : 0;
+}
+
+// Tiles shared by CTAs, enumerated by CTA boundary: boundary b (1 <= b <
+// CTAs owning segments) names the tile its CTA's run starts in when that run
+// starts strictly inside the tile and CTA b-1's run starts at or before the
+// tile's start (b is the tile's first interior boundary); else -1.  Every
+// tile shared by CTAs is named by exactly one boundary.
+__host__ __device__ __forceinline__ int shared_tile_of_boundary(int b, int KB, const SplitConsts& k,
+                                                                int warps) {
+    const int sb = seg_begin(b * warps, k);
+    const int t = sb / KB;
+    if (sb == t * KB) return -1;
+    if (seg_begin((b - 1) * warps, k) > t * KB) return -1;
+    return t;
+}
+
 // Walks seg_begin(g) for g = g_start, g_start + 1, ... with additions only.
 struct SegWalker {
     int sb, r, Q, Rm, G;

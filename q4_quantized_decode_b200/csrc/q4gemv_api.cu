@@ -541,7 +541,7 @@ void build_descriptors(q4gemv_ctx* h, const StackKey& k, std::vector<q4::StackGe
         d.N = (int)n_of[t];
         d.K = (int)k_of[t];
         d.renorm = i == 0 ? 0 : 1;
-        d.pad = 0;
+        d.fill_y = k.trace_y ? 1 : 0;
         const int S = (int)((n_of[t] + 31) / 32 * (k_of[t] / 32));
         const int gmax = h->sms * kWarps;
         d.sc = q4::make_split(S, gmax < S ? gmax : S);
@@ -560,13 +560,14 @@ int enqueue_stack_persistent(q4gemv_ctx* h, const StackKey& k, cudaStream_t st) 
     sa.x_out = static_cast<__half*>(k.x_out);
     sa.hidden = (int)k.hidden;
     sa.ws = h->ws;
+    sa.ws_half = h->sms * 2 * 32;   // [CTAs][2][32] per GEMV parity (ws holds sms * 16 warps * 1 KB)
     sa.cnt = h->cnt;
     sa.err = h->err;
     sa.sync = h->sync;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(h->sms);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = q4::ring_bytes(kWarps, kR1, kC1) + (size_t)kmax * 3;
+    cfg.dynamicSmemBytes = q4::stack_smem_bytes((int)kmax, kWarps, kR1, kC1);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
@@ -638,7 +639,7 @@ int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64
 
     const int64_t kmax_step = hidden > ffn ? hidden : ffn;
     if (h->stack_mode == kStackPersistent && kmax_step <= (int64_t)q4::kStackXChunks * 8 * kThreads &&
-        q4::ring_bytes(kWarps, kR1, kC1) + (size_t)kmax_step * 3 <= kMaxDynSmem) {
+        q4::stack_smem_bytes((int)kmax_step, kWarps, kR1, kC1) <= kMaxDynSmem) {
         if (!h->desc_valid || !(h->desc_key == k)) {
             if (cs != cudaStreamCaptureStatusNone)
                 return fail(h, Q4_EUNSUPPORTED,

@@ -25,7 +25,7 @@ struct StackGemv {
     __half* trace_x;      // nullable: the input vector used
     int N, K;
     int renorm;           // 1: input = renorm(previous output[0:K]); 0: input = x_in
-    int pad;
+    int fill_y;           // 1: also write y of tiles shared by CTAs (y is traced)
     SplitConsts sc;       // split of its segments over the grid's warps
 };
 
@@ -35,17 +35,105 @@ struct StackArgs {
     const __half* x_in;   // input of GEMV 0
     __half* x_out;        // renorm(last output[0:hidden])
     int hidden;
-    float* ws;            // split-tile partials (as q4gemv_run)
-    int* cnt;             // per-tile arrival counters
+    float* ws;            // CTA partials, two GEMV-parity halves of [CTAs][2][32]
+    int ws_half;          // floats per half
+    int* cnt;             // unused (tiles shared by CTAs are combined by the next reader)
     int* err;             // device error word
     int* sync;            // [0] grid arrivals, [1] abort flag; zero at launch
+};
+
+// Outputs of the previous GEMV in tiles shared by several CTAs exist only as
+// per-CTA partials until they are read: every reader sums them in CTA order
+// (the same sum q4gemv_run's kernel takes) and rounds to f16.  prepare()
+// combines, with all threads of the CTA, the shared tiles' 8-element chunks
+// that fall in the staged range into `patch` (shared memory, 16 bytes per
+// chunk), so their loads overlap those of the rest of the vector; apply()
+// then takes chunk q from the patch when its tile is shared.  ws == nullptr:
+// no-op.  A traced step also completes y (fill_y) for those tiles: boundary
+// b's tile is written by CTA b, or every one by the calling CTA (fill_all).
+template <int WARPS>
+struct SplitFix {
+    static constexpr bool kActive = true;
+    const float* ws;      // the previous GEMV's CTA partials [CTAs][2][32]
+    SplitConsts sc;       // its split
+    int KB;               // its blocks per row
+    __half* fill_y;       // nullable: its output, to complete
+    int fill_n;           // its rows
+    bool fill_all;
+
+    // The combined chunk u (rows 8u..8u+7) of shared tile t, whose first
+    // contributing CTA is cf; two contributors are loaded together (the
+    // usual case), any further ones after them; the sum runs from +0.
+    __device__ __forceinline__ uint4 combine(int t, int cf, int u) const {
+        const int cl = warp_of_seg(t * KB + KB - 1, sc) / WARPS;
+        const float4* p0 = reinterpret_cast<const float4*>(
+            ws + ((size_t)cf * 2 + cta_slot_read(cf, cf, t, KB, sc, WARPS)) * 32 + u * 8);
+        const float4* p1 = reinterpret_cast<const float4*>(ws + ((size_t)(cf + 1) * 2) * 32 + u * 8);
+        const float4 a0 = __ldcg(p0), a1 = __ldcg(p0 + 1), b0 = __ldcg(p1), b1 = __ldcg(p1 + 1);
+        float s[8] = {0.f + a0.x, 0.f + a0.y, 0.f + a0.z, 0.f + a0.w,
+                      0.f + a1.x, 0.f + a1.y, 0.f + a1.z, 0.f + a1.w};
+        s[0] += b0.x; s[1] += b0.y; s[2] += b0.z; s[3] += b0.w;
+        s[4] += b1.x; s[5] += b1.y; s[6] += b1.z; s[7] += b1.w;
+        for (int c = cf + 2; c <= cl; ++c) {
+            const float4* pc = reinterpret_cast<const float4*>(ws + ((size_t)c * 2) * 32 + u * 8);
+            const float4 c0 = __ldcg(pc), c1 = __ldcg(pc + 1);
+            s[0] += c0.x; s[1] += c0.y; s[2] += c0.z; s[3] += c0.w;
+            s[4] += c1.x; s[5] += c1.y; s[6] += c1.z; s[7] += c1.w;
+        }
+        uint4 o;
+        __half2* h = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) h[e] = __floats2half2_rn(s[2 * e], s[2 * e + 1]);
+        return o;
+    }
+
+    template <int NT>
+    __device__ __forceinline__ void prepare(int nq, uint32_t patch) const {
+        if (ws == nullptr) return;
+        const int nb = (sc.G + WARPS - 1) / WARPS;      // CTAs owning segments
+        const int total = (nb - 1) * 4;                 // (boundary, chunk) pairs
+        for (int p0 = threadIdx.x; p0 < total; p0 += 2 * NT) {
+            // Two pairs per thread per round, so their loads overlap.
+            int tt[2], qq[2];
+            bool fl[2];
+            uint4 v[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int p = p0 + k * NT;
+                const int b = (p >> 2) + 1;
+                tt[k] = p < total ? shared_tile_of_boundary(b, KB, sc, WARPS) : -1;
+                qq[k] = tt[k] * 4 + (p & 3);
+                fl[k] = fill_y != nullptr && (fill_all || b == (int)blockIdx.x);
+                if (tt[k] >= 0 && (qq[k] < nq || fl[k])) v[k] = combine(tt[k], b - 1, p & 3);
+                else tt[k] = -1;
+            }
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                if (tt[k] < 0) continue;
+                if (qq[k] < nq) sts128(patch + (uint32_t)qq[k] * 16, v[k]);
+                if (fl[k]) {
+                    const __half* h = reinterpret_cast<const __half*>(&v[k]);
+                    for (int e = 0; e < 8; ++e)
+                        if (qq[k] * 8 + e < fill_n) fill_y[(size_t)qq[k] * 8 + e] = h[e];
+                }
+            }
+        }
+    }
+
+    __device__ __forceinline__ uint4 apply(int q, uint4 v, uint32_t patch) const {
+        if (ws == nullptr) return v;
+        const int t = q >> 2;
+        const int cf = warp_of_seg(t * KB, sc) / WARPS, cl = warp_of_seg(t * KB + KB - 1, sc) / WARPS;
+        return cf == cl ? v : lds128(patch + (uint32_t)q * 16);
+    }
 };
 
 // Unit-RMS renorm of in[0:len) into out, same arithmetic and order as the
 // renorm fused into the GEMV prologue (coherent loads: `in` may have been
 // written by other CTAs of the running kernel).  All NT threads of one CTA.
-template <int NT, bool kCoherent, int QN>
-__device__ __forceinline__ void renorm_block(const __half* in, __half* out, int len, float* red) {
+template <int NT, bool kCoherent, int QN, class Fix>
+__device__ __forceinline__ void renorm_block(const __half* in, __half* out, int len, float* red,
+                                             const Fix& fix, uint32_t patch) {
     const int tid = threadIdx.x, lane = tid & 31;
     const int nq = len / 8;
     uint4 xr[QN];
@@ -54,6 +142,13 @@ __device__ __forceinline__ void renorm_block(const __half* in, __half* out, int 
         const int q = tid + NT * i;
         const uint4* src = reinterpret_cast<const uint4*>(in + (size_t)q * 8);
         xr[i] = q < nq ? (kCoherent ? __ldcg(src) : *src) : make_uint4(0, 0, 0, 0);
+    }
+    fix.template prepare<NT>(nq, patch);
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < QN; ++i) {
+        const int q = tid + NT * i;
+        if (q < nq) xr[i] = fix.apply(q, xr[i], patch);
     }
     float part = 0.f;
 #pragma unroll
@@ -73,7 +168,7 @@ __device__ __forceinline__ void renorm_block(const __half* in, __half* out, int 
     float s = 0.f;
 #pragma unroll
     for (int w = 0; w < NT / 32; ++w) s += red[w];
-    const float scale = (s > 0.f) ? __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(s, (float)len))) : 0.f;
+    const float scale = renorm_scale(s, len);
 #pragma unroll
     for (int i = 0; i < QN; ++i) {
         const int q = tid + NT * i;
@@ -112,65 +207,82 @@ __device__ __forceinline__ GemvArgs stack_view(const StackArgs& sa, int i) {
 // Activation chunks per thread in the persistent step: K <= 5 * 8 * threads.
 constexpr int kStackXChunks = 5;
 
-// Issues a warp's chunks (C segments, one bulk copy each) GEMV after GEMV,
-// at most R ahead of consumption.  Every lane tracks the state; lane 0 issues.
-// The descriptor of the GEMV after the current one is loaded a whole GEMV
-// ahead, so advancing never waits on memory.
-template <int R, int C>
-struct StreamProducer {
-    int gi;               // GEMV being issued
-    int ch, nch, nseg;    // chunk within it, chunk count, segment count
-    const uint8_t* src;   // first segment of this warp's run in GEMV gi
-    int issued;           // chunks issued so far (all GEMVs)
-    const uint8_t* nW;    // GEMV gi + 1: matrix and split (prefetched)
-    SplitConsts nsc;
+// Shared memory of the persistent step for inputs of up to kmax elements:
+// ring, int16 activations (2 bytes each), block records (1 byte per
+// element), one tile partial pair per warp.
+__host__ __device__ constexpr size_t stack_smem_bytes(int kmax, int warps, int R, int C) {
+    return ring_bytes(warps, R, C) + (size_t)kmax * 3 + warp_partial_bytes(1, warps);
+}
 
-    __device__ __forceinline__ void load_next(const StackArgs& sa) {
-        if (gi + 1 < sa.n_gemv) {
-            const StackGemv* d = sa.gemv + gi + 1;
-            nW = d->W;
-            nsc = d->sc;
-        }
-    }
-    // Position on GEMV gi or, if this warp owns nothing there, on the next
-    // GEMV where it does.
-    __device__ __forceinline__ void enter(const StackArgs& sa, int gw, const uint8_t* W,
-                                          SplitConsts k) {
-        while (true) {
-            if (gw < k.G) {
-                const int s0 = seg_begin(gw, k), s1 = seg_begin(gw + 1, k);
-                nseg = s1 - s0;
-                nch = (nseg + C - 1) / C;
-                src = W + (size_t)s0 * kSegBytes;
-                ch = 0;
-                load_next(sa);
-                return;
-            }
-            if (++gi >= sa.n_gemv) return;
+// A warp's position in its stream of chunks (C segments each) across the
+// GEMVs of the step: chunk ch of its run in GEMV gi.  Descriptors are read
+// through L1 (they are prefetched there at kernel start).
+template <int C>
+struct StreamCursor {
+    int gi;               // GEMV (n_gemv: past the end)
+    int ch, nch, nseg;    // chunk of the run, chunks, segments
+    const uint8_t* src;   // first segment of the run
+
+    // Position on chunk 0 of GEMV gi or, if warp gw owns nothing there, of
+    // the next GEMV where it does.
+    __device__ __forceinline__ void enter(const StackArgs& sa, int gw) {
+        for (; gi < sa.n_gemv; ++gi) {
             const StackGemv* d = sa.gemv + gi;
-            W = d->W;
-            k = d->sc;
+            SplitConsts k;
+            k.G = __ldg(&d->sc.G);
+            if (gw >= k.G) continue;
+            k.Q = __ldg(&d->sc.Q);
+            k.Rm = __ldg(&d->sc.Rm);
+            k.MG = __ldg(reinterpret_cast<const unsigned long long*>(&d->sc.MG));
+            const uint8_t* W = reinterpret_cast<const uint8_t*>(
+                __ldg(reinterpret_cast<const unsigned long long*>(&d->W)));
+            const int s0 = seg_begin(gw, k), s1 = seg_begin(gw + 1, k);
+            nseg = s1 - s0;
+            nch = (nseg + C - 1) / C;
+            src = W + (size_t)s0 * kSegBytes;
+            ch = 0;
+            return;
         }
     }
     __device__ __forceinline__ void start(const StackArgs& sa, int gw) {
         gi = 0;
+        enter(sa, gw);
+    }
+    __device__ __forceinline__ bool valid(const StackArgs& sa) const { return gi < sa.n_gemv; }
+    __device__ __forceinline__ const uint8_t* addr() const { return src + (size_t)ch * C * kSegBytes; }
+    __device__ __forceinline__ uint32_t bytes() const {
+        return (uint32_t)min(C, nseg - ch * C) * kSegBytes;
+    }
+    __device__ __forceinline__ void advance(const StackArgs& sa, int gw) {
+        if (++ch == nch) {
+            ++gi;
+            enter(sa, gw);
+        }
+    }
+};
+
+// Issues a warp's chunks into its ring of R stages, GEMV after GEMV, at most
+// R ahead of consumption.  Every lane tracks the state; lane 0 issues.
+template <int R, int C>
+struct StreamProducer {
+    StreamCursor<C> cur;
+    int issued;           // chunks issued into the ring so far (all GEMVs)
+
+    __device__ __forceinline__ void start(const StackArgs& sa, int gw) {
+        cur.start(sa, gw);
         issued = 0;
-        enter(sa, gw, sa.gemv[0].W, sa.gemv[0].sc);
     }
     __device__ __forceinline__ void fill(const StackArgs& sa, int gw, int consumed, uint32_t stage0,
                                          uint64_t* bars, int lane) {
-        while (gi < sa.n_gemv && issued - consumed < R) {
+        while (cur.valid(sa) && issued - consumed < R) {
             const int k = issued % R;
-            const uint32_t bytes = (uint32_t)min(C, nseg - ch * C) * kSegBytes;
             if (lane == 0) {
+                const uint32_t bytes = cur.bytes();
                 mbar_arrive_expect_tx(bars + k, bytes);
-                bulk_g2s_addr(stage0 + (uint32_t)k * C * kSegBytes, src + (size_t)ch * C * kSegBytes,
-                              bytes, bars + k);
+                bulk_g2s_addr(stage0 + (uint32_t)k * C * kSegBytes, cur.addr(), bytes, bars + k);
             }
             ++issued;
-            if (++ch == nch) {
-                if (++gi < sa.n_gemv) enter(sa, gw, nW, nsc);
-            }
+            cur.advance(sa, gw);
         }
     }
 };
@@ -211,6 +323,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa
     const uint32_t stage0_base = smem_base;
     const uint32_t xs = smem_base + (uint32_t)ring_bytes(WARPS, R, C);
     const uint32_t rec = xs + (uint32_t)kmax * 2;
+    float* park = reinterpret_cast<float*>(smem + ring_bytes(WARPS, R, C) + (size_t)kmax * 3);
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gw = blockIdx.x * WARPS + warp;
@@ -221,6 +334,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa
         for (int k = 0; k < R; ++k) mbar_init(wbars + k, 1);
         fence_barrier_init();
     }
+    // The descriptors are read again and again by the cursors: pull them into
+    // L1 once.
+    for (int off = threadIdx.x * 128; off < sa.n_gemv * (int)sizeof(StackGemv); off += NT * 128)
+        prefetch_l1(reinterpret_cast<const uint8_t*>(sa.gemv) + off);
     __syncwarp();
 
     StreamProducer<R, C> prod;
@@ -230,12 +347,27 @@ __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa
 
     bool ok = true;
     for (int i = 0; i < sa.n_gemv && ok; ++i) {
-        const GemvArgs a = stack_view(sa, i);
+        GemvArgs a = stack_view(sa, i);
+        a.ws = sa.ws + (size_t)(i & 1) * sa.ws_half;
+        SplitFix<WARPS> fix;
+        fix.ws = nullptr;
+        if (i > 0) {
+            const StackGemv& pd = sa.gemv[i - 1];
+            fix.ws = sa.ws + (size_t)((i - 1) & 1) * sa.ws_half;
+            fix.sc = pd.sc;
+            fix.KB = pd.K / 32;
+            fix.fill_y = pd.fill_y ? pd.y : nullptr;
+            fix.fill_n = pd.N;
+            fix.fill_all = false;
+        }
+        // The warp's share of GEMV i depends on no data: set it up before the
+        // barrier.
+        Dp2aConsumer<1> cons;
+        cons.init(a, gw, xs, rec, park + (size_t)warp * 2 * 32);
         if (i > 0) ok = grid_wait(sa.sync, i * (int)gridDim.x, sa.err, &flag);
         if (!ok) break;
-        stage_activations<1, NT, true, kStackXChunks>(a, xs, rec, red);
-        Dp2aConsumer<1> cons;
-        cons.init(a, gw, xs, rec);
+        if (a.K <= 2 * NT * 8) stage_activations<1, NT, true, 2>(a, xs, rec, red, fix);
+        else stage_activations<1, NT, true, kStackXChunks>(a, xs, rec, red, fix);
         const int nseg = cons.sp.s1 - cons.sp.s0;
         for (int j = 0; j < nseg; j += C) {
             const int k = consumed % R;
@@ -253,15 +385,26 @@ __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa
             fence_proxy_async_smem();
             prod.fill(sa, gw, consumed, stage0, wbars, lane);
         }
-        cons.finish(a);
-        // This CTA is done with GEMV i (outputs and partial combines written).
+        cons.flush_last(a);
+        __syncthreads();
+        int xt[2], xcf[2], xcl[2];   // tiles shared with other CTAs: combined by their readers
+        cons.template combine_cta<WARPS>(a, park, a.ws, xt, xcf, xcl);
+        // This CTA is done with GEMV i (outputs and CTA partials written).
         __syncthreads();
         if (threadIdx.x == 0) red_add_release_gpu(sa.sync, 1);
     }
     if (ok) ok = grid_wait(sa.sync, sa.n_gemv * (int)gridDim.x, sa.err, &flag);
     if (ok) {
-        if (blockIdx.x == 0)
-            renorm_block<NT, true, kStackXChunks>(sa.gemv[sa.n_gemv - 1].y, sa.x_out, sa.hidden, red);
+        const int il = sa.n_gemv - 1;
+        const StackGemv& ld = sa.gemv[il];
+        SplitFix<WARPS> fix;
+        fix.ws = sa.ws + (size_t)(il & 1) * sa.ws_half;
+        fix.sc = ld.sc;
+        fix.KB = ld.K / 32;
+        fix.fill_y = ld.fill_y ? ld.y : nullptr;
+        fix.fill_n = ld.N;
+        fix.fill_all = true;
+        if (blockIdx.x == 0) renorm_block<NT, true, kStackXChunks>(ld.y, sa.x_out, sa.hidden, red, fix, xs);
         return;
     }
     // Abort: let this warp's copies in flight land (bounded) before leaving.

@@ -22,6 +22,12 @@ def probe(tmp_path_factory):
     for f in ("probe_seg_begin", "probe_warp_of_seg"):
         getattr(lib, f).argtypes = [ctypes.c_int] * 3
     lib.probe_walk.argtypes = [ctypes.c_int] * 4
+    lib.probe_warp_split.argtypes = [ctypes.c_int] * 4 + [ctypes.POINTER(ctypes.c_int)]
+    lib.probe_cta_combiner.argtypes = [ctypes.c_int] * 6
+    lib.probe_park_slot_read.argtypes = [ctypes.c_int] * 6
+    lib.probe_cta_slot_write.argtypes = [ctypes.c_int] * 6
+    lib.probe_cta_slot_read.argtypes = [ctypes.c_int] * 7
+    lib.probe_shared_tile_of_boundary.argtypes = [ctypes.c_int] * 5
     lib.probe_xperm_pos.argtypes = [ctypes.c_int]
     return lib
 
@@ -105,3 +111,80 @@ def test_xperm_is_a_permutation_grouping_lane_words(probe):
     for c in range(4):
         group = {pos[j] for j in list(range(4 * c, 4 * c + 4)) + list(range(16 + 4 * c, 20 + 4 * c))}
         assert group == set(range(8 * c, 8 * c + 8))
+
+
+def _split(probe, gw, S, G, KB):
+    out = (ctypes.c_int * 8)()
+    probe.probe_warp_split(gw, S, G, KB, out)
+    return list(out)
+
+
+@pytest.mark.parametrize("S,G,KB", [(25600, 2368, 160), (35840, 2368, 160), (174080, 2368, 160),
+                                    (87040, 2368, 544), (12, 12, 3), (99, 50, 9), (994, 37, 7), (1001, 40, 7), (7 * 130, 148 * 16 // 3, 7),
+                                    (5000, 333, 1), (160, 160, 160), (64, 64, 64), (165, 165, 5),
+                                    (4096, 2368, 4096), (300, 150, 30), (2368 * 3, 2368, 2)])
+def test_two_level_combine_bookkeeping(probe, S, G, KB):
+    """Simulates the two-level combine of the M <= 2 kernel and of the
+    persistent step with the kernel's own decision functions: every parked
+    partial that is read was parked for that tile, every split tile is
+    combined once per contributing CTA, CTA partial slots never collide and
+    the reader finds them, and each tile shared by CTAs has exactly one
+    writer of its output in a traced step."""
+    W = 16
+    T = S // KB
+    sp = {gw: _split(probe, gw, S, G, KB) for gw in range(G)}
+    parked = {}
+    for gw, (s0, s1, tf, tl, gf0, gl0, gf1, gl1) in sp.items():
+        assert s1 > s0
+        for t, gf, gl in ((tf, gf0, gl0), (tl, gf1, gl1)):
+            if gf != gl:
+                parked[(gw, 0 if t == tf else 1)] = t
+    combined, y_written, cta_parked = {}, [0] * T, {}
+    for gw, (s0, s1, tf, tl, gf0, gl0, gf1, gl1) in sp.items():
+        b, cta_lo = gw // W, gw // W * W
+        for e, (t, gf, gl) in enumerate(((tf, gf0, gl0), (tl, gf1, gl1))):
+            if not probe.probe_cta_combiner(gw, e, S, G, KB, W):
+                continue
+            assert gw == max(gf, cta_lo)                 # the CTA's first contributor
+            w_to = min(gl, cta_lo + W - 1)
+            for w in range(gw, w_to + 1):
+                sl = probe.probe_park_slot_read(gw, w, t, S, G, KB)
+                assert parked.get((w, sl)) == t
+            assert (b, t) not in combined
+            combined[(b, t)] = 1
+            if gf >= cta_lo and gl <= cta_lo + W - 1:
+                y_written[t] += 1
+            else:
+                slc = probe.probe_cta_slot_write(b, t, KB, S, G, W)
+                assert (b, slc) not in cta_parked
+                cta_parked[(b, slc)] = t
+    for t in range(T):
+        gf = probe.probe_warp_of_seg(t * KB, S, G)
+        gl = probe.probe_warp_of_seg(t * KB + KB - 1, S, G)
+        if gf == gl:
+            assert y_written[t] == 0                      # written by its warp's flush
+            continue
+        cf, cl = gf // W, gl // W
+        for c in range(cf, cl + 1):
+            assert combined.get((c, t)) == 1
+        if cf == cl:
+            assert y_written[t] == 1
+            continue
+        assert y_written[t] == 0
+        for c in range(cf, cl + 1):
+            sl = probe.probe_cta_slot_read(c, cf, t, KB, S, G, W)
+            assert cta_parked.get((c, sl)) == t
+    # The persistent step's readers enumerate the shared tiles by CTA
+    # boundary: each shared tile exactly once, named with its first CTA b-1.
+    nb = (G + W - 1) // W
+    named = {}
+    for b in range(1, nb):
+        t = probe.probe_shared_tile_of_boundary(b, KB, S, G, W)
+        if t >= 0:
+            assert t not in named
+            named[t] = b
+    shared = {t for t in range(T)
+              if probe.probe_warp_of_seg(t * KB, S, G) // W != probe.probe_warp_of_seg(t * KB + KB - 1, S, G) // W}
+    assert set(named) == shared
+    for t, b in named.items():
+        assert probe.probe_warp_of_seg(t * KB, S, G) // W == b - 1
