@@ -51,6 +51,8 @@ def _configure(lib):
     lib.oracle_repack.restype = None
     lib.oracle_renorm.argtypes = [vp, i64, vp]
     lib.oracle_renorm.restype = None
+    lib.oracle_unit_rms_scale.argtypes = [vp, i64]
+    lib.oracle_unit_rms_scale.restype = ctypes.c_double
     lib.oracle_round_f16.argtypes = [vp, i64, vp]
     lib.oracle_round_f16.restype = None
     return lib
@@ -140,10 +142,17 @@ def repack(gguf: np.ndarray, N: int, K: int) -> np.ndarray:
 
 
 def renorm(v: np.ndarray) -> np.ndarray:
+    """f16(v * unit_rms_scale(v)): the step's final output vector."""
     v = np.ascontiguousarray(v, dtype=np.uint16)
     out = np.empty_like(v)
     _load().oracle_renorm(v.ctypes.data, v.size, out.ctypes.data)
     return out
+
+
+def unit_rms_scale(v: np.ndarray) -> float:
+    """1 / sqrt(mean(v^2)) of an f16 vector in fp64 (0 for an all-zero one)."""
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    return float(_load().oracle_unit_rms_scale(v.ctypes.data, v.size))
 
 
 def stack_step(get_rows, x_in: np.ndarray, n_layers: int, hidden: int,
@@ -151,25 +160,31 @@ def stack_step(get_rows, x_in: np.ndarray, n_layers: int, hidden: int,
     """The renormalised 64-layer-style chain of GEMVs (one decode step, M=1).
 
     Layer l, with matrices QKV (qkv_n x hidden), O (hidden x hidden),
-    gate+up (2*ffn x hidden), down (hidden x ffn):
-        a = renorm(f16(QKV x)[0:hidden])
-        b = renorm(f16(O a))
-        u = renorm(f16(gate_up b)[0:ffn])
-        x = renorm(f16(down u))
-    Each GEMV output is rounded to f16 (the boundary's vector type) before the
-    renorm.  ``get_rows(l, t)`` returns the GGUF bytes of matrix t (0 QKV,
-    1 O, 2 gate+up, 3 down) of layer l.  ``record(i, x_f16, y_f64)`` is
-    called for each GEMV i = 4l + t when given.  Returns the final f16 x.
+    gate+up (2*ffn x hidden), down (hidden x ffn), each GEMV output rounded
+    to f16 (the boundary's vector type) and each next input taken as that
+    f16 vector (its first K entries) scaled to unit RMS by a real scalar:
+        a = f16(QKV x);           b = f16(O (s(a') a'))       a' = a[0:hidden]
+        u = f16(gate_up (s(b) b)); x' = f16(down (s(u') u'))  u' = u[0:ffn]
+    with s(v) = 1/sqrt(mean(v^2)) (0 for v = 0); by linearity each output
+    is f16(s * (W v)), computed here in fp64.  The step returns the next
+    layer's input as an f16 vector, f16(s(x') x').  ``get_rows(l, t)``
+    returns the GGUF bytes of matrix t (0 QKV, 1 O, 2 gate+up, 3 down) of
+    layer l.  ``record(i, x_f16, s, y_f64)`` is called for each GEMV
+    i = 4l + t when given (x_f16: the unscaled input, s its scale, y_f64 the
+    output before rounding).
     """
     dims = [(qkv_n, hidden), (hidden, hidden), (2 * ffn, hidden), (hidden, ffn)]
     x = np.ascontiguousarray(x_in, dtype=np.uint16)
+    s = 1.0
     for l in range(n_layers):
         for t, (N, K) in enumerate(dims):
             assert x.size == K
-            y = q4_gemv(get_rows(l, t), K, x.reshape(1, K), threads=threads)[0]
+            with np.errstate(invalid="ignore"):          # 0 * inf of a non-finite row is NaN
+                y = s * q4_gemv(get_rows(l, t), K, x.reshape(1, K), threads=threads)[0]
             if record is not None:
-                record(4 * l + t, x, y)
+                record(4 * l + t, x, s, y)
             yh = f64_to_f16(y)
             keep = {0: hidden, 1: hidden, 2: ffn, 3: hidden}[t]
-            x = renorm(yh[:keep])
-    return x
+            x = np.ascontiguousarray(yh[:keep])
+            s = unit_rms_scale(x)
+    return renorm(x)

@@ -126,19 +126,22 @@ void oracle_repack(const uint8_t* gguf, int64_t N, int64_t K, uint8_t* packed) {
     }
 }
 
-/* Renormalise an f16 vector to unit RMS: s = sum v_i^2 (fp64), out_i =
- * f16(v_i / sqrt(s / len)); all-zero input gives all-zero output. */
-void oracle_renorm(const uint16_t* v, int64_t len, uint16_t* out) {
+/* Unit-RMS scale of an f16 vector: s = sum v_i^2 (fp64), 1 / sqrt(s / len);
+ * 0 for an all-zero vector (which then stays zero). */
+double oracle_unit_rms_scale(const uint16_t* v, int64_t len) {
     double s = 0.0;
     for (int64_t i = 0; i < len; ++i) {
         const double a = oracle_f16_to_f64(v[i]);
         s += a * a;
     }
-    if (s == 0.0) {
-        for (int64_t i = 0; i < len; ++i) out[i] = 0;
-        return;
-    }
-    const double scale = 1.0 / sqrt(s / (double)len);
+    if (s == 0.0) return 0.0;
+    return 1.0 / sqrt(s / (double)len);
+}
+
+/* Renormalise an f16 vector to unit RMS as an f16 vector: out_i =
+ * f16(v_i * scale). */
+void oracle_renorm(const uint16_t* v, int64_t len, uint16_t* out) {
+    const double scale = oracle_unit_rms_scale(v, len);
     for (int64_t i = 0; i < len; ++i)
         out[i] = oracle_f64_to_f16(oracle_f16_to_f64(v[i]) * scale);
 }

@@ -284,6 +284,43 @@ def test_renorm_invariants():
     assert np.array_equal(oracle.renorm(v ^ 0x8000), r ^ 0x8000)
 
 
+def test_unit_rms_scale_invariants():
+    v = synth.normal_f16(2, synth.act_id(0), 4096)
+    s = oracle.unit_rms_scale(v)
+    # power-of-two scaling of the input divides the scale exactly
+    assert oracle.unit_rms_scale(f16_bits(f16_values(v) * 8.0)) == s / 8.0
+    # constant vectors: 1/|c|; zero: 0; sign-blind
+    assert oracle.unit_rms_scale(f16_bits(np.full(37, -0.75))) == 1.0 / 0.75
+    assert oracle.unit_rms_scale(np.zeros(9, dtype=np.uint16)) == 0.0
+    assert oracle.unit_rms_scale(v ^ 0x8000) == s
+    # renorm is the scaled vector rounded once
+    assert np.array_equal(oracle.renorm(v), oracle.f64_to_f16(f16_values(v) * s))
+
+
+def test_stack_scales_inputs_without_rounding():
+    """One layer whose O matrix selects entry p[n] of its input with weight
+    +-3/64: b[n] = f16(s * (+-3/64 * a[p[n]])) with a = f16(QKV x) and s its
+    unit-RMS scale, rounded once (a second f16 rounding of s*a, before O,
+    would change some entries)."""
+    hidden, qkv_n, ffn = 64, 64, 64
+    qkv = synth.q4_0_matrix(77, synth.weight_id(0), qkv_n, hidden)
+    p_o = RNG.permutation(hidden); s_o = RNG.choice([-1, 1], hidden)
+    o = signed_selection(hidden, hidden, p_o, s_o, d_bits=0x2A00)     # d = 3/64
+    x = synth.normal_f16(77, synth.act_id(0), hidden)
+    seen = {}
+    oracle.stack_step(lambda l, t: {0: qkv, 1: o, 2: synth.q4_0_matrix(77, 3, 2 * ffn, hidden),
+                                    3: synth.q4_0_matrix(77, 4, hidden, ffn)}[t],
+                      x, 1, hidden, qkv_n, ffn, record=lambda i, xf, sc, y: seen.setdefault(i, (xf, sc, y)))
+    a = oracle.f64_to_f16(oracle.q4_gemv(qkv, hidden, x[None, :])[0])
+    s = oracle.unit_rms_scale(a)
+    xf, sc, y = seen[1]
+    assert np.array_equal(xf, a) and sc == s
+    want = oracle.f64_to_f16(s * (s_o * 0.046875 * f16_values(a)[p_o]))
+    assert np.array_equal(oracle.f64_to_f16(y), want)
+    twice = oracle.f64_to_f16(s_o * 0.046875 * f16_values(oracle.f64_to_f16(s * f16_values(a)))[p_o])
+    assert not np.array_equal(twice, want)
+
+
 def signed_selection(N, K, src, sign, junk_from=None, d_bits=0x2800):
     """Q4_0 rows with one nonzero per row: row n = sign[n] * 2^-5 * e_{src[n]}
     (code 9 -> +d, code 7 -> -d, d = 2^-5).  Rows >= junk_from get random
