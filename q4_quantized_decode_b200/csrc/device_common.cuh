@@ -160,6 +160,12 @@ __device__ __forceinline__ float renorm_scale(float s, int len) {
     return (s > 0.f) ? rsqrtf(__fdividef(s, (float)len)) : 0.f;
 }
 
+// Orders this thread's generic-proxy global accesses with async-proxy
+// (bulk copy) accesses to global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // One-line prefetch into L1.
 __device__ __forceinline__ void prefetch_l1(const void* p) {
     asm volatile("prefetch.global.L1 [%0];" ::"l"(p));

@@ -64,12 +64,19 @@ __host__ __device__ constexpr size_t warp_partial_bytes(int M, int warps) {
     return (size_t)warps * 2 * M * 32 * sizeof(float);
 }
 
+// Per-block sums of squares of an activation vector of K entries (fp32,
+// padded to 16 bytes).
+__host__ __device__ constexpr size_t tile_sum_bytes(int K) {
+    return ((size_t)(K / 32) * 4 + 15) / 16 * 16;
+}
+
 // Shared-memory footprint of the M <= 2 kernel: the ring, the int16
 // activations (2 bytes per element), per block and lane group the pair
-// {-8 * sum X, block scale} (8 bytes, 32 per block), then the warp partials.
+// {-8 * sum X, block scale} (8 bytes, 32 per block), the warp partials, then
+// the block sums of squares of vector 0.
 __host__ __device__ constexpr size_t gemv_dp2a_smem_bytes(int M, int K, int warps, int R, int C) {
     return ring_bytes(warps, R, C) + (size_t)M * K * 2 + (size_t)M * (K / 32) * 32 +
-           warp_partial_bytes(M, warps);
+           warp_partial_bytes(M, warps) + tile_sum_bytes(K);
 }
 
 // Position of element j of a 32-column block in the permuted X layout: the
@@ -110,81 +117,159 @@ struct WarpRing {
     }
 };
 
-// Activation staging for the M <= 2 kernel, all threads of the CTA.  Thread
-// t holds the 16-byte chunks q = t, t + NT, ... of x (8 elements each; four
-// chunks make a 32-column block, held by four consecutive lanes).  For M = 1
-// with `renorm`, the vector is first scaled to unit RMS: s = sum v^2 in fp32
-// (fixed order: per thread, then warp xor tree, then warps in order), each v
-// becomes f16(v * 1/sqrt(s/K)), an all-zero vector stays zero.  Each block is
-// then converted to X = rint(v * 2^(14-E)) (E: exponent of the block maximum,
-// so |X| <= 32752 and the maximum is exact) and written in lane order; lane
-// group c of the block gets {-8 * sum of its eight X, 2^(E-14)}.
-// kCoherent: load x through L2 only (it was written by other CTAs of the
-// same running kernel, so an L1 copy could be stale).
-// QN: 16-byte chunks held per thread (M * K <= QN * 8 * NT); all QN rounds
-// run (chunks past the end are zeros), so callers pick the smallest QN that
-// covers the vector: the rounds then overlap instead of running one by one.
-// Fix: completes the loaded input where it exists only as partial sums (the
-// persistent step); NoFix keeps what was loaded.  A Fix with kActive runs
-// prepare() with all threads (it may use the X area of shared memory as
-// scratch), then, after a CTA barrier, apply() per chunk.
-struct NoFix {
-    static constexpr bool kActive = false;
-    template <int NT>
-    __device__ __forceinline__ void prepare(int, uint32_t) const {}
-    __device__ __forceinline__ uint4 apply(int, uint4 v, uint32_t) const { return v; }
-};
+// ---- Activation blocks: exact int16 codes and sums of squares.
+//
+// A 32-entry block v of an f16 activation vector becomes X = rint(v *
+// 2^(14-E)) (E: exponent of the block maximum, so |X| <= 32752 and the
+// maximum is exact), stored in lane order (xperm_pos), and lane group c gets
+// the record {-8 * sum of its eight X, 2^(E-14)}.  X is read from the low
+// mantissa bits of v * 2^(14-E) + 1.5 * 2^23: the product is exact and
+// |X| < 2^22, so the one rounding of the addition is the round to the nearest
+// integer (ties to even) and the bits hold 0x4B400000 + X.  All-zero block:
+// X = 0, scale 0; non-finite block: scale NaN (its products are NaN whatever
+// X holds).
+//
+// The block's sum of squares (for the unit-RMS scale of the next input) is
+// taken in one fixed binary tree: squares rounded to fp32, then pairs of
+// entries whose indices differ in bit 0, then bit 1, ... bit 4, every sum
+// rounded to fp32 (no fused operations).  Two layouts compute the same tree:
+// a chunk layout (four lanes per block, lane u holding entries 8u..8u+7) and
+// a lane layout (one entry per lane, lane 4g + c holding entry g + 8c).
 
-template <int M, int NT, bool kCoherent = false, int QN = kXChunksPerThread, class Fix = NoFix>
+__device__ __forceinline__ void block_exponent(uint32_t mx, float& inv, float& sc) {
+    const int E = (int)(mx >> 23) - 127;                                   // max in [2^E, 2^(E+1))
+    const bool live = mx != 0u && mx < 0x7F800000u;
+    inv = live ? __uint_as_float((uint32_t)(141 - E) << 23) : 0.f;          // 2^(14-E)
+    sc = live ? __uint_as_float((uint32_t)(113 + E) << 23)                  // 2^(E-14)
+              : (mx == 0u ? 0.f : __uint_as_float(0x7FC00000u));
+}
+constexpr float kRoundMagic = 12582912.0f;    // 1.5 * 2^23
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;
+
+// Chunk layout: this lane holds entries 8u..8u+7 (u = lane & 3) of a block
+// in v[]; the four lanes of the block call together (all 32 lanes of the
+// warp execute it).  Outputs: the two 8-byte X words of the lane order
+// positions of its entries, the record sums h0 (group 2(u&1)) and h1 (group
+// 2(u&1)+1), the block scale and the block's sum of squares (all 4 lanes).
+struct ChunkQ {
+    uint2 x0, x1;        // X of entries 8u..8u+3 and 8u+4..8u+7 (int16 pairs)
+    int h0, h1;
+    float sc, sq;
+};
+__device__ __forceinline__ ChunkQ quant_chunk(const float v[8]) {
+    ChunkQ o;
+    uint32_t mx = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mx = max(mx, __float_as_uint(fabsf(v[e])));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    float inv;
+    block_exponent(mx, inv, o.sc);
+    uint32_t xb[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) xb[e] = __float_as_uint(fmaf(v[e], inv, kRoundMagic));
+    o.h0 = (int)(xb[0] + xb[1] + xb[2] + xb[3] - 4u * kRoundMagicBits);
+    o.h1 = (int)(xb[4] + xb[5] + xb[6] + xb[7] - 4u * kRoundMagicBits);
+    o.h0 += __shfl_xor_sync(0xffffffffu, o.h0, 2);      // quarters u and u^2 share lane groups
+    o.h1 += __shfl_xor_sync(0xffffffffu, o.h1, 2);
+    // The low 16 bits of xb[e] are X[e] in two's complement.
+    o.x0 = make_uint2(__byte_perm(xb[0], xb[1], 0x5410), __byte_perm(xb[2], xb[3], 0x5410));
+    o.x1 = make_uint2(__byte_perm(xb[4], xb[5], 0x5410), __byte_perm(xb[6], xb[7], 0x5410));
+    float q[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) q[e] = __fmul_rn(v[e], v[e]);
+    const float a0 = __fadd_rn(q[0], q[1]), a1 = __fadd_rn(q[2], q[3]);
+    const float a2 = __fadd_rn(q[4], q[5]), a3 = __fadd_rn(q[6], q[7]);
+    float t = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
+    t = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, 1));   // entry bit 3 = u bit 0
+    t = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, 2));   // entry bit 4 = u bit 1
+    o.sq = t;
+    return o;
+}
+// Store a chunk's X words and records: block b, quarter u, at X base xb_addr
+// (64 bytes per block) and record base rb_addr (32 bytes per block), shared
+// memory.
+__device__ __forceinline__ void store_chunk_smem(const ChunkQ& o, uint32_t x_base, uint32_t r_base,
+                                                 int b, int u) {
+    const int pos0 = (u & 1) * 16 + (u >> 1) * 4;   // lane order of entries 8u..8u+3 (+8 for the rest)
+    const uint32_t xa = x_base + (uint32_t)b * 64 + pos0 * 2;
+    sts64(xa, o.x0);
+    sts64(xa + 16, o.x1);
+    if (u < 2) {
+        const uint32_t ra = r_base + (uint32_t)b * 32 + (u & 1) * 16;
+        sts64(ra, make_uint2((uint32_t)(-8 * o.h0), __float_as_uint(o.sc)));
+        sts64(ra + 8, make_uint2((uint32_t)(-8 * o.h1), __float_as_uint(o.sc)));
+    }
+}
+
+// Lane layout (all 32 lanes): this lane holds entry j = (lane >> 2) + 8 *
+// (lane & 3) of block b.  Writes X, the records and the sum of squares of
+// the block to global memory (the persistent step's pre-quantised input).
+__device__ __forceinline__ void quant_lane_store(float v, int b, int16_t* xq, uint2* xrec, float* xsq) {
+    const int lane = threadIdx.x & 31;
+    const int j = (lane >> 2) + 8 * (lane & 3);
+    uint32_t mx = __float_as_uint(fabsf(v));
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float inv, sc;
+    block_exponent(mx, inv, sc);
+    const uint32_t xb = __float_as_uint(fmaf(v, inv, kRoundMagic));
+    int h = (int)(xb - kRoundMagicBits);
+    xq[(size_t)b * 32 + xperm_pos(j)] = (int16_t)(xb & 0xFFFFu);
+    // lane group (j & 15) >> 2: entry bits 0, 1 and 4 vary = lane bits 2, 3, 1
+    h += __shfl_xor_sync(0xffffffffu, h, 4);
+    h += __shfl_xor_sync(0xffffffffu, h, 8);
+    h += __shfl_xor_sync(0xffffffffu, h, 2);
+    if ((lane & 0xE) == 0) {
+        const int grp = (j & 15) >> 2;
+        xrec[(size_t)b * 4 + grp] = make_uint2((uint32_t)(-8 * h), __float_as_uint(sc));
+    }
+    // entry bits 0, 1, 2, 3, 4 = lane bits 2, 3, 4, 0, 1
+    float t = __fmul_rn(v, v);
+    t = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, 4));
+    t = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, 8));
+    t = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, 16));
+    t = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, 1));
+    t = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, 2));
+    if (lane == 0) xsq[b] = t;
+}
+
+// Unit-RMS scale from the nb block sums of squares (shared or global
+// memory, any warp): lane l adds blocks l, l + 32, ... (two interleaved
+// accumulators, joined), then the lanes in an xor tree; every lane returns it.
+__device__ __forceinline__ float unit_rms_scale(const float* sq, int nb, int K) {
+    const int lane = threadIdx.x & 31;
+    float a0 = 0.f, a1 = 0.f;
+    int t = lane;
+    for (; t + 32 < nb; t += 64) {
+        a0 = __fadd_rn(a0, sq[t]);
+        a1 = __fadd_rn(a1, sq[t + 32]);
+    }
+    if (t < nb) a0 = __fadd_rn(a0, sq[t]);
+    float a = __fadd_rn(a0, a1);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, o));
+    return renorm_scale(a, K);
+}
+
+// Activation staging for the M <= 2 kernel, all threads of the CTA.  Thread
+// t holds the 16-byte chunks q = t, t + NT, ... of x (8 entries each; four
+// chunks make a 32-entry block, held by four consecutive lanes) and writes
+// the blocks' codes and records to shared memory, and (vector 0) the block
+// sums of squares to sq[].  CTA 0 writes the input it read to trace_x.
+// QN: chunks held per thread (M * K <= QN * 8 * NT); all QN rounds run
+// (chunks past the end are zeros), so callers pick the smallest QN that
+// covers the vector: the rounds then overlap instead of running one by one.
+template <int M, int NT, int QN>
 __device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs, uint32_t rec,
-                                                  float* red, const Fix& fix = Fix()) {
-    const int tid = threadIdx.x, lane = tid & 31;
+                                                  float* sq) {
+    const int tid = threadIdx.x;
     const int nq = M * a.K / 8;
     uint4 xr[QN];
 #pragma unroll
     for (int i = 0; i < QN; ++i) {
         const int q = tid + NT * i;
-        const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)q * 8);
-        xr[i] = q < nq ? (kCoherent ? __ldcg(src) : *src) : make_uint4(0, 0, 0, 0);
-    }
-    if constexpr (Fix::kActive) {
-        fix.template prepare<NT>(nq, xs);
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < QN; ++i) {
-            const int q = tid + NT * i;
-            if (q < nq) xr[i] = fix.apply(q, xr[i], xs);
-        }
-    }
-    if (M == 1 && a.renorm) {
-        float part = 0.f;
-#pragma unroll
-        for (int i = 0; i < QN; ++i) {
-            const __half2* h = reinterpret_cast<const __half2*>(&xr[i]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __half22float2(h[e]);
-                part = fmaf(f.x, f.x, part);
-                part = fmaf(f.y, f.y, part);
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        if (lane == 0) red[tid >> 5] = part;
-        __syncthreads();
-        float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < NT / 32; ++w) s += red[w];
-        const float scale = renorm_scale(s, a.K);
-#pragma unroll
-        for (int i = 0; i < QN; ++i) {
-            __half2* h = reinterpret_cast<__half2*>(&xr[i]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __half22float2(h[e]);
-                h[e] = __floats2half2_rn(f.x * scale, f.y * scale);
-            }
-        }
+        xr[i] = q < nq ? *reinterpret_cast<const uint4*>(a.x + (size_t)q * 8) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int i = 0; i < QN; ++i) {
@@ -192,7 +277,7 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs
         if (M == 1 && a.trace_x != nullptr && blockIdx.x == 0 && q < nq)
             *reinterpret_cast<uint4*>(a.trace_x + (size_t)q * 8) = xr[i];
         // The four chunks of a block sit in lanes 4j..4j+3 (NT*i is a multiple
-        // of 4), so every lane takes part in the shuffles below.
+        // of 4), so every lane takes part in the shuffles.
         const __half2* h = reinterpret_cast<const __half2*>(&xr[i]);
         float v[8];
 #pragma unroll
@@ -201,43 +286,10 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs
             v[2 * e] = f.x;
             v[2 * e + 1] = f.y;
         }
-        uint32_t mx = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mx = max(mx, __float_as_uint(fabsf(v[e])));
-        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        // X = rint(v * 2^(14-E)) (E: exponent of the block maximum), read from
-        // the low mantissa bits of v * 2^(14-E) + 1.5 * 2^23: the product is
-        // exact and |X| <= 32752, so the one rounding of the addition is the
-        // round-to-nearest-even to an integer and the bits hold 0x4B400000 + X.
-        // All-zero block: X = 0, scale 0.  Non-finite block: scale NaN (the
-        // outputs become NaN whatever X holds).
-        const int E = (int)(mx >> 23) - 127;                                   // max in [2^E, 2^(E+1))
-        const bool live = mx != 0u && mx < 0x7F800000u;
-        const float inv = live ? __uint_as_float((uint32_t)(141 - E) << 23) : 0.f;   // 2^(14-E)
-        const float sc = live ? __uint_as_float((uint32_t)(113 + E) << 23)            // 2^(E-14)
-                              : (mx == 0u ? 0.f : __uint_as_float(0x7FC00000u));
-        uint32_t xb[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xb[e] = __float_as_uint(fmaf(v[e], inv, 12582912.0f));
-        int h0 = (int)(xb[0] + xb[1] + xb[2] + xb[3] - 4u * 0x4B400000u);
-        int h1 = (int)(xb[4] + xb[5] + xb[6] + xb[7] - 4u * 0x4B400000u);
-        h0 += __shfl_xor_sync(0xffffffffu, h0, 2);      // quarters u and u^2 share lane groups
-        h1 += __shfl_xor_sync(0xffffffffu, h1, 2);
+        const ChunkQ o = quant_chunk(v);
         if (q < nq) {
-            const int bb = q >> 2, u = q & 3;
-            const int pos0 = (u & 1) * 16 + (u >> 1) * 4;   // elements 8u..8u+3 (then +8 for 8u+4..8u+7)
-            const uint32_t xsb = xs + (uint32_t)bb * 64;
-            // The low 16 bits of xb[e] are X[e] in two's complement.
-            sts64(xsb + pos0 * 2, make_uint2(__byte_perm(xb[0], xb[1], 0x5410), __byte_perm(xb[2], xb[3], 0x5410)));
-            sts64(xsb + pos0 * 2 + 16,
-                  make_uint2(__byte_perm(xb[4], xb[5], 0x5410), __byte_perm(xb[6], xb[7], 0x5410)));
-            if (u < 2) {
-                const int c0 = (u & 1) * 2;
-                const uint32_t rb = rec + (uint32_t)bb * 32 + c0 * 8;
-                sts64(rb, make_uint2((uint32_t)(-8 * h0), __float_as_uint(sc)));
-                sts64(rb + 8, make_uint2((uint32_t)(-8 * h1), __float_as_uint(sc)));
-            }
+            store_chunk_smem(o, xs, rec, q >> 2, q & 3);
+            if ((q & 3) == 0 && q < a.K / 8) sq[q >> 2] = o.sq;
         }
     }
     __syncthreads();
@@ -245,6 +297,16 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs
 
 // One warp's share of one GEMV on the dp2a path: accumulators, position in
 // its run of segments, and the split-tile bookkeeping.
+// Where a GEMV of the persistent step also writes its finished output
+// blocks pre-quantised for the next GEMV (lane-order X, records, sums of
+// squares; lane layout); nb: blocks the next GEMV reads (0: none).
+struct QuantOut {
+    int16_t* x;
+    uint2* rec;
+    float* sq;
+    int nb;
+};
+
 template <int M>
 struct Dp2aConsumer {
     float acc[M][4];
@@ -254,11 +316,15 @@ struct Dp2aConsumer {
     uint32_t x_lane0, r_lane0, xp, rp;   // running shared addresses of block b's X words and record
     uint32_t xstride, rstride;           // per activation vector
     float* park;             // this warp's two parked partials [2][M][32] (shared memory)
+    float oscale;            // outputs are f16(oscale * sum): the input's unit-RMS scale, or 1
+    QuantOut qo;
 
     __device__ __forceinline__ void init(const GemvArgs& a, int gw_, uint32_t xs, uint32_t rec,
                                          float* park_) {
         gw = gw_;
         park = park_;
+        oscale = 1.f;
+        qo.nb = 0;
         lane = threadIdx.x & 31;
         g = lane >> 2;
         c = lane & 3;
@@ -297,7 +363,9 @@ struct Dp2aConsumer {
         for (int m = 0; m < M; ++m) {
             const float val = (c == 0) ? acc[m][0] : (c == 1) ? acc[m][1] : (c == 2) ? acc[m][2] : acc[m][3];
             if (whole) {
-                if (row < a.N) a.y[(size_t)m * a.N + row] = __float2half_rn(val);
+                const __half yh = __float2half_rn(__fmul_rn(oscale, val));
+                if (row < a.N) a.y[(size_t)m * a.N + row] = yh;
+                if (M == 1 && t < qo.nb) quant_lane_store(__half2float(yh), t, qo.x, qo.rec, qo.sq);
             } else {
                 park[(sp.slot(t) * M + m) * 32 + r] = val;
             }
@@ -394,7 +462,7 @@ struct Dp2aConsumer {
     // finished (y written); for a tile shared with other CTAs the CTA's
     // partial goes to ws[cta][slot], slot 0 if the CTA's run starts in the
     // tile, else 1, and the tile is returned in xt[] (at most two, -1: none)
-    // with its contributing CTAs [xcf, xcl].
+    // with its contributing CTAs [xcf, xcl].  Lane 4g + c handles row g + 8c.
     template <int WARPS>
     __device__ __forceinline__ void combine_cta(const GemvArgs& a, const float* park_base, float* ws,
                                                 int xt[2], int xcf[2], int xcl[2]) {
@@ -414,18 +482,21 @@ struct Dp2aConsumer {
                 const int sl = park_slot_read(sp, gw, w, t);
                 const float* p = park_base + ((size_t)(w - cta_lo) * 2 + sl) * M * 32;
 #pragma unroll
-                for (int m = 0; m < M; ++m) sum[m] += p[m * 32 + lane];
+                for (int m = 0; m < M; ++m) sum[m] += p[m * 32 + r];
             }
             if (gf >= cta_lo && gl <= cta_hi) {
-                const int64_t row = (int64_t)t * 32 + lane;
+                const int64_t row = (int64_t)t * 32 + r;
 #pragma unroll
-                for (int m = 0; m < M; ++m)
-                    if (row < a.N) a.y[(size_t)m * a.N + row] = __float2half_rn(sum[m]);
+                for (int m = 0; m < M; ++m) {
+                    const __half yh = __float2half_rn(__fmul_rn(oscale, sum[m]));
+                    if (row < a.N) a.y[(size_t)m * a.N + row] = yh;
+                    if (M == 1 && t < qo.nb) quant_lane_store(__half2float(yh), t, qo.x, qo.rec, qo.sq);
+                }
             } else {
                 const int slc = cta_slot_write(blockIdx.x, t, KB, a.sc, WARPS);
 #pragma unroll
                 for (int m = 0; m < M; ++m)
-                    ws[(((size_t)blockIdx.x * 2 + slc) * M + m) * 32 + lane] = sum[m];
+                    ws[(((size_t)blockIdx.x * 2 + slc) * M + m) * 32 + r] = sum[m];
                 xt[e] = t;
                 xcf[e] = gf / WARPS;
                 xcl[e] = gl / WARPS;
@@ -438,7 +509,8 @@ struct Dp2aConsumer {
 // their arrival; the last to arrive sums the CTA partials in CTA order,
 // writes y and re-arms the counter.  One warp, lane = row.
 template <int M, int WARPS>
-__device__ __forceinline__ void combine_ctas_arrive(const GemvArgs& a, int t, int cf, int cl) {
+__device__ __forceinline__ void combine_ctas_arrive(const GemvArgs& a, int t, int cf, int cl,
+                                                    float oscale) {
     const int lane = threadIdx.x & 31;
     __syncwarp();
     int old = 0;
@@ -472,7 +544,7 @@ __device__ __forceinline__ void combine_ctas_arrive(const GemvArgs& a, int t, in
         const int64_t row = (int64_t)t * 32 + lane;
 #pragma unroll
         for (int m = 0; m < M; ++m)
-            if (row < a.N) a.y[(size_t)m * a.N + row] = __float2half_rn(sum[m]);
+            if (row < a.N) a.y[(size_t)m * a.N + row] = __float2half_rn(__fmul_rn(oscale, sum[m]));
         if (lane == 0) a.cnt[t] = 0;
     } else if (old >= need) {
         if (lane == 0) set_device_error(a.err, kDevConcurrent);
@@ -483,13 +555,13 @@ template <int M, int WARPS, int R, int C>
 __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[WARPS * R];
-    __shared__ float red[WARPS];
 
     const uint32_t smem_base = smem_addr(smem);
     const uint32_t xs = smem_base + (uint32_t)ring_bytes(WARPS, R, C);   // int16 X, lane order
     const uint32_t rec = xs + (uint32_t)(M * a.K * 2);                  // {-8 sum X, scale}
     float* park = reinterpret_cast<float*>(smem + ring_bytes(WARPS, R, C) + (size_t)M * a.K * 2 +
                                            (size_t)M * a.KB * 32);      // [WARPS][2][M][32]
+    float* sq = park + WARPS * 2 * M * 32;                              // block sums of squares
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gw = blockIdx.x * WARPS + warp;
@@ -518,10 +590,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
     {
         constexpr int NT = WARPS * 32;
         const int nq = M * a.K / 8;
-        if (nq <= 2 * NT) stage_activations<M, NT, false, 2>(a, xs, rec, red);
-        else if (nq <= 5 * NT) stage_activations<M, NT, false, 5>(a, xs, rec, red);
-        else stage_activations<M, NT, false, kXChunksPerThread>(a, xs, rec, red);
+        if (nq <= 2 * NT) stage_activations<M, NT, 2>(a, xs, rec, sq);
+        else if (nq <= 5 * NT) stage_activations<M, NT, 5>(a, xs, rec, sq);
+        else stage_activations<M, NT, kXChunksPerThread>(a, xs, rec, sq);
     }
+    // A renormalised input (M = 1) is the loaded vector times its unit-RMS
+    // scale, applied to the outputs.
+    if (M == 1 && a.renorm) cons.oscale = unit_rms_scale(sq, a.KB, a.K);
 
     for (int ch = 0; ch < ring.nch; ++ch) {
         if (!ring.wait(ch)) set_device_error(a.err, kDevTimeout);   // data then unreliable
@@ -541,55 +616,77 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
     __syncthreads();
     int xt[2], xcf[2], xcl[2];
     cons.template combine_cta<WARPS>(a, park, a.ws, xt, xcf, xcl);
-    if (xt[0] >= 0) combine_ctas_arrive<M, WARPS>(a, xt[0], xcf[0], xcl[0]);
-    if (xt[1] >= 0) combine_ctas_arrive<M, WARPS>(a, xt[1], xcf[1], xcl[1]);
+    if (xt[0] >= 0) combine_ctas_arrive<M, WARPS>(a, xt[0], xcf[0], xcl[0], cons.oscale);
+    if (xt[1] >= 0) combine_ctas_arrive<M, WARPS>(a, xt[1], xcf[1], xcl[1], cons.oscale);
 }
 
-// Final renorm of the decode step: out = renorm(in[0:len)), with the same
-// arithmetic (and order) as the renorm fused into the GEMV prologue.
-template <int WARPS>
-__global__ void __launch_bounds__(WARPS * 32, 1) renorm_kernel(const __half* in, __half* out, int len) {
-    __shared__ float red[WARPS];
-    constexpr int NT = WARPS * 32;
-    const int tid = threadIdx.x, lane = tid & 31;
-    pdl_wait();
+// Unit-RMS renorm of in[0:len) into out: out_i = f16(s * in_i), s from the
+// block sums of squares in the fixed tree and order above (the same s the
+// GEMVs apply), all NT threads of one CTA.  Fix completes chunks that exist
+// only as partial sums (the persistent step); sq: scratch for len/32 floats.
+template <int NT, int QN, bool kCoherent, class Fix>
+__device__ __forceinline__ void renorm_block(const __half* in, __half* out, int len, float* sq,
+                                             const Fix& fix, uint32_t patch) {
+    const int tid = threadIdx.x;
     const int nq = len / 8;
-    uint4 xr[kXChunksPerThread];
+    uint4 xr[QN];
 #pragma unroll
-    for (int i = 0; i < kXChunksPerThread; ++i) {
+    for (int i = 0; i < QN; ++i) {
         const int q = tid + NT * i;
-        xr[i] = q < nq ? *reinterpret_cast<const uint4*>(in + (size_t)q * 8) : make_uint4(0, 0, 0, 0);
+        const uint4* src = reinterpret_cast<const uint4*>(in + (size_t)q * 8);
+        xr[i] = q < nq ? (kCoherent ? __ldcg(src) : *src) : make_uint4(0, 0, 0, 0);
     }
-    float part = 0.f;
+    if constexpr (Fix::kActive) {
+        fix.template prepare<NT>(nq, patch);
+        __syncthreads();
 #pragma unroll
-    for (int i = 0; i < kXChunksPerThread; ++i) {
-        const __half2* h = reinterpret_cast<const __half2*>(&xr[i]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(h[e]);
-            part = fmaf(f.x, f.x, part);
-            part = fmaf(f.y, f.y, part);
+        for (int i = 0; i < QN; ++i) {
+            const int q = tid + NT * i;
+            if (q < nq) xr[i] = fix.apply(q, xr[i], patch);
         }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    if (lane == 0) red[tid >> 5] = part;
+    for (int i = 0; i < QN; ++i) {
+        const int q = tid + NT * i;
+        const __half2* h = reinterpret_cast<const __half2*>(&xr[i]);
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(h[e]);
+            v[2 * e] = f.x;
+            v[2 * e + 1] = f.y;
+        }
+        const ChunkQ o = quant_chunk(v);     // only the sum of squares is used
+        if (q < nq && (q & 3) == 0) sq[q >> 2] = o.sq;
+    }
     __syncthreads();
-    float s = 0.f;
+    const float scale = unit_rms_scale(sq, len / 32, len);
 #pragma unroll
-    for (int w = 0; w < WARPS; ++w) s += red[w];
-    const float scale = renorm_scale(s, len);
-#pragma unroll
-    for (int i = 0; i < kXChunksPerThread; ++i) {
+    for (int i = 0; i < QN; ++i) {
         const int q = tid + NT * i;
         __half2* h = reinterpret_cast<__half2*>(&xr[i]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float2 f = __half22float2(h[e]);
-            h[e] = __floats2half2_rn(f.x * scale, f.y * scale);
+            h[e] = __floats2half2_rn(__fmul_rn(scale, f.x), __fmul_rn(scale, f.y));
         }
         if (q < nq) *reinterpret_cast<uint4*>(out + (size_t)q * 8) = xr[i];
     }
+}
+
+struct NoFix {
+    static constexpr bool kActive = false;
+    template <int NT>
+    __device__ __forceinline__ void prepare(int, uint32_t) const {}
+    __device__ __forceinline__ uint4 apply(int, uint4 v, uint32_t) const { return v; }
+};
+
+// Final renorm of the decode step: out = f16(s * in[0:len)).
+template <int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 1) renorm_kernel(const __half* in, __half* out, int len) {
+    __shared__ float sq[(kXChunksPerThread * 8 * WARPS * 32) / 32];
+    pdl_wait();
+    renorm_block<WARPS * 32, kXChunksPerThread, false>(in, out, len, sq, NoFix(), 0u);
 }
 
 // GGUF Q4_0 -> packed layout, one warp per segment (grid-stride).

@@ -31,6 +31,9 @@ constexpr size_t kMaxDynSmem = 224 * 1024;   // opt-in dynamic shared memory per
 #define Q4_MMA_KERNEL_1 q4::gemv_mma_kernel<1, kWarps, kR2, kC2>
 #define Q4_MMA_KERNEL_2 q4::gemv_mma_kernel<2, kWarps, kR2, kC2>
 #define Q4_STACK_KERNEL q4::stack_kernel<kWarps, kR1, kC1>
+// Largest input of a GEMV in the persistent step (its staging holds up to
+// kStackXChunks 16-byte chunks per thread).
+constexpr int kStackKmax = q4::kStackXChunks * 8 * kThreads;
 
 enum StackMode { kStackPersistent = 0, kStackKernels = 1 };
 
@@ -82,6 +85,7 @@ struct q4gemv_ctx {
     StackKey desc_key;
     bool desc_valid = false;
     int* sync = nullptr;             // grid barrier words of the persistent step
+    uint8_t* xq = nullptr;           // pre-quantised inputs of the persistent step (two halves)
     std::string last_error;
 };
 
@@ -387,7 +391,8 @@ int q4gemv_create(q4gemv_t* out, int device) {
         if (cudaMalloc(&h->ws, ws_bytes) != cudaSuccess ||
             cudaMalloc(&h->cnt, (size_t)kMaxTiles * sizeof(int)) != cudaSuccess ||
             cudaMalloc(&h->err, sizeof(int)) != cudaSuccess ||
-            cudaMalloc(&h->sync, 4 * sizeof(int)) != cudaSuccess)
+            cudaMalloc(&h->sync, 4 * sizeof(int)) != cudaSuccess ||
+            cudaMalloc(&h->xq, 2 * q4::stack_xq_half_bytes(kStackKmax)) != cudaSuccess)
             rc = fail(h, Q4_ENOMEM, "workspace allocation failed");
         const char* mode = getenv("Q4GEMV_STACK_MODE");
         if (mode && !strcmp(mode, "kernels")) h->stack_mode = kStackKernels;
@@ -417,6 +422,7 @@ int q4gemv_create(q4gemv_t* out, int device) {
         cudaFree(h->cnt);
         cudaFree(h->err);
         cudaFree(h->sync);
+        cudaFree(h->xq);
         if (h->cap) cudaStreamDestroy(h->cap);
         delete h;
         return rc;
@@ -437,6 +443,7 @@ int q4gemv_destroy(q4gemv_t h) {
     cudaFree(h->act);
     cudaFree(h->desc);
     cudaFree(h->sync);
+    cudaFree(h->xq);
     delete h;
     return Q4_OK;
 }
@@ -564,6 +571,9 @@ int enqueue_stack_persistent(q4gemv_ctx* h, const StackKey& k, cudaStream_t st) 
     sa.cnt = h->cnt;
     sa.err = h->err;
     sa.sync = h->sync;
+    sa.xq = h->xq;
+    sa.xq_half = (int)q4::stack_xq_half_bytes(kStackKmax);
+    sa.kmax = (int)kmax;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(h->sms);
     cfg.blockDim = dim3(kThreads);
@@ -638,7 +648,7 @@ int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64
     }
 
     const int64_t kmax_step = hidden > ffn ? hidden : ffn;
-    if (h->stack_mode == kStackPersistent && kmax_step <= (int64_t)q4::kStackXChunks * 8 * kThreads &&
+    if (h->stack_mode == kStackPersistent && kmax_step <= (int64_t)kStackKmax &&
         q4::stack_smem_bytes((int)kmax_step, kWarps, kR1, kC1) <= kMaxDynSmem) {
         if (!h->desc_valid || !(h->desc_key == k)) {
             if (cs != cudaStreamCaptureStatusNone)

@@ -22,9 +22,9 @@ namespace q4 {
 struct StackGemv {
     const uint8_t* W;     // packed matrix
     __half* y;            // output, N entries
-    __half* trace_x;      // nullable: the input vector used
+    __half* trace_x;      // nullable: the input vector before its scale (filled at the end)
     int N, K;
-    int renorm;           // 1: input = renorm(previous output[0:K]); 0: input = x_in
+    int renorm;           // 1: input = unit-RMS scale * previous output[0:K]; 0: input = x_in
     int fill_y;           // 1: also write y of tiles shared by CTAs (y is traced)
     SplitConsts sc;       // split of its segments over the grid's warps
 };
@@ -33,10 +33,13 @@ struct StackArgs {
     const StackGemv* gemv;
     int n_gemv;
     const __half* x_in;   // input of GEMV 0
-    __half* x_out;        // renorm(last output[0:hidden])
+    __half* x_out;        // f16(s * last output[0:hidden])
     int hidden;
     float* ws;            // CTA partials, two GEMV-parity halves of [CTAs][2][32]
     int ws_half;          // floats per half
+    uint8_t* xq;          // pre-quantised inputs, two GEMV-parity halves of xq_half bytes:
+    int xq_half;          //   X [kmax] int16 (lane order), records [kmax / 32][4] {-8 sum X, scale},
+    int kmax;             //   block sums of squares [kmax / 32] fp32
     int* cnt;             // unused (tiles shared by CTAs are combined by the next reader)
     int* err;             // device error word
     int* sync;            // [0] grid arrivals, [1] abort flag; zero at launch
@@ -44,26 +47,29 @@ struct StackArgs {
 
 // Outputs of the previous GEMV in tiles shared by several CTAs exist only as
 // per-CTA partials until they are read: every reader sums them in CTA order
-// (the same sum q4gemv_run's kernel takes) and rounds to f16.  prepare()
-// combines, with all threads of the CTA, the shared tiles' 8-element chunks
-// that fall in the staged range into `patch` (shared memory, 16 bytes per
-// chunk), so their loads overlap those of the rest of the vector; apply()
-// then takes chunk q from the patch when its tile is shared.  ws == nullptr:
-// no-op.  A traced step also completes y (fill_y) for those tiles: boundary
-// b's tile is written by CTA b, or every one by the calling CTA (fill_all).
+// (the same sum q4gemv_run's kernel takes), scales by the previous GEMV's
+// output scale and rounds to f16.  combine() gives one 8-row chunk of such a
+// tile.  For the step's final renorm, prepare() combines, with all threads
+// of the CTA, the shared tiles' chunks in the staged range into `patch`
+// (shared memory, 16 bytes per chunk), so their loads overlap those of the
+// rest of the vector, and apply() takes chunk q from the patch when its tile
+// is shared.  ws == nullptr: no-op.  A traced step also completes y (fill_y)
+// for those tiles: boundary b's tile is written by CTA b, or every one by
+// the calling CTA (fill_all).
 template <int WARPS>
 struct SplitFix {
     static constexpr bool kActive = true;
     const float* ws;      // the previous GEMV's CTA partials [CTAs][2][32]
     SplitConsts sc;       // its split
     int KB;               // its blocks per row
+    float oscale;         // its output scale
     __half* fill_y;       // nullable: its output, to complete
     int fill_n;           // its rows
     bool fill_all;
 
-    // The combined chunk u (rows 8u..8u+7) of shared tile t, whose first
-    // contributing CTA is cf; two contributors are loaded together (the
-    // usual case), any further ones after them; the sum runs from +0.
+    // Chunk u (rows 8u..8u+7) of shared tile t, whose first contributing
+    // CTA is cf; two contributors are loaded together (the usual case), any
+    // further ones after them; the sum runs from +0.
     __device__ __forceinline__ uint4 combine(int t, int cf, int u) const {
         const int cl = warp_of_seg(t * KB + KB - 1, sc) / WARPS;
         const float4* p0 = reinterpret_cast<const float4*>(
@@ -83,8 +89,14 @@ struct SplitFix {
         uint4 o;
         __half2* h = reinterpret_cast<__half2*>(&o);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) h[e] = __floats2half2_rn(s[2 * e], s[2 * e + 1]);
+        for (int e = 0; e < 4; ++e)
+            h[e] = __floats2half2_rn(__fmul_rn(oscale, s[2 * e]), __fmul_rn(oscale, s[2 * e + 1]));
         return o;
+    }
+    __device__ __forceinline__ void fill(int t, int u, uint4 v) const {
+        const __half* h = reinterpret_cast<const __half*>(&v);
+        for (int e = 0; e < 8; ++e)
+            if (t * 32 + u * 8 + e < fill_n) fill_y[(size_t)t * 32 + u * 8 + e] = h[e];
     }
 
     template <int NT>
@@ -111,11 +123,7 @@ struct SplitFix {
             for (int k = 0; k < 2; ++k) {
                 if (tt[k] < 0) continue;
                 if (qq[k] < nq) sts128(patch + (uint32_t)qq[k] * 16, v[k]);
-                if (fl[k]) {
-                    const __half* h = reinterpret_cast<const __half*>(&v[k]);
-                    for (int e = 0; e < 8; ++e)
-                        if (qq[k] * 8 + e < fill_n) fill_y[(size_t)qq[k] * 8 + e] = h[e];
-                }
+                if (fl[k]) fill(tt[k], qq[k] & 3, v[k]);
             }
         }
     }
@@ -128,58 +136,66 @@ struct SplitFix {
     }
 };
 
-// Unit-RMS renorm of in[0:len) into out, same arithmetic and order as the
-// renorm fused into the GEMV prologue (coherent loads: `in` may have been
-// written by other CTAs of the running kernel).  All NT threads of one CTA.
-template <int NT, bool kCoherent, int QN, class Fix>
-__device__ __forceinline__ void renorm_block(const __half* in, __half* out, int len, float* red,
-                                             const Fix& fix, uint32_t patch) {
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int nq = len / 8;
-    uint4 xr[QN];
-#pragma unroll
-    for (int i = 0; i < QN; ++i) {
-        const int q = tid + NT * i;
-        const uint4* src = reinterpret_cast<const uint4*>(in + (size_t)q * 8);
-        xr[i] = q < nq ? (kCoherent ? __ldcg(src) : *src) : make_uint4(0, 0, 0, 0);
+// Staging of GEMV i >= 1 of the step from the pre-quantised input that GEMV
+// i-1's CTAs wrote for their finished tiles: one bulk copy each of the codes,
+// records and block sums of squares into shared memory, while all threads
+// combine, scale, round and quantise the tiles shared by CTAs (the copy holds
+// no valid data for those) and write them over the copy once it has landed.
+// K: entries of GEMV i's input; xbar: this CTA's copy barrier, phase parity.
+template <int WARPS, int NT>
+__device__ __forceinline__ void stage_prequant(const StackArgs& sa, int i, int K,
+                                               const SplitFix<WARPS>& fx, uint32_t xs, uint32_t rec,
+                                               float* sq, uint64_t* xbar, uint32_t parity) {
+    const int KB = K / 32;
+    const uint8_t* base = sa.xq + (size_t)(i & 1) * sa.xq_half;
+    if (threadIdx.x == 0) {
+        // Other CTAs wrote these bytes with ordinary stores before the grid
+        // barrier, and this CTA last read the destination with ordinary
+        // loads: order both before the bulk copies.
+        fence_proxy_async_global();
+        fence_proxy_async_smem();
+        const uint32_t bx = (uint32_t)K * 2, br = (uint32_t)K, bs = (uint32_t)tile_sum_bytes(K);
+        mbar_arrive_expect_tx(xbar, bx + br + bs);
+        bulk_g2s_addr(xs, base, bx, xbar);
+        bulk_g2s_addr(rec, base + (size_t)sa.kmax * 2, br, xbar);
+        bulk_g2s_addr(smem_addr(sq), base + (size_t)sa.kmax * 3, bs, xbar);
     }
-    fix.template prepare<NT>(nq, patch);
-    __syncthreads();
+    // Shared tiles of GEMV i-1, enumerated by CTA boundary and chunk (four
+    // consecutive threads per tile, so the quantiser's shuffles stay inside
+    // one tile); every lane runs the quantiser, idle ones on zeros.
+    const int nb = (fx.sc.G + WARPS - 1) / WARPS;
+    const int total = (nb - 1) * 4;
+    constexpr int kRounds = 2;                          // total <= 2 * NT: up to 257 CTAs
+    ChunkQ o[kRounds];
+    int tq[kRounds];
 #pragma unroll
-    for (int i = 0; i < QN; ++i) {
-        const int q = tid + NT * i;
-        if (q < nq) xr[i] = fix.apply(q, xr[i], patch);
-    }
-    float part = 0.f;
-#pragma unroll
-    for (int i = 0; i < QN; ++i) {
-        const __half2* h = reinterpret_cast<const __half2*>(&xr[i]);
+    for (int k = 0; k < kRounds; ++k) {
+        const int p = (int)threadIdx.x + k * NT;
+        const int b = (p >> 2) + 1, u = p & 3;
+        const int t = p < total ? shared_tile_of_boundary(b, fx.KB, fx.sc, WARPS) : -1;
+        const bool fl = t >= 0 && fx.fill_y != nullptr && b == (int)blockIdx.x;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (t >= 0 && (t < KB || fl)) v = fx.combine(t, b - 1, u);
+        if (fl) fx.fill(t, u, v);
+        float f[8];
+        const __half2* h = reinterpret_cast<const __half2*>(&v);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(h[e]);
-            part = fmaf(f.x, f.x, part);
-            part = fmaf(f.y, f.y, part);
+            const float2 g = __half22float2(h[e]);
+            f[2 * e] = g.x;
+            f[2 * e + 1] = g.y;
         }
+        o[k] = quant_chunk(f);
+        tq[k] = (t >= 0 && t < KB) ? t * 4 + u : -1;
     }
+    if (!mbar_wait_bounded(xbar, parity, 1u << 22)) set_device_error(sa.err, kDevTimeout);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    if (lane == 0) red[tid >> 5] = part;
+    for (int k = 0; k < kRounds; ++k) {
+        if (tq[k] < 0) continue;
+        store_chunk_smem(o[k], xs, rec, tq[k] >> 2, tq[k] & 3);
+        if ((tq[k] & 3) == 0) sq[tq[k] >> 2] = o[k].sq;
+    }
     __syncthreads();
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < NT / 32; ++w) s += red[w];
-    const float scale = renorm_scale(s, len);
-#pragma unroll
-    for (int i = 0; i < QN; ++i) {
-        const int q = tid + NT * i;
-        __half2* h = reinterpret_cast<__half2*>(&xr[i]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(h[e]);
-            h[e] = __floats2half2_rn(f.x * scale, f.y * scale);
-        }
-        if (q < nq) *reinterpret_cast<uint4*>(out + (size_t)q * 8) = xr[i];
-    }
 }
 
 // The view of GEMV i that the per-warp consumer and the staging work on.
@@ -209,9 +225,15 @@ constexpr int kStackXChunks = 5;
 
 // Shared memory of the persistent step for inputs of up to kmax elements:
 // ring, int16 activations (2 bytes each), block records (1 byte per
-// element), one tile partial pair per warp.
+// element), one tile partial pair per warp, block sums of squares.
 __host__ __device__ constexpr size_t stack_smem_bytes(int kmax, int warps, int R, int C) {
-    return ring_bytes(warps, R, C) + (size_t)kmax * 3 + warp_partial_bytes(1, warps);
+    return ring_bytes(warps, R, C) + (size_t)kmax * 3 + warp_partial_bytes(1, warps) +
+           tile_sum_bytes(kmax);
+}
+
+// Bytes of one parity half of the pre-quantised input buffer.
+__host__ __device__ constexpr size_t stack_xq_half_bytes(int kmax) {
+    return ((size_t)kmax * 3 + tile_sum_bytes(kmax) + 255) / 256 * 256;
 }
 
 // A warp's position in its stream of chunks (C segments each) across the
@@ -315,7 +337,7 @@ template <int WARPS, int R, int C>
 __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa, int kmax) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[WARPS * R];
-    __shared__ float red[WARPS];
+    __shared__ __align__(8) uint64_t xbar;
     __shared__ int flag;
     constexpr int NT = WARPS * 32;
 
@@ -324,6 +346,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa
     const uint32_t xs = smem_base + (uint32_t)ring_bytes(WARPS, R, C);
     const uint32_t rec = xs + (uint32_t)kmax * 2;
     float* park = reinterpret_cast<float*>(smem + ring_bytes(WARPS, R, C) + (size_t)kmax * 3);
+    float* sq = park + WARPS * 2 * 32;
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gw = blockIdx.x * WARPS + warp;
@@ -332,13 +355,14 @@ __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa
 
     if (lane == 0) {
         for (int k = 0; k < R; ++k) mbar_init(wbars + k, 1);
+        if (warp == 0) mbar_init(&xbar, 1);
         fence_barrier_init();
     }
     // The descriptors are read again and again by the cursors: pull them into
     // L1 once.
     for (int off = threadIdx.x * 128; off < sa.n_gemv * (int)sizeof(StackGemv); off += NT * 128)
         prefetch_l1(reinterpret_cast<const uint8_t*>(sa.gemv) + off);
-    __syncwarp();
+    __syncthreads();
 
     StreamProducer<R, C> prod;
     prod.start(sa, gw);
@@ -346,28 +370,39 @@ __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa
     prod.fill(sa, gw, consumed, stage0, wbars, lane);
 
     bool ok = true;
+    float s_prev = 1.f;                   // output scale of GEMV i-1
     for (int i = 0; i < sa.n_gemv && ok; ++i) {
         GemvArgs a = stack_view(sa, i);
         a.ws = sa.ws + (size_t)(i & 1) * sa.ws_half;
-        SplitFix<WARPS> fix;
-        fix.ws = nullptr;
-        if (i > 0) {
+        // The warp's share of GEMV i depends on no data: set it up before the
+        // barrier.  Finished output blocks go out pre-quantised for GEMV i+1.
+        Dp2aConsumer<1> cons;
+        cons.init(a, gw, xs, rec, park + (size_t)warp * 2 * 32);
+        if (i + 1 < sa.n_gemv) {
+            uint8_t* ob = sa.xq + (size_t)((i + 1) & 1) * sa.xq_half;
+            cons.qo.x = reinterpret_cast<int16_t*>(ob);
+            cons.qo.rec = reinterpret_cast<uint2*>(ob + (size_t)sa.kmax * 2);
+            cons.qo.sq = reinterpret_cast<float*>(ob + (size_t)sa.kmax * 3);
+            cons.qo.nb = sa.gemv[i + 1].K / 32;
+        }
+        if (i > 0) ok = grid_wait(sa.sync, i * (int)gridDim.x, sa.err, &flag);
+        if (!ok) break;
+        if (i == 0) {
+            if (a.K <= 2 * NT * 8) stage_activations<1, NT, 2>(a, xs, rec, sq);
+            else stage_activations<1, NT, kStackXChunks>(a, xs, rec, sq);
+        } else {
             const StackGemv& pd = sa.gemv[i - 1];
+            SplitFix<WARPS> fix;
             fix.ws = sa.ws + (size_t)((i - 1) & 1) * sa.ws_half;
             fix.sc = pd.sc;
             fix.KB = pd.K / 32;
+            fix.oscale = s_prev;
             fix.fill_y = pd.fill_y ? pd.y : nullptr;
             fix.fill_n = pd.N;
             fix.fill_all = false;
+            stage_prequant<WARPS, NT>(sa, i, a.K, fix, xs, rec, sq, &xbar, (uint32_t)((i - 1) & 1));
+            cons.oscale = unit_rms_scale(sq, a.KB, a.K);
         }
-        // The warp's share of GEMV i depends on no data: set it up before the
-        // barrier.
-        Dp2aConsumer<1> cons;
-        cons.init(a, gw, xs, rec, park + (size_t)warp * 2 * 32);
-        if (i > 0) ok = grid_wait(sa.sync, i * (int)gridDim.x, sa.err, &flag);
-        if (!ok) break;
-        if (a.K <= 2 * NT * 8) stage_activations<1, NT, true, 2>(a, xs, rec, red, fix);
-        else stage_activations<1, NT, true, kStackXChunks>(a, xs, rec, red, fix);
         const int nseg = cons.sp.s1 - cons.sp.s0;
         for (int j = 0; j < nseg; j += C) {
             const int k = consumed % R;
@@ -389,7 +424,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa
         __syncthreads();
         int xt[2], xcf[2], xcl[2];   // tiles shared with other CTAs: combined by their readers
         cons.template combine_cta<WARPS>(a, park, a.ws, xt, xcf, xcl);
-        // This CTA is done with GEMV i (outputs and CTA partials written).
+        s_prev = cons.oscale;
+        // This CTA is done with GEMV i (outputs, CTA partials and the next
+        // input's blocks written; the latter are read by bulk copies).
+        fence_proxy_async_global();
         __syncthreads();
         if (threadIdx.x == 0) red_add_release_gpu(sa.sync, 1);
     }
@@ -397,14 +435,26 @@ __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa
     if (ok) {
         const int il = sa.n_gemv - 1;
         const StackGemv& ld = sa.gemv[il];
-        SplitFix<WARPS> fix;
-        fix.ws = sa.ws + (size_t)(il & 1) * sa.ws_half;
-        fix.sc = ld.sc;
-        fix.KB = ld.K / 32;
-        fix.fill_y = ld.fill_y ? ld.y : nullptr;
-        fix.fill_n = ld.N;
-        fix.fill_all = true;
-        if (blockIdx.x == 0) renorm_block<NT, true, kStackXChunks>(ld.y, sa.x_out, sa.hidden, red, fix, xs);
+        if (blockIdx.x == 0) {
+            SplitFix<WARPS> fix;
+            fix.ws = sa.ws + (size_t)(il & 1) * sa.ws_half;
+            fix.sc = ld.sc;
+            fix.KB = ld.K / 32;
+            fix.oscale = s_prev;
+            fix.fill_y = ld.fill_y ? ld.y : nullptr;
+            fix.fill_n = ld.N;
+            fix.fill_all = true;
+            renorm_block<NT, kStackXChunks, true>(ld.y, sa.x_out, sa.hidden, sq, fix, xs);
+        }
+        // Traced inputs: GEMV j read x_in (j = 0) or GEMV j-1's output, all
+        // complete now (j - 1 is not the last GEMV).
+        for (int j = blockIdx.x; j < sa.n_gemv; j += gridDim.x) {
+            const StackGemv& d = sa.gemv[j];
+            if (d.trace_x == nullptr) continue;
+            const __half* src = j == 0 ? sa.x_in : sa.gemv[j - 1].y;
+            for (int q = threadIdx.x; q < d.K / 8; q += NT)
+                reinterpret_cast<uint4*>(d.trace_x)[q] = __ldcg(reinterpret_cast<const uint4*>(src) + q);
+        }
         return;
     }
     // Abort: let this warp's copies in flight land (bounded) before leaving.
