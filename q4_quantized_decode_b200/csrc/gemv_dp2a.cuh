@@ -122,7 +122,10 @@ struct WarpRing {
 // A 32-entry block v of an f16 activation vector becomes X = rint(v *
 // 2^(14-E)) (E: exponent of the block maximum, so |X| <= 32752 and the
 // maximum is exact), stored in lane order (xperm_pos), and lane group c gets
-// the record {-8 * sum of its eight X, 2^(E-14)}.  X is read from the low
+// the record {0x4B400000 - 8 * sum of its eight X, 2^(E-14)}: started from
+// that word, the dp2a sum of a lane's four rows ends as the bit pattern of
+// the float 1.5 * 2^23 + sum (q - 8) X (exact: the sum is below 2^22 in
+// magnitude), so one subtraction makes it a float.  X is read from the low
 // mantissa bits of v * 2^(14-E) + 1.5 * 2^23: the product is exact and
 // |X| < 2^22, so the one rounding of the addition is the round to the nearest
 // integer (ties to even) and the bits hold 0x4B400000 + X.  All-zero block:
@@ -197,8 +200,8 @@ __device__ __forceinline__ void store_chunk_smem(const ChunkQ& o, uint32_t x_bas
     sts64(xa + 16, o.x1);
     if (u < 2) {
         const uint32_t ra = r_base + (uint32_t)b * 32 + (u & 1) * 16;
-        sts64(ra, make_uint2((uint32_t)(-8 * o.h0), __float_as_uint(o.sc)));
-        sts64(ra + 8, make_uint2((uint32_t)(-8 * o.h1), __float_as_uint(o.sc)));
+        sts64(ra, make_uint2(kRoundMagicBits - 8u * (uint32_t)o.h0, __float_as_uint(o.sc)));
+        sts64(ra + 8, make_uint2(kRoundMagicBits - 8u * (uint32_t)o.h1, __float_as_uint(o.sc)));
     }
 }
 
@@ -222,7 +225,7 @@ __device__ __forceinline__ void quant_lane_store(float v, int b, int16_t* xq, ui
     h += __shfl_xor_sync(0xffffffffu, h, 2);
     if ((lane & 0xE) == 0) {
         const int grp = (j & 15) >> 2;
-        xrec[(size_t)b * 4 + grp] = make_uint2((uint32_t)(-8 * h), __float_as_uint(sc));
+        xrec[(size_t)b * 4 + grp] = make_uint2(kRoundMagicBits - 8u * (uint32_t)h, __float_as_uint(sc));
     }
     // entry bits 0, 1, 2, 3, 4 = lane bits 2, 3, 4, 0, 1
     float t = __fmul_rn(v, v);
@@ -403,14 +406,17 @@ struct Dp2aConsumer {
                 v[m][i] = dp2a_hi(xq[m].w, hi, t);
             }
         }
+        const float2 mm = make_float2(-kRoundMagic, -kRoundMagic);
 #pragma unroll
         for (int m = 0; m < M; ++m) {
             const float sbm = __uint_as_float(rc[m].y);
             const float2 s2 = make_float2(sbm, sbm);
             const float2 ds01 = fmul2(d01, s2), ds23 = fmul2(d23, s2);
             float2 a01 = make_float2(acc[m][0], acc[m][1]), a23 = make_float2(acc[m][2], acc[m][3]);
-            a01 = ffma2(make_float2((float)v[m][0], (float)v[m][1]), ds01, a01);
-            a23 = ffma2(make_float2((float)v[m][2], (float)v[m][3]), ds23, a23);
+            const float2 f01 = fadd2(make_float2(__int_as_float(v[m][0]), __int_as_float(v[m][1])), mm);
+            const float2 f23 = fadd2(make_float2(__int_as_float(v[m][2]), __int_as_float(v[m][3])), mm);
+            a01 = ffma2(f01, ds01, a01);
+            a23 = ffma2(f23, ds23, a23);
             acc[m][0] = a01.x;
             acc[m][1] = a01.y;
             acc[m][2] = a23.x;
