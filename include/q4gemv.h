@@ -72,11 +72,7 @@ typedef enum {
 } q4gemv_status;
 
 /* Limits checked by validation.  Besides these, ceil(N/32) * (K/32) must be
- * below 2^31, and on the tensor-core path (M >= 3, or M <= 2 with K beyond
- * the CUDA-core kernel's staging) a matrix wider than the activations one
- * CTA can stage (about 9700 columns for M <= 8, 4800 for M <= 16) is
- * accepted up to about 3839 * that many columns' worth of 32-row tiles
- * (Q4_ESHAPE beyond). */
+ * below 2^31. */
 #define Q4GEMV_MAX_M 16
 #define Q4GEMV_MAX_N (1 << 22)     /* rows */
 #define Q4GEMV_MAX_K (1 << 20)     /* columns */
@@ -140,7 +136,14 @@ Q4GEMV_API int q4gemv_repack(q4gemv_t h, const void* gguf, void* packed,
  * exactly (elements within a factor 16 of it are exact; others are rounded
  * to 2^-15 of the block maximum) and the per-block dot products are exact
  * integers.  Deterministic: the same inputs on the same device give the
- * same bits. */
+ * same bits.
+ * For M >= 3 (and M <= 2 with K beyond the CUDA-core kernel's activation
+ * staging) the tensor-core kernel runs; a matrix wider than the activation
+ * slice one CTA can hold (about 9,700 columns for M <= 8, 6,000 for M <= 16)
+ * is covered by several launches over column panels whose sums are added in
+ * fp32, in panel order, in an accumulator of M*N floats owned by the handle
+ * (preallocated for M*N <= 2^21; a larger first call grows it, which
+ * synchronises the device and must not happen during a stream capture). */
 Q4GEMV_API int q4gemv_run(q4gemv_t h, const void* W_packed, const void* x, void* y,
                int M, int64_t N, int64_t K, q4gemv_stream_t stream);
 

@@ -28,6 +28,12 @@
 
 namespace q4 {
 
+// One launch covers a column panel of the matrix: blocks [p0, p0 + KBv) of
+// every row (the whole row when KBv == KB).  Its segments are numbered in
+// panel order, v = t * KBv + j for block p0 + j of tile t, and split flat over
+// the launch's warps.  A matrix too wide for one CTA's activation staging is
+// covered by several panel launches whose sums are added in panel order in
+// fp32 (mode 1: yacc = sum, 2: yacc += sum, 3: y = f16(yacc + sum)).
 struct MmaArgs {
     const uint8_t* W;    // packed matrix (segments of 576 bytes)
     const __half* x;     // [M][K]
@@ -35,10 +41,59 @@ struct MmaArgs {
     float* ws;           // [G][2][16][32] split-tile partials
     int* cnt;            // [T] arrival counters, zero between calls
     int* err;
+    float* yacc;         // [M][N] fp32 sum of earlier panels (modes 1..3)
     int64_t N;
-    int K, KB, T, S, G;
+    int K, KB, T, S, G;  // S = T * KBv
+    int KBv, p0;         // panel: blocks per tile, first block
+    int mode;            // 0: y = f16(sum); 1..3: panel modes above
     int M;               // 1..16 (columns >= M are zero-padded)
     SplitConsts sc;      // make_split(S, G)
+};
+
+// A warp's ring over a panel: stage k holds C consecutive panel segments of
+// the warp's run [s0, s1), filled by one bulk copy per contiguous piece (a
+// stage that crosses a tile boundary of a narrower panel takes two or more).
+template <int R, int C>
+struct PanelRing {
+    uint32_t stage0;
+    uint64_t* bars;
+    const uint8_t* W;
+    int s0, nseg, nch, KBv, KB, p0;
+
+    __device__ void init(uint32_t ring_base, uint64_t* bar_base, int warp, const MmaArgs& a, int s0_,
+                         int s1_) {
+        stage0 = ring_base + (uint32_t)warp * R * C * kSegBytes;
+        bars = bar_base + warp * R;
+        W = a.W;
+        s0 = s0_;
+        nseg = s1_ - s0_;
+        nch = (nseg + C - 1) / C;
+        KBv = a.KBv;
+        KB = a.KB;
+        p0 = a.p0;
+    }
+    __device__ uint32_t stage(int k) const { return stage0 + (uint32_t)k * C * kSegBytes; }
+    // Lane 0 only.
+    __device__ void issue(int ch) const {
+        const int k = ch % R;
+        int n = min(C, nseg - ch * C);
+        const int v = s0 + ch * C;
+        int t = v / KBv, j = v - t * KBv;
+        mbar_arrive_expect_tx(bars + k, (uint32_t)n * kSegBytes);
+        uint32_t dst = stage(k);
+        while (n > 0) {
+            const int len = min(n, KBv - j);
+            bulk_g2s_addr(dst, W + ((size_t)t * KB + p0 + j) * kSegBytes, (uint32_t)len * kSegBytes,
+                          bars + k);
+            dst += (uint32_t)len * kSegBytes;
+            n -= len;
+            ++t;
+            j = 0;
+        }
+    }
+    __device__ bool wait(int ch) const {
+        return mbar_wait_bounded(bars + (ch % R), (uint32_t)((ch / R) & 1), 1u << 22);
+    }
 };
 
 // Bytes per staged activation vector for `nblk` blocks: 64 per block, padded
@@ -108,9 +163,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
     const int g = lane >> 2, c = lane & 3;
     const int gw = blockIdx.x * WARPS + warp;
     WarpSplit sp;
-    sp.init(gw, a.sc, a.KB);
+    sp.init(gw, a.sc, a.KBv);
     const int s0 = sp.s0, s1 = sp.s1;
-    const int KB = a.KB;
+    const int KB = a.KBv;                       // blocks per tile of this panel
 
     // The CTA's blocks: its warps own one contiguous run of segments.
     const int w_lo = blockIdx.x * WARPS;
@@ -121,8 +176,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
     const int b0 = (cs1 - cs0 >= KB) ? 0 : (cs0 % KB);
     const int vstride = mma_vstride(nblk);
 
-    WarpRing<R, C> ring;
-    ring.init(smem_base, bars, warp, a.W, s0, s1);
+    PanelRing<R, C> ring;
+    ring.init(smem_base, bars, warp, a, s0, s1);
     if (lane == 0) {
         for (int k = 0; k < R; ++k) mbar_init(bars + warp * R + k, 1);
         fence_barrier_init();
@@ -147,7 +202,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
                     const int vv = p / (nblk * 4), rem = p - vv * nblk * 4;
                     int b = b0 + (rem >> 2);
                     if (b >= KB) b -= KB;
-                    v[u] = *reinterpret_cast<const uint4*>(a.x + (size_t)vv * a.K + b * 32 + (rem & 3) * 8);
+                    v[u] = *reinterpret_cast<const uint4*>(a.x + (size_t)vv * a.K + (a.p0 + b) * 32 +
+                                                           (rem & 3) * 8);
                 }
             }
 #pragma unroll
@@ -182,6 +238,15 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
     const int t_first = sp.t_first;
     int t_cur = t_first;
 
+    // A finished output (all blocks of this panel summed).
+    auto emit = [&](int col, int64_t row, float v) {
+        const size_t o = (size_t)col * a.N + row;
+        if (a.mode == 0) a.y[o] = __float2half_rn(v);
+        else if (a.mode == 1) a.yacc[o] = v;
+        else if (a.mode == 2) a.yacc[o] = a.yacc[o] + v;
+        else a.y[o] = __float2half_rn(a.yacc[o] + v);
+    };
+
     // Output (row, column) held by acc[tt][nt][i]:
     //   row = 16*tt + g + 8*(i >> 1), column = 8*nt + 2c + (i & 1).
     auto flush = [&](int t) {
@@ -197,8 +262,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
                     const int col = 8 * nt + 2 * c + (i & 1);
                     const int64_t row = (int64_t)t * 32 + r;
                     if (whole) {
-                        if (col < a.M && row < a.N)
-                            a.y[(size_t)col * a.N + row] = __float2half_rn(acc[tt][nt][i]);
+                        if (col < a.M && row < a.N) emit(col, row, acc[tt][nt][i]);
                     } else {
                         a.ws[(((size_t)gw * 2 + slot) * 16 + col) * 32 + r] = acc[tt][nt][i];
                     }
@@ -265,43 +329,97 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
     }
     if (s1 > s0) flush(t_cur);
 
-    auto arrive = [&](int t, int gf, int gl) {
-        if (gf == gl) return;
-        __syncwarp();
-        int old = 0;
-        if (lane == 0) old = atom_add_acq_rel_gpu(a.cnt + t, 1);
-        old = __shfl_sync(0xffffffffu, old, 0);
-        __syncwarp();                       // order the lanes' reads after lane 0's acquire
-        const int need = gl - gf + 1;
-        if (old == need - 1) {
-            const int64_t row = (int64_t)t * 32 + lane;
-            for (int col = 0; col < a.M; ++col) {
-                float sum = 0.f;
-                SegWalker wk;
-                wk.init(gf, a.sc);
-                for (int g0 = gf; g0 <= gl; g0 += 8) {
-                    float pv[8];
+    // Split tiles, two levels, each summed in a fixed order.  Level 1: all
+    // threads of the CTA sum, per output, the parked partials of the CTA's
+    // contributing warps in warp order (loads of many outputs in flight at
+    // once); a tile inside the CTA is then finished.  Level 2: a tile shared
+    // with other CTAs leaves the CTA's partial (slot 0 if the CTA's run starts
+    // in it, else 1) and the last CTA to arrive (per-tile counter) sums the
+    // CTA partials in CTA order.
+    __shared__ int tl_t[2 * WARPS], tl_gf[2 * WARPS], tl_gl[2 * WARPS], tl_s0[2 * WARPS];
+    __shared__ int tl_n, tl_k2[2], tl_old[2];
+    if (threadIdx.x == 0) tl_n = 0;
+    __syncthreads();
+    const int cta_lo = w_lo, cta_hi = w_hi - 1;
+    if (s1 > s0 && lane == 0) {
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int gg = g0 + u;
-                        const int sl = (wk.sb >= t * KB) ? 0 : 1;
-                        pv[u] = gg <= gl ? ld_relaxed_gpu(a.ws + (((size_t)gg * 2 + sl) * 16 + col) * 32 + lane)
-                                         : 0.f;
-                        wk.next();
-                    }
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) sum += pv[u];
-                }
-                if (row < a.N) a.y[(size_t)col * a.N + row] = __float2half_rn(sum);
-            }
-            if (lane == 0) a.cnt[t] = 0;
-        } else if (old >= need) {
-            if (lane == 0) set_device_error(a.err, kDevConcurrent);
+        for (int e = 0; e < 2; ++e) {
+            if (!cta_combiner(sp, e, gw, cta_lo)) continue;
+            const int k = atomicAdd(&tl_n, 1);
+            tl_t[k] = e == 0 ? sp.t_first : sp.t_last;
+            tl_gf[k] = e == 0 ? sp.gf0 : sp.gf1;
+            tl_gl[k] = e == 0 ? sp.gl0 : sp.gl1;
+            tl_s0[k] = park_slot_read(sp, gw, gw, tl_t[k]);   // this (first) warp's slot
         }
-    };
-    if (s1 > s0) {
-        arrive(sp.t_first, sp.gf0, sp.gl0);
-        if (sp.t_last != sp.t_first) arrive(sp.t_last, sp.gf1, sp.gl1);
+    }
+    __syncthreads();
+    const int ntl = tl_n;
+    float* ws_cta = a.ws + (size_t)a.G * 2 * 16 * 32;       // [CTAs][2][16][32]
+    const int per_tile = 32 * a.M;
+    for (int idx = threadIdx.x; idx < ntl * per_tile; idx += NT) {
+        const int k = idx / per_tile, rem = idx - k * per_tile;
+        const int col = rem >> 5, r = rem & 31;
+        const int t = tl_t[k], gf = tl_gf[k], gl = tl_gl[k];
+        const int wf = max(gf, cta_lo), wl = min(gl, cta_hi);
+        float sum = 0.f;
+        // Eight contributors per round: their loads are issued together, the
+        // sum still runs in warp order.
+        for (int w0 = wf; w0 <= wl; w0 += 8) {
+            float pv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int w = w0 + u;
+                const int sl = w == wf ? tl_s0[k] : 0;
+                pv[u] = w <= wl ? ld_relaxed_gpu(a.ws + (((size_t)w * 2 + sl) * 16 + col) * 32 + r) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (w0 + u <= wl) sum += pv[u];
+        }
+        if (gf >= cta_lo && gl <= cta_hi) {
+            const int64_t row = (int64_t)t * 32 + r;
+            if (row < a.N) emit(col, row, sum);
+        } else {
+            const int slc = cta_slot_write(blockIdx.x, t, KB, a.sc, WARPS);
+            ws_cta[(((size_t)blockIdx.x * 2 + slc) * 16 + col) * 32 + r] = sum;
+        }
+    }
+    __syncthreads();
+    // Level 2: the listed tiles this CTA shares with others (at most two: its
+    // first tile, j = 0, and its last, j = 1).
+    if (threadIdx.x == 0) {
+        tl_k2[0] = tl_k2[1] = -1;
+        for (int k = 0; k < ntl; ++k) {
+            if (tl_gf[k] >= cta_lo && tl_gl[k] <= cta_hi) continue;
+            const int j = (tl_gf[k] < cta_lo) ? 0 : 1;
+            tl_k2[j] = k;
+            tl_old[j] = atom_add_acq_rel_gpu(a.cnt + tl_t[k], 1);
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int k = tl_k2[j];
+        if (k < 0) continue;
+        const int old = tl_old[j];
+        const int t = tl_t[k];
+        const int cf = tl_gf[k] / WARPS, cl = tl_gl[k] / WARPS;
+        const int need = cl - cf + 1;
+        if (old == need - 1) {
+            for (int idx = threadIdx.x; idx < per_tile; idx += NT) {
+                const int col = idx >> 5, r = idx & 31;
+                float sum = 0.f;
+                for (int cc = cf; cc <= cl; ++cc) {
+                    const int sl = cta_slot_read(cc, cf, t, KB, a.sc, WARPS);
+                    sum += ld_relaxed_gpu(ws_cta + (((size_t)cc * 2 + sl) * 16 + col) * 32 + r);
+                }
+                const int64_t row = (int64_t)t * 32 + r;
+                if (row < a.N) emit(col, row, sum);
+            }
+            if (threadIdx.x == 0) a.cnt[t] = 0;
+        } else if (old >= need) {
+            if (threadIdx.x == 0) set_device_error(a.err, kDevConcurrent);
+        }
     }
 }
 

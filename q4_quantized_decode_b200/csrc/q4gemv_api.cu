@@ -21,15 +21,19 @@ constexpr int kWarps = 16;                 // warps per CTA of the GEMV kernels
 constexpr int kThreads = kWarps * 32;
 // Per-warp TMA ring (stages x segments per stage) of each kernel.
 constexpr int kR1 = 3, kC1 = 6;            // M = 1 and the decode step
-constexpr int kR2 = 2, kC2 = 4;            // M = 2 and the tensor-core kernel
+constexpr int kR2 = 2, kC2 = 4;            // M = 2
+constexpr int kRm1 = 2, kCm1 = 4;          // tensor-core kernel, M <= 8
+constexpr int kRm2 = 2, kCm2 = 2;          // tensor-core kernel, M <= 16 (small ring: a whole
+                                           // 160-block activation slice fits beside it)
 constexpr int kMinSegsPerWarp = 4;         // small problems use fewer warps
 constexpr int kMaxTiles = Q4GEMV_MAX_N / 32;
 constexpr size_t kMaxDynSmem = 224 * 1024;   // opt-in dynamic shared memory per CTA
+constexpr size_t kYaccPrealloc = (size_t)1 << 21;   // fp32 panel accumulator floats at create
 
 #define Q4_DP2A_KERNEL_1 q4::gemv_dp2a_kernel<1, kWarps, kR1, kC1>
 #define Q4_DP2A_KERNEL_2 q4::gemv_dp2a_kernel<2, kWarps, kR2, kC2>
-#define Q4_MMA_KERNEL_1 q4::gemv_mma_kernel<1, kWarps, kR2, kC2>
-#define Q4_MMA_KERNEL_2 q4::gemv_mma_kernel<2, kWarps, kR2, kC2>
+#define Q4_MMA_KERNEL_1 q4::gemv_mma_kernel<1, kWarps, kRm1, kCm1>
+#define Q4_MMA_KERNEL_2 q4::gemv_mma_kernel<2, kWarps, kRm2, kCm2>
 #define Q4_STACK_KERNEL q4::stack_kernel<kWarps, kR1, kC1>
 // Largest input of a GEMV in the persistent step (its staging holds up to
 // kStackXChunks 16-byte chunks per thread).
@@ -86,6 +90,8 @@ struct q4gemv_ctx {
     bool desc_valid = false;
     int* sync = nullptr;             // grid barrier words of the persistent step
     uint8_t* xq = nullptr;           // pre-quantised inputs of the persistent step (two halves)
+    float* yacc = nullptr;           // fp32 panel sums of wide tensor-core GEMVs
+    size_t yacc_floats = 0;
     std::string last_error;
 };
 
@@ -208,83 +214,94 @@ int ensure_ws(q4gemv_ctx* h, int warps, cudaStream_t st) {
 
 // Largest block count one CTA of the tensor-core kernel may stage (nt8 = 1:
 // up to 8 vectors, 2: up to 16).
+size_t mma_ring(int nt8) {
+    return nt8 == 1 ? q4::ring_bytes(kWarps, kRm1, kCm1) : q4::ring_bytes(kWarps, kRm2, kCm2);
+}
+
 int mma_xcap(int nt8) {
-    const size_t ring = q4::ring_bytes(kWarps, kR2, kC2);
+    const size_t ring = mma_ring(nt8);
     int xcap = 1;
     while (ring + q4::gemv_mma_smem_bytes(nt8, xcap + 1) <= kMaxDynSmem) ++xcap;
     return xcap;
 }
 
-// Wide-K problems on the tensor-core path launch ceil(S / xcap) CTAs rounded
-// up to whole waves; the warp count must stay within the split's limit for
-// any wave of up to 256 SMs.
-constexpr int64_t kMmaMaxRunCtas = q4::kMaxSplitWarps / kWarps - 256;
-
-bool mma_split_fits(int M, int64_t N, int64_t K) {
-    const int64_t KB = K / 32, S = (N + 31) / 32 * KB;
-    const int xcap = mma_xcap(M <= 8 ? 1 : 2);
-    return KB <= xcap || (S + xcap - 1) / xcap <= kMmaMaxRunCtas;
+// fp32 accumulator of the column panels of a wide tensor-core GEMV.
+int ensure_yacc(q4gemv_ctx* h, size_t floats, cudaStream_t st) {
+    if (floats <= h->yacc_floats) return Q4_OK;
+    if (h->fault == kFaultAlloc) return fail(h, Q4_EFAULTINJ, "injected allocation failure");
+    cudaStreamSynchronize(st);
+    cudaFree(h->yacc);
+    h->yacc = nullptr;
+    h->yacc_floats = 0;
+    if (cudaMalloc(&h->yacc, floats * sizeof(float)) != cudaSuccess)
+        return fail(h, Q4_ENOMEM, "panel accumulator of %zu floats failed", floats);
+    h->yacc_floats = floats;
+    return Q4_OK;
 }
 
-// Launch one GEMV on the tensor-core path (any M in 1..16, any K).
+// Launch one GEMV on the tensor-core path (any M in 1..16, any K).  When the
+// activation slice of a whole row (KB blocks of 8 or 16 vectors) does not fit
+// beside the ring, the matrix is covered by P column panels of at most xcap
+// blocks, one launch each, summed in panel order in fp32.
 int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M, int64_t N,
                     int64_t K, cudaStream_t st) {
     if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
     const int nt8 = M <= 8 ? 1 : 2;
     const int KB = (int)(K / 32);
     const int T = (int)((N + 31) / 32);
-    const int S = T * KB;
-    // Largest block count one CTA may stage; a CTA whose run of segments is
-    // at least KB stages all KB blocks, so KB must fit or runs stay shorter.
     const int xcap = mma_xcap(nt8);
-    const int wave = h->sms;                   // resident CTAs (one per SM)
-    int64_t ctas;
-    if (KB <= xcap) {
-        // Any run length fits: one wave, fewer for small problems.
-        ctas = wave;
+    const int P = (KB + xcap - 1) / xcap;
+    const int Wf = (KB + P - 1) / P;                 // panel width (the last may be narrower)
+    if (P > 1) {
+        const int rc = ensure_yacc(h, (size_t)M * (size_t)N, st);
+        if (rc != Q4_OK) return rc;
+    }
+    for (int p = 0; p < P; ++p) {
+        const int p0 = p * Wf;
+        const int KBv = KB - p0 < Wf ? KB - p0 : Wf;
+        const int64_t S = (int64_t)T * KBv;
+        // One wave, fewer CTAs for small problems: any run length fits, since
+        // a CTA stages at most KBv <= xcap blocks.
+        int64_t ctas = h->sms;
         const int64_t cap = S / (kWarps * kMinSegsPerWarp);
         if (ctas > cap) ctas = cap < 1 ? 1 : cap;
-    } else {
-        // Runs must stay within xcap blocks: whole waves of short runs.
-        ctas = (S + xcap - 1) / xcap;
-        ctas = (ctas + wave - 1) / wave * wave;
+        int64_t G = ctas * kWarps;
+        if (G > S) G = S;
+        // warp partials [G][2][16][32], then CTA partials [ctas][2][16][32]
+        const int rc = ensure_ws(h, (int)(G + ctas), st);
+        if (rc != Q4_OK) return rc;
+        q4::MmaArgs a;
+        a.W = static_cast<const uint8_t*>(W);
+        a.x = x;
+        a.y = y;
+        a.ws = h->ws;
+        a.cnt = h->cnt;
+        a.err = h->err;
+        a.yacc = h->yacc;
+        a.N = N;
+        a.K = (int)K;
+        a.KB = KB;
+        a.T = T;
+        a.S = (int)S;
+        a.G = (int)G;
+        a.KBv = KBv;
+        a.p0 = p0;
+        a.mode = P == 1 ? 0 : (p == 0 ? 1 : (p == P - 1 ? 3 : 2));
+        a.M = M;
+        a.sc = q4::make_split(a.S, a.G);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)ctas);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = mma_ring(nt8) + q4::gemv_mma_smem_bytes(nt8, KBv);
+        cfg.stream = st;
+        cfg.numAttrs = 0;
+        cudaError_t e;
+        if (nt8 == 1)
+            e = cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_1, a);
+        else
+            e = cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_2, a);
+        if (e != cudaSuccess) return cuda_fail(h, e, "gemv (mma) launch");
     }
-    int64_t G = ctas * kWarps;
-    if (G > S) G = S;
-    // Capping G would lengthen the CTAs' runs past xcap blocks of staged
-    // activations: refuse such (very large, very wide) problems instead.
-    if (G > q4::kMaxSplitWarps)
-        return fail(h, Q4_ESHAPE, "run: N * K too large for the M >= 3 / wide-K path");
-    const int rc = ensure_ws(h, (int)G, st);
-    if (rc != Q4_OK) return rc;
-    const int nblk_max = (KB <= xcap) ? KB : xcap;
-    q4::MmaArgs a;
-    a.W = static_cast<const uint8_t*>(W);
-    a.x = x;
-    a.y = y;
-    a.ws = h->ws;
-    a.cnt = h->cnt;
-    a.err = h->err;
-    a.N = N;
-    a.K = (int)K;
-    a.KB = KB;
-    a.T = T;
-    a.S = S;
-    a.G = (int)G;
-    a.M = M;
-    a.sc = q4::make_split(a.S, a.G);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)ctas);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = q4::ring_bytes(kWarps, kR2, kC2) + q4::gemv_mma_smem_bytes(nt8, nblk_max);
-    cfg.stream = st;
-    cfg.numAttrs = 0;
-    cudaError_t e;
-    if (nt8 == 1)
-        e = cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_1, a);
-    else
-        e = cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_2, a);
-    if (e != cudaSuccess) return cuda_fail(h, e, "gemv (mma) launch");
     return Q4_OK;
 }
 
@@ -352,7 +369,6 @@ int q4gemv_validate(int M, int64_t N, int64_t K, const void* W, const void* x, c
     if (M < 1 || M > Q4GEMV_MAX_M) return Q4_EUNSUPPORTED;
     const int sh = check_shape(N, K);
     if (sh != Q4_OK) return sh;
-    if (!dp2a_fits(M, K) && !mma_split_fits(M, N, K)) return Q4_ESHAPE;
     if (!W || !x || !y) return Q4_EINVAL;
     if (!aligned16(W) || !aligned16(x) || !aligned16(y)) return Q4_EALIGN;
     return Q4_OK;
@@ -392,8 +408,11 @@ int q4gemv_create(q4gemv_t* out, int device) {
             cudaMalloc(&h->cnt, (size_t)kMaxTiles * sizeof(int)) != cudaSuccess ||
             cudaMalloc(&h->err, sizeof(int)) != cudaSuccess ||
             cudaMalloc(&h->sync, 4 * sizeof(int)) != cudaSuccess ||
-            cudaMalloc(&h->xq, 2 * q4::stack_xq_half_bytes(kStackKmax)) != cudaSuccess)
+            cudaMalloc(&h->xq, 2 * q4::stack_xq_half_bytes(kStackKmax)) != cudaSuccess ||
+            cudaMalloc(&h->yacc, kYaccPrealloc * sizeof(float)) != cudaSuccess)
             rc = fail(h, Q4_ENOMEM, "workspace allocation failed");
+        else
+            h->yacc_floats = kYaccPrealloc;
         const char* mode = getenv("Q4GEMV_STACK_MODE");
         if (mode && !strcmp(mode, "kernels")) h->stack_mode = kStackKernels;
     }
@@ -423,6 +442,7 @@ int q4gemv_create(q4gemv_t* out, int device) {
         cudaFree(h->err);
         cudaFree(h->sync);
         cudaFree(h->xq);
+        cudaFree(h->yacc);
         if (h->cap) cudaStreamDestroy(h->cap);
         delete h;
         return rc;
@@ -444,6 +464,7 @@ int q4gemv_destroy(q4gemv_t h) {
     cudaFree(h->desc);
     cudaFree(h->sync);
     cudaFree(h->xq);
+    cudaFree(h->yacc);
     delete h;
     return Q4_OK;
 }
