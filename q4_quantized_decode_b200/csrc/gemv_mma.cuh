@@ -122,8 +122,7 @@ __device__ __forceinline__ uint32_t lop_mask_or(uint32_t w, uint32_t mask, uint3
 __device__ __forceinline__ void mma_16816(float& d0, float& d1, float& d2, float& d3, uint32_t a0,
                                           uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                           uint32_t b1, float c0, float c1, float c2, float c3) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%10,%11,%12,%13};"
         : "=f"(d0), "=f"(d1), "=f"(d2), "=f"(d3)
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(c2),
@@ -188,15 +187,15 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
     pdl_launch_dependents();
     pdl_wait();
 
-    // Stage the CTA's activation blocks with plain 16-byte loads (four per
+    // Stage the CTA's activation blocks with plain 16-byte loads (eight per
     // round per thread), reordered into lane order; zero vectors pad M up to
     // 8*NT8.
     {
         const int nchunk = a.M * nblk * 4;
-        for (int p0 = threadIdx.x; p0 < nchunk; p0 += 4 * NT) {
-            uint4 v[4];
+        for (int p0 = threadIdx.x; p0 < nchunk; p0 += 8 * NT) {
+            uint4 v[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 const int p = p0 + u * NT;
                 if (p < nchunk) {
                     const int vv = p / (nblk * 4), rem = p - vv * nblk * 4;
@@ -207,7 +206,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
                 }
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 const int p = p0 + u * NT;
                 if (p < nchunk) {
                     const int vv = p / (nblk * 4), rem = p - vv * nblk * 4;
@@ -275,13 +274,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
     if (jb < 0) jb += KB;
     const uint32_t x_lane = xsm + (uint32_t)g * vstride + (uint32_t)c * 16;
 
-    auto segment = [&](uint32_t seg) {
+    auto segment = [&](uint32_t seg, int jbs) {
         const uint4 w = lds128(seg + lane * 16);
         const uint2 dd = lds64(seg + kSegSclOff + g * 8);
         uint4 xv[NT8];
 #pragma unroll
         for (int nt = 0; nt < NT8; ++nt)
-            xv[nt] = lds128(x_lane + (uint32_t)(8 * nt) * vstride + (uint32_t)jb * 64);
+            xv[nt] = lds128(x_lane + (uint32_t)(8 * nt) * vstride + (uint32_t)jbs * 64);
         const float2 d01 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
         const float2 d23 = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
         const float dA[2] = {d01.x, d23.x};   // rows g, g+16
@@ -311,17 +310,27 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
         if (!ring.wait(ch)) set_device_error(a.err, kDevTimeout);   // data then unreliable
         const uint32_t st = ring.stage(ch % R);
         const int n = min(C, ring.nseg - ch * C);
-        for (int j = 0; j < n; ++j) {
-            if (b == KB) {
-                flush(t_cur);
-                ++t_cur;
-                b = 0;
-                jb = KB - b0;
-                if (jb >= KB) jb -= KB;
+        if (n == C && b + C <= KB && jb + C <= KB) {
+            // No tile ends inside this stage: its segments at constant
+            // offsets, free to interleave.
+#pragma unroll
+            for (int j = 0; j < C; ++j) segment(st + j * kSegBytes, jb + j);
+            b += C;
+            jb += C;
+            if (jb == KB) jb = 0;
+        } else {
+            for (int j = 0; j < n; ++j) {
+                if (b == KB) {
+                    flush(t_cur);
+                    ++t_cur;
+                    b = 0;
+                    jb = KB - b0;
+                    if (jb >= KB) jb -= KB;
+                }
+                segment(st + j * kSegBytes, jb);
+                ++b;
+                if (++jb == KB) jb = 0;
             }
-            segment(st + j * kSegBytes);
-            ++b;
-            if (++jb == KB) jb = 0;
         }
         __syncwarp();
         fence_proxy_async_smem();
