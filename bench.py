@@ -57,6 +57,20 @@ WORKLOAD = ("27B-shaped decode step, M=1: 64 layers x (QKV 5120->7168, O 5120->5
             "matrices, one persistent kernel launch per step")
 
 
+KERNEL_SOURCES = ["stack.cuh", "gemv_dp2a.cuh", "partition.cuh", "device_common.cuh"]
+
+
+def kernel_source_hash() -> str:
+    """sha256 over the sources of the decode-step kernel (ties the ncu
+    traffic figure in profiles/ to the code it was measured on)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "q4_quantized_decode_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -348,11 +362,15 @@ def run_ours(args, rank: int, world: int, dist):
         "frac_of_nominal_8TBps": per_rank_gbs / NOMINAL_HBM_GBS,
     }
     traffic = os.path.join(ROOT, "profiles", "traffic_per_launch.json")
-    if os.path.exists(traffic):
+    if os.path.exists(traffic) and L == 64:
         with open(traffic) as f:
             tr = json.load(f)
-        roofline["traffic"] = tr.get("bytes_per_step_equivalent")
-        roofline["traffic_note"] = tr.get("note")
+        # Counters taken on another version of the kernel's source do not count.
+        if tr.get("source_sha256") == kernel_source_hash():
+            roofline["traffic"] = tr.get("bytes_per_launch")
+            roofline["traffic_note"] = tr.get("note")
+        else:
+            roofline["traffic_note"] = "kernel source changed since the ncu capture: traffic unknown"
     cpu = None
     if not args.no_cpu_baseline:
         threads = os.cpu_count() or 1
