@@ -158,29 +158,38 @@ typedef struct {
 /* One synthetic decode step (M = 1) through n_layers layers of four Q4_0
  * GEMVs each, the 27B-shaped workload of the pages (hidden 5120: taozi.news
  * page, section "技术架构"; 64 layers: originshq.com page, section "The
- * Architecture: Layers Distributed, Activations in Flight"):
- *     a = renorm(f16(QKV x)[0:hidden])
- *     b = renorm(f16(O a))
- *     u = renorm(f16(gate_up b)[0:ffn])
- *     x = renorm(f16(down u))
- * renorm(v) scales v to unit RMS: s = sum v_i^2 in fp32, v_i * (1/sqrt(s/len))
- * in fp32 rounded to binary16; an all-zero v stays zero.  The pages give no
- * layer math beyond the GEMVs, so this chain (Q slice in place of attention,
- * gate half without an activation) is the reading adopted.
+ * Architecture: Layers Distributed, Activations in Flight").  Every GEMV
+ * output is rounded to binary16; the next GEMV reads its first K entries v
+ * scaled to unit RMS by the real scalar s(v) = 1/sqrt(mean(v^2)) (0 for an
+ * all-zero v), i.e. it computes f16(s(v) * (W v)):
+ *     a = f16(QKV x),   b = f16(s(a') O a'),  a' = a[0:hidden]
+ *     u = f16(s(b) gate_up b),   x' = f16(s(u') down u'),  u' = u[0:ffn]
+ * and x_out = f16(s(x') x').  The pages give no layer math beyond the GEMVs,
+ * so this chain (Q slice in place of attention, gate half without an
+ * activation, a unit-RMS scale in place of the norm) is the reading adopted.
+ * On the GPU s is taken in fp32: block sums of squares in a fixed binary tree,
+ * blocks in a fixed order, the hardware's approximate reciprocal square root.
  *   layers  : HOST array of n_layers entries (device pointers inside)
- *   x_in    : device, hidden binary16 (not modified)
- *   x_out   : device, hidden binary16 (may alias x_in)
+ *   x_in    : hidden binary16 (not modified); device (16-byte aligned) or
+ *             host memory, pinned or pageable: a host vector is copied to
+ *             the device on `stream` inside the call
+ *   x_out   : hidden binary16 (may alias x_in); device or host memory (a host
+ *             vector is copied back on `stream` inside the call)
  *   trace_x : device or NULL; [4*n_layers][max(hidden, ffn)] binary16: the
  *             input vector of GEMV i = 4l + t (t = 0 QKV, 1 O, 2 gate_up,
- *             3 down) in its first K_i entries
+ *             3 down), before its scale, in its first K_i entries
  *   trace_y : device or NULL; [4*n_layers][max(qkv_n, hidden, 2*ffn)]
  *             binary16: the raw output of GEMV i in its first N_i entries
- * Requires qkv_n >= hidden, qkv_n % 8 == 0, 1 <= n_layers <= 4096.  The first call with a
- * given set of arguments captures the whole step (4*n_layers GEMVs, each
- * with the renorm of its input fused in, plus one final renorm) as a CUDA
- * graph on an internal stream; later calls with the same arguments replay it
- * with one cudaGraphLaunch on `stream`.  If `stream` is capturing, the
- * kernels are launched directly into the caller's capture instead. */
+ * Requires qkv_n >= hidden, qkv_n % 8 == 0, 1 <= n_layers <= 4096,
+ * max(hidden, ffn) within one CTA's activation staging.  The step runs as ONE
+ * cooperative persistent kernel (plus a 16-byte reset of its barrier words);
+ * the first call with a given set of arguments uploads its descriptors and
+ * must happen outside any stream capture, later calls only launch.  With the
+ * environment variable Q4GEMV_STACK_MODE=kernels (read at create) the step
+ * runs instead as a CUDA graph of one kernel per GEMV, captured on the first
+ * call and replayed, or launched into the caller's capture when `stream` is
+ * capturing; both modes give the same bits.  Host vectors are not accepted
+ * while `stream` is capturing. */
 Q4GEMV_API int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers,
                      int64_t hidden, int64_t qkv_n, int64_t ffn,
                      const void* x_in, void* x_out, void* trace_x,

@@ -92,6 +92,8 @@ struct q4gemv_ctx {
     uint8_t* xq = nullptr;           // pre-quantised inputs of the persistent step (two halves)
     float* yacc = nullptr;           // fp32 panel sums of wide tensor-core GEMVs
     size_t yacc_floats = 0;
+    __half* hio = nullptr;           // device copies of host x_in / x_out of run_stack
+    int64_t hio_elems = 0;           // per vector
     std::string last_error;
 };
 
@@ -120,6 +122,16 @@ int cuda_fail(q4gemv_ctx* h, cudaError_t e, const char* what) {
     } while (0)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Host memory (pinned or pageable) rather than device or managed memory.
+bool is_host_pointer(const void* p) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();           // clear: an unknown pointer is pageable host memory
+        return true;
+    }
+    return at.type == cudaMemoryTypeHost || at.type == cudaMemoryTypeUnregistered;
+}
 
 int check_shape(int64_t N, int64_t K) {
     if (N <= 0 || K <= 0 || K % 32 != 0) return Q4_ESHAPE;
@@ -465,6 +477,7 @@ int q4gemv_destroy(q4gemv_t h) {
     cudaFree(h->sync);
     cudaFree(h->xq);
     cudaFree(h->yacc);
+    cudaFree(h->hio);
     delete h;
     return Q4_OK;
 }
@@ -510,6 +523,15 @@ int q4gemv_run(q4gemv_t h, const void* W, const void* x, void* y, int M, int64_t
 }
 
 namespace {
+
+// After a step whose x_out is host memory: copy the device result out on
+// the same stream.
+int finish_host_out(q4gemv_ctx* h, int rc, bool host_out, void* user_out, const void* dev_out,
+                    int64_t hidden, cudaStream_t st) {
+    if (rc != Q4_OK || !host_out) return rc;
+    Q4_CUDA(h, cudaMemcpyAsync(user_out, dev_out, hidden * sizeof(__half), cudaMemcpyDeviceToHost, st));
+    return Q4_OK;
+}
 
 // Enqueue the whole decode step on `st`.
 int enqueue_stack(q4gemv_ctx* h, const StackKey& k, cudaStream_t st) {
@@ -627,7 +649,11 @@ int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64
         if (s != Q4_OK) return fail(h, s, "run_stack: invalid matrix shape");
         if (!dp2a_fits(1, d[1])) return fail(h, Q4_EUNSUPPORTED, "run_stack: K too large");
     }
-    if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(trace_x) || !aligned16(trace_y))
+    // x_in / x_out may be host memory (pinned or pageable): staged through
+    // device copies on the same stream, inside this call.
+    const bool host_in = is_host_pointer(x_in), host_out = is_host_pointer(x_out);
+    if ((!host_in && !aligned16(x_in)) || (!host_out && !aligned16(x_out)) || !aligned16(trace_x) ||
+        !aligned16(trace_y))
         return fail(h, Q4_EALIGN, "run_stack: misaligned pointer");
     for (int l = 0; l < n_layers; ++l) {
         const q4gemv_layer& L = layers[l];
@@ -638,6 +664,29 @@ int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64
     }
     Q4_CUDA(h, cudaSetDevice(h->device));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void* x_out_user = x_out;
+    if (host_in || host_out) {
+        cudaStreamCaptureStatus cs0 = cudaStreamCaptureStatusNone;
+        Q4_CUDA(h, cudaStreamIsCapturing(st, &cs0));
+        if (cs0 != cudaStreamCaptureStatusNone)
+            return fail(h, Q4_EUNSUPPORTED, "run_stack: host vectors cannot be used during stream capture");
+        if (hidden > h->hio_elems) {
+            if (h->fault == kFaultAlloc) return fail(h, Q4_EFAULTINJ, "injected allocation failure");
+            Q4_CUDA(h, cudaStreamSynchronize(st));
+            cudaFree(h->hio);
+            h->hio = nullptr;
+            h->hio_elems = 0;
+            const int64_t n = (hidden + 7) / 8 * 8;
+            if (cudaMalloc(&h->hio, 2 * n * sizeof(__half)) != cudaSuccess)
+                return fail(h, Q4_ENOMEM, "run_stack: host-vector staging allocation failed");
+            h->hio_elems = n;
+        }
+        if (host_in) {
+            Q4_CUDA(h, cudaMemcpyAsync(h->hio, x_in, hidden * sizeof(__half), cudaMemcpyHostToDevice, st));
+            x_in = h->hio;
+        }
+        if (host_out) x_out = h->hio + h->hio_elems;
+    }
 
     StackKey k;
     k.layers.assign(layers, layers + n_layers);
@@ -693,7 +742,8 @@ int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64
             h->desc_key = k;
             h->desc_valid = true;
         }
-        return enqueue_stack_persistent(h, k, st);
+        return finish_host_out(h, enqueue_stack_persistent(h, k, st), host_out, x_out_user, x_out,
+                               hidden, st);
     }
     if (cs != cudaStreamCaptureStatusNone) return enqueue_stack(h, k, st);
 
@@ -721,7 +771,7 @@ int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64
         h->key = k;
     }
     Q4_CUDA(h, cudaGraphLaunch(h->exec, st));
-    return Q4_OK;
+    return finish_host_out(h, Q4_OK, host_out, x_out_user, x_out, hidden, st);
 }
 
 int q4gemv_sync_status(q4gemv_t h, q4gemv_stream_t stream) {

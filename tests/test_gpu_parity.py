@@ -271,6 +271,28 @@ def test_stack_small_end_to_end_and_teacher_forced(eng):
     assert np.array_equal(out, out2)
 
 
+def test_stack_host_vectors(eng):
+    """x_in / x_out in host memory (pinned or pageable) give the same bits as
+    device vectors; the copies happen inside the call."""
+    L, hidden, qkv_n, ffn = 1, 256, 384, 512
+    layers, _ = build_stack(eng, L, hidden, qkv_n, ffn, 99)
+    x = synth.normal_f16(99, synth.act_id(0), hidden)
+    want = bits_of(eng.run_stack(layers, f16_dev(x), hidden, qkv_n, ffn))
+    for pinned in (True, False):
+        xh = torch.from_numpy(x.view(np.float16).copy())
+        oh = torch.empty(hidden, dtype=torch.float16)
+        if pinned:
+            xh, oh = xh.pin_memory(), oh.pin_memory()
+        eng.run_stack(layers, xh, hidden, qkv_n, ffn, x_out=oh)
+        torch.cuda.synchronize()
+        assert eng.sync_status() == q4.Q4_OK
+        assert np.array_equal(oh.numpy().view(np.uint16), want), pinned
+    # host in, device out
+    od = torch.empty(hidden, dtype=torch.float16, device="cuda")
+    eng.run_stack(layers, torch.from_numpy(x.view(np.float16).copy()), hidden, qkv_n, ffn, x_out=od)
+    assert np.array_equal(bits_of(od), want)
+
+
 def test_stack_signed_permutation_closed_form(eng):
     from tests.test_oracle_pins import make_perm_stack, perm_stack_expected
     L, hidden, qkv_n, ffn = 3, 64, 96, 128
