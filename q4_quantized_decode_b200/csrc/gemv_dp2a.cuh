@@ -39,7 +39,7 @@ constexpr int kXChunksPerThread = 9; // activation staging: M*K <= 9 * 8 * threa
 
 struct GemvArgs {
     const uint8_t* W;       // packed matrix (segments of 576 bytes)
-    const __half* x;        // [M][K] activations, or the renorm source (M == 1)
+    const __half* x;        // [M][K] activations (renorm: the previous f16 output, unscaled)
     __half* y;              // [M][N]
     float* ws;              // CTA partials of tiles shared by CTAs [CTAs][2][M][32]
     int* cnt;               // per-tile arrival counters [T], zero between calls
@@ -49,7 +49,8 @@ struct GemvArgs {
     int K, KB, T;
     int S;                  // segments = T * KB
     int G;                  // warps that own segments (G <= S)
-    int renorm;             // 1: the input is renorm(x[0:K]) (M == 1 only)
+    int renorm;             // 1 (M == 1): the input is s * x[0:K], s its unit-RMS scale, applied
+                            // to the outputs; 0: the input is x
     SplitConsts sc;         // make_split(S, G)
 };
 

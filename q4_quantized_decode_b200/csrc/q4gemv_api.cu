@@ -611,7 +611,6 @@ int enqueue_stack_persistent(q4gemv_ctx* h, const StackKey& k, cudaStream_t st) 
     sa.hidden = (int)k.hidden;
     sa.ws = h->ws;
     sa.ws_half = h->sms * 2 * 32;   // [CTAs][2][32] per GEMV parity (ws holds sms * 16 warps * 1 KB)
-    sa.cnt = h->cnt;
     sa.err = h->err;
     sa.sync = h->sync;
     sa.xq = h->xq;

@@ -1,17 +1,19 @@
-// The whole synthetic decode step (4 * n_layers renormalised M = 1 GEMVs) as
-// one persistent kernel: one CTA per SM, a grid-wide barrier between
-// consecutive GEMVs, and each warp's weight stream running ahead across GEMV
-// boundaries.
+// The whole synthetic decode step (4 * n_layers M = 1 GEMVs, each input the
+// previous f16 output scaled to unit RMS) as one persistent kernel: one CTA
+// per SM, a grid-wide barrier between consecutive GEMVs, and each warp's
+// weight stream running ahead across GEMV boundaries.
 //
 // The pages keep the GPU fed with one command submission per token
 // (originshq.com page, section "The Engine: ~50 WGSL Kernels Written From
 // Scratch").  Here one launch covers the step, and the dependency between
-// GEMVs (the next input is the renormalised previous output) no longer
-// drains the memory pipe: weights do not depend on activations, so while a
-// CTA waits at the barrier and restages x, its warps' rings already hold the
-// next GEMV's first segments (up to ~150 KB per SM).  Each GEMV is computed by
-// the same per-warp consumer as q4gemv_run's M = 1 kernel, over the same
-// balanced segment split, so results are identical to chaining that kernel.
+// GEMVs (the next input is the previous output) no longer drains the memory
+// pipe: weights do not depend on activations, so while a CTA waits at the
+// barrier and stages its input, its warps' rings already hold the next
+// GEMV's first segments (~166 KB per SM).  Each GEMV's finished output blocks
+// are also written converted for the next GEMV, which stages them with bulk
+// copies.  Each GEMV is computed by the same per-warp consumer as
+// q4gemv_run's M = 1 kernel, over the same balanced segment split and with
+// the same combine order, so results are identical to chaining that kernel.
 #pragma once
 
 #include "gemv_dp2a.cuh"
@@ -40,7 +42,6 @@ struct StackArgs {
     uint8_t* xq;          // pre-quantised inputs, two GEMV-parity halves of xq_half bytes:
     int xq_half;          //   X [kmax] int16 (lane order), records [kmax / 32][4] {-8 sum X, scale},
     int kmax;             //   block sums of squares [kmax / 32] fp32
-    int* cnt;             // unused (tiles shared by CTAs are combined by the next reader)
     int* err;             // device error word
     int* sync;            // [0] grid arrivals, [1] abort flag; zero at launch
 };
@@ -49,7 +50,7 @@ struct StackArgs {
 // per-CTA partials until they are read: every reader sums them in CTA order
 // (the same sum q4gemv_run's kernel takes), scales by the previous GEMV's
 // output scale and rounds to f16.  combine() gives one 8-row chunk of such a
-// tile.  For the step's final renorm, prepare() combines, with all threads
+// tile.  For the step's final output, prepare() combines, with all threads
 // of the CTA, the shared tiles' chunks in the staged range into `patch`
 // (shared memory, 16 bytes per chunk), so their loads overlap those of the
 // rest of the vector, and apply() takes chunk q from the patch when its tile
@@ -206,7 +207,7 @@ __device__ __forceinline__ GemvArgs stack_view(const StackArgs& sa, int i) {
     a.x = (i == 0) ? sa.x_in : sa.gemv[i - 1].y;
     a.y = d.y;
     a.ws = sa.ws;
-    a.cnt = sa.cnt;
+    a.cnt = nullptr;      // no arrival counters: shared tiles are combined by the next reader
     a.err = sa.err;
     a.trace_x = d.trace_x;
     a.N = d.N;
