@@ -59,6 +59,7 @@ struct PanelRing {
     uint64_t* bars;
     const uint8_t* W;
     int s0, nseg, nch, KBv, KB, p0;
+    int it, ij;           // issue cursor: tile and block (in the panel) of the next chunk
 
     __device__ void init(uint32_t ring_base, uint64_t* bar_base, int warp, const MmaArgs& a, int s0_,
                          int s1_) {
@@ -71,24 +72,27 @@ struct PanelRing {
         KBv = a.KBv;
         KB = a.KB;
         p0 = a.p0;
+        it = s0_ / KBv;
+        ij = s0_ - it * KBv;
     }
     __device__ uint32_t stage(int k) const { return stage0 + (uint32_t)k * C * kSegBytes; }
-    // Lane 0 only.
-    __device__ void issue(int ch) const {
+    // Lane 0 only, chunks in order.
+    __device__ void issue(int ch) {
         const int k = ch % R;
         int n = min(C, nseg - ch * C);
-        const int v = s0 + ch * C;
-        int t = v / KBv, j = v - t * KBv;
         mbar_arrive_expect_tx(bars + k, (uint32_t)n * kSegBytes);
         uint32_t dst = stage(k);
         while (n > 0) {
-            const int len = min(n, KBv - j);
-            bulk_g2s_addr(dst, W + ((size_t)t * KB + p0 + j) * kSegBytes, (uint32_t)len * kSegBytes,
+            const int len = min(n, KBv - ij);
+            bulk_g2s_addr(dst, W + ((size_t)it * KB + p0 + ij) * kSegBytes, (uint32_t)len * kSegBytes,
                           bars + k);
             dst += (uint32_t)len * kSegBytes;
             n -= len;
-            ++t;
-            j = 0;
+            ij += len;
+            if (ij == KBv) {
+                ij = 0;
+                ++it;
+            }
         }
     }
     __device__ bool wait(int ch) const {
@@ -113,12 +117,6 @@ __host__ __device__ __forceinline__ int mma_xpos(int e) {
     return ((e & 15) >> 2) * 8 + (e >> 4) * 4 + (((r & 1) << 1) | (r >> 1));
 }
 
-__device__ __forceinline__ uint32_t lop_mask_or(uint32_t w, uint32_t mask, uint32_t magic) {
-    uint32_t d;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "r"(mask), "r"(magic));  // (a & b) | c
-    return d;
-}
-
 __device__ __forceinline__ void mma_16816(float& d0, float& d1, float& d2, float& d3, uint32_t a0,
                                           uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                           uint32_t b1, float c0, float c1, float c2, float c3) {
@@ -129,25 +127,27 @@ __device__ __forceinline__ void mma_16816(float& d0, float& d1, float& d2, float
           "f"(c3));
 }
 
-__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
-__device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
-
 // Exact (q - 8) f16 pairs from one code word: lo/hi nibbles of bytes (0, 2)
 // and (1, 3).
 struct CodePairs {
     uint32_t p, q, r, s;   // p: k(4c, 4c+2)  q: k(4c+1, 4c+3)  r: k(4c+16, 4c+18)  s: k(4c+17, 4c+19)
 };
 __device__ __forceinline__ CodePairs unpack_pairs(uint32_t w) {
-    const uint32_t magic = 0x64006400u;     // f16 1024.0 in both halves
-    const uint32_t w8 = w >> 8;
-    const __half2 off_lo = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));  // 1032
-    const __half2 sixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));  // 1/16
-    const __half2 m72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));  // -72
+    // Codes into the mantissa of f16 1024 (0x6400): 1024 + q (low nibbles)
+    // or 1024 + 16q (high nibbles); then - 1032, or * 1/16 - 72: exact q - 8.
     CodePairs o;
-    o.p = h2_bits(__hsub2(bits_h2(lop_mask_or(w, 0x000F000Fu, magic)), off_lo));
-    o.q = h2_bits(__hsub2(bits_h2(lop_mask_or(w8, 0x000F000Fu, magic)), off_lo));
-    o.r = h2_bits(__hfma2(bits_h2(lop_mask_or(w, 0x00F000F0u, magic)), sixteenth, m72));
-    o.s = h2_bits(__hfma2(bits_h2(lop_mask_or(w8, 0x00F000F0u, magic)), sixteenth, m72));
+    asm("{\n\t.reg .b32 w8, t0, t1, t2, t3;\n\t"
+        "shr.b32 w8, %4, 8;\n\t"
+        "lop3.b32 t0, %4, 0x000F000F, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 t1, w8, 0x000F000F, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 t2, %4, 0x00F000F0, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 t3, w8, 0x00F000F0, 0x64006400, 0xEA;\n\t"
+        "sub.rn.f16x2 %0, t0, %5;\n\t"
+        "sub.rn.f16x2 %1, t1, %5;\n\t"
+        "fma.rn.f16x2 %2, t2, %6, %7;\n\t"
+        "fma.rn.f16x2 %3, t3, %6, %7;\n\t}"
+        : "=r"(o.p), "=r"(o.q), "=r"(o.r), "=r"(o.s)
+        : "r"(w), "r"(0x64086408u), "r"(0x2C002C00u), "r"(0xD480D480u));
     return o;
 }
 

@@ -22,9 +22,11 @@ constexpr int kThreads = kWarps * 32;
 // Per-warp TMA ring (stages x segments per stage) of each kernel.
 constexpr int kR1 = 3, kC1 = 6;            // M = 1 and the decode step
 constexpr int kR2 = 2, kC2 = 4;            // M = 2
-constexpr int kRm1 = 2, kCm1 = 4;          // tensor-core kernel, M <= 8
-constexpr int kRm2 = 2, kCm2 = 2;          // tensor-core kernel, M <= 16 (small ring: a whole
-                                           // 160-block activation slice fits beside it)
+// Tensor-core kernel: for each vector group (M <= 8, M <= 16) a deeper ring
+// used when a whole row's activation slice still fits beside it ("full"), and
+// a shallower one that leaves room for wider column panels ("panel").
+constexpr int kRmF1 = 2, kCmF1 = 7, kRmP1 = 2, kCmP1 = 4;   // M <= 8
+constexpr int kRmF2 = 2, kCmF2 = 3, kRmP2 = 2, kCmP2 = 2;   // M <= 16
 constexpr int kMinSegsPerWarp = 4;         // small problems use fewer warps
 constexpr int kMaxTiles = Q4GEMV_MAX_N / 32;
 constexpr size_t kMaxDynSmem = 224 * 1024;   // opt-in dynamic shared memory per CTA
@@ -32,8 +34,10 @@ constexpr size_t kYaccPrealloc = (size_t)1 << 21;   // fp32 panel accumulator fl
 
 #define Q4_DP2A_KERNEL_1 q4::gemv_dp2a_kernel<1, kWarps, kR1, kC1>
 #define Q4_DP2A_KERNEL_2 q4::gemv_dp2a_kernel<2, kWarps, kR2, kC2>
-#define Q4_MMA_KERNEL_1 q4::gemv_mma_kernel<1, kWarps, kRm1, kCm1>
-#define Q4_MMA_KERNEL_2 q4::gemv_mma_kernel<2, kWarps, kRm2, kCm2>
+#define Q4_MMA_KERNEL_F1 q4::gemv_mma_kernel<1, kWarps, kRmF1, kCmF1>
+#define Q4_MMA_KERNEL_P1 q4::gemv_mma_kernel<1, kWarps, kRmP1, kCmP1>
+#define Q4_MMA_KERNEL_F2 q4::gemv_mma_kernel<2, kWarps, kRmF2, kCmF2>
+#define Q4_MMA_KERNEL_P2 q4::gemv_mma_kernel<2, kWarps, kRmP2, kCmP2>
 #define Q4_STACK_KERNEL q4::stack_kernel<kWarps, kR1, kC1>
 // Largest input of a GEMV in the persistent step (its staging holds up to
 // kStackXChunks 16-byte chunks per thread).
@@ -224,14 +228,16 @@ int ensure_ws(q4gemv_ctx* h, int warps, cudaStream_t st) {
     return Q4_OK;
 }
 
-// Largest block count one CTA of the tensor-core kernel may stage (nt8 = 1:
-// up to 8 vectors, 2: up to 16).
-size_t mma_ring(int nt8) {
-    return nt8 == 1 ? q4::ring_bytes(kWarps, kRm1, kCm1) : q4::ring_bytes(kWarps, kRm2, kCm2);
+// Ring bytes of the tensor-core kernel (nt8 = 1: up to 8 vectors, 2: up to
+// 16; full: the deeper ring).
+size_t mma_ring(int nt8, bool full) {
+    if (nt8 == 1) return full ? q4::ring_bytes(kWarps, kRmF1, kCmF1) : q4::ring_bytes(kWarps, kRmP1, kCmP1);
+    return full ? q4::ring_bytes(kWarps, kRmF2, kCmF2) : q4::ring_bytes(kWarps, kRmP2, kCmP2);
 }
 
-int mma_xcap(int nt8) {
-    const size_t ring = mma_ring(nt8);
+// Largest block count one CTA may stage beside the given ring.
+int mma_xcap(int nt8, bool full) {
+    const size_t ring = mma_ring(nt8, full);
     int xcap = 1;
     while (ring + q4::gemv_mma_smem_bytes(nt8, xcap + 1) <= kMaxDynSmem) ++xcap;
     return xcap;
@@ -261,7 +267,10 @@ int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, in
     const int nt8 = M <= 8 ? 1 : 2;
     const int KB = (int)(K / 32);
     const int T = (int)((N + 31) / 32);
-    const int xcap = mma_xcap(nt8);
+    // The deeper ring when a whole row's activation slice fits beside it,
+    // else the shallower one with wider panels.
+    const bool full = KB <= mma_xcap(nt8, true);
+    const int xcap = mma_xcap(nt8, full);
     const int P = (KB + xcap - 1) / xcap;
     const int Wf = (KB + P - 1) / P;                 // panel width (the last may be narrower)
     if (P > 1) {
@@ -304,14 +313,14 @@ int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, in
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)ctas);
         cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = mma_ring(nt8) + q4::gemv_mma_smem_bytes(nt8, KBv);
+        cfg.dynamicSmemBytes = mma_ring(nt8, full) + q4::gemv_mma_smem_bytes(nt8, KBv);
         cfg.stream = st;
         cfg.numAttrs = 0;
         cudaError_t e;
         if (nt8 == 1)
-            e = cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_1, a);
+            e = full ? cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_F1, a) : cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_P1, a);
         else
-            e = cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_2, a);
+            e = full ? cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_F2, a) : cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_P2, a);
         if (e != cudaSuccess) return cuda_fail(h, e, "gemv (mma) launch");
     }
     return Q4_OK;
@@ -435,7 +444,8 @@ int q4gemv_create(q4gemv_t* out, int device) {
     }
     if (rc == Q4_OK) {
         if (set_smem_attr(Q4_DP2A_KERNEL_1) || set_smem_attr(Q4_DP2A_KERNEL_2) ||
-            set_smem_attr(Q4_MMA_KERNEL_1) || set_smem_attr(Q4_MMA_KERNEL_2) ||
+            set_smem_attr(Q4_MMA_KERNEL_F1) || set_smem_attr(Q4_MMA_KERNEL_P1) ||
+            set_smem_attr(Q4_MMA_KERNEL_F2) || set_smem_attr(Q4_MMA_KERNEL_P2) ||
             set_smem_attr(Q4_STACK_KERNEL) ||
             0)
             rc = fail(h, Q4_ECUDA, "cudaFuncSetAttribute failed");
