@@ -138,12 +138,13 @@ Q4GEMV_API int q4gemv_repack(q4gemv_t h, const void* gguf, void* packed,
  * integers.  Deterministic: the same inputs on the same device give the
  * same bits.
  * For M >= 3 (and M <= 2 with K beyond the CUDA-core kernel's activation
- * staging) the tensor-core kernel runs; a matrix wider than the activation
- * slice one CTA can hold (about 9,700 columns for M <= 8, 6,000 for M <= 16)
- * is covered by several launches over column panels whose sums are added in
- * fp32, in panel order, in an accumulator of M*N floats owned by the handle
- * (preallocated for M*N <= 2^21; a larger first call grows it, which
- * synchronises the device and must not happen during a stream capture). */
+ * staging) the tensor-core kernel runs, as a grid of P column panels whose
+ * fp32 sums a second small kernel adds in panel order (P = 1 for large N and
+ * K up to about 6,000 columns; more panels for narrow N, so a CTA stages a
+ * short activation slice, and for wider K).  The panel sums live in a buffer
+ * of P*M*N floats owned by the handle (preallocated for P*M*N <= 2^21; a
+ * larger first call grows it, which synchronises the device and must not
+ * happen during a stream capture). */
 Q4GEMV_API int q4gemv_run(q4gemv_t h, const void* W_packed, const void* x, void* y,
                int M, int64_t N, int64_t K, q4gemv_stream_t stream);
 

@@ -28,27 +28,66 @@
 
 namespace q4 {
 
-// One launch covers a column panel of the matrix: blocks [p0, p0 + KBv) of
-// every row (the whole row when KBv == KB).  Its segments are numbered in
-// panel order, v = t * KBv + j for block p0 + j of tile t, and split flat over
-// the launch's warps.  A matrix too wide for one CTA's activation staging is
-// covered by several panel launches whose sums are added in panel order in
-// fp32 (mode 1: yacc = sum, 2: yacc += sum, 3: y = f16(yacc + sum)).
+// The launch is a grid of P column panels (blockIdx.y) × CTAs (blockIdx.x).
+// Panel p covers blocks [p0, p0 + KBv) of every row (p0 = p * KBv; the last
+// panel takes what is left); its segments are numbered in panel order,
+// v = t * KBv + j for block p0 + j of tile t, and split flat over the panel's
+// warps.  With one panel the outputs are written as f16; with several, each
+// panel writes its fp32 sums to ypart[p] and panel_reduce_kernel adds them in
+// panel order.  Narrow panels let a CTA stage a short activation slice for
+// many rows, and make matrices wider than one CTA's staging possible.
 struct MmaArgs {
     const uint8_t* W;    // packed matrix (segments of 576 bytes)
     const __half* x;     // [M][K]
     __half* y;           // [M][N]
-    float* ws;           // [G][2][16][32] split-tile partials
-    int* cnt;            // [T] arrival counters, zero between calls
+    float* ws;           // per panel: [G][2][16][32] warp partials, [CTAs][2][16][32] CTA partials
+    int* cnt;            // per panel: [T] arrival counters, zero between calls
     int* err;
-    float* yacc;         // [M][N] fp32 sum of earlier panels (modes 1..3)
+    float* ypart;        // [P][M][N] fp32 panel sums (P > 1)
     int64_t N;
-    int K, KB, T, S, G;  // S = T * KBv
+    int K, KB, T, S, G;  // S = T * KBv; G: the panel's warps that own segments
     int KBv, p0;         // panel: blocks per tile, first block
-    int mode;            // 0: y = f16(sum); 1..3: panel modes above
     int M;               // 1..16 (columns >= M are zero-padded)
     SplitConsts sc;      // make_split(S, G)
+    int P;               // panels
+    int S_last, G_last;  // the last panel's segments, warps and split
+    SplitConsts sc_last;
+    int64_t ws_panel;    // floats of ws per panel
 };
+
+// This CTA's view of the launch: its panel's geometry, split and slices of
+// the scratch.
+__device__ __forceinline__ MmaArgs panel_view(const MmaArgs& in) {
+    MmaArgs a = in;
+    const int p = blockIdx.y;
+    if (in.P > 1) {
+        const bool last = p == in.P - 1;
+        a.p0 = p * in.KBv;
+        if (last) {
+            a.KBv = in.KB - a.p0;
+            a.S = in.S_last;
+            a.G = in.G_last;
+            a.sc = in.sc_last;
+        }
+        a.ws = in.ws + (size_t)p * in.ws_panel;
+        a.cnt = in.cnt + (size_t)p * in.T;
+        a.ypart = in.ypart + (size_t)p * in.M * in.N;
+    }
+    return a;
+}
+
+// y = f16(sum of the panels' fp32 sums, in panel order).
+static __global__ void __launch_bounds__(256) panel_reduce_kernel(const float* __restrict__ part,
+                                                                __half* __restrict__ y, int P,
+                                                                int64_t MN) {
+    pdl_wait();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < MN; i += stride) {
+        float sum = 0.f;
+        for (int p = 0; p < P; ++p) sum += part[(size_t)p * MN + i];
+        y[i] = __float2half_rn(sum);
+    }
+}
 
 // A warp's ring over a panel: stage k holds C consecutive panel segments of
 // the warp's run [s0, s1), filled by one bulk copy per contiguous piece (a
@@ -152,7 +191,8 @@ __device__ __forceinline__ CodePairs unpack_pairs(uint32_t w) {
 }
 
 template <int NT8, int WARPS, int R, int C>
-__global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a) {
+__global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a_in) {
+    const MmaArgs a = panel_view(a_in);
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[WARPS * R];
     constexpr int NT = WARPS * 32;
@@ -240,10 +280,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
     // A finished output (all blocks of this panel summed).
     auto emit = [&](int col, int64_t row, float v) {
         const size_t o = (size_t)col * a.N + row;
-        if (a.mode == 0) a.y[o] = __float2half_rn(v);
-        else if (a.mode == 1) a.yacc[o] = v;
-        else if (a.mode == 2) a.yacc[o] = a.yacc[o] + v;
-        else a.y[o] = __float2half_rn(a.yacc[o] + v);
+        if (a.P == 1) a.y[o] = __float2half_rn(v);
+        else a.ypart[o] = v;
     };
 
     // Output (row, column) held by acc[tt][nt][i]:

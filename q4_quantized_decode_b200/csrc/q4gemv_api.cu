@@ -22,11 +22,8 @@ constexpr int kThreads = kWarps * 32;
 // Per-warp TMA ring (stages x segments per stage) of each kernel.
 constexpr int kR1 = 3, kC1 = 6;            // M = 1 and the decode step
 constexpr int kR2 = 2, kC2 = 4;            // M = 2
-// Tensor-core kernel: for each vector group (M <= 8, M <= 16) a deeper ring
-// used when a whole row's activation slice still fits beside it ("full"), and
-// a shallower one that leaves room for wider column panels ("panel").
-constexpr int kRmF1 = 2, kCmF1 = 7, kRmP1 = 2, kCmP1 = 4;   // M <= 8
-constexpr int kRmF2 = 2, kCmF2 = 3, kRmP2 = 2, kCmP2 = 2;   // M <= 16
+constexpr int kRm1 = 2, kCm1 = 7;          // tensor-core kernel, M <= 8
+constexpr int kRm2 = 2, kCm2 = 3;          // tensor-core kernel, M <= 16
 constexpr int kMinSegsPerWarp = 4;         // small problems use fewer warps
 constexpr int kMaxTiles = Q4GEMV_MAX_N / 32;
 constexpr size_t kMaxDynSmem = 224 * 1024;   // opt-in dynamic shared memory per CTA
@@ -34,10 +31,8 @@ constexpr size_t kYaccPrealloc = (size_t)1 << 21;   // fp32 panel accumulator fl
 
 #define Q4_DP2A_KERNEL_1 q4::gemv_dp2a_kernel<1, kWarps, kR1, kC1>
 #define Q4_DP2A_KERNEL_2 q4::gemv_dp2a_kernel<2, kWarps, kR2, kC2>
-#define Q4_MMA_KERNEL_F1 q4::gemv_mma_kernel<1, kWarps, kRmF1, kCmF1>
-#define Q4_MMA_KERNEL_P1 q4::gemv_mma_kernel<1, kWarps, kRmP1, kCmP1>
-#define Q4_MMA_KERNEL_F2 q4::gemv_mma_kernel<2, kWarps, kRmF2, kCmF2>
-#define Q4_MMA_KERNEL_P2 q4::gemv_mma_kernel<2, kWarps, kRmP2, kCmP2>
+#define Q4_MMA_KERNEL_1 q4::gemv_mma_kernel<1, kWarps, kRm1, kCm1>
+#define Q4_MMA_KERNEL_2 q4::gemv_mma_kernel<2, kWarps, kRm2, kCm2>
 #define Q4_STACK_KERNEL q4::stack_kernel<kWarps, kR1, kC1>
 // Largest input of a GEMV in the persistent step (its staging holds up to
 // kStackXChunks 16-byte chunks per thread).
@@ -80,7 +75,8 @@ struct q4gemv_ctx {
     int fault = kFaultNone;
     float* ws = nullptr;          // [ws_warps][2][MAX_M][32] fp32
     int ws_warps = 0;
-    int* cnt = nullptr;           // [kMaxTiles]
+    int* cnt = nullptr;           // arrival counters, zero between calls
+    int64_t cnt_elems = 0;
     int* err = nullptr;           // device error word
     __half* act = nullptr;        // stack intermediates
     size_t act_elems = 0;
@@ -228,22 +224,20 @@ int ensure_ws(q4gemv_ctx* h, int warps, cudaStream_t st) {
     return Q4_OK;
 }
 
-// Ring bytes of the tensor-core kernel (nt8 = 1: up to 8 vectors, 2: up to
-// 16; full: the deeper ring).
-size_t mma_ring(int nt8, bool full) {
-    if (nt8 == 1) return full ? q4::ring_bytes(kWarps, kRmF1, kCmF1) : q4::ring_bytes(kWarps, kRmP1, kCmP1);
-    return full ? q4::ring_bytes(kWarps, kRmF2, kCmF2) : q4::ring_bytes(kWarps, kRmP2, kCmP2);
+// Ring bytes of the tensor-core kernel (nt8 = 1: up to 8 vectors, 2: up to 16).
+size_t mma_ring(int nt8) {
+    return nt8 == 1 ? q4::ring_bytes(kWarps, kRm1, kCm1) : q4::ring_bytes(kWarps, kRm2, kCm2);
 }
 
-// Largest block count one CTA may stage beside the given ring.
-int mma_xcap(int nt8, bool full) {
-    const size_t ring = mma_ring(nt8, full);
+// Largest block count one CTA may stage beside the ring.
+int mma_xcap(int nt8) {
+    const size_t ring = mma_ring(nt8);
     int xcap = 1;
     while (ring + q4::gemv_mma_smem_bytes(nt8, xcap + 1) <= kMaxDynSmem) ++xcap;
     return xcap;
 }
 
-// fp32 accumulator of the column panels of a wide tensor-core GEMV.
+// fp32 panel sums of a tensor-core GEMV run as several column panels.
 int ensure_yacc(q4gemv_ctx* h, size_t floats, cudaStream_t st) {
     if (floats <= h->yacc_floats) return Q4_OK;
     if (h->fault == kFaultAlloc) return fail(h, Q4_EFAULTINJ, "injected allocation failure");
@@ -252,76 +246,108 @@ int ensure_yacc(q4gemv_ctx* h, size_t floats, cudaStream_t st) {
     h->yacc = nullptr;
     h->yacc_floats = 0;
     if (cudaMalloc(&h->yacc, floats * sizeof(float)) != cudaSuccess)
-        return fail(h, Q4_ENOMEM, "panel accumulator of %zu floats failed", floats);
+        return fail(h, Q4_ENOMEM, "panel sums of %zu floats failed", floats);
     h->yacc_floats = floats;
     return Q4_OK;
 }
 
-// Launch one GEMV on the tensor-core path (any M in 1..16, any K).  When the
-// activation slice of a whole row (KB blocks of 8 or 16 vectors) does not fit
-// beside the ring, the matrix is covered by P column panels of at most xcap
-// blocks, one launch each, summed in panel order in fp32.
+// Arrival counters for `n` (panel, tile) pairs, zero between calls.
+int ensure_cnt(q4gemv_ctx* h, int64_t n, cudaStream_t st) {
+    if (n <= h->cnt_elems) return Q4_OK;
+    if (h->fault == kFaultAlloc) return fail(h, Q4_EFAULTINJ, "injected allocation failure");
+    cudaStreamSynchronize(st);
+    cudaFree(h->cnt);
+    h->cnt = nullptr;
+    h->cnt_elems = 0;
+    if (cudaMalloc(&h->cnt, (size_t)n * sizeof(int)) != cudaSuccess ||
+        cudaMemset(h->cnt, 0, (size_t)n * sizeof(int)) != cudaSuccess)
+        return fail(h, Q4_ENOMEM, "arrival counters for %lld tiles failed", (long long)n);
+    h->cnt_elems = n;
+    return Q4_OK;
+}
+
+// Launch one GEMV on the tensor-core path (any M in 1..16, any K) as a grid
+// of P column panels × CTAs.  P makes every panel fit one CTA's activation
+// staging and keeps the staged slice (panel width × 8 or 16 vectors × 64 B)
+// at most half the weight bytes a CTA streams; P > 1 adds a reduce launch.
 int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M, int64_t N,
                     int64_t K, cudaStream_t st) {
     if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
     const int nt8 = M <= 8 ? 1 : 2;
     const int KB = (int)(K / 32);
     const int T = (int)((N + 31) / 32);
-    // The deeper ring when a whole row's activation slice fits beside it,
-    // else the shallower one with wider panels.
-    const bool full = KB <= mma_xcap(nt8, true);
-    const int xcap = mma_xcap(nt8, full);
-    const int P = (KB + xcap - 1) / xcap;
-    const int Wf = (KB + P - 1) / P;                 // panel width (the last may be narrower)
+    const int xcap = mma_xcap(nt8);
+    int64_t P = (KB + xcap - 1) / xcap;
+    // staging per CTA <= half its weights: P >= 2 * 64 * vecs * sms / (576 * T)
+    const int64_t p_ratio = (2 * 64 * 8 * nt8 * (int64_t)h->sms + 576 * (int64_t)T - 1) / (576 * (int64_t)T);
+    if (P < p_ratio) P = p_ratio;
+    if (P > KB) P = KB;
+    if (P > h->sms) P = h->sms;
+    const int Wf = (int)((KB + P - 1) / P);          // panel width
+    P = (KB + Wf - 1) / Wf;                          // no empty panel
+    const int Wl = KB - (int)(P - 1) * Wf;           // the last panel's width
+    int64_t cpp = h->sms / P;                        // CTAs per panel: about one wave in all
+    const int64_t S = (int64_t)T * Wf, S_last = (int64_t)T * Wl;
+    const int64_t cap = S_last / (kWarps * kMinSegsPerWarp);
+    if (cpp > cap) cpp = cap;
+    if (cpp < 1) cpp = 1;
+    const int64_t Gmax = cpp * kWarps;
+    const int64_t G = Gmax < S ? Gmax : S, G_last = Gmax < S_last ? Gmax : S_last;
+    int rc = ensure_ws(h, (int)(P * (Gmax + cpp)), st);
+    if (rc != Q4_OK) return rc;
+    rc = ensure_cnt(h, P * T, st);
+    if (rc != Q4_OK) return rc;
     if (P > 1) {
-        const int rc = ensure_yacc(h, (size_t)M * (size_t)N, st);
+        rc = ensure_yacc(h, (size_t)P * M * (size_t)N, st);
         if (rc != Q4_OK) return rc;
     }
-    for (int p = 0; p < P; ++p) {
-        const int p0 = p * Wf;
-        const int KBv = KB - p0 < Wf ? KB - p0 : Wf;
-        const int64_t S = (int64_t)T * KBv;
-        // One wave, fewer CTAs for small problems: any run length fits, since
-        // a CTA stages at most KBv <= xcap blocks.
-        int64_t ctas = h->sms;
-        const int64_t cap = S / (kWarps * kMinSegsPerWarp);
-        if (ctas > cap) ctas = cap < 1 ? 1 : cap;
-        int64_t G = ctas * kWarps;
-        if (G > S) G = S;
-        // warp partials [G][2][16][32], then CTA partials [ctas][2][16][32]
-        const int rc = ensure_ws(h, (int)(G + ctas), st);
-        if (rc != Q4_OK) return rc;
-        q4::MmaArgs a;
-        a.W = static_cast<const uint8_t*>(W);
-        a.x = x;
-        a.y = y;
-        a.ws = h->ws;
-        a.cnt = h->cnt;
-        a.err = h->err;
-        a.yacc = h->yacc;
-        a.N = N;
-        a.K = (int)K;
-        a.KB = KB;
-        a.T = T;
-        a.S = (int)S;
-        a.G = (int)G;
-        a.KBv = KBv;
-        a.p0 = p0;
-        a.mode = P == 1 ? 0 : (p == 0 ? 1 : (p == P - 1 ? 3 : 2));
-        a.M = M;
-        a.sc = q4::make_split(a.S, a.G);
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)ctas);
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = mma_ring(nt8, full) + q4::gemv_mma_smem_bytes(nt8, KBv);
-        cfg.stream = st;
-        cfg.numAttrs = 0;
-        cudaError_t e;
-        if (nt8 == 1)
-            e = full ? cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_F1, a) : cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_P1, a);
-        else
-            e = full ? cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_F2, a) : cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_P2, a);
-        if (e != cudaSuccess) return cuda_fail(h, e, "gemv (mma) launch");
+    q4::MmaArgs a;
+    a.W = static_cast<const uint8_t*>(W);
+    a.x = x;
+    a.y = y;
+    a.ws = h->ws;
+    a.cnt = h->cnt;
+    a.err = h->err;
+    a.ypart = h->yacc;
+    a.N = N;
+    a.K = (int)K;
+    a.KB = KB;
+    a.T = T;
+    a.S = (int)S;
+    a.G = (int)G;
+    a.KBv = Wf;
+    a.p0 = 0;
+    a.M = M;
+    a.sc = q4::make_split(a.S, a.G);
+    a.P = (int)P;
+    a.S_last = (int)S_last;
+    a.G_last = (int)G_last;
+    a.sc_last = q4::make_split(a.S_last, a.G_last);
+    a.ws_panel = (Gmax + cpp) * 2 * 16 * 32;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cpp, (unsigned)P);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = mma_ring(nt8) + q4::gemv_mma_smem_bytes(nt8, Wf);
+    cfg.stream = st;
+    cfg.numAttrs = 0;
+    cudaError_t e = nt8 == 1 ? cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_1, a)
+                             : cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_2, a);
+    if (e != cudaSuccess) return cuda_fail(h, e, "gemv (mma) launch");
+    if (P > 1) {
+        const int64_t MN = (int64_t)M * N;
+        int64_t blocks = (MN + 255) / 256;
+        if (blocks > (int64_t)h->sms * 8) blocks = (int64_t)h->sms * 8;
+        cudaLaunchConfig_t rcfg = {};
+        rcfg.gridDim = dim3((unsigned)blocks);
+        rcfg.blockDim = dim3(256);
+        rcfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        rcfg.attrs = attr;
+        rcfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&rcfg, q4::panel_reduce_kernel, (const float*)h->yacc, y, (int)P, MN);
+        if (e != cudaSuccess) return cuda_fail(h, e, "panel reduce launch");
     }
     return Q4_OK;
 }
@@ -432,8 +458,10 @@ int q4gemv_create(q4gemv_t* out, int device) {
             cudaMalloc(&h->xq, 2 * q4::stack_xq_half_bytes(kStackKmax)) != cudaSuccess ||
             cudaMalloc(&h->yacc, kYaccPrealloc * sizeof(float)) != cudaSuccess)
             rc = fail(h, Q4_ENOMEM, "workspace allocation failed");
-        else
+        else {
             h->yacc_floats = kYaccPrealloc;
+            h->cnt_elems = kMaxTiles;
+        }
         const char* mode = getenv("Q4GEMV_STACK_MODE");
         if (mode && !strcmp(mode, "kernels")) h->stack_mode = kStackKernels;
     }
@@ -444,8 +472,7 @@ int q4gemv_create(q4gemv_t* out, int device) {
     }
     if (rc == Q4_OK) {
         if (set_smem_attr(Q4_DP2A_KERNEL_1) || set_smem_attr(Q4_DP2A_KERNEL_2) ||
-            set_smem_attr(Q4_MMA_KERNEL_F1) || set_smem_attr(Q4_MMA_KERNEL_P1) ||
-            set_smem_attr(Q4_MMA_KERNEL_F2) || set_smem_attr(Q4_MMA_KERNEL_P2) ||
+            set_smem_attr(Q4_MMA_KERNEL_1) || set_smem_attr(Q4_MMA_KERNEL_2) ||
             set_smem_attr(Q4_STACK_KERNEL) ||
             0)
             rc = fail(h, Q4_ECUDA, "cudaFuncSetAttribute failed");
