@@ -239,21 +239,27 @@ __device__ __forceinline__ void quant_lane_store(float v, int b, int16_t* xq, ui
 }
 
 // Unit-RMS scale from the nb block sums of squares (shared or global
-// memory, any warp): lane l adds blocks l, l + 32, ... (two interleaved
-// accumulators, joined), then the lanes in an xor tree; every lane returns it.
+// memory, any warp; every lane returns it).  Lane l takes blocks l + 32j in
+// rounds of eight j (loads issued together, zeros past nb), each round summed
+// in a fixed three-level tree and added to the lane's sum in round order;
+// then the lanes in an xor tree.
 __device__ __forceinline__ float unit_rms_scale(const float* sq, int nb, int K) {
     const int lane = threadIdx.x & 31;
-    float a0 = 0.f, a1 = 0.f;
-    int t = lane;
-    for (; t + 32 < nb; t += 64) {
-        a0 = __fadd_rn(a0, sq[t]);
-        a1 = __fadd_rn(a1, sq[t + 32]);
-    }
-    if (t < nb) a0 = __fadd_rn(a0, sq[t]);
-    float a = __fadd_rn(a0, a1);
+    float acc = 0.f;
+    for (int j0 = 0; j0 * 32 < nb; j0 += 8) {
+        float v[8];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, o));
-    return renorm_scale(a, K);
+        for (int u = 0; u < 8; ++u) {
+            const int t = lane + 32 * (j0 + u);
+            v[u] = t < nb ? sq[t] : 0.f;
+        }
+        const float a0 = __fadd_rn(v[0], v[1]), a1 = __fadd_rn(v[2], v[3]);
+        const float a2 = __fadd_rn(v[4], v[5]), a3 = __fadd_rn(v[6], v[7]);
+        acc = __fadd_rn(acc, __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3)));
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+    return renorm_scale(acc, K);
 }
 
 // Activation staging for the M <= 2 kernel, all threads of the CTA.  Thread

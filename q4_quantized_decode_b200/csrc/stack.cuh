@@ -329,9 +329,8 @@ __device__ __forceinline__ bool grid_wait(int* sync, int target, int* err, int* 
         *flag_smem = ok;
     }
     __syncthreads();
-    const bool ok = *flag_smem != 0;
-    __syncthreads();
-    return ok;
+    // flag_smem is written again only after the CTA's next barriers.
+    return *flag_smem != 0;
 }
 
 template <int WARPS, int R, int C>
