@@ -51,6 +51,10 @@ def _configure(lib):
     lib.oracle_repack.restype = None
     lib.oracle_renorm.argtypes = [vp, i64, vp]
     lib.oracle_renorm.restype = None
+    lib.oracle_q8_gemv.argtypes = [vp, i64, i64, vp, i64, vp]
+    lib.oracle_q8_gemv.restype = None
+    lib.oracle_repack_q8.argtypes = [vp, i64, i64, vp]
+    lib.oracle_repack_q8.restype = None
     lib.oracle_unit_rms_scale.argtypes = [vp, i64]
     lib.oracle_unit_rms_scale.restype = ctypes.c_double
     lib.oracle_round_f16.argtypes = [vp, i64, vp]
@@ -100,17 +104,25 @@ def f64_to_f16(v) -> np.ndarray:
 def q4_gemv(rows: np.ndarray, K: int, x: np.ndarray, threads: int = 1) -> np.ndarray:
     """y[M][nrows] (fp64) for GGUF rows (nrows, K/32*18) uint8 and x[M][K]
     f16 bit patterns.  ``threads`` > 1 splits the rows across threads."""
-    lib = _load()
+    return _gemv(_load().oracle_q4_gemv, 18, rows, K, x, threads)
+
+
+def q8_gemv(rows: np.ndarray, K: int, x: np.ndarray, threads: int = 1) -> np.ndarray:
+    """As q4_gemv, for GGUF Q8_0 rows (nrows, K/32*34) uint8."""
+    return _gemv(_load().oracle_q8_gemv, 34, rows, K, x, threads)
+
+
+def _gemv(fn, block_bytes: int, rows: np.ndarray, K: int, x: np.ndarray, threads: int) -> np.ndarray:
     rows = np.ascontiguousarray(rows, dtype=np.uint8)
     x = np.ascontiguousarray(np.atleast_2d(x), dtype=np.uint16)
     M = x.shape[0]
     assert x.shape[1] == K and K % 32 == 0
-    rb = (K // 32) * 18
+    rb = (K // 32) * block_bytes
     nrows = rows.size // rb
     assert rows.size == nrows * rb
     y = np.empty((M, nrows), dtype=np.float64)
     if threads <= 1 or nrows < 2 * threads:
-        lib.oracle_q4_gemv(rows.ctypes.data, nrows, K, x.ctypes.data, M, y.ctypes.data)
+        fn(rows.ctypes.data, nrows, K, x.ctypes.data, M, y.ctypes.data)
         return y
     # partition rows; each worker writes its own [M][chunk] block
     bounds = np.linspace(0, nrows, threads + 1).astype(np.int64)
@@ -120,8 +132,7 @@ def q4_gemv(rows: np.ndarray, K: int, x: np.ndarray, threads: int = 1) -> np.nda
     def work(i):
         r0, r1 = int(bounds[i]), int(bounds[i + 1])
         if r1 > r0:
-            lib.oracle_q4_gemv(rows.ctypes.data + r0 * rb, r1 - r0, K,
-                               x.ctypes.data, M, parts[i].ctypes.data)
+            fn(rows.ctypes.data + r0 * rb, r1 - r0, K, x.ctypes.data, M, parts[i].ctypes.data)
 
     with ThreadPoolExecutor(threads) as ex:
         list(ex.map(work, range(threads)))
@@ -138,6 +149,19 @@ def repack(gguf: np.ndarray, N: int, K: int) -> np.ndarray:
     g = np.ascontiguousarray(gguf, dtype=np.uint8)
     assert g.size == N * (K // 32) * 18
     _load().oracle_repack(g.ctypes.data, N, K, out.ctypes.data)
+    return out
+
+
+def packed_bytes_q8(N: int, K: int) -> int:
+    Np = (N + 31) // 32 * 32
+    return Np * (K // 32) * 34
+
+
+def repack_q8(gguf: np.ndarray, N: int, K: int) -> np.ndarray:
+    out = np.empty(packed_bytes_q8(N, K), dtype=np.uint8)
+    g = np.ascontiguousarray(gguf, dtype=np.uint8)
+    assert g.size == N * (K // 32) * 34
+    _load().oracle_repack_q8(g.ctypes.data, N, K, out.ctypes.data)
     return out
 
 

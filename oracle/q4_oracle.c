@@ -126,6 +126,60 @@ void oracle_repack(const uint8_t* gguf, int64_t N, int64_t K, uint8_t* packed) {
     }
 }
 
+/* ---- Q8_0: GGUF's other block format, named by the pages (taozi.news page,
+ * section "支持模型与限制") without a layout.  The plainest reading, GGUF's
+ * Q8_0 block: 34 bytes per 32 weights, an f16 scale d (little-endian) then
+ * 32 signed 8-bit codes; weight j is qs[j] * d. */
+static double q8_0_weight(const uint8_t* row, int64_t k) {
+    const uint8_t* blk = row + (k / 32) * 34;
+    const uint16_t dbits = (uint16_t)(blk[0] | (blk[1] << 8));
+    const double d = oracle_f16_to_f64(dbits);
+    const int q = (int)(int8_t)blk[2 + k % 32];
+    return (double)q * d;
+}
+
+/* As oracle_q4_gemv, for Q8_0 rows of K/32*34 bytes. */
+void oracle_q8_gemv(const uint8_t* rows, int64_t nrows, int64_t K,
+                    const uint16_t* x, int64_t M, double* y) {
+    const int64_t rb = (K / 32) * 34;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t r = 0; r < nrows; ++r) {
+            const uint8_t* row = rows + r * rb;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += q8_0_weight(row, k) * oracle_f16_to_f64(x[m * K + k]);
+            y[m * nrows + r] = acc;
+        }
+    }
+}
+
+/* The packed Q8_0 layout, restated from the library's documented contract:
+ * rows padded to Np = ceil(N/32)*32 (padding rows: codes 0, d = +0), tiles of
+ * 32 rows, segment s = t*KB + b in the 1088 bytes from 1088*s; row
+ * n = 32t + g + 8i (g in [0,8), i in [0,4)):
+ *   byte 1088*s + 32*(4g + c) + 8i + e      <-  qs[4c + e]        (c, e in [0,4))
+ *   byte 1088*s + 32*(4g + c) + 8i + 4 + e  <-  qs[16 + 4c + e]
+ *   bytes 1088*s + 1024 + 8g + 2i + {0,1}   <-  d (little-endian f16)       */
+void oracle_repack_q8(const uint8_t* gguf, int64_t N, int64_t K, uint8_t* packed) {
+    const int64_t KB = K / 32;
+    const int64_t Np = (N + 31) / 32 * 32;
+    for (int64_t n = 0; n < Np; ++n) {
+        const int64_t t = n / 32, r = n % 32;
+        const int64_t g = r % 8, i = r / 8;
+        for (int64_t b = 0; b < KB; ++b) {
+            uint8_t* seg = packed + 1088 * (t * KB + b);
+            uint8_t blk[34];
+            for (int h = 0; h < 34; ++h) blk[h] = (n < N) ? gguf[(n * KB + b) * 34 + h] : 0x00;
+            for (int64_t c = 0; c < 4; ++c)
+                for (int64_t e = 0; e < 4; ++e) {
+                    seg[32 * (4 * g + c) + 8 * i + e] = blk[2 + 4 * c + e];
+                    seg[32 * (4 * g + c) + 8 * i + 4 + e] = blk[2 + 16 + 4 * c + e];
+                }
+            for (int64_t h = 0; h < 2; ++h) seg[1024 + 8 * g + 2 * i + h] = blk[h];
+        }
+    }
+}
+
 /* Unit-RMS scale of an f16 vector: s = sum v_i^2 (fp64), 1 / sqrt(s / len);
  * 0 for an all-zero vector (which then stays zero). */
 double oracle_unit_rms_scale(const uint16_t* v, int64_t len) {

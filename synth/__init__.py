@@ -61,6 +61,8 @@ def _load():
             lib.synth_q4_0_rows.argtypes = [u64, u64, i64, i64, i64, vp]
             lib.synth_q4_0_rows.restype = None
             lib.synth_normal_f16.argtypes = [u64, u64, i64, i64, vp]
+            lib.synth_q8_0_rows.argtypes = [u64, u64, i64, i64, i64, vp]
+            lib.synth_q8_0_rows.restype = None
             lib.synth_normal_f16.restype = None
             _lib = lib
     return _lib
@@ -141,6 +143,41 @@ def q4_0_row_list(seed: int, tensor_id: int, K: int, rows) -> np.ndarray:
     for i, r in enumerate(rows):
         lib.synth_q4_0_rows(seed, tensor_id, K, int(r), 1, out[i].ctypes.data)
     return out
+
+
+def q8_0_block_bytes(K: int) -> int:
+    return (K // 32) * 34
+
+
+def q8_0_rows(seed: int, tensor_id: int, K: int, row0: int, nrows: int,
+              threads: int | None = None) -> np.ndarray:
+    """GGUF Q8_0 bytes of rows [row0, row0+nrows) of a K-column matrix,
+    shape (nrows, K/32*34) uint8."""
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    rb = q8_0_block_bytes(K)
+    out = np.empty((nrows, rb), dtype=np.uint8)
+    lib = _load()
+    t = _threads(nrows, threads)
+    if t == 1 or nrows * rb < (1 << 20):
+        lib.synth_q8_0_rows(seed, tensor_id, K, row0, nrows, out.ctypes.data)
+        return out
+    chunk = (nrows + t - 1) // t
+    base = out.ctypes.data
+
+    def work(i):
+        r0 = i * chunk
+        n = min(chunk, nrows - r0)
+        if n > 0:
+            lib.synth_q8_0_rows(seed, tensor_id, K, row0 + r0, n, base + r0 * rb)
+
+    with ThreadPoolExecutor(t) as ex:
+        list(ex.map(work, range(t)))
+    return out
+
+
+def q8_0_matrix(seed: int, tensor_id: int, N: int, K: int, threads: int | None = None) -> np.ndarray:
+    return q8_0_rows(seed, tensor_id, K, 0, N, threads=threads)
 
 
 def normal_f16(seed: int, tensor_id: int, n: int, i0: int = 0) -> np.ndarray:

@@ -108,6 +108,34 @@ void synth_q4_0_rows(uint64_t seed, uint64_t tensor_id, int64_t K,
     }
 }
 
+/* Rows [row0, row0 + nrows) of a Q8_0 matrix with K columns (K % 32 == 0),
+ * written as GGUF blocks of 34 bytes: f16 d (little-endian), then 32 int8
+ * codes.  d = f16(+-(0.002 + 0.048 u) / 16) (u, sign: draw 5bi) keeps the
+ * weights in the range of the Q4_0 matrices; the codes are the raw bytes of
+ * draws 5bi+1 .. 5bi+4 (uniform over -128..127). */
+void synth_q8_0_rows(uint64_t seed, uint64_t tensor_id, int64_t K,
+                     int64_t row0, int64_t nrows, uint8_t* out) {
+    const uint64_t key = synth_stream_key(seed, tensor_id);
+    const int64_t nb = K / 32;
+    for (int64_t r = 0; r < nrows; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const uint64_t bi = (uint64_t)(row0 + r) * (uint64_t)nb + (uint64_t)b;
+            const uint64_t r0 = synth_splitmix64_at(key, 5 * bi);
+            const double u = (double)(r0 & ((1ULL << 53) - 1)) * 0x1p-53;
+            double mag = (0.002 + 0.048 * u) / 16.0;
+            if (r0 >> 63) mag = -mag;
+            const uint16_t d = synth_f64_to_f16(mag);
+            uint8_t* blk = out + (r * nb + b) * 34;
+            blk[0] = (uint8_t)(d & 0xFF);
+            blk[1] = (uint8_t)(d >> 8);
+            for (int w = 0; w < 4; ++w) {
+                const uint64_t rw = synth_splitmix64_at(key, 5 * bi + 1 + (uint64_t)w);
+                for (int j = 0; j < 8; ++j) blk[2 + 8 * w + j] = (uint8_t)(rw >> (8 * j));
+            }
+        }
+    }
+}
+
 /* Elements [i0, i0 + n) of an f16 N(0,1) vector. */
 void synth_normal_f16(uint64_t seed, uint64_t tensor_id, int64_t i0, int64_t n,
                       uint16_t* out) {

@@ -7,6 +7,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_pins as pins
+from tests import test_oracle_q8_pins as q8pins
 
 SRC = open(os.path.join(os.path.dirname(oracle.__file__), "q4_oracle.c")).read()
 
@@ -29,6 +30,17 @@ MUTANTS = {
     "repack_pad_code": ("(h < 2 ? 0x00 : 0x88)", "(h < 2 ? 0x00 : 0x00)"),
     "renorm_no_len": ("sqrt(s / (double)len)", "sqrt(s)"),
     "rne_ties_up": ("(frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0))", "(frac >= 0.5)"),
+}
+
+# Planted in the Q8_0 part; caught by the Q8_0 pins.
+Q8_MUTANTS = {
+    "q8_codes_unsigned": ("(int)(int8_t)blk[2 + k % 32]", "(int)blk[2 + k % 32]"),
+    "q8_block_stride_32": ("row + (k / 32) * 34", "row + (k / 32) * 32"),
+    "q8_code_offset_1": ("blk[2 + k % 32]", "blk[1 + k % 32]"),
+    "q8_repack_halves_swapped": ("seg[32 * (4 * g + c) + 8 * i + 4 + e] = blk[2 + 16 + 4 * c + e]",
+                                 "seg[32 * (4 * g + c) + 8 * i + 4 + e] = blk[2 + 4 * c + e]"),
+    "q8_repack_scale_slot": ("seg[1024 + 8 * g + 2 * i + h]", "seg[1024 + 8 * i + 2 * g + h]"),
+    "q8_repack_segment_stride": ("packed + 1088 * (t * KB + b)", "packed + 1024 * (t * KB + b)"),
 }
 
 PIN_TESTS = [
@@ -70,3 +82,35 @@ def test_mutant_is_caught(name, tmp_path):
     finally:
         oracle._restore_library(prev)
     assert failed, f"mutant {name} survived every pin"
+
+
+Q8_PIN_TESTS = [
+    q8pins.test_zero_codes_give_zero,
+    q8pins.test_unit_vectors_pin_code_order_sign_and_scale,
+    q8pins.test_scale_linearity_powers_of_two,
+    q8pins.test_exact_rationals_brute_force,
+    q8pins.test_dense_equivalence_synthetic_matrix,
+    q8pins.test_repack_q8_round_trip_and_padding,
+]
+
+
+@pytest.mark.parametrize("name", sorted(Q8_MUTANTS))
+def test_q8_mutant_is_caught(name, tmp_path):
+    old, new = Q8_MUTANTS[name]
+    assert old in SRC, f"mutation anchor for {name} no longer in the oracle"
+    src = tmp_path / "mut.c"
+    src.write_text(SRC.replace(old, new, 1))
+    so = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+                           str(src), "-o", str(so), "-lm"])
+    prev = oracle._swap_library(str(so))
+    try:
+        caught = 0
+        for t in Q8_PIN_TESTS:
+            try:
+                t()
+            except (AssertionError, ValueError, IndexError):
+                caught += 1
+        assert caught > 0, f"no Q8_0 pin catches mutant {name}"
+    finally:
+        oracle._restore_library(prev)
