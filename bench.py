@@ -410,22 +410,29 @@ def run_case(args):
     import q4_quantized_decode_b200 as q4
     N, K = (int(v) for v in args.shape.lower().split("x"))
     M = args.M
+    q8 = args.format == "q8_0"
     eng = q4.Q4Gemv(0)
     seed = synth.config_seed(args.config_seed)
-    gguf = synth.q4_0_matrix(seed, synth.weight_id(0), N, K)
-    W0 = eng.repack(torch.from_numpy(gguf.reshape(-1)).cuda(), N, K)
+    if q8:
+        gguf = synth.q8_0_matrix(seed, synth.weight_id(0), N, K)
+        W0 = eng.repack_q8_0(torch.from_numpy(gguf.reshape(-1)).cuda(), N, K)
+        run = eng.run_q8_0
+    else:
+        gguf = synth.q4_0_matrix(seed, synth.weight_id(0), N, K)
+        W0 = eng.repack(torch.from_numpy(gguf.reshape(-1)).cuda(), N, K)
+        run = eng.run
     l2 = torch.cuda.get_device_properties(0).L2_cache_size
     R = args.rotate or max(2, -(-4 * l2 // W0.numel()))
     mats = [W0] + [W0.clone() for _ in range(R - 1)]
     x = torch.from_numpy(synth.activations(seed, M, K).view(np.float16)).cuda()
     y = torch.empty(M, N, dtype=torch.float16, device="cuda")
-    eng.run(mats[0], x, N, K, out=y)
+    run(mats[0], x, N, K, out=y)
     torch.cuda.synchronize()
     s = torch.cuda.Stream()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
         for W in mats:
-            eng.run(W, x, N, K, out=y)
+            run(W, x, N, K, out=y)
     for _ in range(args.warmup):
         g.replay()
     torch.cuda.synchronize()
@@ -438,9 +445,9 @@ def run_case(args):
     if eng.sync_status() != q4.Q4_OK:
         raise RuntimeError("device status")
     us = e0.elapsed_time(e1) * 1e3 / (args.steps * R)
-    nbytes = N * (K // 32) * 18 + 2 * M * (K + N)
+    nbytes = N * (K // 32) * (34 if q8 else 18) + 2 * M * (K + N)
     peak, kind = measured_peaks()
-    print(json.dumps({"case": f"gemv M={M} {N}x{K}", "N": N, "K": K, "M": M, "rotate": R,
+    print(json.dumps({"case": f"gemv {args.format} M={M} {N}x{K}", "N": N, "K": K, "M": M, "rotate": R,
                       "us_per_launch": us, "GB/s": nbytes / us / 1e3,
                       "frac_of_peak": nbytes / us / 1e3 / peak, "peak": peak, "peak_kind": kind,
                       "rows_per_s": N / us * 1e6, "tflops": 2 * M * N * K / us / 1e6,
@@ -474,6 +481,7 @@ def main():
     ap.add_argument("--M", type=int, default=1)
     ap.add_argument("--rotate", type=int, default=0, help="matrix copies in rotation (0: > 4x L2)")
     ap.add_argument("--config-seed", type=int, default=2)
+    ap.add_argument("--format", choices=["q4_0", "q8_0"], default="q4_0", help="weights of --case gemv")
     ap.add_argument("--layers", type=int, default=64, help="layers of the step (profiling only)")
     args = ap.parse_args()
     if args.layers != 64:

@@ -148,6 +148,45 @@ Q4GEMV_API int q4gemv_repack(q4gemv_t h, const void* gguf, void* packed,
 Q4GEMV_API int q4gemv_run(q4gemv_t h, const void* W_packed, const void* x, void* y,
                int M, int64_t N, int64_t K, q4gemv_stream_t stream);
 
+/* ---- Q8_0 matrices (the other GGUF format the pages name: taozi.news page,
+ * section "支持模型与限制"; layout from GGUF).  A row holds K/32 blocks of 34
+ * bytes: an f16 scale d (little-endian), then 32 signed 8-bit codes; weight
+ * j of a block is qs[j] * d. */
+
+/* Bytes of a GGUF Q8_0 matrix: N * (K/32) * 34; 0 if the shape is invalid. */
+Q4GEMV_API size_t q4gemv_q8_0_gguf_bytes(int64_t N, int64_t K);
+
+/* Bytes of the packed Q8_0 matrix: Np * (K/32) * 34, Np = ceil(N/32)*32; 0 if
+ * the shape is invalid.  Packed layout: rows padded to Np (padding rows hold
+ * codes 0 and d = +0), tiles of 32 rows; segment s = t*KB + b (KB = K/32)
+ * holds block b of the rows of tile t in the 1088 bytes from 1088*s; row
+ * n = 32t + g + 8i (g in [0,8), i in [0,4)):
+ *   segment bytes 32*(4g + c) + 8i + e      = qs[4c + e]       (c, e in [0,4))
+ *   segment bytes 32*(4g + c) + 8i + 4 + e  = qs[16 + 4c + e]
+ *   segment bytes 1024 + 8g + 2i, +1        = d (little-endian)
+ * A lane (g, c) of a warp thus finds the codes it multiplies with the
+ * activations' lane group c, for its four rows, in 32 contiguous bytes. */
+Q4GEMV_API size_t q4gemv_q8_0_packed_bytes(int64_t N, int64_t K);
+
+/* One-time repack of a GGUF Q8_0 matrix (arguments and errors as
+ * q4gemv_repack; gguf any alignment >= 2).  Bit-exact. */
+Q4GEMV_API int q4gemv_q8_0_repack(q4gemv_t h, const void* gguf, void* packed,
+                       int64_t N, int64_t K, q4gemv_stream_t stream);
+
+/* Host-only check of q4gemv_q8_0_run's arguments: Q4_EUNSUPPORTED for M
+ * outside {1, 2} or M*K beyond the kernel's activation staging (M*K <=
+ * 36,864 and the shared-memory budget), else as q4gemv_validate. */
+Q4GEMV_API int q4gemv_q8_0_validate(int M, int64_t N, int64_t K, const void* W_packed,
+                         const void* x, const void* y);
+
+/* y[M][N] = W x[M][K]^T for a packed Q8_0 W, M in {1, 2} (buffers as
+ * q4gemv_run).  The activations are converted per 32-column block as for
+ * Q4_0 (exact for the block maximum), each block's dot product with the
+ * 8-bit codes is an exact integer, converted to fp32 once and scaled by d;
+ * fp32 accumulation; y rounded to binary16 once.  Deterministic. */
+Q4GEMV_API int q4gemv_q8_0_run(q4gemv_t h, const void* W_packed, const void* x, void* y,
+                    int M, int64_t N, int64_t K, q4gemv_stream_t stream);
+
 /* One layer's packed matrices for q4gemv_run_stack. */
 typedef struct {
     const void* qkv;      /* qkv_n  x hidden */

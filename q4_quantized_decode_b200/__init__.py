@@ -62,6 +62,11 @@ def _load_library():
         "q4gemv_last_error": ([vp], ctypes.c_char_p),
         "q4gemv_set_fault": ([vp, ctypes.c_char_p], ci),
         "q4gemv_run_noalloc": ([vp, vp, vp, ci, i64, i64, vp], ci),
+        "q4gemv_q8_0_gguf_bytes": ([i64, i64], ctypes.c_size_t),
+        "q4gemv_q8_0_packed_bytes": ([i64, i64], ctypes.c_size_t),
+        "q4gemv_q8_0_repack": ([vp, vp, vp, i64, i64, vp], ci),
+        "q4gemv_q8_0_validate": ([ci, i64, i64, vp, vp, vp], ci),
+        "q4gemv_q8_0_run": ([vp, vp, vp, vp, ci, i64, i64, vp], ci),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
@@ -135,6 +140,26 @@ def q4gemv_run_noalloc(W, x, y, M, N, K, stream) -> int:
     return _lib.q4gemv_run_noalloc(W, x, y, M, N, K, stream)
 
 
+def q4gemv_q8_0_gguf_bytes(N: int, K: int) -> int:
+    return _lib.q4gemv_q8_0_gguf_bytes(N, K)
+
+
+def q4gemv_q8_0_packed_bytes(N: int, K: int) -> int:
+    return _lib.q4gemv_q8_0_packed_bytes(N, K)
+
+
+def q4gemv_q8_0_repack(h, gguf, packed, N, K, stream) -> int:
+    return _lib.q4gemv_q8_0_repack(h, gguf, packed, N, K, stream)
+
+
+def q4gemv_q8_0_validate(M, N, K, W, x, y) -> int:
+    return _lib.q4gemv_q8_0_validate(M, N, K, W, x, y)
+
+
+def q4gemv_q8_0_run(h, W, x, y, M, N, K, stream) -> int:
+    return _lib.q4gemv_q8_0_run(h, W, x, y, M, N, K, stream)
+
+
 def _ptr(t) -> int | None:
     if t is None:
         return None
@@ -193,6 +218,25 @@ class Q4Gemv:
             out = torch.empty((M, N), dtype=torch.float16, device=x.device)
         self._check(q4gemv_run(self.h, _ptr(W_packed), _ptr(x2), _ptr(out), M, N, K,
                                _stream(stream)))
+        return out
+
+    def repack_q8_0(self, gguf, N: int, K: int, out=None, stream=None):
+        """gguf: uint8 CUDA tensor of N*(K/32)*34 bytes -> packed Q8_0 tensor."""
+        import torch
+        if out is None:
+            out = torch.empty(q4gemv_q8_0_packed_bytes(N, K), dtype=torch.uint8, device=gguf.device)
+        self._check(q4gemv_q8_0_repack(self.h, _ptr(gguf), _ptr(out), N, K, _stream(stream)))
+        return out
+
+    def run_q8_0(self, W_packed, x, N: int, K: int, out=None, stream=None):
+        """x: f16 CUDA tensor [M][K] (M <= 2) -> y f16 [M][N] for a packed Q8_0 W."""
+        import torch
+        x2 = x.reshape(-1, K)
+        M = x2.shape[0]
+        if out is None:
+            out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+        self._check(q4gemv_q8_0_run(self.h, _ptr(W_packed), _ptr(x2), _ptr(out), M, N, K,
+                                    _stream(stream)))
         return out
 
     def run_stack(self, layers, x_in, hidden: int, qkv_n: int, ffn: int, x_out=None,

@@ -33,6 +33,17 @@ __device__ __forceinline__ int dp2a_hi(uint32_t a, uint32_t b, int acc) {
     asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(acc));
     return d;
 }
+// The same with signed 8-bit bytes in b.
+__device__ __forceinline__ int dp2a_lo_s8(uint32_t a, uint32_t b, int acc) {
+    int d;
+    asm("dp2a.lo.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(acc));
+    return d;
+}
+__device__ __forceinline__ int dp2a_hi_s8(uint32_t a, uint32_t b, int acc) {
+    int d;
+    asm("dp2a.hi.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(acc));
+    return d;
+}
 
 // Packed fp32 pairs (sm_100 f32x2 pipes): d = a * b + c and d = a * b.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {

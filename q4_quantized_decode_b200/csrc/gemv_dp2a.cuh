@@ -33,8 +33,18 @@
 
 namespace q4 {
 
-constexpr int kSegBytes = 576;       // one segment: 512 bytes of codes, then 64 of scales
+constexpr int kSegBytes = 576;       // one Q4_0 segment: 512 bytes of codes, then 64 of scales
 constexpr int kSegSclOff = 512;
+// Q8_0 segments (32 rows x one block of 32 signed 8-bit codes): 1024 bytes
+// of codes, then the same 64 bytes of scales.  Lane (g, c) finds, for row
+// g + 8i, codes 4c..4c+3 and 16+4c..16+4c+3 in the 8 bytes at 32*(4g+c) + 8i.
+constexpr int kSegBytesQ8 = 1088;
+constexpr int kSegSclOffQ8 = 1024;
+template <bool Q8>
+struct SegFmt {
+    static constexpr int kBytes = Q8 ? kSegBytesQ8 : kSegBytes;
+    static constexpr int kScl = Q8 ? kSegSclOffQ8 : kSegSclOff;
+};
 constexpr int kXChunksPerThread = 9; // activation staging: M*K <= 9 * 8 * threads
 
 struct GemvArgs {
@@ -55,8 +65,8 @@ struct GemvArgs {
 };
 
 // Per-warp ring of R stages of C segments.
-__host__ __device__ constexpr size_t ring_bytes(int warps, int R, int C) {
-    return (size_t)warps * R * C * kSegBytes;
+__host__ __device__ constexpr size_t ring_bytes(int warps, int R, int C, int seg = kSegBytes) {
+    return (size_t)warps * R * C * seg;
 }
 
 // Per warp, two parked tile partials (the first and the last tile of its
@@ -75,8 +85,9 @@ __host__ __device__ constexpr size_t tile_sum_bytes(int K) {
 // activations (2 bytes per element), per block and lane group the pair
 // {-8 * sum X, block scale} (8 bytes, 32 per block), the warp partials, then
 // the block sums of squares of vector 0.
-__host__ __device__ constexpr size_t gemv_dp2a_smem_bytes(int M, int K, int warps, int R, int C) {
-    return ring_bytes(warps, R, C) + (size_t)M * K * 2 + (size_t)M * (K / 32) * 32 +
+__host__ __device__ constexpr size_t gemv_dp2a_smem_bytes(int M, int K, int warps, int R, int C,
+                                                        int seg = kSegBytes) {
+    return ring_bytes(warps, R, C, seg) + (size_t)M * K * 2 + (size_t)M * (K / 32) * 32 +
            warp_partial_bytes(M, warps) + tile_sum_bytes(K);
 }
 
@@ -89,7 +100,7 @@ __host__ __device__ __forceinline__ int xperm_pos(int j) {
 
 // A warp's private ring: stage k holds C consecutive segments of the warp's
 // run [s0, s1), filled by one elected lane with one bulk copy.
-template <int R, int C>
+template <int R, int C, int SEG = kSegBytes>
 struct WarpRing {
     uint32_t stage0;        // shared address of this warp's first stage
     uint64_t* bars;         // R full-barriers
@@ -99,19 +110,19 @@ struct WarpRing {
 
     __device__ void init(uint32_t ring_base, uint64_t* bar_base, int warp, const uint8_t* W, int s0,
                          int s1) {
-        stage0 = ring_base + (uint32_t)warp * R * C * kSegBytes;
+        stage0 = ring_base + (uint32_t)warp * R * C * SEG;
         bars = bar_base + warp * R;
-        src = W + (size_t)s0 * kSegBytes;
+        src = W + (size_t)s0 * SEG;
         nseg = s1 - s0;
         nch = (nseg + C - 1) / C;
     }
-    __device__ uint32_t stage(int k) const { return stage0 + (uint32_t)k * C * kSegBytes; }
+    __device__ uint32_t stage(int k) const { return stage0 + (uint32_t)k * C * SEG; }
     // Lane 0 only.
     __device__ void issue(int ch) const {
         const int k = ch % R;
-        const uint32_t bytes = (uint32_t)min(C, nseg - ch * C) * kSegBytes;
+        const uint32_t bytes = (uint32_t)min(C, nseg - ch * C) * SEG;
         mbar_arrive_expect_tx(bars + k, bytes);
-        bulk_g2s_addr(stage(k), src + (size_t)ch * C * kSegBytes, bytes, bars + k);
+        bulk_g2s_addr(stage(k), src + (size_t)ch * C * SEG, bytes, bars + k);
     }
     __device__ bool wait(int ch) const {
         return mbar_wait_bounded(bars + (ch % R), (uint32_t)((ch / R) & 1), 1u << 22);
@@ -317,8 +328,9 @@ struct QuantOut {
     int nb;
 };
 
-template <int M>
+template <int M, bool Q8 = false>
 struct Dp2aConsumer {
+    static constexpr int SEG = SegFmt<Q8>::kBytes;
     float acc[M][4];
     WarpSplit sp;
     int gw, lane, g, c, r;   // r: the tile row this lane emits
@@ -388,6 +400,10 @@ struct Dp2aConsumer {
     // are at xb and rb: codes and scales from a ring stage, X from the staged
     // activations.  Rows are handled in pairs on the packed fp32x2 pipes.
     __device__ __forceinline__ void segment(uint32_t seg, uint32_t xb, uint32_t rb) {
+        if constexpr (Q8) {
+            segment_q8(seg, xb, rb);
+            return;
+        }
         const uint4 w = lds128(seg + lane * 16);
         const uint2 dd = lds64(seg + kSegSclOff + g * 8);
         const float2 d01 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
@@ -431,6 +447,32 @@ struct Dp2aConsumer {
         }
     }
 
+    // Q8_0 segment: per row, two words of four signed codes (columns 4c.. and
+    // 16+4c..) against the same int16 activation words; the block sum is an
+    // exact integer (|sum| < 2^26) converted to fp32 once.
+    __device__ __forceinline__ void segment_q8(uint32_t seg, uint32_t xb, uint32_t rb) {
+        const uint4 w01 = lds128(seg + lane * 32), w23 = lds128(seg + lane * 32 + 16);
+        const uint2 dd = lds64(seg + kSegSclOffQ8 + g * 8);
+        const float2 d01 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
+        const float2 d23 = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
+        const uint32_t wa[4] = {w01.x, w01.z, w23.x, w23.z};   // codes 4c..4c+3 of rows g + 8i
+        const uint32_t wb[4] = {w01.y, w01.w, w23.y, w23.w};   // codes 16+4c..
+        const float dr[4] = {d01.x, d01.y, d23.x, d23.y};
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const uint4 xq = lds128(xb + (uint32_t)m * xstride);
+            const float sbm = __uint_as_float(lds64(rb + (uint32_t)m * rstride).y);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                int t = dp2a_lo_s8(xq.x, wa[i], 0);
+                t = dp2a_hi_s8(xq.y, wa[i], t);
+                t = dp2a_lo_s8(xq.z, wb[i], t);
+                t = dp2a_hi_s8(xq.w, wb[i], t);
+                acc[m][i] = fmaf((float)t, __fmul_rn(dr[i], sbm), acc[m][i]);
+            }
+        }
+    }
+
     // Next segment of the run (flushing a finished tile first).
     __device__ __forceinline__ void step(const GemvArgs& a, uint32_t seg) {
         if (b == KB) {
@@ -453,13 +495,13 @@ struct Dp2aConsumer {
         if (b + C <= KB) {
 #pragma unroll
             for (int j = 0; j < C; ++j)
-                segment(st + j * kSegBytes, xp + j * 64, rp + j * 32);
+                segment(st + j * SEG, xp + j * 64, rp + j * 32);
             b += C;
             xp += C * 64;
             rp += C * 32;
         } else {
 #pragma unroll
-            for (int j = 0; j < C; ++j) step(a, st + j * kSegBytes);
+            for (int j = 0; j < C; ++j) step(a, st + j * SEG);
         }
     }
 
@@ -564,15 +606,16 @@ __device__ __forceinline__ void combine_ctas_arrive(const GemvArgs& a, int t, in
     }
 }
 
-template <int M, int WARPS, int R, int C>
+template <int M, int WARPS, int R, int C, bool Q8 = false>
 __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs a) {
+    constexpr int SEG = SegFmt<Q8>::kBytes;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[WARPS * R];
 
     const uint32_t smem_base = smem_addr(smem);
-    const uint32_t xs = smem_base + (uint32_t)ring_bytes(WARPS, R, C);   // int16 X, lane order
+    const uint32_t xs = smem_base + (uint32_t)ring_bytes(WARPS, R, C, SEG);   // int16 X, lane order
     const uint32_t rec = xs + (uint32_t)(M * a.K * 2);                  // {-8 sum X, scale}
-    float* park = reinterpret_cast<float*>(smem + ring_bytes(WARPS, R, C) + (size_t)M * a.K * 2 +
+    float* park = reinterpret_cast<float*>(smem + ring_bytes(WARPS, R, C, SEG) + (size_t)M * a.K * 2 +
                                            (size_t)M * a.KB * 32);      // [WARPS][2][M][32]
     float* sq = park + WARPS * 2 * M * 32;                              // block sums of squares
 
@@ -580,8 +623,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
     const int gw = blockIdx.x * WARPS + warp;
     // G <= S, so every warp below G owns at least one segment; warps of the
     // last CTA beyond G only help stage the activations.
-    Dp2aConsumer<M> cons;
-    WarpRing<R, C> ring;
+    Dp2aConsumer<M, Q8> cons;
+    WarpRing<R, C, SEG> ring;
     {
         WarpSplit sp;
         sp.init(gw, a.sc, a.KB);
@@ -618,7 +661,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
         if (n == C) {
             cons.template stage_full<C>(a, st);
         } else {
-            for (int j = 0; j < n; ++j) cons.step(a, st + j * kSegBytes);
+            for (int j = 0; j < n; ++j) cons.step(a, st + j * SEG);
         }
         // Stage fully read: hand it back to the async proxy for the refill.
         __syncwarp();
@@ -700,6 +743,45 @@ __global__ void __launch_bounds__(WARPS * 32, 1) renorm_kernel(const __half* in,
     __shared__ float sq[(kXChunksPerThread * 8 * WARPS * 32) / 32];
     pdl_wait();
     renorm_block<WARPS * 32, kXChunksPerThread, false>(in, out, len, sq, NoFix(), 0u);
+}
+
+// GGUF Q8_0 -> packed layout, one warp per segment (grid-stride): lane
+// (g, c) writes the 32 code bytes of its four rows and lane group 0 the
+// scales.
+static __global__ void __launch_bounds__(256) repack_q8_kernel(const uint8_t* __restrict__ gguf,
+                                                          uint8_t* __restrict__ packed, int64_t N,
+                                                          int KB, int64_t S) {
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t s = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); s < S; s += nwarps) {
+        const int64_t t = s / KB, b = s - t * KB;
+        uint32_t words[8];
+        uint16_t dv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int64_t row = t * 32 + g + 8 * i;
+            if (row < N) {
+                const uint8_t* blk = gguf + (row * KB + b) * 34;
+                // codes start at byte 2 of the block: 2-byte aligned only
+                const uint16_t* h = reinterpret_cast<const uint16_t*>(blk);
+                words[2 * i] = (uint32_t)h[1 + 2 * c] | ((uint32_t)h[2 + 2 * c] << 16);
+                words[2 * i + 1] = (uint32_t)h[9 + 2 * c] | ((uint32_t)h[10 + 2 * c] << 16);
+                dv[i] = h[0];
+            } else {
+                words[2 * i] = words[2 * i + 1] = 0u;
+                dv[i] = 0;
+            }
+        }
+        uint8_t* seg = packed + s * kSegBytesQ8;
+        *reinterpret_cast<uint4*>(seg + lane * 32) = make_uint4(words[0], words[1], words[2], words[3]);
+        *reinterpret_cast<uint4*>(seg + lane * 32 + 16) = make_uint4(words[4], words[5], words[6], words[7]);
+        if (c == 0) {
+            *reinterpret_cast<uint2*>(seg + kSegSclOffQ8 + g * 8) =
+                make_uint2((uint32_t)dv[0] | ((uint32_t)dv[1] << 16),
+                           (uint32_t)dv[2] | ((uint32_t)dv[3] << 16));
+        }
+    }
 }
 
 // GGUF Q4_0 -> packed layout, one warp per segment (grid-stride).

@@ -31,6 +31,11 @@ constexpr size_t kYaccPrealloc = (size_t)1 << 21;   // fp32 panel accumulator fl
 
 #define Q4_DP2A_KERNEL_1 q4::gemv_dp2a_kernel<1, kWarps, kR1, kC1>
 #define Q4_DP2A_KERNEL_2 q4::gemv_dp2a_kernel<2, kWarps, kR2, kC2>
+// Q8_0 (1088-byte segments): stages of three segments, about the bytes of
+// six Q4_0 ones.
+constexpr int kRq1 = 3, kCq1 = 3, kRq2 = 2, kCq2 = 3;
+#define Q4_Q8_KERNEL_1 q4::gemv_dp2a_kernel<1, kWarps, kRq1, kCq1, true>
+#define Q4_Q8_KERNEL_2 q4::gemv_dp2a_kernel<2, kWarps, kRq2, kCq2, true>
 #define Q4_MMA_KERNEL_1 q4::gemv_mma_kernel<1, kWarps, kRm1, kCm1>
 #define Q4_MMA_KERNEL_2 q4::gemv_mma_kernel<2, kWarps, kRm2, kCm2>
 #define Q4_STACK_KERNEL q4::stack_kernel<kWarps, kR1, kC1>
@@ -40,7 +45,10 @@ constexpr int kStackKmax = q4::kStackXChunks * 8 * kThreads;
 
 enum StackMode { kStackPersistent = 0, kStackKernels = 1 };
 
-size_t dp2a_smem(int M, int64_t K) {
+size_t dp2a_smem(int M, int64_t K, bool q8 = false) {
+    if (q8)
+        return M == 1 ? q4::gemv_dp2a_smem_bytes(1, (int)K, kWarps, kRq1, kCq1, q4::kSegBytesQ8)
+                      : q4::gemv_dp2a_smem_bytes(2, (int)K, kWarps, kRq2, kCq2, q4::kSegBytesQ8);
     return M == 1 ? q4::gemv_dp2a_smem_bytes(1, (int)K, kWarps, kR1, kC1)
                   : q4::gemv_dp2a_smem_bytes(2, (int)K, kWarps, kR2, kC2);
 }
@@ -159,7 +167,7 @@ int set_smem_attr(F* kernel) {
 // Launch one GEMV (M <= 2 path).  `pdl` adds the programmatic-dependent-
 // launch attribute (only used between the library's own kernels).
 int launch_gemv(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M, int64_t N,
-                int64_t K, int renorm, __half* trace_x, cudaStream_t st, bool pdl) {
+                int64_t K, int renorm, __half* trace_x, cudaStream_t st, bool pdl, bool q8 = false) {
     if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
     const int KB = (int)(K / 32);
     const int T = (int)((N + 31) / 32);
@@ -184,7 +192,7 @@ int launch_gemv(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M,
     a.G = ctas * kWarps < S ? ctas * kWarps : S;   // every owning warp gets >= 1 segment
     a.renorm = renorm;
     a.sc = q4::make_split(a.S, a.G);
-    const size_t smem = dp2a_smem(M, K);
+    const size_t smem = dp2a_smem(M, K, q8);
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ctas);
@@ -197,7 +205,9 @@ int launch_gemv(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M,
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
     cudaError_t e;
-    if (M == 1)
+    if (q8)
+        e = M == 1 ? cudaLaunchKernelEx(&cfg, Q4_Q8_KERNEL_1, a) : cudaLaunchKernelEx(&cfg, Q4_Q8_KERNEL_2, a);
+    else if (M == 1)
         e = cudaLaunchKernelEx(&cfg, Q4_DP2A_KERNEL_1, a);
     else
         e = cudaLaunchKernelEx(&cfg, Q4_DP2A_KERNEL_2, a);
@@ -472,6 +482,7 @@ int q4gemv_create(q4gemv_t* out, int device) {
     }
     if (rc == Q4_OK) {
         if (set_smem_attr(Q4_DP2A_KERNEL_1) || set_smem_attr(Q4_DP2A_KERNEL_2) ||
+            set_smem_attr(Q4_Q8_KERNEL_1) || set_smem_attr(Q4_Q8_KERNEL_2) ||
             set_smem_attr(Q4_MMA_KERNEL_1) || set_smem_attr(Q4_MMA_KERNEL_2) ||
             set_smem_attr(Q4_STACK_KERNEL) ||
             0)
@@ -557,6 +568,62 @@ int q4gemv_run(q4gemv_t h, const void* W, const void* x, void* y, int M, int64_t
                            0, nullptr, st, false);
     return launch_gemv_mma(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K,
                            st);
+}
+ 
+size_t q4gemv_q8_0_gguf_bytes(int64_t N, int64_t K) {
+    if (check_shape(N, K) != Q4_OK) return 0;
+    return (size_t)N * (size_t)(K / 32) * 34;
+}
+
+size_t q4gemv_q8_0_packed_bytes(int64_t N, int64_t K) {
+    if (check_shape(N, K) != Q4_OK) return 0;
+    return (size_t)((N + 31) / 32 * 32) * (size_t)(K / 32) * 34;
+}
+
+int q4gemv_q8_0_repack(q4gemv_t h, const void* gguf, void* packed, int64_t N, int64_t K,
+                       q4gemv_stream_t stream) {
+    if (!h) return Q4_EINVAL;
+    const int sh = check_shape(N, K);
+    if (sh != Q4_OK) return fail(h, sh, "q8_0 repack: invalid shape N=%lld K=%lld", (long long)N, (long long)K);
+    if (!gguf || !packed) return fail(h, Q4_EINVAL, "q8_0 repack: null pointer");
+    if ((reinterpret_cast<uintptr_t>(gguf) & 1u) || !aligned16(packed))
+        return fail(h, Q4_EALIGN, "q8_0 repack: misaligned pointer");
+    const uintptr_t g0 = reinterpret_cast<uintptr_t>(gguf), g1 = g0 + q4gemv_q8_0_gguf_bytes(N, K);
+    const uintptr_t p0 = reinterpret_cast<uintptr_t>(packed), p1 = p0 + q4gemv_q8_0_packed_bytes(N, K);
+    if (g0 < p1 && p0 < g1) return fail(h, Q4_EINVAL, "q8_0 repack: gguf and packed overlap");
+    if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
+    Q4_CUDA(h, cudaSetDevice(h->device));
+    const int KB = (int)(K / 32);
+    const int64_t S = (N + 31) / 32 * KB;
+    int64_t blocks = (S + 7) / 8;
+    if (blocks > (int64_t)h->sms * 32) blocks = (int64_t)h->sms * 32;
+    q4::repack_q8_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint8_t*>(gguf), static_cast<uint8_t*>(packed), N, KB, S);
+    Q4_CUDA(h, cudaGetLastError());
+    return Q4_OK;
+}
+
+int q4gemv_q8_0_validate(int M, int64_t N, int64_t K, const void* W, const void* x, const void* y) {
+    if (M < 1 || M > 2) return Q4_EUNSUPPORTED;
+    const int sh = check_shape(N, K);
+    if (sh != Q4_OK) return sh;
+    if (M * K > (int64_t)q4::kXChunksPerThread * 8 * kThreads || dp2a_smem(M, K, true) > kMaxDynSmem)
+        return Q4_EUNSUPPORTED;
+    if (!W || !x || !y) return Q4_EINVAL;
+    if (!aligned16(W) || !aligned16(x) || !aligned16(y)) return Q4_EALIGN;
+    return Q4_OK;
+}
+
+int q4gemv_q8_0_run(q4gemv_t h, const void* W, const void* x, void* y, int M, int64_t N, int64_t K,
+                    q4gemv_stream_t stream) {
+    if (!h) return Q4_EINVAL;
+    const int v = q4gemv_q8_0_validate(M, N, K, W, x, y);
+    if (v != Q4_OK)
+        return fail(h, v, "q8_0 run: %s (M=%d N=%lld K=%lld)", q4gemv_strerror(v), M, (long long)N,
+                    (long long)K);
+    Q4_CUDA(h, cudaSetDevice(h->device));
+    return launch_gemv(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K, 0, nullptr,
+                       static_cast<cudaStream_t>(stream), false, true);
 }
 
 namespace {
