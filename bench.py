@@ -80,6 +80,15 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense f16/bf16 tensor throughput (TFLOP/s, burst) and its source."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
 # ------------------------------------------------------------------ multi-rank helpers
 
 def max_over_ranks(dist, values, device=None):
@@ -447,11 +456,17 @@ def run_case(args):
     us = e0.elapsed_time(e1) * 1e3 / (args.steps * R)
     nbytes = N * (K // 32) * (34 if q8 else 18) + 2 * M * (K + N)
     peak, kind = measured_peaks()
-    print(json.dumps({"case": f"gemv {args.format} M={M} {N}x{K}", "N": N, "K": K, "M": M, "rotate": R,
-                      "us_per_launch": us, "GB/s": nbytes / us / 1e3,
-                      "frac_of_peak": nbytes / us / 1e3 / peak, "peak": peak, "peak_kind": kind,
-                      "rows_per_s": N / us * 1e6, "tflops": 2 * M * N * K / us / 1e6,
-                      "launches": args.steps * R}), flush=True)
+    line = {"case": f"gemv {args.format} M={M} {N}x{K}", "N": N, "K": K, "M": M, "rotate": R,
+            "us_per_launch": us, "GB/s": nbytes / us / 1e3,
+            "frac_of_peak": nbytes / us / 1e3 / peak, "peak": peak, "peak_kind": kind,
+            "rows_per_s": N / us * 1e6, "tflops": 2 * M * N * K / us / 1e6,
+            "launches": args.steps * R}
+    if M > q4.MAX_M_GEMV:
+        # tensor-core GEMM: f16 products, bound by the tensor pipe (f16 = bf16 rate)
+        tp, tkind = measured_tensor_peak()
+        line.update({"tensor_peak_tflops": tp, "tensor_peak_kind": tkind,
+                     "tensor_frac": line["tflops"] / tp})
+    print(json.dumps(line), flush=True)
     eng.close()
     return 0
 

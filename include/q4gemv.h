@@ -65,7 +65,7 @@ typedef enum {
     Q4_EALIGN = -3,        /* a device pointer is not 16-byte aligned */
     Q4_ENOMEM = -4,        /* device or host allocation failed */
     Q4_ECUDA = -5,         /* a CUDA runtime call failed (see q4gemv_last_error) */
-    Q4_EUNSUPPORTED = -6,  /* M outside [1, 16], or the device is not sm_100 */
+    Q4_EUNSUPPORTED = -6,  /* M outside [1, 256], or the device is not sm_100 */
     Q4_ETIMEOUT = -7,      /* a bounded device-side wait gave up */
     Q4_EFAULTINJ = -8,     /* a host step failed on purpose (fault injection) */
     Q4_ECONCURRENT = -9    /* kernels saw overlapping calls on one handle */
@@ -73,7 +73,8 @@ typedef enum {
 
 /* Limits checked by validation.  Besides these, ceil(N/32) * (K/32) must be
  * below 2^31. */
-#define Q4GEMV_MAX_M 16
+#define Q4GEMV_MAX_M 256            /* vectors per q4gemv_run call */
+#define Q4GEMV_MAX_M_GEMV 16        /* above this, the tensor-core GEMM path */
 #define Q4GEMV_MAX_N (1 << 22)     /* rows */
 #define Q4GEMV_MAX_K (1 << 20)     /* columns */
 
@@ -128,7 +129,7 @@ Q4GEMV_API int q4gemv_repack(q4gemv_t h, const void* gguf, void* packed,
  *   W_packed : device, q4gemv_packed_bytes(N, K) bytes
  *   x        : device, M*K binary16, row-major
  *   y        : device, M*N binary16, row-major (written, never read)
- * 1 <= M <= 16, K % 32 == 0.  Accumulation is fp32 or exact integer; y is
+ * 1 <= M <= 256, K % 32 == 0.  Accumulation is fp32 or exact integer; y is
  * rounded to nearest even once.  Results beyond the binary16 range become
  * +-Inf; a non-finite x element makes the affected outputs NaN.  For M <= 2
  * the activations of each 32-column block are converted to 16-bit integers
@@ -144,7 +145,17 @@ Q4GEMV_API int q4gemv_repack(q4gemv_t h, const void* gguf, void* packed,
  * short activation slice, and for wider K).  The panel sums live in a buffer
  * of P*M*N floats owned by the handle (preallocated for P*M*N <= 2^21; a
  * larger first call grows it, which synchronises the device and must not
- * happen during a stream capture). */
+ * happen during a stream capture).
+ * For M = 17..256 (prefill chunks) a dense-contraction path on the tcgen05
+ * tensor cores runs instead: "dequantise the weight tile, then multiply" --
+ * each weight becomes the binary16 value (q - 8) * d, rounded to nearest even
+ * once (relative error <= 2^-11 per weight; (q - 8) and the products are
+ * exact), and the sums accumulate in fp32.  A first kernel writes x into an
+ * activation image owned by the handle (ceil(K/64) * Mp * 128 bytes, Mp = M
+ * rounded up to 16; preallocated up to 16 MiB, grown like the panel sums);
+ * the GEMM kernel covers 256 rows per CTA, and for narrow N splits K so the
+ * grid fills the SMs, its fp32 split sums (P*M*N floats, the same buffer as
+ * the panel sums) added in split order by the reduce kernel. */
 Q4GEMV_API int q4gemv_run(q4gemv_t h, const void* W_packed, const void* x, void* y,
                int M, int64_t N, int64_t K, q4gemv_stream_t stream);
 

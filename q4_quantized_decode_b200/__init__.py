@@ -25,7 +25,8 @@ Q4_EUNSUPPORTED = -6
 Q4_ETIMEOUT = -7
 Q4_EFAULTINJ = -8
 Q4_ECONCURRENT = -9
-MAX_M = 16
+MAX_M = 256        # vectors per q4gemv_run call
+MAX_M_GEMV = 16    # above this, the tensor-core GEMM path
 
 
 class Q4Error(RuntimeError):

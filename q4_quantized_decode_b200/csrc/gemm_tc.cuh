@@ -1,0 +1,370 @@
+// Q4_0 GEMM for M = 17..256 activation vectors (prefill chunks) on the
+// 5th-generation tensor cores: Y[m][n] = sum_k W[n][k] * X[m][k].
+//
+// Dequantise-then-multiply, the reading of "dequantise a weight tile once and
+// apply it to every vector": each weight becomes the f16 value (q - 8) * d
+// (one rounding; (q - 8) itself is exact), the f16 x f16 products are exact and
+// accumulate in fp32 in tensor memory.  With this many vectors the work is a
+// dense contraction (2 * M flops per 0.5625 weight bytes), so it runs on
+// tcgen05.mma rather than on the CUDA cores.
+//
+// One CTA computes 256 output rows (two M = 128 accumulators) for all vectors
+// over its share of K (a split of the K steps when N alone gives too few CTAs):
+//   warps 0..7  dequantise the stage's weights into the A tiles and, at the
+//               end, read the accumulators back (warp w: accumulator w / 4,
+//               TMEM lanes 32 (w % 4) ..);
+//   warp 8      issues the bulk copies of each stage: the stage's packed
+//               segments (the 576-byte tiles of 32 rows x one block) and the
+//               stage's slice of the activation image;
+//   warp 9      one thread issues the MMAs and commits them to the stage's
+//               "empty" barrier and finally to the accumulator barrier.
+// A stage covers 64 columns (two blocks).  Operands sit in shared memory in
+// the K-major, 128-byte-swizzled canonical layout: row r of a tile is 128
+// bytes at r * 128, its 16-byte chunk c stored at chunk position c ^ (r % 8);
+// groups of 8 rows are 1024 bytes apart.  The activation image (written by
+// tc_ximg_kernel) already holds each stage's [Mp][64] slice in that byte
+// order, so one bulk copy brings it in.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+
+#include "device_common.cuh"
+
+namespace q4 {
+
+constexpr int kTcAcc = 2;                       // 128-row accumulators per CTA
+constexpr int kTcRows = 128 * kTcAcc;           // output rows per CTA
+constexpr int kTcTiles = kTcRows / 32;          // packed 32-row tiles per CTA
+constexpr int kTcKStep = 64;                    // columns per stage
+constexpr int kTcDqWarps = 4 * kTcAcc;          // dequantise / epilogue warps
+constexpr int kTcThreads = 32 * (kTcDqWarps + 2);
+constexpr int kTcMaxVec = 256;                  // MMA N limit (vectors)
+constexpr int kTcAccCols = 256;                 // TMEM columns per accumulator
+constexpr int kTcTmemCols = kTcAcc * kTcAccCols;
+constexpr int kTcATile = 128 * 128;             // bytes of one 128-row A tile
+constexpr int kTcRawBytes = kTcTiles * 2 * 576; // packed bytes of one stage
+
+// Bytes of one pipeline stage for Mp vectors (A tiles, B slice, packed bytes),
+// a multiple of 1024 so every tile starts on a swizzle-pattern boundary.
+__host__ __device__ constexpr uint32_t tc_stage_bytes(int Mp) {
+    return (uint32_t)((kTcAcc * kTcATile + Mp * 128 + kTcRawBytes + 1023) / 1024 * 1024);
+}
+// Dynamic shared memory of the kernel for S stages: 1024 bytes of alignment
+// slack, the stages, 3 barriers per stage + 1, the TMEM address word.
+__host__ __device__ constexpr uint32_t tc_smem_bytes(int Mp, int S) {
+    return 1024 + (uint32_t)S * tc_stage_bytes(Mp) + 8u * (3 * S + 1) + 16;
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16: f16 A and B, both K-major,
+// fp32 accumulator, no negation or sparsity, shape m x n.
+__host__ __device__ constexpr uint32_t tc_idesc_f16(int m, int n) {
+    return (1u << 4)                         // accumulator format: f32
+           | (0u << 7) | (0u << 10)          // A, B format: f16
+           | (0u << 15) | (0u << 16)         // A, B: K-major
+           | ((uint32_t)(n >> 3) << 17)      // N / 8
+           | ((uint32_t)(m >> 4) << 24);     // M / 16
+}
+
+// Shared-memory matrix descriptor of a K-major, 128-byte-swizzled operand
+// whose 8-row groups are 1024 bytes apart, starting at shared address `saddr`.
+__host__ __device__ constexpr uint64_t tc_sdesc_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu)          // start address / 16
+           | ((uint64_t)1 << 16)                       // leading offset (unused when swizzled)
+           | ((uint64_t)(1024 >> 4) << 32)             // stride offset: next 8-row group
+           | ((uint64_t)1 << 46)                       // descriptor version (sm_100)
+           | ((uint64_t)2 << 61);                      // 128-byte swizzle
+}
+
+// ---- tcgen05 wrappers -----------------------------------------------------
+
+__device__ __forceinline__ void tc_alloc(uint32_t* slot, uint32_t ncols) {   // whole warp
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_addr(slot)), "r"(ncols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tc_dealloc(uint32_t taddr, uint32_t ncols) {   // whole warp
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                 :: "r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D (+)= A * B^T for one 16-column K slice; `acc` = 0 overwrites D.
+__device__ __forceinline__ void tc_mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t acc) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc) : "memory");
+}
+// Arrives once on `bar` when every MMA this thread issued so far has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(smem_addr(bar)) : "memory");
+}
+// 16 consecutive fp32 columns of this thread's TMEM lane, waited for in the
+// same statement so no use of the registers can move above the wait.
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                   "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+                   "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+                 : "r"(taddr) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// Bounded wait that also gives up as soon as another role has aborted.
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    for (uint32_t i = 0; i < (1u << 22); ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63) == 63 && *abort_flag) return false;
+    }
+    return false;
+}
+
+struct TcArgs {
+    const uint8_t* W;    // packed Q4_0 matrix (576-byte segments, tiles of 32 rows)
+    const uint8_t* xi;   // activation image: [nk][Mp][128 bytes], swizzled rows
+    __half* y;           // [M][N] (P == 1)
+    float* ypart;        // [P][M][N] fp32 split sums (P > 1)
+    int* err;
+    int64_t N;
+    int KB, T;           // blocks per row, packed tiles ceil(N / 32)
+    int M, Mp;           // vectors; MMA N = Mp = M rounded up to 16
+    int nk, nkp, P;      // K steps, steps per split, splits
+    int S;               // pipeline stages
+    uint32_t idesc;      // tc_idesc_f16(128, Mp)
+};
+
+// Four weights of one packed word (bytes e = 0..3; low nibbles are codes
+// 4c + e, high nibbles codes 16 + 4c + e) as f16 (q - 8) * d, in code order:
+// lo = low-nibble weights, hi = high-nibble weights, 8 bytes each.
+// 0x6400 | q is the f16 1024 + q; 0x5400 | (q << 4) is the f16 64 + q.
+__device__ __forceinline__ void tc_dequant_word(uint32_t w, __half2 dd, uint2& lo, uint2& hi) {
+    const uint32_t p01 = __byte_perm(w, 0u, 0x4140);   // bytes 0, 1 -> 16-bit lanes
+    const uint32_t p23 = __byte_perm(w, 0u, 0x4342);   // bytes 2, 3
+    const __half2 k1032 = __half2half2(__ushort_as_half((unsigned short)0x6408));   // 1032
+    const __half2 k72 = __half2half2(__ushort_as_half((unsigned short)0x5480));     // 72
+    const uint32_t l01 = (p01 & 0x000F000Fu) | 0x64006400u;
+    const uint32_t l23 = (p23 & 0x000F000Fu) | 0x64006400u;
+    const uint32_t h01 = (p01 & 0x00F000F0u) | 0x54005400u;
+    const uint32_t h23 = (p23 & 0x00F000F0u) | 0x54005400u;
+    const __half2 a = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&l01), k1032), dd);
+    const __half2 b = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&l23), k1032), dd);
+    const __half2 c = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&h01), k72), dd);
+    const __half2 e = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&h23), k72), dd);
+    lo = make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+    hi = make_uint2(*reinterpret_cast<const uint32_t*>(&c), *reinterpret_cast<const uint32_t*>(&e));
+}
+
+static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) {
+    extern __shared__ uint8_t tc_smem_raw[];
+    const int S = a.S;
+    const uint32_t stage_bytes = tc_stage_bytes(a.Mp);
+    const uint32_t raw0 = smem_addr(tc_smem_raw);
+    const uint32_t base = (raw0 + 1023u) & ~1023u;               // swizzle needs 1024-byte tiles
+    uint8_t* gbase = tc_smem_raw + (base - raw0);
+    uint64_t* full = reinterpret_cast<uint64_t*>(gbase + (size_t)S * stage_bytes);
+    uint64_t* aready = full + S;
+    uint64_t* empty = aready + S;
+    uint64_t* accbar = empty + S;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(accbar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = blockIdx.x * kTcTiles;                       // first packed tile
+    const int p = blockIdx.y;
+    const int k0 = p * a.nkp;
+    const int ns = min(a.nk, k0 + a.nkp) - k0;                  // this split's K steps (>= 1)
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(aready + s, 32 * kTcDqWarps);
+            mbar_init(empty + s, 1);
+        }
+        mbar_init(accbar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) tc_alloc(tslot, kTcTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+
+    if (warp == kTcDqWarps) {
+        // ---- producer: bulk copies of each stage ----
+        if (lane == 0) {
+            const int ntiles = min(kTcTiles, a.T - t0);
+            const uint32_t bbytes = (uint32_t)a.Mp * 128u;
+            int i = 0;
+            for (; i < ns; ++i) {
+                const int s = i % S;
+                if (i >= S && !tc_wait(empty + s, (uint32_t)((i / S - 1) & 1), abort_flag)) {
+                    *abort_flag = 1;
+                    set_device_error(a.err, kDevTimeout);
+                    break;
+                }
+                const int ks = k0 + i, b0 = 2 * ks;
+                const int nb = min(2, a.KB - b0);
+                const uint32_t st = base + (uint32_t)s * stage_bytes;
+                const uint32_t sB = st + kTcAcc * kTcATile, sraw = sB + bbytes;
+                mbar_arrive_expect_tx(full + s, (uint32_t)(ntiles * nb * 576) + bbytes);
+                for (int j = 0; j < ntiles; ++j)
+                    bulk_g2s_addr(sraw + (uint32_t)j * 1152u,
+                                  a.W + ((size_t)(t0 + j) * a.KB + b0) * 576, (uint32_t)nb * 576u,
+                                  full + s);
+                bulk_g2s_addr(sB, a.xi + (size_t)ks * bbytes, bbytes, full + s);
+            }
+            // Copies still in flight must land before the CTA exits: wait for
+            // the last phase issued on every stage (already complete normally).
+            for (int s = 0; s < S && s < i; ++s) {
+                const int last = s + ((i - 1 - s) / S) * S;
+                mbar_wait_bounded(full + s, (uint32_t)((last / S) & 1), 1u << 22);
+            }
+        }
+    } else if (warp == kTcDqWarps + 1) {
+        // ---- MMA issuer ----
+        if (lane == 0) {
+            for (int i = 0; i < ns; ++i) {
+                const int s = i % S;
+                const uint32_t ph = (uint32_t)((i / S) & 1);
+                if (!tc_wait(aready + s, ph, abort_flag) || !tc_wait(full + s, ph, abort_flag)) {
+                    *abort_flag = 1;
+                    set_device_error(a.err, kDevTimeout);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t st = base + (uint32_t)s * stage_bytes;
+                const uint32_t sB = st + kTcAcc * kTcATile;
+#pragma unroll
+                for (int acc = 0; acc < kTcAcc; ++acc)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma_f16(tmem + (uint32_t)(acc * kTcAccCols),
+                                   tc_sdesc_sw128(st + (uint32_t)(acc * kTcATile + 32 * kk)),
+                                   tc_sdesc_sw128(sB + (uint32_t)(32 * kk)), a.idesc,
+                                   (uint32_t)(i | kk));
+                tc_commit(empty + s);
+            }
+            tc_commit(accbar);        // also after an abort: tracks every MMA issued
+        }
+    } else {
+        // ---- dequantise: thread (warp w, lane 4g + c) takes the 16 bytes of
+        // lane 4g + c of tile w's segments: rows g + 8i (i = 0..3), codes
+        // 4c..4c+3 and 16+4c..16+4c+3 of each block ----
+        const int g = lane >> 2, c = lane & 3;
+        const int acc = warp >> 2;
+        const uint32_t arow0 = (uint32_t)((warp & 3) * 32 + g);      // A row of i = 0
+        for (int i = 0; i < ns; ++i) {
+            const int s = i % S;
+            if (!tc_wait(full + s, (uint32_t)((i / S) & 1), abort_flag)) {
+                *abort_flag = 1;
+                set_device_error(a.err, kDevTimeout);
+                break;
+            }
+            const uint32_t st = base + (uint32_t)s * stage_bytes;
+            const uint32_t sA = st + (uint32_t)(acc * kTcATile);
+            const uint32_t sraw = st + kTcAcc * kTcATile + (uint32_t)a.Mp * 128u + (uint32_t)warp * 1152u;
+            const int nb = min(2, a.KB - 2 * (k0 + i));
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint4 wq = make_uint4(0, 0, 0, 0);
+                uint2 sc = make_uint2(0, 0);
+                if (h < nb) {
+                    wq = lds128(sraw + (uint32_t)(h * 576 + 16 * lane));
+                    sc = lds64(sraw + (uint32_t)(h * 576 + 512 + 8 * g));
+                }
+                const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
+                const uint32_t sv[4] = {sc.x, sc.x >> 16, sc.y, sc.y >> 16};
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii) {
+                    const __half2 dd = __half2half2(__ushort_as_half((unsigned short)(sv[ii] & 0xFFFFu)));
+                    uint2 lo, hi;
+                    tc_dequant_word(wv[ii], dd, lo, hi);
+                    if (h >= nb) { lo = make_uint2(0, 0); hi = lo; }
+                    const uint32_t r = arow0 + 8u * (uint32_t)ii;    // r % 8 == g
+                    const uint32_t rowa = sA + r * 128u + (uint32_t)(c & 1) * 8u;
+                    const uint32_t chl = (uint32_t)(4 * h + (c >> 1));   // columns 32h + 4c ..
+                    const uint32_t chh = chl + 2u;                       // columns 32h + 16 + 4c ..
+                    sts64(rowa + ((chl ^ (uint32_t)g) << 4), lo);
+                    sts64(rowa + ((chh ^ (uint32_t)g) << 4), hi);
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(aready + s);
+        }
+
+        // ---- epilogue: accumulator rows -> y (or the split's fp32 sums) ----
+        // tcgen05.ld is warp-collective: the decision to read is made per warp.
+        const bool ok = __all_sync(0xFFFFFFFFu, tc_wait(accbar, 0u, abort_flag) && !*abort_flag);
+        tc_fence_after();
+        if (ok) {
+            const int64_t n = (int64_t)blockIdx.x * kTcRows + acc * 128 + (warp & 3) * 32 + lane;
+            const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(acc * kTcAccCols);
+            for (int c0 = 0; c0 < a.Mp; c0 += 16) {
+                uint32_t v[16];
+                tc_ld16(taddr + (uint32_t)c0, v);
+                if (n < a.N) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int m = c0 + j;
+                        if (m < a.M) {
+                            const float f = __uint_as_float(v[j]);
+                            if (a.P == 1)
+                                a.y[(size_t)m * a.N + n] = __float2half_rn(f);
+                            else
+                                a.ypart[((size_t)p * a.M + m) * a.N + n] = f;
+                        }
+                    }
+                }
+            }
+        } else if (threadIdx.x == 0) {
+            set_device_error(a.err, kDevTimeout);
+        }
+    }
+
+    __syncwarp();        // single-lane roles rejoin their warps
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tc_dealloc(tmem, kTcTmemCols);
+    }
+}
+
+// Activation image of x[M][K] for gemm_tc_kernel: for each 64-column step ks,
+// Mp rows of 128 bytes, row m's 16-byte chunk c (columns 64 ks + 8c ..) at
+// chunk position c ^ (m % 8); rows m >= M and columns >= K are zero.
+static __global__ void __launch_bounds__(256) tc_ximg_kernel(const __half* __restrict__ x,
+                                                           uint8_t* __restrict__ img, int M, int K,
+                                                           int Mp, int nk) {
+    const int64_t total = (int64_t)nk * Mp * 8;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < total; q += stride) {
+        const int64_t ks = q / ((int64_t)Mp * 8);
+        const int rem = (int)(q - ks * Mp * 8);
+        const int m = rem >> 3, c = rem & 7;
+        const int64_t k = ks * 64 + c * 8;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (m < M && k < K) v = *reinterpret_cast<const uint4*>(x + (size_t)m * K + k);
+        *reinterpret_cast<uint4*>(img + ((size_t)ks * Mp + m) * 128 + ((c ^ (m & 7)) << 4)) = v;
+    }
+}
+
+}  // namespace q4

@@ -12,6 +12,7 @@
 
 #include "../../include/q4gemv.h"
 #include "gemv_dp2a.cuh"
+#include "gemm_tc.cuh"
 #include "gemv_mma.cuh"
 #include "stack.cuh"
 
@@ -28,6 +29,7 @@ constexpr int kMinSegsPerWarp = 4;         // small problems use fewer warps
 constexpr int kMaxTiles = Q4GEMV_MAX_N / 32;
 constexpr size_t kMaxDynSmem = 224 * 1024;   // opt-in dynamic shared memory per CTA
 constexpr size_t kYaccPrealloc = (size_t)1 << 21;   // fp32 panel accumulator floats at create
+constexpr size_t kXimgPrealloc = (size_t)1 << 24;   // GEMM activation image bytes at create
 
 #define Q4_DP2A_KERNEL_1 q4::gemv_dp2a_kernel<1, kWarps, kR1, kC1>
 #define Q4_DP2A_KERNEL_2 q4::gemv_dp2a_kernel<2, kWarps, kR2, kC2>
@@ -81,7 +83,7 @@ struct q4gemv_ctx {
     int device = 0;
     int sms = 0;
     int fault = kFaultNone;
-    float* ws = nullptr;          // [ws_warps][2][MAX_M][32] fp32
+    float* ws = nullptr;          // [ws_warps][2][MAX_M_GEMV][32] fp32
     int ws_warps = 0;
     int* cnt = nullptr;           // arrival counters, zero between calls
     int64_t cnt_elems = 0;
@@ -101,6 +103,8 @@ struct q4gemv_ctx {
     float* yacc = nullptr;           // fp32 panel sums of wide tensor-core GEMVs
     size_t yacc_floats = 0;
     __half* hio = nullptr;           // device copies of host x_in / x_out of run_stack
+    uint8_t* ximg = nullptr;         // activation image of the tensor-core GEMM
+    size_t ximg_bytes = 0;
     int64_t hio_elems = 0;           // per vector
     std::string last_error;
 };
@@ -228,7 +232,7 @@ int ensure_ws(q4gemv_ctx* h, int warps, cudaStream_t st) {
     cudaFree(h->ws);
     h->ws = nullptr;
     h->ws_warps = 0;
-    if (cudaMalloc(&h->ws, (size_t)warps * 2 * Q4GEMV_MAX_M * 32 * sizeof(float)) != cudaSuccess)
+    if (cudaMalloc(&h->ws, (size_t)warps * 2 * Q4GEMV_MAX_M_GEMV * 32 * sizeof(float)) != cudaSuccess)
         return fail(h, Q4_ENOMEM, "workspace growth to %d warps failed", warps);
     h->ws_warps = warps;
     return Q4_OK;
@@ -362,6 +366,92 @@ int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, in
     return Q4_OK;
 }
 
+// Activation image of the tensor-core GEMM (grows like the panel sums).
+int ensure_ximg(q4gemv_ctx* h, size_t bytes, cudaStream_t st) {
+    if (bytes <= h->ximg_bytes) return Q4_OK;
+    if (h->fault == kFaultAlloc) return fail(h, Q4_EFAULTINJ, "injected allocation failure");
+    cudaStreamSynchronize(st);
+    cudaFree(h->ximg);
+    h->ximg = nullptr;
+    h->ximg_bytes = 0;
+    if (cudaMalloc(&h->ximg, bytes) != cudaSuccess)
+        return fail(h, Q4_ENOMEM, "activation image of %zu bytes failed", bytes);
+    h->ximg_bytes = bytes;
+    return Q4_OK;
+}
+
+// Launch the M = 17..256 product on the tcgen05 tensor cores: the activation
+// image, the GEMM over ceil(N/256) row tiles x P splits of the K steps (P as
+// large as keeps the grid within one wave of the SMs), and for P > 1 the
+// reduce of the fp32 split sums in split order.
+int launch_gemm_tc(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M, int64_t N,
+                   int64_t K, cudaStream_t st) {
+    if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
+    const int KB = (int)(K / 32);
+    const int nk = (KB + 1) / 2;
+    const int Mp = (M + 15) / 16 * 16;
+    const int64_t tiles = (N + q4::kTcRows - 1) / q4::kTcRows;
+    int64_t P = h->sms / tiles;
+    if (P < 1) P = 1;
+    if (P > nk) P = nk;
+    const int nkp = (int)((nk + P - 1) / P);
+    P = (nk + nkp - 1) / nkp;                        // every split has steps
+    const uint32_t sb = q4::tc_stage_bytes(Mp);
+    int S = (int)((kMaxDynSmem - 2048) / sb);
+    if (S > 6) S = 6;
+    size_t smem = q4::tc_smem_bytes(Mp, S);
+    // One CTA per SM: each holds all 512 TMEM columns.
+    if (smem < 116 * 1024) smem = 116 * 1024;
+    int rc = ensure_ximg(h, (size_t)nk * Mp * 128, st);
+    if (rc != Q4_OK) return rc;
+    if (P > 1) {
+        rc = ensure_yacc(h, (size_t)P * M * (size_t)N, st);
+        if (rc != Q4_OK) return rc;
+    }
+    const int64_t chunks = (int64_t)nk * Mp * 8;
+    int64_t blocks = (chunks + 255) / 256;
+    if (blocks > (int64_t)h->sms * 8) blocks = (int64_t)h->sms * 8;
+    q4::tc_ximg_kernel<<<(unsigned)blocks, 256, 0, st>>>(x, h->ximg, M, (int)K, Mp, nk);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(h, e, "activation image launch");
+    q4::TcArgs a;
+    a.W = static_cast<const uint8_t*>(W);
+    a.xi = h->ximg;
+    a.y = y;
+    a.ypart = h->yacc;
+    a.err = h->err;
+    a.N = N;
+    a.KB = KB;
+    a.T = (int)((N + 31) / 32);
+    a.M = M;
+    a.Mp = Mp;
+    a.nk = nk;
+    a.nkp = nkp;
+    a.P = (int)P;
+    a.S = S;
+    a.idesc = q4::tc_idesc_f16(128, Mp);
+    q4::gemm_tc_kernel<<<dim3((unsigned)tiles, (unsigned)P), q4::kTcThreads, smem, st>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(h, e, "gemm (tcgen05) launch");
+    if (P > 1) {
+        const int64_t MN = (int64_t)M * N;
+        int64_t rb = (MN + 255) / 256;
+        if (rb > (int64_t)h->sms * 8) rb = (int64_t)h->sms * 8;
+        cudaLaunchConfig_t rcfg = {};
+        rcfg.gridDim = dim3((unsigned)rb);
+        rcfg.blockDim = dim3(256);
+        rcfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        rcfg.attrs = attr;
+        rcfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&rcfg, q4::panel_reduce_kernel, (const float*)h->yacc, y, (int)P, MN);
+        if (e != cudaSuccess) return cuda_fail(h, e, "split reduce launch");
+    }
+    return Q4_OK;
+}
+
 int launch_renorm(q4gemv_ctx* h, const __half* in, __half* out, int len, cudaStream_t st,
                   bool pdl) {
     if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
@@ -460,16 +550,18 @@ int q4gemv_create(q4gemv_t* out, int device) {
     if (rc == Q4_OK && h->fault == kFaultAlloc) rc = fail(h, Q4_EFAULTINJ, "injected allocation failure");
     if (rc == Q4_OK) {
         h->ws_warps = h->sms * kWarps;
-        const size_t ws_bytes = (size_t)h->ws_warps * 2 * Q4GEMV_MAX_M * 32 * sizeof(float);
+        const size_t ws_bytes = (size_t)h->ws_warps * 2 * Q4GEMV_MAX_M_GEMV * 32 * sizeof(float);
         if (cudaMalloc(&h->ws, ws_bytes) != cudaSuccess ||
             cudaMalloc(&h->cnt, (size_t)kMaxTiles * sizeof(int)) != cudaSuccess ||
             cudaMalloc(&h->err, sizeof(int)) != cudaSuccess ||
             cudaMalloc(&h->sync, 4 * sizeof(int)) != cudaSuccess ||
             cudaMalloc(&h->xq, 2 * q4::stack_xq_half_bytes(kStackKmax)) != cudaSuccess ||
-            cudaMalloc(&h->yacc, kYaccPrealloc * sizeof(float)) != cudaSuccess)
+            cudaMalloc(&h->yacc, kYaccPrealloc * sizeof(float)) != cudaSuccess ||
+            cudaMalloc(&h->ximg, kXimgPrealloc) != cudaSuccess)
             rc = fail(h, Q4_ENOMEM, "workspace allocation failed");
         else {
             h->yacc_floats = kYaccPrealloc;
+            h->ximg_bytes = kXimgPrealloc;
             h->cnt_elems = kMaxTiles;
         }
         const char* mode = getenv("Q4GEMV_STACK_MODE");
@@ -484,7 +576,7 @@ int q4gemv_create(q4gemv_t* out, int device) {
         if (set_smem_attr(Q4_DP2A_KERNEL_1) || set_smem_attr(Q4_DP2A_KERNEL_2) ||
             set_smem_attr(Q4_Q8_KERNEL_1) || set_smem_attr(Q4_Q8_KERNEL_2) ||
             set_smem_attr(Q4_MMA_KERNEL_1) || set_smem_attr(Q4_MMA_KERNEL_2) ||
-            set_smem_attr(Q4_STACK_KERNEL) ||
+            set_smem_attr(Q4_STACK_KERNEL) || set_smem_attr(q4::gemm_tc_kernel) ||
             0)
             rc = fail(h, Q4_ECUDA, "cudaFuncSetAttribute failed");
     }
@@ -503,6 +595,7 @@ int q4gemv_create(q4gemv_t* out, int device) {
         cudaFree(h->sync);
         cudaFree(h->xq);
         cudaFree(h->yacc);
+        cudaFree(h->ximg);
         if (h->cap) cudaStreamDestroy(h->cap);
         delete h;
         return rc;
@@ -526,6 +619,7 @@ int q4gemv_destroy(q4gemv_t h) {
     cudaFree(h->xq);
     cudaFree(h->yacc);
     cudaFree(h->hio);
+    cudaFree(h->ximg);
     delete h;
     return Q4_OK;
 }
@@ -563,6 +657,9 @@ int q4gemv_run(q4gemv_t h, const void* W, const void* x, void* y, int M, int64_t
                     (long long)K);
     Q4_CUDA(h, cudaSetDevice(h->device));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (M > Q4GEMV_MAX_M_GEMV)
+        return launch_gemm_tc(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N,
+                              K, st);
     if (dp2a_fits(M, K))
         return launch_gemv(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K,
                            0, nullptr, st, false);

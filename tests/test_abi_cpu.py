@@ -62,7 +62,9 @@ def test_validate_paths():
     assert v(1, 5120, 5120, A, A, A) == q4.Q4_OK
     assert v(2, 5120, 17408, A, A, A) == q4.Q4_OK
     assert v(0, 32, 32, A, A, A) == q4.Q4_EUNSUPPORTED
-    assert v(17, 32, 32, A, A, A) == q4.Q4_EUNSUPPORTED
+    assert v(17, 32, 32, A, A, A) == q4.Q4_OK          # tensor-core GEMM path
+    assert v(256, 32, 32, A, A, A) == q4.Q4_OK
+    assert v(257, 32, 32, A, A, A) == q4.Q4_EUNSUPPORTED
     assert v(1, 32, 48, A, A, A) == q4.Q4_ESHAPE
     assert v(1, 0, 32, A, A, A) == q4.Q4_ESHAPE
     assert v(1, 32, 32, None, A, A) == q4.Q4_EINVAL
