@@ -148,9 +148,10 @@ Q4GEMV_API int q4gemv_repack(q4gemv_t h, const void* gguf, void* packed,
  * happen during a stream capture).
  * For M = 17..256 (prefill chunks) a dense-contraction path on the tcgen05
  * tensor cores runs instead: "dequantise the weight tile, then multiply" --
- * each weight becomes the binary16 value (q - 8) * d, rounded to nearest even
- * once (relative error <= 2^-11 per weight; (q - 8) and the products are
- * exact), and the sums accumulate in fp32.  A first kernel writes x into an
+ * each weight (q - 8) * d is split exactly into two binary16 parts (the
+ * rounded value and its remainder), both multiply x (exact products), and
+ * the sums accumulate in fp32.  Scales |d| >= 8192 overflow binary16 in the
+ * split and give non-finite outputs.  A first kernel writes x into an
  * activation image owned by the handle (ceil(K/64) * Mp * 128 bytes, Mp = M
  * rounded up to 16; preallocated up to 16 MiB, grown like the panel sums);
  * the GEMM kernel covers 256 rows per CTA, and for narrow N splits K so the

@@ -2,15 +2,20 @@
 // 5th-generation tensor cores: Y[m][n] = sum_k W[n][k] * X[m][k].
 //
 // Dequantise-then-multiply, the reading of "dequantise a weight tile once and
-// apply it to every vector": each weight becomes the f16 value (q - 8) * d
-// (one rounding; (q - 8) itself is exact), the f16 x f16 products are exact and
-// accumulate in fp32 in tensor memory.  With this many vectors the work is a
-// dense contraction (2 * M flops per 0.5625 weight bytes), so it runs on
-// tcgen05.mma rather than on the CUDA cores.
+// apply it to every vector".  A weight (q - 8) * d has up to 14 significant
+// bits, more than binary16 holds, so it is split exactly into two binary16
+// values: main = RN((q - 8) * d) and rest = (q - 8) * d - main (a multiple of
+// d's last bit below main's last bit: at most 4 bits, always representable).
+// Both parts multiply the same activations, so every weight costs two f16
+// products; these are exact in fp32 and accumulate in fp32 in tensor memory,
+// which leaves fp32 summation as the only error before the output rounding.
+// With this many vectors the work is a dense contraction (4 * M tensor flops
+// per 0.5625 weight bytes), so it runs on tcgen05.mma, not the CUDA cores.
 //
 // One CTA computes 256 output rows (two M = 128 accumulators) for all vectors
 // over its share of K (a split of the K steps when N alone gives too few CTAs):
-//   warps 0..7  dequantise the stage's weights into the A tiles and, at the
+//   warps 0..7  dequantise the stage's weights into the A tiles (main and
+//               rest parts, one tile each per accumulator) and, at the
 //               end, read the accumulators back (warp w: accumulator w / 4,
 //               TMEM lanes 32 (w % 4) ..);
 //   warp 8      issues the bulk copies of each stage: the stage's packed
@@ -45,10 +50,12 @@ constexpr int kTcTmemCols = kTcAcc * kTcAccCols;
 constexpr int kTcATile = 128 * 128;             // bytes of one 128-row A tile
 constexpr int kTcRawBytes = kTcTiles * 2 * 576; // packed bytes of one stage
 
+constexpr int kTcABytes = 2 * kTcAcc * kTcATile; // main + rest tiles of a stage
+
 // Bytes of one pipeline stage for Mp vectors (A tiles, B slice, packed bytes),
 // a multiple of 1024 so every tile starts on a swizzle-pattern boundary.
 __host__ __device__ constexpr uint32_t tc_stage_bytes(int Mp) {
-    return (uint32_t)((kTcAcc * kTcATile + Mp * 128 + kTcRawBytes + 1023) / 1024 * 1024);
+    return (uint32_t)((kTcABytes + Mp * 128 + kTcRawBytes + 1023) / 1024 * 1024);
 }
 // Dynamic shared memory of the kernel for S stages: 1024 bytes of alignment
 // slack, the stages, 3 barriers per stage + 1, the TMEM address word.
@@ -150,11 +157,22 @@ struct TcArgs {
     uint32_t idesc;      // tc_idesc_f16(128, Mp)
 };
 
+// Exact split of one (q - 8) * d pair: main = RN(q * d), rest = q * d - main
+// (the fused multiply-add rounds the exact remainder, which is representable).
+__device__ __forceinline__ void tc_split2(__half2 q, __half2 dd, uint32_t& m, uint32_t& r) {
+    const __half2 hm = __hmul2(q, dd);
+    const __half2 hr = __hfma2(q, dd, __hneg2(hm));
+    m = *reinterpret_cast<const uint32_t*>(&hm);
+    r = *reinterpret_cast<const uint32_t*>(&hr);
+}
+
 // Four weights of one packed word (bytes e = 0..3; low nibbles are codes
-// 4c + e, high nibbles codes 16 + 4c + e) as f16 (q - 8) * d, in code order:
-// lo = low-nibble weights, hi = high-nibble weights, 8 bytes each.
-// 0x6400 | q is the f16 1024 + q; 0x5400 | (q << 4) is the f16 64 + q.
-__device__ __forceinline__ void tc_dequant_word(uint32_t w, __half2 dd, uint2& lo, uint2& hi) {
+// 4c + e, high nibbles codes 16 + 4c + e), in code order, 8 bytes per set:
+// lm / lr = main / rest parts of the low-nibble weights, hm / hr of the high.
+// 0x6400 | q is the f16 1024 + q; 0x5400 | (q << 4) is the f16 64 + q; the
+// subtractions leave q - 8 exactly.
+__device__ __forceinline__ void tc_dequant_word(uint32_t w, __half2 dd, uint2& lm, uint2& lr,
+                                                uint2& hm, uint2& hr) {
     const uint32_t p01 = __byte_perm(w, 0u, 0x4140);   // bytes 0, 1 -> 16-bit lanes
     const uint32_t p23 = __byte_perm(w, 0u, 0x4342);   // bytes 2, 3
     const __half2 k1032 = __half2half2(__ushort_as_half((unsigned short)0x6408));   // 1032
@@ -163,12 +181,10 @@ __device__ __forceinline__ void tc_dequant_word(uint32_t w, __half2 dd, uint2& l
     const uint32_t l23 = (p23 & 0x000F000Fu) | 0x64006400u;
     const uint32_t h01 = (p01 & 0x00F000F0u) | 0x54005400u;
     const uint32_t h23 = (p23 & 0x00F000F0u) | 0x54005400u;
-    const __half2 a = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&l01), k1032), dd);
-    const __half2 b = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&l23), k1032), dd);
-    const __half2 c = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&h01), k72), dd);
-    const __half2 e = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&h23), k72), dd);
-    lo = make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
-    hi = make_uint2(*reinterpret_cast<const uint32_t*>(&c), *reinterpret_cast<const uint32_t*>(&e));
+    tc_split2(__hsub2(*reinterpret_cast<const __half2*>(&l01), k1032), dd, lm.x, lr.x);
+    tc_split2(__hsub2(*reinterpret_cast<const __half2*>(&l23), k1032), dd, lm.y, lr.y);
+    tc_split2(__hsub2(*reinterpret_cast<const __half2*>(&h01), k72), dd, hm.x, hr.x);
+    tc_split2(__hsub2(*reinterpret_cast<const __half2*>(&h23), k72), dd, hm.y, hr.y);
 }
 
 static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) {
@@ -223,7 +239,7 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
                 const int ks = k0 + i, b0 = 2 * ks;
                 const int nb = min(2, a.KB - b0);
                 const uint32_t st = base + (uint32_t)s * stage_bytes;
-                const uint32_t sB = st + kTcAcc * kTcATile, sraw = sB + bbytes;
+                const uint32_t sB = st + kTcABytes, sraw = sB + bbytes;
                 mbar_arrive_expect_tx(full + s, (uint32_t)(ntiles * nb * 576) + bbytes);
                 for (int j = 0; j < ntiles; ++j)
                     bulk_g2s_addr(sraw + (uint32_t)j * 1152u,
@@ -251,15 +267,19 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
                 }
                 tc_fence_after();
                 const uint32_t st = base + (uint32_t)s * stage_bytes;
-                const uint32_t sB = st + kTcAcc * kTcATile;
+                const uint32_t sB = st + kTcABytes;
 #pragma unroll
                 for (int acc = 0; acc < kTcAcc; ++acc)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t bdesc = tc_sdesc_sw128(sB + (uint32_t)(32 * kk));
+                        const uint32_t am = st + (uint32_t)(acc * kTcATile + 32 * kk);
+                        tc_mma_f16(tmem + (uint32_t)(acc * kTcAccCols), tc_sdesc_sw128(am), bdesc,
+                                   a.idesc, (uint32_t)(i | kk));
                         tc_mma_f16(tmem + (uint32_t)(acc * kTcAccCols),
-                                   tc_sdesc_sw128(st + (uint32_t)(acc * kTcATile + 32 * kk)),
-                                   tc_sdesc_sw128(sB + (uint32_t)(32 * kk)), a.idesc,
-                                   (uint32_t)(i | kk));
+                                   tc_sdesc_sw128(am + (uint32_t)(kTcAcc * kTcATile)), bdesc,
+                                   a.idesc, 1u);
+                    }
                 tc_commit(empty + s);
             }
             tc_commit(accbar);        // also after an abort: tracks every MMA issued
@@ -279,8 +299,9 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
                 break;
             }
             const uint32_t st = base + (uint32_t)s * stage_bytes;
-            const uint32_t sA = st + (uint32_t)(acc * kTcATile);
-            const uint32_t sraw = st + kTcAcc * kTcATile + (uint32_t)a.Mp * 128u + (uint32_t)warp * 1152u;
+            const uint32_t sA = st + (uint32_t)(acc * kTcATile);               // main part
+            const uint32_t sR = sA + (uint32_t)(kTcAcc * kTcATile);            // rest part
+            const uint32_t sraw = st + kTcABytes + (uint32_t)a.Mp * 128u + (uint32_t)warp * 1152u;
             const int nb = min(2, a.KB - 2 * (k0 + i));
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -295,15 +316,19 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
 #pragma unroll
                 for (int ii = 0; ii < 4; ++ii) {
                     const __half2 dd = __half2half2(__ushort_as_half((unsigned short)(sv[ii] & 0xFFFFu)));
-                    uint2 lo, hi;
-                    tc_dequant_word(wv[ii], dd, lo, hi);
-                    if (h >= nb) { lo = make_uint2(0, 0); hi = lo; }
+                    uint2 lm, lr, hm, hr;
+                    tc_dequant_word(wv[ii], dd, lm, lr, hm, hr);
+                    if (h >= nb) { lm = make_uint2(0, 0); lr = lm; hm = lm; hr = lm; }
                     const uint32_t r = arow0 + 8u * (uint32_t)ii;    // r % 8 == g
-                    const uint32_t rowa = sA + r * 128u + (uint32_t)(c & 1) * 8u;
+                    const uint32_t off = r * 128u + (uint32_t)(c & 1) * 8u;
                     const uint32_t chl = (uint32_t)(4 * h + (c >> 1));   // columns 32h + 4c ..
                     const uint32_t chh = chl + 2u;                       // columns 32h + 16 + 4c ..
-                    sts64(rowa + ((chl ^ (uint32_t)g) << 4), lo);
-                    sts64(rowa + ((chh ^ (uint32_t)g) << 4), hi);
+                    const uint32_t ol = off + ((chl ^ (uint32_t)g) << 4);
+                    const uint32_t oh = off + ((chh ^ (uint32_t)g) << 4);
+                    sts64(sA + ol, lm);
+                    sts64(sA + oh, hm);
+                    sts64(sR + ol, lr);
+                    sts64(sR + oh, hr);
                 }
             }
             fence_proxy_async_smem();
