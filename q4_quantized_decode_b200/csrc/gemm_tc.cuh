@@ -18,12 +18,16 @@
 //               rest parts, one tile each per accumulator) and, at the
 //               end, read the accumulators back (warp w: accumulator w / 4,
 //               TMEM lanes 32 (w % 4) ..);
-//   warp 8      issues the bulk copies of each stage: the stage's packed
-//               segments (the 576-byte tiles of 32 rows x one block) and the
-//               stage's slice of the activation image;
-//   warp 9      one thread issues the MMAs and commits them to the stage's
-//               "empty" barrier and finally to the accumulator barrier.
-// A stage covers 64 columns (two blocks).  Operands sit in shared memory in
+//   warp 8      issues the bulk copies of each K step into a ring of L load
+//               stages: the step's packed segments (the 576-byte tiles of 32
+//               rows x one block) and its slice of the activation image;
+//   warp 9      one thread issues the MMAs and commits them to the load
+//               stage's and the A buffer's "empty" barriers, finally to the
+//               accumulator barrier.
+// A K step covers 64 columns (two blocks).  The A tiles (main and rest parts
+// of 256 rows, 64 KB) are double-buffered apart from the load ring, so the
+// copies run L steps ahead while dequantising step i + 1 overlaps the MMAs of
+// step i.  Operands sit in shared memory in
 // the K-major, 128-byte-swizzled canonical layout: row r of a tile is 128
 // bytes at r * 128, its 16-byte chunk c stored at chunk position c ^ (r % 8);
 // groups of 8 rows are 1024 bytes apart.  The activation image (written by
@@ -50,17 +54,21 @@ constexpr int kTcTmemCols = kTcAcc * kTcAccCols;
 constexpr int kTcATile = 128 * 128;             // bytes of one 128-row A tile
 constexpr int kTcRawBytes = kTcTiles * 2 * 576; // packed bytes of one stage
 
-constexpr int kTcABytes = 2 * kTcAcc * kTcATile; // main + rest tiles of a stage
+constexpr int kTcABytes = 2 * kTcAcc * kTcATile; // main + rest tiles of one A buffer
+constexpr int kTcABufs = 2;                      // A buffers: dequantise one, multiply the other
 
-// Bytes of one pipeline stage for Mp vectors (A tiles, B slice, packed bytes),
-// a multiple of 1024 so every tile starts on a swizzle-pattern boundary.
-__host__ __device__ constexpr uint32_t tc_stage_bytes(int Mp) {
-    return (uint32_t)((kTcABytes + Mp * 128 + kTcRawBytes + 1023) / 1024 * 1024);
+// Bytes of one load stage for Mp vectors (the activation slice, then the
+// packed bytes), a multiple of 1024 so every slice starts on a swizzle-pattern
+// boundary.
+__host__ __device__ constexpr uint32_t tc_load_stage_bytes(int Mp) {
+    return (uint32_t)((Mp * 128 + kTcRawBytes + 1023) / 1024 * 1024);
 }
-// Dynamic shared memory of the kernel for S stages: 1024 bytes of alignment
-// slack, the stages, 3 barriers per stage + 1, the TMEM address word.
-__host__ __device__ constexpr uint32_t tc_smem_bytes(int Mp, int S) {
-    return 1024 + (uint32_t)S * tc_stage_bytes(Mp) + 8u * (3 * S + 1) + 16;
+// Dynamic shared memory of the kernel with L load stages: 1024 bytes of
+// alignment slack, the A buffers, the load stages, the barriers (2 per load
+// stage, 2 per A buffer, 1), the TMEM address word and the abort flag.
+__host__ __device__ constexpr uint32_t tc_smem_bytes(int Mp, int L) {
+    return 1024 + (uint32_t)(kTcABufs * kTcABytes) + (uint32_t)L * tc_load_stage_bytes(Mp) +
+           8u * (2 * L + 2 * kTcABufs + 1) + 16;
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16: f16 A and B, both K-major,
@@ -153,7 +161,7 @@ struct TcArgs {
     int KB, T;           // blocks per row, packed tiles ceil(N / 32)
     int M, Mp;           // vectors; MMA N = Mp = M rounded up to 16
     int nk, nkp, P;      // K steps, steps per split, splits
-    int S;               // pipeline stages
+    int L;               // load stages
     uint32_t idesc;      // tc_idesc_f16(128, Mp)
 };
 
@@ -189,15 +197,17 @@ __device__ __forceinline__ void tc_dequant_word(uint32_t w, __half2 dd, uint2& l
 
 static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) {
     extern __shared__ uint8_t tc_smem_raw[];
-    const int S = a.S;
-    const uint32_t stage_bytes = tc_stage_bytes(a.Mp);
+    const int L = a.L;
+    const uint32_t ld_bytes = tc_load_stage_bytes(a.Mp);
     const uint32_t raw0 = smem_addr(tc_smem_raw);
     const uint32_t base = (raw0 + 1023u) & ~1023u;               // swizzle needs 1024-byte tiles
-    uint8_t* gbase = tc_smem_raw + (base - raw0);
-    uint64_t* full = reinterpret_cast<uint64_t*>(gbase + (size_t)S * stage_bytes);
-    uint64_t* aready = full + S;
-    uint64_t* empty = aready + S;
-    uint64_t* accbar = empty + S;
+    const uint32_t ld0 = base + (uint32_t)(kTcABufs * kTcABytes);  // first load stage
+    uint8_t* gbar = tc_smem_raw + (ld0 - raw0) + (size_t)L * ld_bytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(gbar);          // [L] copies landed
+    uint64_t* lempty = full + L;                                 // [L] MMAs done with the stage
+    uint64_t* aready = lempty + L;                               // [2] A buffer written
+    uint64_t* aempty = aready + kTcABufs;                        // [2] MMAs done with the buffer
+    uint64_t* accbar = aempty + kTcABufs;
     uint32_t* tslot = reinterpret_cast<uint32_t*>(accbar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
 
@@ -206,12 +216,16 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
     const int p = blockIdx.y;
     const int k0 = p * a.nkp;
     const int ns = min(a.nk, k0 + a.nkp) - k0;                  // this split's K steps (>= 1)
+    const uint32_t bbytes = (uint32_t)a.Mp * 128u;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(full + s, 1);
-            mbar_init(aready + s, 32 * kTcDqWarps);
-            mbar_init(empty + s, 1);
+        for (int j = 0; j < L; ++j) {
+            mbar_init(full + j, 1);
+            mbar_init(lempty + j, 1);
+        }
+        for (int b = 0; b < kTcABufs; ++b) {
+            mbar_init(aready + b, 32 * kTcDqWarps);
+            mbar_init(aempty + b, 1);
         }
         mbar_init(accbar, 1);
         *abort_flag = 0;
@@ -224,63 +238,62 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
     const uint32_t tmem = *tslot;
 
     if (warp == kTcDqWarps) {
-        // ---- producer: bulk copies of each stage ----
+        // ---- producer: bulk copies of each K step into load stage i % L ----
         if (lane == 0) {
             const int ntiles = min(kTcTiles, a.T - t0);
-            const uint32_t bbytes = (uint32_t)a.Mp * 128u;
             int i = 0;
             for (; i < ns; ++i) {
-                const int s = i % S;
-                if (i >= S && !tc_wait(empty + s, (uint32_t)((i / S - 1) & 1), abort_flag)) {
+                const int j = i % L;
+                if (i >= L && !tc_wait(lempty + j, (uint32_t)((i / L - 1) & 1), abort_flag)) {
                     *abort_flag = 1;
                     set_device_error(a.err, kDevTimeout);
                     break;
                 }
                 const int ks = k0 + i, b0 = 2 * ks;
                 const int nb = min(2, a.KB - b0);
-                const uint32_t st = base + (uint32_t)s * stage_bytes;
-                const uint32_t sB = st + kTcABytes, sraw = sB + bbytes;
-                mbar_arrive_expect_tx(full + s, (uint32_t)(ntiles * nb * 576) + bbytes);
-                for (int j = 0; j < ntiles; ++j)
-                    bulk_g2s_addr(sraw + (uint32_t)j * 1152u,
-                                  a.W + ((size_t)(t0 + j) * a.KB + b0) * 576, (uint32_t)nb * 576u,
-                                  full + s);
-                bulk_g2s_addr(sB, a.xi + (size_t)ks * bbytes, bbytes, full + s);
+                const uint32_t sB = ld0 + (uint32_t)j * ld_bytes, sraw = sB + bbytes;
+                mbar_arrive_expect_tx(full + j, (uint32_t)(ntiles * nb * 576) + bbytes);
+                for (int t = 0; t < ntiles; ++t)
+                    bulk_g2s_addr(sraw + (uint32_t)t * 1152u,
+                                  a.W + ((size_t)(t0 + t) * a.KB + b0) * 576, (uint32_t)nb * 576u,
+                                  full + j);
+                bulk_g2s_addr(sB, a.xi + (size_t)ks * bbytes, bbytes, full + j);
             }
             // Copies still in flight must land before the CTA exits: wait for
             // the last phase issued on every stage (already complete normally).
-            for (int s = 0; s < S && s < i; ++s) {
-                const int last = s + ((i - 1 - s) / S) * S;
-                mbar_wait_bounded(full + s, (uint32_t)((last / S) & 1), 1u << 22);
+            for (int j = 0; j < L && j < i; ++j) {
+                const int last = j + ((i - 1 - j) / L) * L;
+                mbar_wait_bounded(full + j, (uint32_t)((last / L) & 1), 1u << 22);
             }
         }
     } else if (warp == kTcDqWarps + 1) {
         // ---- MMA issuer ----
         if (lane == 0) {
             for (int i = 0; i < ns; ++i) {
-                const int s = i % S;
-                const uint32_t ph = (uint32_t)((i / S) & 1);
-                if (!tc_wait(aready + s, ph, abort_flag) || !tc_wait(full + s, ph, abort_flag)) {
+                const int j = i % L, b = i & 1;
+                if (!tc_wait(aready + b, (uint32_t)((i >> 1) & 1), abort_flag) ||
+                    !tc_wait(full + j, (uint32_t)((i / L) & 1), abort_flag)) {
                     *abort_flag = 1;
                     set_device_error(a.err, kDevTimeout);
                     break;
                 }
                 tc_fence_after();
-                const uint32_t st = base + (uint32_t)s * stage_bytes;
-                const uint32_t sB = st + kTcABytes;
+                const uint32_t sA = base + (uint32_t)(b * kTcABytes);
+                const uint32_t sB = ld0 + (uint32_t)j * ld_bytes;
 #pragma unroll
                 for (int acc = 0; acc < kTcAcc; ++acc)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t bdesc = tc_sdesc_sw128(sB + (uint32_t)(32 * kk));
-                        const uint32_t am = st + (uint32_t)(acc * kTcATile + 32 * kk);
+                        const uint32_t am = sA + (uint32_t)(acc * kTcATile + 32 * kk);
                         tc_mma_f16(tmem + (uint32_t)(acc * kTcAccCols), tc_sdesc_sw128(am), bdesc,
                                    a.idesc, (uint32_t)(i | kk));
                         tc_mma_f16(tmem + (uint32_t)(acc * kTcAccCols),
                                    tc_sdesc_sw128(am + (uint32_t)(kTcAcc * kTcATile)), bdesc,
                                    a.idesc, 1u);
                     }
-                tc_commit(empty + s);
+                tc_commit(lempty + j);
+                tc_commit(aempty + b);
             }
             tc_commit(accbar);        // also after an abort: tracks every MMA issued
         }
@@ -292,16 +305,16 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
         const int acc = warp >> 2;
         const uint32_t arow0 = (uint32_t)((warp & 3) * 32 + g);      // A row of i = 0
         for (int i = 0; i < ns; ++i) {
-            const int s = i % S;
-            if (!tc_wait(full + s, (uint32_t)((i / S) & 1), abort_flag)) {
+            const int j = i % L, b = i & 1;
+            if (!tc_wait(full + j, (uint32_t)((i / L) & 1), abort_flag) ||
+                (i >= kTcABufs && !tc_wait(aempty + b, (uint32_t)(((i >> 1) - 1) & 1), abort_flag))) {
                 *abort_flag = 1;
                 set_device_error(a.err, kDevTimeout);
                 break;
             }
-            const uint32_t st = base + (uint32_t)s * stage_bytes;
-            const uint32_t sA = st + (uint32_t)(acc * kTcATile);               // main part
-            const uint32_t sR = sA + (uint32_t)(kTcAcc * kTcATile);            // rest part
-            const uint32_t sraw = st + kTcABytes + (uint32_t)a.Mp * 128u + (uint32_t)warp * 1152u;
+            const uint32_t sA = base + (uint32_t)(b * kTcABytes + acc * kTcATile);   // main part
+            const uint32_t sR = sA + (uint32_t)(kTcAcc * kTcATile);                 // rest part
+            const uint32_t sraw = ld0 + (uint32_t)j * ld_bytes + bbytes + (uint32_t)warp * 1152u;
             const int nb = min(2, a.KB - 2 * (k0 + i));
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -332,7 +345,7 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
                 }
             }
             fence_proxy_async_smem();
-            mbar_arrive(aready + s);
+            mbar_arrive(aready + b);
         }
 
         // ---- epilogue: accumulator rows -> y (or the split's fp32 sums) ----
@@ -347,10 +360,10 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
                 tc_ld16(taddr + (uint32_t)c0, v);
                 if (n < a.N) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int m = c0 + j;
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int m = c0 + jj;
                         if (m < a.M) {
-                            const float f = __uint_as_float(v[j]);
+                            const float f = __uint_as_float(v[jj]);
                             if (a.P == 1)
                                 a.y[(size_t)m * a.N + n] = __float2half_rn(f);
                             else

@@ -396,10 +396,12 @@ int launch_gemm_tc(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int
     if (P > nk) P = nk;
     const int nkp = (int)((nk + P - 1) / P);
     P = (nk + nkp - 1) / nkp;                        // every split has steps
-    const uint32_t sb = q4::tc_stage_bytes(Mp);
-    int S = (int)((kMaxDynSmem - 2048) / sb);
-    if (S > 6) S = 6;
-    size_t smem = q4::tc_smem_bytes(Mp, S);
+    // Load stages: as many as fit beside the two A buffers (at least 2).
+    const size_t fixed = q4::tc_smem_bytes(Mp, 0);
+    const size_t lsb = q4::tc_load_stage_bytes(Mp) + 16;
+    int L = (int)((kMaxDynSmem - fixed) / lsb);
+    if (L > 8) L = 8;
+    size_t smem = q4::tc_smem_bytes(Mp, L);
     // One CTA per SM: each holds all 512 TMEM columns.
     if (smem < 116 * 1024) smem = 116 * 1024;
     int rc = ensure_ximg(h, (size_t)nk * Mp * 128, st);
@@ -428,7 +430,7 @@ int launch_gemm_tc(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int
     a.nk = nk;
     a.nkp = nkp;
     a.P = (int)P;
-    a.S = S;
+    a.L = L;
     a.idesc = q4::tc_idesc_f16(128, Mp);
     q4::gemm_tc_kernel<<<dim3((unsigned)tiles, (unsigned)P), q4::kTcThreads, smem, st>>>(a);
     e = cudaGetLastError();
