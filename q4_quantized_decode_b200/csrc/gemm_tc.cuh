@@ -224,7 +224,7 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
             mbar_init(lempty + j, 1);
         }
         for (int b = 0; b < kTcABufs; ++b) {
-            mbar_init(aready + b, 32 * kTcDqWarps);
+            mbar_init(aready + b, kTcDqWarps);
             mbar_init(aempty + b, 1);
         }
         mbar_init(accbar, 1);
@@ -298,16 +298,22 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
             tc_commit(accbar);        // also after an abort: tracks every MMA issued
         }
     } else {
-        // ---- dequantise: thread (warp w, lane 4g + c) takes the 16 bytes of
-        // lane 4g + c of tile w's segments: rows g + 8i (i = 0..3), codes
-        // 4c..4c+3 and 16+4c..16+4c+3 of each block ----
-        const int g = lane >> 2, c = lane & 3;
+        // ---- dequantise: the thread with pair (g, c) takes the 16 bytes at
+        // 16 (4g + c) of tile w's segments: rows g + 8i (i = 0..3), codes
+        // 4c..4c+3 and 16+4c..16+4c+3 of each block.  The lane -> (g, c) map
+        // (g bits: lane bit 0, bit 3, bit 0 ^ bit 4; c: lane bits 1-2) makes
+        // every quarter-warp's 16-byte loads and every half-warp's 8-byte
+        // swizzled stores hit distinct banks ----
+        const int g = (lane & 1) | ((lane >> 2) & 2) | (((lane ^ (lane >> 4)) & 1) << 2);
+        const int c = (lane >> 1) & 3;
         const int acc = warp >> 2;
         const uint32_t arow0 = (uint32_t)((warp & 3) * 32 + g);      // A row of i = 0
         for (int i = 0; i < ns; ++i) {
             const int j = i % L, b = i & 1;
-            if (!tc_wait(full + j, (uint32_t)((i / L) & 1), abort_flag) ||
-                (i >= kTcABufs && !tc_wait(aempty + b, (uint32_t)(((i >> 1) - 1) & 1), abort_flag))) {
+            const bool got = tc_wait(full + j, (uint32_t)((i / L) & 1), abort_flag) &&
+                             (i < kTcABufs ||
+                              tc_wait(aempty + b, (uint32_t)(((i >> 1) - 1) & 1), abort_flag));
+            if (!__all_sync(0xFFFFFFFFu, got)) {       // the warp leaves together
                 *abort_flag = 1;
                 set_device_error(a.err, kDevTimeout);
                 break;
@@ -321,7 +327,7 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
                 uint4 wq = make_uint4(0, 0, 0, 0);
                 uint2 sc = make_uint2(0, 0);
                 if (h < nb) {
-                    wq = lds128(sraw + (uint32_t)(h * 576 + 16 * lane));
+                    wq = lds128(sraw + (uint32_t)(h * 576 + 16 * (4 * g + c)));
                     sc = lds64(sraw + (uint32_t)(h * 576 + 512 + 8 * g));
                 }
                 const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
@@ -344,8 +350,9 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
                     sts64(sR + oh, hr);
                 }
             }
-            fence_proxy_async_smem();
-            mbar_arrive(aready + b);
+            fence_proxy_async_smem();      // this thread's tile writes -> tensor-core reads
+            __syncwarp();
+            if (lane == 0) mbar_arrive(aready + b);
         }
 
         // ---- epilogue: accumulator rows -> y (or the split's fp32 sums) ----
