@@ -186,16 +186,20 @@ Q4GEMV_API int q4gemv_q8_0_repack(q4gemv_t h, const void* gguf, void* packed,
                        int64_t N, int64_t K, q4gemv_stream_t stream);
 
 /* Host-only check of q4gemv_q8_0_run's arguments: Q4_EUNSUPPORTED for M
- * outside {1, 2} or M*K beyond the kernel's activation staging (M*K <=
- * 36,864 and the shared-memory budget), else as q4gemv_validate. */
+ * outside [1, 256], else as q4gemv_validate. */
 Q4GEMV_API int q4gemv_q8_0_validate(int M, int64_t N, int64_t K, const void* W_packed,
                          const void* x, const void* y);
 
-/* y[M][N] = W x[M][K]^T for a packed Q8_0 W, M in {1, 2} (buffers as
- * q4gemv_run).  The activations are converted per 32-column block as for
- * Q4_0 (exact for the block maximum), each block's dot product with the
- * 8-bit codes is an exact integer, converted to fp32 once and scaled by d;
- * fp32 accumulation; y rounded to binary16 once.  Deterministic. */
+/* y[M][N] = W x[M][K]^T for a packed Q8_0 W, 1 <= M <= 256 (buffers as
+ * q4gemv_run).  M <= 2 with M*K <= 36,864 (and the kernel's shared memory):
+ * the activations are converted per 32-column block as for Q4_0 (exact for
+ * the block maximum), each block's dot product with the 8-bit codes is an
+ * exact integer, converted to fp32 once and scaled by d.  Otherwise the
+ * tcgen05 GEMM of q4gemv_run's M > 16 path runs with Q8_0 segments: each
+ * weight q * d (up to 18 significant bits) is split exactly into two binary16
+ * parts; scales |d| >= 512 overflow the split (non-finite outputs); its
+ * activation image and split sums live in the same handle buffers.  fp32
+ * accumulation; y rounded to binary16 once.  Deterministic. */
 Q4GEMV_API int q4gemv_q8_0_run(q4gemv_t h, const void* W_packed, const void* x, void* y,
                     int M, int64_t N, int64_t K, q4gemv_stream_t stream);
 

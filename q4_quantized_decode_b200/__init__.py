@@ -230,7 +230,7 @@ class Q4Gemv:
         return out
 
     def run_q8_0(self, W_packed, x, N: int, K: int, out=None, stream=None):
-        """x: f16 CUDA tensor [M][K] (M <= 2) -> y f16 [M][N] for a packed Q8_0 W."""
+        """x: f16 CUDA tensor [M][K] (M <= 256) -> y f16 [M][N] for a packed Q8_0 W."""
         import torch
         x2 = x.reshape(-1, K)
         M = x2.shape[0]

@@ -19,8 +19,9 @@
 //               end, read the accumulators back (warp w: accumulator w / 4,
 //               TMEM lanes 32 (w % 4) ..);
 //   warp 8      issues the bulk copies of each K step into a ring of L load
-//               stages: the step's packed segments (the 576-byte tiles of 32
-//               rows x one block) and its slice of the activation image;
+//               stages: the step's packed segments (the 576-byte Q4_0 or
+//               1088-byte Q8_0 tiles of 32 rows x one block) and its slice of
+//               the activation image;
 //   warp 9      one thread issues the MMAs and commits them to the load
 //               stage's and the A buffer's "empty" barriers, finally to the
 //               accumulator barrier.
@@ -52,7 +53,11 @@ constexpr int kTcMaxVec = 256;                  // MMA N limit (vectors)
 constexpr int kTcAccCols = 256;                 // TMEM columns per accumulator
 constexpr int kTcTmemCols = kTcAcc * kTcAccCols;
 constexpr int kTcATile = 128 * 128;             // bytes of one 128-row A tile
-constexpr int kTcRawBytes = kTcTiles * 2 * 576; // packed bytes of one stage
+// Packed segment of one 32-row tile and one block: Q4_0 576 bytes (codes at
+// 16 (4g + c) + 4i, scales at 512), Q8_0 1088 bytes (codes at 32 (4g + c) + 8i,
+// scales at 1024); a load stage holds two segments of each of the CTA's tiles.
+__host__ __device__ constexpr int tc_seg_bytes(bool q8) { return q8 ? 1088 : 576; }
+__host__ __device__ constexpr int tc_raw_bytes(bool q8) { return kTcTiles * 2 * tc_seg_bytes(q8); }
 
 constexpr int kTcABytes = 2 * kTcAcc * kTcATile; // main + rest tiles of one A buffer
 constexpr int kTcABufs = 2;                      // A buffers: dequantise one, multiply the other
@@ -60,14 +65,14 @@ constexpr int kTcABufs = 2;                      // A buffers: dequantise one, m
 // Bytes of one load stage for Mp vectors (the activation slice, then the
 // packed bytes), a multiple of 1024 so every slice starts on a swizzle-pattern
 // boundary.
-__host__ __device__ constexpr uint32_t tc_load_stage_bytes(int Mp) {
-    return (uint32_t)((Mp * 128 + kTcRawBytes + 1023) / 1024 * 1024);
+__host__ __device__ constexpr uint32_t tc_load_stage_bytes(int Mp, bool q8 = false) {
+    return (uint32_t)((Mp * 128 + tc_raw_bytes(q8) + 1023) / 1024 * 1024);
 }
 // Dynamic shared memory of the kernel with L load stages: 1024 bytes of
 // alignment slack, the A buffers, the load stages, the barriers (2 per load
 // stage, 2 per A buffer, 1), the TMEM address word and the abort flag.
-__host__ __device__ constexpr uint32_t tc_smem_bytes(int Mp, int L) {
-    return 1024 + (uint32_t)(kTcABufs * kTcABytes) + (uint32_t)L * tc_load_stage_bytes(Mp) +
+__host__ __device__ constexpr uint32_t tc_smem_bytes(int Mp, int L, bool q8 = false) {
+    return 1024 + (uint32_t)(kTcABufs * kTcABytes) + (uint32_t)L * tc_load_stage_bytes(Mp, q8) +
            8u * (2 * L + 2 * kTcABufs + 1) + 16;
 }
 
@@ -152,7 +157,7 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 }
 
 struct TcArgs {
-    const uint8_t* W;    // packed Q4_0 matrix (576-byte segments, tiles of 32 rows)
+    const uint8_t* W;    // packed Q4_0 (576-byte segments) or Q8_0 (1088-byte) matrix
     const uint8_t* xi;   // activation image: [nk][Mp][128 bytes], swizzled rows
     __half* y;           // [M][N] (P == 1)
     float* ypart;        // [P][M][N] fp32 split sums (P > 1)
@@ -195,10 +200,23 @@ __device__ __forceinline__ void tc_dequant_word(uint32_t w, __half2 dd, uint2& l
     tc_split2(__hsub2(*reinterpret_cast<const __half2*>(&h23), k72), dd, hm.y, hr.y);
 }
 
-static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) {
+// Four signed 8-bit codes of one word (byte e = code e), as f16 q * d in code
+// order, split into main and rest parts (8 bytes each).  (b ^ 0x80) | 0x6400 is
+// the f16 1024 + (q + 128); subtracting 1152 leaves q exactly.
+__device__ __forceinline__ void tc_dequant_word_q8(uint32_t w, __half2 dd, uint2& m, uint2& r) {
+    const __half2 k1152 = __half2half2(__ushort_as_half((unsigned short)0x6480));   // 1152
+    const uint32_t p01 = (__byte_perm(w, 0u, 0x4140) ^ 0x00800080u) | 0x64006400u;
+    const uint32_t p23 = (__byte_perm(w, 0u, 0x4342) ^ 0x00800080u) | 0x64006400u;
+    tc_split2(__hsub2(*reinterpret_cast<const __half2*>(&p01), k1152), dd, m.x, r.x);
+    tc_split2(__hsub2(*reinterpret_cast<const __half2*>(&p23), k1152), dd, m.y, r.y);
+}
+
+template <bool Q8>
+__global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) {
+    constexpr int SEG = tc_seg_bytes(Q8), SCL = Q8 ? 1024 : 512;
     extern __shared__ uint8_t tc_smem_raw[];
     const int L = a.L;
-    const uint32_t ld_bytes = tc_load_stage_bytes(a.Mp);
+    const uint32_t ld_bytes = tc_load_stage_bytes(a.Mp, Q8);
     const uint32_t raw0 = smem_addr(tc_smem_raw);
     const uint32_t base = (raw0 + 1023u) & ~1023u;               // swizzle needs 1024-byte tiles
     const uint32_t ld0 = base + (uint32_t)(kTcABufs * kTcABytes);  // first load stage
@@ -252,10 +270,10 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
                 const int ks = k0 + i, b0 = 2 * ks;
                 const int nb = min(2, a.KB - b0);
                 const uint32_t sB = ld0 + (uint32_t)j * ld_bytes, sraw = sB + bbytes;
-                mbar_arrive_expect_tx(full + j, (uint32_t)(ntiles * nb * 576) + bbytes);
+                mbar_arrive_expect_tx(full + j, (uint32_t)(ntiles * nb * SEG) + bbytes);
                 for (int t = 0; t < ntiles; ++t)
-                    bulk_g2s_addr(sraw + (uint32_t)t * 1152u,
-                                  a.W + ((size_t)(t0 + t) * a.KB + b0) * 576, (uint32_t)nb * 576u,
+                    bulk_g2s_addr(sraw + (uint32_t)(t * 2 * SEG),
+                                  a.W + ((size_t)(t0 + t) * a.KB + b0) * SEG, (uint32_t)(nb * SEG),
                                   full + j);
                 bulk_g2s_addr(sB, a.xi + (size_t)ks * bbytes, bbytes, full + j);
             }
@@ -320,23 +338,42 @@ static __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcA
             }
             const uint32_t sA = base + (uint32_t)(b * kTcABytes + acc * kTcATile);   // main part
             const uint32_t sR = sA + (uint32_t)(kTcAcc * kTcATile);                 // rest part
-            const uint32_t sraw = ld0 + (uint32_t)j * ld_bytes + bbytes + (uint32_t)warp * 1152u;
+            const uint32_t sraw = ld0 + (uint32_t)j * ld_bytes + bbytes + (uint32_t)(warp * 2 * SEG);
             const int nb = min(2, a.KB - 2 * (k0 + i));
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                uint4 wq = make_uint4(0, 0, 0, 0);
+                // Q4_0: one 16-byte word per row i (row g + 8i), low nibbles codes
+                // 4c.., high nibbles 16 + 4c..; Q8_0: two words per row, codes 4c..
+                // then 16 + 4c...
+                uint32_t wv[Q8 ? 8 : 4];
                 uint2 sc = make_uint2(0, 0);
                 if (h < nb) {
-                    wq = lds128(sraw + (uint32_t)(h * 576 + 16 * (4 * g + c)));
-                    sc = lds64(sraw + (uint32_t)(h * 576 + 512 + 8 * g));
+                    const uint32_t seg = sraw + (uint32_t)(h * SEG);
+                    if constexpr (Q8) {
+                        const uint4 u0 = lds128(seg + (uint32_t)(32 * (4 * g + c)));
+                        const uint4 u1 = lds128(seg + (uint32_t)(32 * (4 * g + c) + 16));
+                        wv[0] = u0.x; wv[1] = u0.y; wv[2] = u0.z; wv[3] = u0.w;
+                        wv[4] = u1.x; wv[5] = u1.y; wv[6] = u1.z; wv[7] = u1.w;
+                    } else {
+                        const uint4 u0 = lds128(seg + (uint32_t)(16 * (4 * g + c)));
+                        wv[0] = u0.x; wv[1] = u0.y; wv[2] = u0.z; wv[3] = u0.w;
+                    }
+                    sc = lds64(seg + (uint32_t)(SCL + 8 * g));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < (Q8 ? 8 : 4); ++e) wv[e] = 0;
                 }
-                const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
                 const uint32_t sv[4] = {sc.x, sc.x >> 16, sc.y, sc.y >> 16};
 #pragma unroll
                 for (int ii = 0; ii < 4; ++ii) {
                     const __half2 dd = __half2half2(__ushort_as_half((unsigned short)(sv[ii] & 0xFFFFu)));
                     uint2 lm, lr, hm, hr;
-                    tc_dequant_word(wv[ii], dd, lm, lr, hm, hr);
+                    if constexpr (Q8) {
+                        tc_dequant_word_q8(wv[2 * ii], dd, lm, lr);
+                        tc_dequant_word_q8(wv[2 * ii + 1], dd, hm, hr);
+                    } else {
+                        tc_dequant_word(wv[ii], dd, lm, lr, hm, hr);
+                    }
                     if (h >= nb) { lm = make_uint2(0, 0); lr = lm; hm = lm; hr = lm; }
                     const uint32_t r = arow0 + 8u * (uint32_t)ii;    // r % 8 == g
                     const uint32_t off = r * 128u + (uint32_t)(c & 1) * 8u;

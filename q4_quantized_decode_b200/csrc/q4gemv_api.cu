@@ -385,7 +385,7 @@ int ensure_ximg(q4gemv_ctx* h, size_t bytes, cudaStream_t st) {
 // large as keeps the grid within one wave of the SMs), and for P > 1 the
 // reduce of the fp32 split sums in split order.
 int launch_gemm_tc(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M, int64_t N,
-                   int64_t K, cudaStream_t st) {
+                   int64_t K, cudaStream_t st, bool q8 = false) {
     if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
     const int KB = (int)(K / 32);
     const int nk = (KB + 1) / 2;
@@ -396,12 +396,14 @@ int launch_gemm_tc(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int
     if (P > nk) P = nk;
     const int nkp = (int)((nk + P - 1) / P);
     P = (nk + nkp - 1) / nkp;                        // every split has steps
-    // Load stages: as many as fit beside the two A buffers (at least 2).
-    const size_t fixed = q4::tc_smem_bytes(Mp, 0);
-    const size_t lsb = q4::tc_load_stage_bytes(Mp) + 16;
+    // Load stages: as many as fit beside the two A buffers (2..8; Q8_0 with
+    // more than 240 vectors fits one, which serialises copies and MMAs).
+    const size_t fixed = q4::tc_smem_bytes(Mp, 0, q8);
+    const size_t lsb = q4::tc_load_stage_bytes(Mp, q8) + 16;
     int L = (int)((kMaxDynSmem - fixed) / lsb);
     if (L > 8) L = 8;
-    size_t smem = q4::tc_smem_bytes(Mp, L);
+    if (L < 1) L = 1;
+    size_t smem = q4::tc_smem_bytes(Mp, L, q8);
     // One CTA per SM: each holds all 512 TMEM columns.
     if (smem < 116 * 1024) smem = 116 * 1024;
     int rc = ensure_ximg(h, (size_t)nk * Mp * 128, st);
@@ -432,7 +434,10 @@ int launch_gemm_tc(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int
     a.P = (int)P;
     a.L = L;
     a.idesc = q4::tc_idesc_f16(128, Mp);
-    q4::gemm_tc_kernel<<<dim3((unsigned)tiles, (unsigned)P), q4::kTcThreads, smem, st>>>(a);
+    if (q8)
+        q4::gemm_tc_kernel<true><<<dim3((unsigned)tiles, (unsigned)P), q4::kTcThreads, smem, st>>>(a);
+    else
+        q4::gemm_tc_kernel<false><<<dim3((unsigned)tiles, (unsigned)P), q4::kTcThreads, smem, st>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(h, e, "gemm (tcgen05) launch");
     if (P > 1) {
@@ -478,6 +483,13 @@ int launch_renorm(q4gemv_ctx* h, const __half* in, __half* out, int len, cudaStr
 bool dp2a_fits(int M, int64_t K) {
     return M <= 2 && M * K <= (int64_t)q4::kXChunksPerThread * 8 * kThreads &&
            dp2a_smem(M, K) <= kMaxDynSmem;
+}
+
+// Q8_0: the CUDA-core kernel for M <= 2 where its activation staging fits,
+// the tensor-core GEMM otherwise.
+bool q8_dp2a_fits(int M, int64_t K) {
+    return M <= 2 && M * K <= (int64_t)q4::kXChunksPerThread * 8 * kThreads &&
+           dp2a_smem(M, K, true) <= kMaxDynSmem;
 }
 
 }  // namespace
@@ -578,7 +590,8 @@ int q4gemv_create(q4gemv_t* out, int device) {
         if (set_smem_attr(Q4_DP2A_KERNEL_1) || set_smem_attr(Q4_DP2A_KERNEL_2) ||
             set_smem_attr(Q4_Q8_KERNEL_1) || set_smem_attr(Q4_Q8_KERNEL_2) ||
             set_smem_attr(Q4_MMA_KERNEL_1) || set_smem_attr(Q4_MMA_KERNEL_2) ||
-            set_smem_attr(Q4_STACK_KERNEL) || set_smem_attr(q4::gemm_tc_kernel) ||
+            set_smem_attr(Q4_STACK_KERNEL) || set_smem_attr(q4::gemm_tc_kernel<false>) ||
+            set_smem_attr(q4::gemm_tc_kernel<true>) ||
             0)
             rc = fail(h, Q4_ECUDA, "cudaFuncSetAttribute failed");
     }
@@ -703,11 +716,9 @@ int q4gemv_q8_0_repack(q4gemv_t h, const void* gguf, void* packed, int64_t N, in
 }
 
 int q4gemv_q8_0_validate(int M, int64_t N, int64_t K, const void* W, const void* x, const void* y) {
-    if (M < 1 || M > 2) return Q4_EUNSUPPORTED;
+    if (M < 1 || M > Q4GEMV_MAX_M) return Q4_EUNSUPPORTED;
     const int sh = check_shape(N, K);
     if (sh != Q4_OK) return sh;
-    if (M * K > (int64_t)q4::kXChunksPerThread * 8 * kThreads || dp2a_smem(M, K, true) > kMaxDynSmem)
-        return Q4_EUNSUPPORTED;
     if (!W || !x || !y) return Q4_EINVAL;
     if (!aligned16(W) || !aligned16(x) || !aligned16(y)) return Q4_EALIGN;
     return Q4_OK;
@@ -721,8 +732,11 @@ int q4gemv_q8_0_run(q4gemv_t h, const void* W, const void* x, void* y, int M, in
         return fail(h, v, "q8_0 run: %s (M=%d N=%lld K=%lld)", q4gemv_strerror(v), M, (long long)N,
                     (long long)K);
     Q4_CUDA(h, cudaSetDevice(h->device));
-    return launch_gemv(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K, 0, nullptr,
-                       static_cast<cudaStream_t>(stream), false, true);
+    if (q8_dp2a_fits(M, K))
+        return launch_gemv(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K, 0,
+                           nullptr, static_cast<cudaStream_t>(stream), false, true);
+    return launch_gemm_tc(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K,
+                          static_cast<cudaStream_t>(stream), true);
 }
 
 namespace {

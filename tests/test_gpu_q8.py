@@ -95,9 +95,49 @@ def test_q8_deterministic(eng):
     assert np.array_equal(a, b)
 
 
-def test_q8_rejects_unsupported(eng):
+def test_q8_validate_limits(eng):
     A = 1 << 20
-    assert q4.q4gemv_q8_0_validate(3, 32, 32, A, A, A) == q4.Q4_EUNSUPPORTED
-    assert q4.q4gemv_q8_0_validate(1, 32, 65536, A, A, A) == q4.Q4_EUNSUPPORTED
+    assert q4.q4gemv_q8_0_validate(3, 32, 32, A, A, A) == q4.Q4_OK          # tensor-core GEMM
+    assert q4.q4gemv_q8_0_validate(256, 32, 32, A, A, A) == q4.Q4_OK
+    assert q4.q4gemv_q8_0_validate(1, 32, 65536, A, A, A) == q4.Q4_OK      # wide K: GEMM path
+    assert q4.q4gemv_q8_0_validate(0, 32, 32, A, A, A) == q4.Q4_EUNSUPPORTED
+    assert q4.q4gemv_q8_0_validate(257, 32, 32, A, A, A) == q4.Q4_EUNSUPPORTED
     assert q4.q4gemv_q8_0_validate(1, 32, 48, A, A, A) == q4.Q4_ESHAPE
     assert q4.q4gemv_q8_0_validate(1, 32, 32, A + 8, A, A) == q4.Q4_EALIGN
+
+
+# ---------------------------------------------------------------- M >= 3: tensor-core GEMM
+
+@pytest.mark.parametrize("N,K,M", [(256, 64, 3), (300, 96, 4), (520, 160, 16), (33, 1056, 17),
+                                   (1024, 1024, 86), (5, 32, 256), (2048, 5120, 169),
+                                   (96, 65536, 1), (40, 40960, 2)])
+def test_q8_gemm_shapes_full(eng, N, K, M):
+    gguf, x, y = q8_case(eng, N, K, M, 1300 + N + K + M)
+    ref = oracle.q8_gemv(gguf, K, x, threads=THREADS)
+    err = rel_err(y, ref)
+    assert err <= 5.2e-4, err            # exact two-part weights: output rounding only
+
+
+@pytest.mark.parametrize("M", [16, 169])
+@pytest.mark.parametrize("N,K", [(34816, 5120), (5120, 17408)])
+def test_q8_gemm_full_shapes_sampled(eng, M, N, K):
+    gguf, x, y = q8_case(eng, N, K, M, synth.config_seed(3) + 2000 + M, tid=0 if K == 5120 else 1)
+    y = y.reshape(M, N)
+    rng = np.random.default_rng(M)
+    rows = np.unique(np.concatenate([rng.choice(N, 160, replace=False), [0, 255, 256, N - 1]]))
+    ref = oracle.q8_gemv(np.ascontiguousarray(gguf[rows]), K, x, threads=THREADS)
+    assert rel_err(np.ascontiguousarray(y[:, rows]), ref) <= TOL
+
+
+def test_q8_gemm_extreme_codes_and_deterministic(eng):
+    N, K, M = 300, 512, 40
+    g = synth.q8_0_matrix(15, synth.weight_id(2), N, K).reshape(N, K // 32, 34)
+    g[:, :, 2:] = np.where(np.arange(32) % 3 == 0, 0x80, np.where(np.arange(32) % 3 == 1, 0x7F, 0xFF))
+    g = g.reshape(N, -1)
+    x = synth.activations(15, M, K)
+    W = packed_q8(eng, g, N, K)
+    xd = f16_dev(x).reshape(M, K)
+    a = bits_of(eng.run_q8_0(W, xd, N, K))
+    b = bits_of(eng.run_q8_0(W, xd, N, K))
+    assert np.array_equal(a, b)
+    assert rel_err(a, oracle.q8_gemv(g, K, x)) <= 5.2e-4
