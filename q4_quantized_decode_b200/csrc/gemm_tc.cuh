@@ -46,7 +46,6 @@ namespace q4 {
 constexpr int kTcAcc = 2;                       // 128-row accumulators per CTA
 constexpr int kTcRows = 128 * kTcAcc;           // output rows per CTA
 constexpr int kTcTiles = kTcRows / 32;          // packed 32-row tiles per CTA
-constexpr int kTcKStep = 64;                    // columns per stage
 constexpr int kTcDqWarps = 4 * kTcAcc;          // dequantise / epilogue warps
 constexpr int kTcThreads = 32 * (kTcDqWarps + 2);
 constexpr int kTcMaxVec = 256;                  // MMA N limit (vectors)
@@ -140,11 +139,6 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_addr(bar)) : "memory");
-}
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-    uint32_t v;
-    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
 }
 
 // Bounded wait that also gives up as soon as another role has aborted.

@@ -30,6 +30,7 @@ constexpr int kMaxTiles = Q4GEMV_MAX_N / 32;
 constexpr size_t kMaxDynSmem = 224 * 1024;   // opt-in dynamic shared memory per CTA
 constexpr size_t kYaccPrealloc = (size_t)1 << 21;   // fp32 panel accumulator floats at create
 constexpr size_t kXimgPrealloc = (size_t)1 << 24;   // GEMM activation image bytes at create
+static_assert(q4::kTcMaxVec == Q4GEMV_MAX_M, "the GEMM's MMA width bounds M");
 
 #define Q4_DP2A_KERNEL_1 q4::gemv_dp2a_kernel<1, kWarps, kR1, kC1>
 #define Q4_DP2A_KERNEL_2 q4::gemv_dp2a_kernel<2, kWarps, kR2, kC2>
