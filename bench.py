@@ -41,7 +41,7 @@ METRIC = "achieved HBM GB/s (% of B200 peak) for Q4_0 GEMV; 27B-shaped decode st
 L, HIDDEN, QKV_N, FFN = 64, 5120, 7168, 17408   # L: layers of the step (--layers)
 DIMS = [(QKV_N, HIDDEN), (HIDDEN, HIDDEN), (2 * FFN, HIDDEN), (HIDDEN, FFN)]
 SHAPE_NAMES = ["qkv_5120x7168", "o_5120x5120", "gate_up_5120x34816", "down_17408x5120"]
-CONFIG_SEED = synth.config_seed(4)
+STEP_SEED = synth.workload_seed(4)
 NOMINAL_HBM_GBS = 8000.0
 
 
@@ -171,11 +171,11 @@ def oracle_sample(min_seconds: float, threads: int):
     matrices) until at least `min_seconds` have elapsed; returns GB/s of
     Q4_0 bytes (+x,y) and a description of the sample."""
     import oracle
-    x = synth.normal_f16(CONFIG_SEED, synth.act_id(0), max(HIDDEN, FFN))
+    x = synth.normal_f16(STEP_SEED, synth.act_id(0), max(HIDDEN, FFN))
     done_bytes, elapsed, layers = 0, 0.0, 0
     while elapsed < min_seconds and layers < L:
         for t, (N, K) in enumerate(DIMS):
-            rows = synth.q4_0_matrix(CONFIG_SEED, synth.weight_id(4 * layers + t), N, K)
+            rows = synth.q4_0_matrix(STEP_SEED, synth.weight_id(4 * layers + t), N, K)
             t0 = time.perf_counter()
             oracle.q4_gemv(rows, K, x[None, :K], threads=threads)
             elapsed += time.perf_counter() - t0
@@ -191,9 +191,9 @@ def oracle_rows_step(i: int, threads: int, frac: int = 64):
     l, t = (i // 4) % L, i % 4
     N, K = DIMS[t]
     sel = np.arange(0, N, frac)
-    rows = synth.q4_0_row_list(CONFIG_SEED, synth.weight_id(4 * l + t), K, sel) if len(sel) < 64 else \
-        synth.q4_0_matrix(CONFIG_SEED, synth.weight_id(4 * l + t), N, K)[sel]
-    x = synth.normal_f16(CONFIG_SEED, synth.act_id(0), K)
+    rows = synth.q4_0_row_list(STEP_SEED, synth.weight_id(4 * l + t), K, sel) if len(sel) < 64 else \
+        synth.q4_0_matrix(STEP_SEED, synth.weight_id(4 * l + t), N, K)[sel]
+    x = synth.normal_f16(STEP_SEED, synth.act_id(0), K)
     t0 = time.perf_counter()
     oracle.q4_gemv(rows, K, x[None, :], threads=threads)
     dt = time.perf_counter() - t0
@@ -239,7 +239,7 @@ def build_weights(eng, torch, rank: int):
     for l in range(L):
         mats = []
         for t, (N, K) in enumerate(DIMS):
-            synth.q4_0_matrix(CONFIG_SEED, synth.weight_id(4 * l + t), N, K, out=host[t])
+            synth.q4_0_matrix(STEP_SEED, synth.weight_id(4 * l + t), N, K, out=host[t])
             g = staging[: host[t].size]
             g.copy_(torch.from_numpy(host[t].reshape(-1)))
             torch.cuda.synchronize()
@@ -287,7 +287,7 @@ def time_prefill(eng, torch, layers, M: int = 169, reps: int = 3):
     tokens) on the step's 64 distinct gate+up matrices (larger than L2): a
     CUDA graph of 64 launches.  Outside the timed step; context only."""
     N, K = DIMS[2]
-    x = torch.from_numpy(synth.activations(CONFIG_SEED + 169, M, K).view(np.float16)).cuda()
+    x = torch.from_numpy(synth.activations(STEP_SEED + 169, M, K).view(np.float16)).cuda()
     y = torch.empty(M, N, device="cuda", dtype=torch.float16)
     eng.run(layers[0][2], x, N, K, out=y)
     torch.cuda.synchronize()
@@ -322,7 +322,7 @@ def run_ours(args, rank: int, world: int, dist):
     dev = torch.device("cuda", local)
     eng = q4.Q4Gemv(local)
     layers, t_repack = build_weights(eng, torch, rank)
-    x_host = torch.from_numpy(synth.normal_f16(CONFIG_SEED, synth.act_id(rank), HIDDEN).view(np.float16)).pin_memory()
+    x_host = torch.from_numpy(synth.normal_f16(STEP_SEED, synth.act_id(rank), HIDDEN).view(np.float16)).pin_memory()
     out_host = torch.empty(HIDDEN, dtype=torch.float16).pin_memory()
     x_in = x_host.to(dev)
     x_out = torch.empty(HIDDEN, dtype=torch.float16, device=dev)
@@ -427,7 +427,7 @@ def run_ours(args, rank: int, world: int, dist):
         "config": {"workload": WORKLOAD, "bytes_per_step": STEP_GEMV_BYTES,
                    "weight_bytes_per_step": STEP_WEIGHT_BYTES,
                    "l2": "inputs larger than L2 (11.9 GB of weights per step)",
-                   "parallelism": f"replicas x{world}", "seed": CONFIG_SEED},
+                   "parallelism": f"replicas x{world}", "seed": STEP_SEED},
         "decode_steps_per_s": steps_per_s,
         "pct_of_8TBps_nominal": 100.0 * per_rank_gbs / NOMINAL_HBM_GBS,
         "roofline": roofline,
@@ -446,7 +446,7 @@ def run_ours(args, rank: int, world: int, dist):
 
 
 def run_case(args):
-    """Standalone GEMV timing on one shape (configs 0-3 and profiling): R
+    """Standalone GEMV timing on one shape (single-shape workloads and profiling): R
     copies of one packed matrix (R * size > 4 x L2 unless --rotate is given)
     launched in rotation inside a CUDA graph; prints one JSON line."""
     import torch
@@ -455,7 +455,7 @@ def run_case(args):
     M = args.M
     q8 = args.format == "q8_0"
     eng = q4.Q4Gemv(0)
-    seed = synth.config_seed(args.config_seed)
+    seed = synth.workload_seed(args.workload_seed)
     if q8:
         gguf = synth.q8_0_matrix(seed, synth.weight_id(0), N, K)
         W0 = eng.repack_q8_0(torch.from_numpy(gguf.reshape(-1)).cuda(), N, K)
@@ -529,7 +529,7 @@ def main():
     ap.add_argument("--shape", default="34816x5120", help="NxK for --case gemv")
     ap.add_argument("--M", type=int, default=1)
     ap.add_argument("--rotate", type=int, default=0, help="matrix copies in rotation (0: > 4x L2)")
-    ap.add_argument("--config-seed", type=int, default=2)
+    ap.add_argument("--workload-seed", type=int, default=2)
     ap.add_argument("--format", choices=["q4_0", "q8_0"], default="q4_0", help="weights of --case gemv")
     ap.add_argument("--layers", type=int, default=64, help="layers of the step (profiling only)")
     args = ap.parse_args()

@@ -10,7 +10,10 @@ Workload recipe (value distributions of the 27B-shaped decode workload):
   * Q4_0 scale d ~ U[0.002, 0.05] with a random sign, rounded to f16;
     nibbles q ~ U{0..15};
   * activations x ~ N(0, 1) rounded to f16;
-  * seeds: ``config_seed(c) = 0x5EED0000 + c``;
+  * seeds: ``workload_seed(w) = 0x5EED0000 + w`` with w = 0 for the single
+    1024 x 1024 GEMV, 1 for the 5120 x 5120 GEMV, 2 for the FFN GEMVs (gate+up
+    34816 x 5120, down 5120 x 17408), 3 for the small-M batches on those
+    shapes, 4 for the 64-layer decode step;
   * tensor ids: weight matrix j -> ``weight_id(j)``, activation row m ->
     ``act_id(m)`` (separate id spaces, so every tensor is its own stream).
 """
@@ -68,8 +71,8 @@ def _load():
     return _lib
 
 
-def config_seed(c: int) -> int:
-    return 0x5EED0000 + int(c)
+def workload_seed(w: int) -> int:
+    return 0x5EED0000 + int(w)
 
 
 def weight_id(j: int) -> int:

@@ -71,8 +71,8 @@ def test_gemm_prefill_widths_full_shapes_sampled(eng, M, N, K):
     """The gate+up and down shapes at the pages' prompt lengths; the oracle
     computes a sample of rows (all vectors) one by one."""
     tid = 0 if K == 5120 else 1
-    gguf = synth.q4_0_matrix(synth.config_seed(3) + M, synth.weight_id(tid), N, K)
-    x = synth.activations(synth.config_seed(3) + 1000 + M, M, K)
+    gguf = synth.q4_0_matrix(synth.workload_seed(3) + M, synth.weight_id(tid), N, K)
+    x = synth.activations(synth.workload_seed(3) + 1000 + M, M, K)
     y = run_case(eng, gguf, x, N, K)
     rows = sampled_rows(N, seed=M)
     ref = oracle.q4_gemv(np.ascontiguousarray(gguf[rows]), K, x, threads=THREADS)

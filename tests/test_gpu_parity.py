@@ -49,18 +49,18 @@ def test_repack_bit_exact(eng, N, K):
 
 # ---------------------------------------------------------------- GEMV, M = 1, 2
 
-CONFIGS = {
-    "c0_1024x1024": (1024, 1024, 0),
-    "c1_5120x5120": (5120, 5120, 1),
-    "c2a_gateup_34816x5120": (34816, 5120, 2),
-    "c2b_down_5120x17408": (5120, 17408, 2),
+M1_SHAPES = {
+    "gemv_1024x1024": (1024, 1024, 0),
+    "o_5120x5120": (5120, 5120, 1),
+    "gate_up_34816x5120": (34816, 5120, 2),
+    "down_5120x17408": (5120, 17408, 2),
 }
 
 
-@pytest.mark.parametrize("name", list(CONFIGS))
-def test_gemv_m1_configs(eng, name):
-    N, K, c = CONFIGS[name]
-    gguf, x, y = gemv_case(eng, N, K, 1, synth.config_seed(c), tid=0 if "down" not in name else 1)
+@pytest.mark.parametrize("name", list(M1_SHAPES))
+def test_gemv_m1_shapes(eng, name):
+    N, K, c = M1_SHAPES[name]
+    gguf, x, y = gemv_case(eng, N, K, 1, synth.workload_seed(c), tid=0 if "down" not in name else 1)
     ref = oracle.q4_gemv(gguf, K, x, threads=THREADS)
     err = rel_err(y, ref)
     assert err <= TOL, err
@@ -75,9 +75,9 @@ def test_gemv_m2(eng, N, K):
 
 @pytest.mark.parametrize("M", [4, 16])
 @pytest.mark.parametrize("N,K", [(34816, 5120), (5120, 17408)])
-def test_gemv_small_m_configs(eng, M, N, K):
-    """Config 3: speculative-verify batch (M=4) and prefill chunk (M=16)."""
-    gguf, x, y = gemv_case(eng, N, K, M, synth.config_seed(3) + M, tid=0 if K == 5120 else 1)
+def test_gemv_small_m_shapes(eng, M, N, K):
+    """Speculative-verify batch (M=4) and prefill chunk (M=16) on the FFN shapes."""
+    gguf, x, y = gemv_case(eng, N, K, M, synth.workload_seed(3) + M, tid=0 if K == 5120 else 1)
     ref = oracle.q4_gemv(gguf, K, x, threads=THREADS)
     err = rel_err(y, ref)
     assert err <= TOL, err
@@ -352,7 +352,7 @@ def test_stack_full_27b_teacher_forced_sampled():
     on sampled rows from the GPU's own traced inputs."""
     eng = q4.Q4Gemv(0)
     L, hidden, qkv_n, ffn = 64, 5120, 7168, 17408
-    seed = synth.config_seed(4)
+    seed = synth.workload_seed(4)
     dims = [(qkv_n, hidden), (hidden, hidden), (2 * ffn, hidden), (hidden, ffn)]
     layers = []
     for l in range(L):

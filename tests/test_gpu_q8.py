@@ -48,7 +48,7 @@ def test_q8_repack_bit_exact(eng, N, K):
 
 @pytest.mark.parametrize("N,K", [(1024, 1024), (5120, 5120), (34816, 5120), (5120, 17408)])
 def test_q8_gemv_m1_config_shapes(eng, N, K):
-    gguf, x, y = q8_case(eng, N, K, 1, synth.config_seed(1) + 80)
+    gguf, x, y = q8_case(eng, N, K, 1, synth.workload_seed(1) + 80)
     ref = oracle.q8_gemv(gguf, K, x, threads=THREADS)
     err = rel_err(y, ref)
     assert err <= TOL, err
@@ -121,7 +121,7 @@ def test_q8_gemm_shapes_full(eng, N, K, M):
 @pytest.mark.parametrize("M", [16, 169])
 @pytest.mark.parametrize("N,K", [(34816, 5120), (5120, 17408)])
 def test_q8_gemm_full_shapes_sampled(eng, M, N, K):
-    gguf, x, y = q8_case(eng, N, K, M, synth.config_seed(3) + 2000 + M, tid=0 if K == 5120 else 1)
+    gguf, x, y = q8_case(eng, N, K, M, synth.workload_seed(3) + 2000 + M, tid=0 if K == 5120 else 1)
     y = y.reshape(M, N)
     rng = np.random.default_rng(M)
     rows = np.unique(np.concatenate([rng.choice(N, 160, replace=False), [0, 255, 256, N - 1]]))

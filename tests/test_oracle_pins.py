@@ -42,7 +42,7 @@ def test_generator_counter_access_is_consistent():
 
 
 def test_generator_distributions():
-    g = synth.q4_0_matrix(synth.config_seed(1), synth.weight_id(0), 512, 1024)
+    g = synth.q4_0_matrix(synth.workload_seed(1), synth.weight_id(0), 512, 1024)
     blocks = g.reshape(-1, 18)
     d = f16_values(blocks[:, 0].astype(np.uint16) | (blocks[:, 1].astype(np.uint16) << 8))
     assert 0.0019 < np.abs(d).min() and np.abs(d).max() <= 0.05
@@ -50,7 +50,7 @@ def test_generator_distributions():
     nib = np.concatenate([blocks[:, 2:] & 15, blocks[:, 2:] >> 4]).ravel()
     counts = np.bincount(nib, minlength=16) / nib.size
     assert np.all(np.abs(counts - 1 / 16) < 0.002)
-    x = f16_values(synth.normal_f16(synth.config_seed(1), synth.act_id(0), 200000))
+    x = f16_values(synth.normal_f16(synth.workload_seed(1), synth.act_id(0), 200000))
     assert abs(x.mean()) < 0.01 and abs(x.std() - 1) < 0.01
 
 
