@@ -252,6 +252,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) 
     if (warp == kTcDqWarps) {
         // ---- producer: bulk copies of each K step into load stage i % L ----
         if (lane == 0) {
+            // Launched as a dependent of the activation-image kernel: the
+            // image (and anything earlier in the stream) is complete and
+            // visible after this wait; the prologue above overlapped it.
+            pdl_wait();
             const int ntiles = min(kTcTiles, a.T - t0);
             int i = 0;
             for (; i < ns; ++i) {
@@ -430,6 +434,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) 
 static __global__ void __launch_bounds__(256) tc_ximg_kernel(const __half* __restrict__ x,
                                                            uint8_t* __restrict__ img, int M, int K,
                                                            int Mp, int nk) {
+    pdl_launch_dependents();      // the GEMM may start its prologue now
     const int64_t total = (int64_t)nk * Mp * 8;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < total; q += stride) {

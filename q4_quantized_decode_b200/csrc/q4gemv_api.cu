@@ -435,11 +435,18 @@ int launch_gemm_tc(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int
     a.P = (int)P;
     a.L = L;
     a.idesc = q4::tc_idesc_f16(128, Mp);
-    if (q8)
-        q4::gemm_tc_kernel<true><<<dim3((unsigned)tiles, (unsigned)P), q4::kTcThreads, smem, st>>>(a);
-    else
-        q4::gemm_tc_kernel<false><<<dim3((unsigned)tiles, (unsigned)P), q4::kTcThreads, smem, st>>>(a);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t gcfg = {};
+    gcfg.gridDim = dim3((unsigned)tiles, (unsigned)P);
+    gcfg.blockDim = dim3(q4::kTcThreads);
+    gcfg.dynamicSmemBytes = smem;
+    gcfg.stream = st;
+    cudaLaunchAttribute gattr[1];
+    gattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    gattr[0].val.programmaticStreamSerializationAllowed = 1;
+    gcfg.attrs = gattr;
+    gcfg.numAttrs = 1;
+    e = q8 ? cudaLaunchKernelEx(&gcfg, q4::gemm_tc_kernel<true>, a)
+           : cudaLaunchKernelEx(&gcfg, q4::gemm_tc_kernel<false>, a);
     if (e != cudaSuccess) return cuda_fail(h, e, "gemm (tcgen05) launch");
     if (P > 1) {
         const int64_t MN = (int64_t)M * N;
