@@ -138,8 +138,9 @@ Q4GEMV_API int q4gemv_repack(q4gemv_t h, const void* gguf, void* packed,
  * to 2^-15 of the block maximum) and the per-block dot products are exact
  * integers.  Deterministic: the same inputs on the same device give the
  * same bits.
- * For M >= 3 (and M <= 2 with K beyond the CUDA-core kernel's activation
- * staging) the tensor-core kernel runs, as a grid of P column panels whose
+ * For 3 <= M <= 16 (and M <= 2 with K beyond the CUDA-core kernel's
+ * activation staging) the mma.sync tensor-core kernel runs, as a grid of P
+ * column panels whose
  * fp32 sums a second small kernel adds in panel order (P = 1 for large N and
  * K up to about 6,000 columns; more panels for narrow N, so a CTA stages a
  * short activation slice, and for wider K).  The panel sums live in a buffer
