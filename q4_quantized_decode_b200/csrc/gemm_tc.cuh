@@ -1,11 +1,14 @@
-// Q4_0 GEMM for M = 17..256 activation vectors (prefill chunks) on the
-// 5th-generation tensor cores: Y[m][n] = sum_k W[n][k] * X[m][k].
+// Q4_0 / Q8_0 GEMM for M = 17..256 activation vectors (prefill chunks; Q8_0
+// also for M = 3..16 and wide K) on the 5th-generation tensor cores:
+// Y[m][n] = sum_k W[n][k] * X[m][k].
 //
 // Dequantise-then-multiply, the reading of "dequantise a weight tile once and
-// apply it to every vector".  A weight (q - 8) * d has up to 14 significant
-// bits, more than binary16 holds, so it is split exactly into two binary16
-// values: main = RN((q - 8) * d) and rest = (q - 8) * d - main (a multiple of
-// d's last bit below main's last bit: at most 4 bits, always representable).
+// apply it to every vector".  A weight w = q * d (q = the nibble - 8, or the
+// signed byte) has up to 14 (Q4_0) or 18 (Q8_0) significant bits, more than
+// binary16 holds, so it is split exactly into two binary16 values:
+// main = RN(w) and rest = w - main (a multiple of d's last bit below main's
+// last bit, so it has at most 7 significant bits and is representable unless
+// main overflowed).
 // Both parts multiply the same activations, so every weight costs two f16
 // products; these are exact in fp32 and accumulate in fp32 in tensor memory,
 // which leaves fp32 summation as the only error before the output rounding.
