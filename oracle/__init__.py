@@ -1,12 +1,13 @@
 """ORACLE -- test infrastructure only.
 
 Plain fp64 CPU restatement of the Q4_0 dequantise-and-multiply GEMV, the
-repack layout and the renormalised layer chain (see ``q4_oracle.c`` for the
-citations).  Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's
+repack layout, the renormalised layer chain and the SiLU-gated input of the
+down GEMV (see ``q4_oracle.c`` for the citations and readings).  Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's
 CPU-baseline / reference leg may import this package; the CUDA product path
 never does and shares no code with it.
 
-Every function here is pinned in ``tests/test_oracle_pins.py``.  The layer
+Every function here is pinned in ``tests/test_oracle_pins.py`` (SiLU gating:
+``tests/test_oracle_swiglu_pins.py``).  The layer
 chain (``stack_step``) is pinned by signed-permutation stacks whose result has
 a closed form.
 """
@@ -59,6 +60,10 @@ def _configure(lib):
     lib.oracle_unit_rms_scale.restype = ctypes.c_double
     lib.oracle_round_f16.argtypes = [vp, i64, vp]
     lib.oracle_round_f16.restype = None
+    lib.oracle_swiglu.argtypes = [vp, i64, i64, vp]
+    lib.oracle_swiglu.restype = None
+    lib.oracle_q4_gemv_f64.argtypes = [vp, i64, i64, vp, i64, vp]
+    lib.oracle_q4_gemv_f64.restype = None
     return lib
 
 
@@ -137,6 +142,49 @@ def _gemv(fn, block_bytes: int, rows: np.ndarray, K: int, x: np.ndarray, threads
     with ThreadPoolExecutor(threads) as ex:
         list(ex.map(work, range(threads)))
     return np.concatenate(parts, axis=1)
+
+
+def swiglu(gate_up: np.ndarray) -> np.ndarray:
+    """u[M][K] = SiLU(gate) * up (fp64) for f16 bit patterns [M][2K] laid out
+    as [gate | up] (see ``q4_oracle.c`` for the reading)."""
+    v = np.ascontiguousarray(np.atleast_2d(gate_up), dtype=np.uint16)
+    M, K2 = v.shape
+    assert K2 % 2 == 0
+    u = np.empty((M, K2 // 2), dtype=np.float64)
+    _load().oracle_swiglu(v.ctypes.data, K2 // 2, M, u.ctypes.data)
+    return u
+
+
+def q4_gemv_f64(rows: np.ndarray, K: int, x: np.ndarray, threads: int = 1) -> np.ndarray:
+    """As q4_gemv with an fp64 input x[M][K]."""
+    rows = np.ascontiguousarray(rows, dtype=np.uint8)
+    x = np.ascontiguousarray(np.atleast_2d(x), dtype=np.float64)
+    M = x.shape[0]
+    assert x.shape[1] == K and K % 32 == 0
+    rb = (K // 32) * 18
+    nrows = rows.size // rb
+    assert rows.size == nrows * rb
+    fn = _load().oracle_q4_gemv_f64
+    if threads <= 1 or nrows < 2 * threads:
+        y = np.empty((M, nrows), dtype=np.float64)
+        fn(rows.ctypes.data, nrows, K, x.ctypes.data, M, y.ctypes.data)
+        return y
+    bounds = np.linspace(0, nrows, threads + 1).astype(np.int64)
+    parts = [np.empty((M, int(bounds[i + 1] - bounds[i])), dtype=np.float64) for i in range(threads)]
+
+    def work(i):
+        r0, r1 = int(bounds[i]), int(bounds[i + 1])
+        if r1 > r0:
+            fn(rows.ctypes.data + r0 * rb, r1 - r0, K, x.ctypes.data, M, parts[i].ctypes.data)
+
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(work, range(threads)))
+    return np.concatenate(parts, axis=1)
+
+
+def q4_gemv_swiglu(rows: np.ndarray, K: int, gate_up: np.ndarray, threads: int = 1) -> np.ndarray:
+    """y = W (SiLU(gate) * up): the down GEMV fed by the gate+up output."""
+    return q4_gemv_f64(rows, K, swiglu(gate_up), threads)
 
 
 def packed_bytes(N: int, K: int) -> int:

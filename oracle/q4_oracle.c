@@ -204,3 +204,35 @@ void oracle_renorm(const uint16_t* v, int64_t len, uint16_t* out) {
 void oracle_round_f16(const double* v, int64_t n, uint16_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_f64_to_f16(v[i]);
 }
+
+/* SiLU(gate) * up for a 2K-entry f16 vector [gate | up] (the gate+up GEMV's
+ * output), in fp64: u_k = g_k / (1 + exp(-g_k)) * up_k.  The pages name the
+ * model family (Qwen 3.8 27B: taozi.news page, section "支持模型与限制";
+ * originshq.com page, "Limitations and Open Questions") but not its FFN
+ * activation; the reading used is that family's gated unit: SiLU of the gate
+ * half times the up half, fed to the down GEMV unrounded. */
+void oracle_swiglu(const uint16_t* gate_up, int64_t K, int64_t M, double* u) {
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t* v = gate_up + m * 2 * K;
+        for (int64_t k = 0; k < K; ++k) {
+            const double g = oracle_f16_to_f64(v[k]);
+            const double p = oracle_f16_to_f64(v[K + k]);
+            u[m * K + k] = g / (1.0 + exp(-g)) * p;
+        }
+    }
+}
+
+/* As oracle_q4_gemv with an fp64 input x[M][K] (not f16 bit patterns). */
+void oracle_q4_gemv_f64(const uint8_t* rows, int64_t nrows, int64_t K,
+                        const double* x, int64_t M, double* y) {
+    const int64_t rb = (K / 32) * 18;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t r = 0; r < nrows; ++r) {
+            const uint8_t* row = rows + r * rb;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += q4_0_weight(row, k) * x[m * K + k];
+            y[m * nrows + r] = acc;
+        }
+    }
+}

@@ -8,6 +8,7 @@ import pytest
 import oracle
 from tests import test_oracle_pins as pins
 from tests import test_oracle_q8_pins as q8pins
+from tests import test_oracle_swiglu_pins as swpins
 
 SRC = open(os.path.join(os.path.dirname(oracle.__file__), "q4_oracle.c")).read()
 
@@ -112,5 +113,46 @@ def test_q8_mutant_is_caught(name, tmp_path):
             except (AssertionError, ValueError, IndexError):
                 caught += 1
         assert caught > 0, f"no Q8_0 pin catches mutant {name}"
+    finally:
+        oracle._restore_library(prev)
+
+
+# Planted in the SiLU-gated input of the down GEMV; caught by its pins.
+SWIGLU_MUTANTS = {
+    "silu_exponent_sign": ("g / (1.0 + exp(-g)) * p", "g / (1.0 + exp(g)) * p"),
+    "up_read_from_gate_half": ("oracle_f16_to_f64(v[K + k])", "oracle_f16_to_f64(v[k])"),
+    "gate_without_silu": ("g / (1.0 + exp(-g)) * p", "g * p"),
+    "f64_gemv_drops_last_column": ("for (int64_t k = 0; k < K; ++k)\n                acc += q4_0_weight(row, k) * x[m * K + k];",
+                                   "for (int64_t k = 0; k < K - 1; ++k)\n                acc += q4_0_weight(row, k) * x[m * K + k];"),
+}
+
+SWIGLU_PIN_TESTS = [
+    swpins.test_odd_part_of_silu_is_the_identity,
+    swpins.test_taylor_series_at_zero_fixes_the_sign_of_the_exponent,
+    swpins.test_limits,
+    swpins.test_linear_in_the_up_half_and_gate_is_the_first_half,
+    swpins.test_f64_gemv_matches_the_f16_gemv_on_f16_inputs,
+    swpins.test_gated_gemv_dense_brute_force,
+]
+
+
+@pytest.mark.parametrize("name", sorted(SWIGLU_MUTANTS))
+def test_swiglu_mutant_is_caught(name, tmp_path):
+    old, new = SWIGLU_MUTANTS[name]
+    assert old in SRC, f"mutation anchor for {name} no longer in the oracle"
+    src = tmp_path / "mut.c"
+    src.write_text(SRC.replace(old, new, 1))
+    so = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+                           str(src), "-o", str(so), "-lm"])
+    prev = oracle._swap_library(str(so))
+    try:
+        caught = 0
+        for t in SWIGLU_PIN_TESTS:
+            try:
+                t()
+            except (AssertionError, ValueError, IndexError):
+                caught += 1
+        assert caught > 0, f"no SiLU pin catches mutant {name}"
     finally:
         oracle._restore_library(prev)
