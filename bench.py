@@ -454,6 +454,9 @@ def run_case(args):
     N, K = (int(v) for v in args.shape.lower().split("x"))
     M = args.M
     q8 = args.format == "q8_0"
+    gated = args.act == "swiglu"
+    if gated and (q8 or M != 1):
+        raise SystemExit("--act swiglu: Q4_0 and M = 1 only")
     eng = q4.Q4Gemv(0)
     seed = synth.workload_seed(args.workload_seed)
     if q8:
@@ -464,10 +467,13 @@ def run_case(args):
         gguf = synth.q4_0_matrix(seed, synth.weight_id(0), N, K)
         W0 = eng.repack(torch.from_numpy(gguf.reshape(-1)).cuda(), N, K)
         run = eng.run
+        if gated:      # the down GEMV fed by a [gate | up] vector of 2K entries
+            def run(W, x, N, K, out=None):
+                return eng.run_swiglu(W, x.reshape(-1), N, K, out=out)
     l2 = torch.cuda.get_device_properties(0).L2_cache_size
     R = args.rotate or max(2, -(-4 * l2 // W0.numel()))
     mats = [W0] + [W0.clone() for _ in range(R - 1)]
-    x = torch.from_numpy(synth.activations(seed, M, K).view(np.float16)).cuda()
+    x = torch.from_numpy(synth.activations(seed, M, 2 * K if gated else K).view(np.float16)).cuda()
     y = torch.empty(M, N, dtype=torch.float16, device="cuda")
     run(mats[0], x, N, K, out=y)
     torch.cuda.synchronize()
@@ -488,9 +494,9 @@ def run_case(args):
     if eng.sync_status() != q4.Q4_OK:
         raise RuntimeError("device status")
     us = e0.elapsed_time(e1) * 1e3 / (args.steps * R)
-    nbytes = N * (K // 32) * (34 if q8 else 18) + 2 * M * (K + N)
+    nbytes = N * (K // 32) * (34 if q8 else 18) + 2 * M * ((2 * K if gated else K) + N)
     peak, kind = measured_peaks()
-    line = {"case": f"gemv {args.format} M={M} {N}x{K}", "N": N, "K": K, "M": M, "rotate": R,
+    line = {"case": f"gemv {args.format}{' swiglu' if gated else ''} M={M} {N}x{K}", "N": N, "K": K, "M": M, "rotate": R,
             "us_per_launch": us, "GB/s": nbytes / us / 1e3,
             "frac_of_peak": nbytes / us / 1e3 / peak, "peak": peak, "peak_kind": kind,
             "rows_per_s": N / us * 1e6, "tflops": 2 * M * N * K / us / 1e6,
@@ -531,6 +537,8 @@ def main():
     ap.add_argument("--rotate", type=int, default=0, help="matrix copies in rotation (0: > 4x L2)")
     ap.add_argument("--workload-seed", type=int, default=2)
     ap.add_argument("--format", choices=["q4_0", "q8_0"], default="q4_0", help="weights of --case gemv")
+    ap.add_argument("--act", choices=["none", "swiglu"], default="none",
+                    help="--case gemv: feed the GEMV SiLU(gate) * up of a 2K input (M = 1)")
     ap.add_argument("--layers", type=int, default=64, help="layers of the step (profiling only)")
     args = ap.parse_args()
     if args.layers != 64:

@@ -166,6 +166,20 @@ Q4GEMV_API int q4gemv_run(q4gemv_t h, const void* W_packed, const void* x, void*
  * bytes: an f16 scale d (little-endian), then 32 signed 8-bit codes; weight
  * j of a block is qs[j] * d. */
 
+/* The down GEMV fed directly by the gate+up GEMV: y[N] = W u for a packed
+ * Q4_0 W (N x K), with u_k = SiLU(g_k) * up_k = g_k / (1 + e^-g_k) * up_k and
+ * gate_up = [g | up] the 2K-entry binary16 output of the gate+up GEMV (gate
+ * half first).  The pages name the model family but not its FFN activation;
+ * this is that family's gated unit.  u is computed in fp32 inside the kernel
+ * (never written) and converted per 32-column block like any M = 1 input;
+ * exact integer block sums, fp32 accumulation, y rounded once.
+ *   gate_up : device, 2K binary16, 16-byte aligned
+ *   y       : device, N binary16
+ * Q4_EUNSUPPORTED for K beyond the M = 1 kernel's staging (K <= 36,864 and
+ * its shared memory); otherwise errors as q4gemv_run.  Deterministic. */
+Q4GEMV_API int q4gemv_run_swiglu(q4gemv_t h, const void* W_packed, const void* gate_up,
+                      void* y, int64_t N, int64_t K, q4gemv_stream_t stream);
+
 /* Bytes of a GGUF Q8_0 matrix: N * (K/32) * 34; 0 if the shape is invalid. */
 Q4GEMV_API size_t q4gemv_q8_0_gguf_bytes(int64_t N, int64_t K);
 

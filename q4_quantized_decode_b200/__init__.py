@@ -56,6 +56,7 @@ def _load_library():
         "q4gemv_validate": ([ci, i64, i64, vp, vp, vp], ci),
         "q4gemv_repack": ([vp, vp, vp, i64, i64, vp], ci),
         "q4gemv_run": ([vp, vp, vp, vp, ci, i64, i64, vp], ci),
+        "q4gemv_run_swiglu": ([vp, vp, vp, vp, i64, i64, vp], ci),
         "q4gemv_run_stack": ([vp, ctypes.POINTER(q4gemv_layer), ci, i64, i64, i64,
                               vp, vp, vp, vp, vp], ci),
         "q4gemv_sync_status": ([vp, vp], ci),
@@ -120,6 +121,10 @@ def q4gemv_repack(h, gguf, packed, N, K, stream) -> int:
 
 def q4gemv_run(h, W, x, y, M, N, K, stream) -> int:
     return _lib.q4gemv_run(h, W, x, y, M, N, K, stream)
+
+
+def q4gemv_run_swiglu(h, W, gate_up, y, N, K, stream) -> int:
+    return _lib.q4gemv_run_swiglu(h, W, gate_up, y, N, K, stream)
 
 
 def q4gemv_run_stack(h, layers, n_layers, hidden, qkv_n, ffn, x_in, x_out,
@@ -219,6 +224,15 @@ class Q4Gemv:
             out = torch.empty((M, N), dtype=torch.float16, device=x.device)
         self._check(q4gemv_run(self.h, _ptr(W_packed), _ptr(x2), _ptr(out), M, N, K,
                                _stream(stream)))
+        return out
+
+    def run_swiglu(self, W_packed, gate_up, N: int, K: int, out=None, stream=None):
+        """gate_up: f16 CUDA tensor [2K] ([gate | up]) -> y f16 [N] = W (SiLU(gate) * up)."""
+        import torch
+        if out is None:
+            out = torch.empty(N, dtype=torch.float16, device=gate_up.device)
+        self._check(q4gemv_run_swiglu(self.h, _ptr(W_packed), _ptr(gate_up), _ptr(out), N, K,
+                                      _stream(stream)))
         return out
 
     def repack_q8_0(self, gguf, N: int, K: int, out=None, stream=None):

@@ -14,6 +14,7 @@
 #include "gemv_dp2a.cuh"
 #include "gemm_tc.cuh"
 #include "gemv_mma.cuh"
+#include "gemv_swiglu.cuh"
 #include "stack.cuh"
 
 namespace {
@@ -42,6 +43,7 @@ constexpr int kRq1 = 3, kCq1 = 3, kRq2 = 2, kCq2 = 3;
 #define Q4_MMA_KERNEL_1 q4::gemv_mma_kernel<1, kWarps, kRm1, kCm1>
 #define Q4_MMA_KERNEL_2 q4::gemv_mma_kernel<2, kWarps, kRm2, kCm2>
 #define Q4_STACK_KERNEL q4::stack_kernel<kWarps, kR1, kC1>
+#define Q4_SWIGLU_KERNEL q4::gemv_swiglu_kernel<kWarps, kR1, kC1>
 // Largest input of a GEMV in the persistent step (its staging holds up to
 // kStackXChunks 16-byte chunks per thread).
 constexpr int kStackKmax = q4::kStackXChunks * 8 * kThreads;
@@ -172,7 +174,8 @@ int set_smem_attr(F* kernel) {
 // Launch one GEMV (M <= 2 path).  `pdl` adds the programmatic-dependent-
 // launch attribute (only used between the library's own kernels).
 int launch_gemv(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M, int64_t N,
-                int64_t K, int renorm, __half* trace_x, cudaStream_t st, bool pdl, bool q8 = false) {
+                int64_t K, int renorm, __half* trace_x, cudaStream_t st, bool pdl, bool q8 = false,
+                bool swiglu = false) {
     if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
     const int KB = (int)(K / 32);
     const int T = (int)((N + 31) / 32);
@@ -210,7 +213,9 @@ int launch_gemv(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M,
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
     cudaError_t e;
-    if (q8)
+    if (swiglu)
+        e = cudaLaunchKernelEx(&cfg, Q4_SWIGLU_KERNEL, a);   // M == 1, gated input
+    else if (q8)
         e = M == 1 ? cudaLaunchKernelEx(&cfg, Q4_Q8_KERNEL_1, a) : cudaLaunchKernelEx(&cfg, Q4_Q8_KERNEL_2, a);
     else if (M == 1)
         e = cudaLaunchKernelEx(&cfg, Q4_DP2A_KERNEL_1, a);
@@ -598,7 +603,8 @@ int q4gemv_create(q4gemv_t* out, int device) {
         if (set_smem_attr(Q4_DP2A_KERNEL_1) || set_smem_attr(Q4_DP2A_KERNEL_2) ||
             set_smem_attr(Q4_Q8_KERNEL_1) || set_smem_attr(Q4_Q8_KERNEL_2) ||
             set_smem_attr(Q4_MMA_KERNEL_1) || set_smem_attr(Q4_MMA_KERNEL_2) ||
-            set_smem_attr(Q4_STACK_KERNEL) || set_smem_attr(q4::gemm_tc_kernel<false>) ||
+            set_smem_attr(Q4_STACK_KERNEL) || set_smem_attr(Q4_SWIGLU_KERNEL) ||
+            set_smem_attr(q4::gemm_tc_kernel<false>) ||
             set_smem_attr(q4::gemm_tc_kernel<true>) ||
             0)
             rc = fail(h, Q4_ECUDA, "cudaFuncSetAttribute failed");
@@ -690,6 +696,19 @@ int q4gemv_run(q4gemv_t h, const void* W, const void* x, void* y, int M, int64_t
                            st);
 }
  
+int q4gemv_run_swiglu(q4gemv_t h, const void* W, const void* gate_up, void* y, int64_t N,
+                      int64_t K, q4gemv_stream_t stream) {
+    if (!h) return Q4_EINVAL;
+    int v = q4gemv_validate(1, N, K, W, gate_up, y);
+    if (v == Q4_OK && !dp2a_fits(1, K)) v = Q4_EUNSUPPORTED;
+    if (v != Q4_OK)
+        return fail(h, v, "run_swiglu: %s (N=%lld K=%lld)", q4gemv_strerror(v), (long long)N,
+                    (long long)K);
+    Q4_CUDA(h, cudaSetDevice(h->device));
+    return launch_gemv(h, W, static_cast<const __half*>(gate_up), static_cast<__half*>(y), 1, N, K,
+                       0, nullptr, static_cast<cudaStream_t>(stream), false, false, true);
+}
+
 size_t q4gemv_q8_0_gguf_bytes(int64_t N, int64_t K) {
     if (check_shape(N, K) != Q4_OK) return 0;
     return (size_t)N * (size_t)(K / 32) * 34;
