@@ -169,8 +169,10 @@ Q4GEMV_API int q4gemv_run(q4gemv_t h, const void* W_packed, const void* x, void*
 /* The down GEMV fed directly by the gate+up GEMV: y[N] = W u for a packed
  * Q4_0 W (N x K), with u_k = SiLU(g_k) * up_k = g_k / (1 + e^-g_k) * up_k and
  * gate_up = [g | up] the 2K-entry binary16 output of the gate+up GEMV (gate
- * half first).  The pages name the model family but not its FFN activation;
- * this is that family's gated unit.  u is computed in fp32 inside the kernel
+ * half first).  The pages name the model family (Qwen 3.8 27B: taozi.news
+ * page, section "支持模型与限制"; originshq.com page, section "Limitations
+ * and Open Questions") but not its FFN activation; this is that family's
+ * gated unit.  u is computed in fp32 inside the kernel
  * (never written) and converted per 32-column block like any M = 1 input;
  * exact integer block sums, fp32 accumulation, y rounded once.
  *   gate_up : device, 2K binary16, 16-byte aligned
@@ -286,9 +288,10 @@ Q4GEMV_API int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_la
  *
  * Arguments as q4gemv_run (device pointers, 16-byte aligned, packed W), on
  * the current CUDA device, asynchronous on `stream`.  Limits: 1 <= M <= 2
- * (else Q4_EUNSUPPORTED); K % 32 == 0, N <= Q4GEMV_NOALLOC_MAX_N, M*K <=
- * 36864 (else Q4_ESHAPE); at most 2560 warps are used.  Device-side error
- * reports are not surfaced.
+ * (else Q4_EUNSUPPORTED); K % 32 == 0, N <= Q4GEMV_NOALLOC_MAX_N, and K <=
+ * 24,896 for M = 1 or K <= 18,432 for M = 2 (the kernel's shared memory and
+ * activation staging; else Q4_ESHAPE); at most 2560 warps are used.
+ * Device-side error reports are not surfaced.
  *
  * The first call on a device sets that device up (resolves the array's
  * device address with cudaGetSymbolAddress, queries the SM count, sets the
@@ -311,11 +314,17 @@ Q4GEMV_API const char* q4gemv_strerror(int status);
  * call on the handle. */
 Q4GEMV_API const char* q4gemv_last_error(q4gemv_t h);
 
-/* Host fault injection for tests: makes the named host step of later calls
- * fail with Q4_EFAULTINJ.  which: "none", "alloc" (workspace or buffer
- * allocation), "launch" (kernel launch), "graph" (graph capture or
- * instantiation).  The environment variable Q4GEMV_FAULT sets the initial
- * value at q4gemv_create. */
+/* Fault injection for tests.  which: "none"; "alloc" (workspace or buffer
+ * allocation), "launch" (kernel launch) or "graph" (graph capture or
+ * instantiation) make that host step of later calls fail with
+ * Q4_EFAULTINJ; "timeout" makes later persistent decode steps
+ * (q4gemv_run_stack) give every bounded device wait a budget of 1,024 polls
+ * and ask their first inter-GEMV wait for a condition that never holds, so
+ * the wait gives up, the kernel records Q4_ETIMEOUT in the handle's error
+ * word, every CTA returns (after its copies in flight have landed) and the
+ * next q4gemv_sync_status reports Q4_ETIMEOUT; the handle stays usable.  No
+ * GPU fault, trap or unbounded wait is involved.  The environment variable
+ * Q4GEMV_FAULT sets the initial value at q4gemv_create. */
 Q4GEMV_API int q4gemv_set_fault(q4gemv_t h, const char* which);
 
 #ifdef __cplusplus

@@ -58,7 +58,7 @@ size_t dp2a_smem(int M, int64_t K, bool q8 = false) {
                   : q4::gemv_dp2a_smem_bytes(2, (int)K, kWarps, kR2, kC2);
 }
 
-enum Fault { kFaultNone = 0, kFaultAlloc, kFaultLaunch, kFaultGraph };
+enum Fault { kFaultNone = 0, kFaultAlloc, kFaultLaunch, kFaultGraph, kFaultTimeout };
 
 struct StackKey {
     std::vector<q4gemv_layer> layers;
@@ -161,6 +161,7 @@ int parse_fault(const char* s) {
     if (!strcmp(s, "alloc")) return kFaultAlloc;
     if (!strcmp(s, "launch")) return kFaultLaunch;
     if (!strcmp(s, "graph")) return kFaultGraph;
+    if (!strcmp(s, "timeout")) return kFaultTimeout;
     return -1;
 }
 
@@ -860,6 +861,10 @@ int enqueue_stack_persistent(q4gemv_ctx* h, const StackKey& k, cudaStream_t st) 
     sa.xq = h->xq;
     sa.xq_half = (int)q4::stack_xq_half_bytes(kStackKmax);
     sa.kmax = (int)kmax;
+    // A test of the device-side timeout: few polls, and a first grid wait
+    // that no arrival count satisfies.
+    sa.poll_limit = h->fault == kFaultTimeout ? (1u << 10) : (1u << 26);
+    sa.unreachable = h->fault == kFaultTimeout ? 1 : 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(h->sms);
     cfg.blockDim = dim3(kThreads);

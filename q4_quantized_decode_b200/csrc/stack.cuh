@@ -44,6 +44,8 @@ struct StackArgs {
     int kmax;             //   block sums of squares [kmax / 32] fp32
     int* err;             // device error word
     int* sync;            // [0] grid arrivals, [1] abort flag; zero at launch
+    uint32_t poll_limit;  // polls of a grid wait before it gives up
+    int unreachable;      // test knob: the first grid wait asks for one arrival too many
 };
 
 // Outputs of the previous GEMV in tiles shared by several CTAs exist only as
@@ -312,10 +314,11 @@ struct StreamProducer {
 
 // Grid barrier: CTA-wide arrival already made; thread 0 waits (bounded) until
 // `target` arrivals or an abort.  Returns false on timeout or abort.
-__device__ __forceinline__ bool grid_wait(int* sync, int target, int* err, int* flag_smem) {
+__device__ __forceinline__ bool grid_wait(int* sync, int target, int* err, int* flag_smem,
+                                          uint32_t poll_limit) {
     if (threadIdx.x == 0) {
         int ok = 0;
-        for (uint32_t it = 0; it < (1u << 26); ++it) {
+        for (uint32_t it = 0; it < poll_limit; ++it) {
             if (ld_acquire_gpu(sync) >= target) {
                 ok = 1;
                 break;
@@ -385,7 +388,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa
             cons.qo.sq = reinterpret_cast<float*>(ob + (size_t)sa.kmax * 3);
             cons.qo.nb = sa.gemv[i + 1].K / 32;
         }
-        if (i > 0) ok = grid_wait(sa.sync, i * (int)gridDim.x, sa.err, &flag);
+        if (i > 0)
+            ok = grid_wait(sa.sync, i * (int)gridDim.x + (i == 1 ? sa.unreachable : 0), sa.err, &flag,
+                           sa.poll_limit);
         if (!ok) break;
         if (i == 0) {
             if (a.K <= 2 * NT * 8) stage_activations<1, NT, 2>(a, xs, rec, sq);
@@ -431,7 +436,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa
         __syncthreads();
         if (threadIdx.x == 0) red_add_release_gpu(sa.sync, 1);
     }
-    if (ok) ok = grid_wait(sa.sync, sa.n_gemv * (int)gridDim.x, sa.err, &flag);
+    if (ok) ok = grid_wait(sa.sync, sa.n_gemv * (int)gridDim.x, sa.err, &flag, sa.poll_limit);
     if (ok) {
         const int il = sa.n_gemv - 1;
         const StackGemv& ld = sa.gemv[il];
