@@ -16,6 +16,11 @@ reported workload then says so).
 Under torchrun (N > 1) every rank runs an independent replica (same weights,
 its own activation stream); there is no data-path collective, only a barrier
 and a max-reduction of the timings.  Rank 0 prints one JSON line.
+
+--shard runs the row-sharded step instead (q4gemv_run_stack_sharded): each
+rank holds 1/N of every matrix's rows and the outputs are all-gathered over
+NCCL after every GEMV, so N GPUs share ONE decode step (strong scaling; the
+reported bytes are the model's once per step).
 """
 from __future__ import annotations
 
@@ -55,6 +60,10 @@ STEP_WEIGHT_BYTES = L * sum(N * (K // 32) * 18 for N, K in DIMS)
 WORKLOAD = ("27B-shaped decode step, M=1: 64 layers x (QKV 5120->7168, O 5120->5120, "
             "gate+up 5120->34816, down 17408->5120) Q4_0 GEMVs with unit-RMS renorm between "
             "matrices, one persistent kernel launch per step")
+WORKLOAD_SHARD = ("27B-shaped decode step, M=1: 64 layers x (QKV 5120->7168, O 5120->5120, "
+                  "gate+up 5120->34816, down 17408->5120) Q4_0 GEMVs with unit-RMS renorm between "
+                  "matrices, every matrix row-sharded over the GPUs: per GEMV one kernel on each "
+                  "GPU's rows and an NCCL all-gather, replayed as one CUDA graph")
 
 
 KERNEL_SOURCES = ["stack.cuh", "gemv_dp2a.cuh", "partition.cuh", "device_common.cuh"]
@@ -314,6 +323,32 @@ def time_prefill(eng, torch, layers, M: int = 169, reps: int = 3):
             "note": "each weight enters the MMA as two exact binary16 parts: 2x the useful flops"}
 
 
+def build_weights_sharded(eng, torch, q4, rank: int, world: int):
+    """This rank's row slices of the 64-layer step's matrices (the rows
+    q4gemv_shard_rows assigns it), repacked on the device; None for a slice
+    of no rows."""
+    layers = []
+    t_repack = 0.0
+    for l in range(L):
+        mats = []
+        for t, (N, K) in enumerate(DIMS):
+            st, row0, rows, _ = q4.q4gemv_shard_rows(N, world, rank)
+            if st != q4.Q4_OK:
+                raise RuntimeError(f"shard_rows status {st}")
+            if rows == 0:
+                mats.append(None)
+                continue
+            full = synth.q4_0_matrix(STEP_SEED, synth.weight_id(4 * l + t), N, K)
+            g = torch.from_numpy(np.ascontiguousarray(full[row0:row0 + rows]).reshape(-1)).cuda()
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            mats.append(eng.repack(g, rows, K))
+            torch.cuda.synchronize()
+            t_repack += time.perf_counter() - t0
+        layers.append(tuple(mats))
+    return layers, t_repack
+
+
 def run_ours(args, rank: int, world: int, dist):
     import torch
     import q4_quantized_decode_b200 as q4
@@ -321,15 +356,38 @@ def run_ours(args, rank: int, world: int, dist):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     eng = q4.Q4Gemv(local)
-    layers, t_repack = build_weights(eng, torch, rank)
-    x_host = torch.from_numpy(synth.normal_f16(STEP_SEED, synth.act_id(rank), HIDDEN).view(np.float16)).pin_memory()
+    if args.shard:
+        # One communicator for the row-sharded step: rank 0's NCCL id, sent
+        # to the others over the process group.
+        uid = [q4.q4gemv_comm_unique_id()[1] if rank == 0 else None]
+        if dist is not None and world > 1:
+            dist.broadcast_object_list(uid, src=0)
+        eng.init_comm(world, rank, uid[0])
+        layers, t_repack = build_weights_sharded(eng, torch, q4, rank, world)
+    else:
+        layers, t_repack = build_weights(eng, torch, rank)
+    act = 0 if args.shard else rank          # the sharded ranks share one step's input
+    x_host = torch.from_numpy(synth.normal_f16(STEP_SEED, synth.act_id(act), HIDDEN).view(np.float16)).pin_memory()
     out_host = torch.empty(HIDDEN, dtype=torch.float16).pin_memory()
     x_in = x_host.to(dev)
     x_out = torch.empty(HIDDEN, dtype=torch.float16, device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
-        eng.run_stack(layers, x_in, HIDDEN, QKV_N, FFN, x_out=x_out)
+        if args.shard:
+            eng.run_stack_sharded(layers, x_in, HIDDEN, QKV_N, FFN, x_out=x_out)
+        else:
+            eng.run_stack(layers, x_in, HIDDEN, QKV_N, FFN, x_out=x_out)
+
+    def step_e2e():
+        if args.shard:
+            # the sharded call takes device vectors: the copies from and to
+            # pinned host memory are made around it, every step
+            x_in.copy_(x_host, non_blocking=True)
+            eng.run_stack_sharded(layers, x_in, HIDDEN, QKV_N, FFN, x_out=x_out)
+            out_host.copy_(x_out, non_blocking=True)
+        else:
+            eng.run_stack(layers, x_host, HIDDEN, QKV_N, FFN, x_out=out_host)
 
     for _ in range(args.warmup):
         step()
@@ -368,20 +426,21 @@ def run_ours(args, rank: int, world: int, dist):
 
     # ---- end-to-end: the C-ABI call with HOST vectors (pinned), which copies
     # x to the device and the result back inside the call, every step
-    eng.run_stack(layers, x_host, HIDDEN, QKV_N, FFN, x_out=out_host)   # descriptors for these pointers
+    step_e2e()   # descriptors (or the graph) for these pointers
     barrier()
     torch.cuda.synchronize()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
     for _ in range(args.steps):
-        eng.run_stack(layers, x_host, HIDDEN, QKV_N, FFN, x_out=out_host)
+        step_e2e()
     f1.record(stream)
     torch.cuda.synchronize()
     barrier()
     ms_e2e = f0.elapsed_time(f1)
 
-    per_shape = time_shapes(eng, torch, layers) if (rank == 0 and not args.no_per_shape) else None
-    prefill = time_prefill(eng, torch, layers) if (rank == 0 and not args.no_per_shape) else None
+    extras = rank == 0 and not args.no_per_shape and not args.shard
+    per_shape = time_shapes(eng, torch, layers) if extras else None
+    prefill = time_prefill(eng, torch, layers) if extras else None
     if eng.sync_status() != q4.Q4_OK:
         raise RuntimeError("device status after timing")
 
@@ -390,10 +449,12 @@ def run_ours(args, rank: int, world: int, dist):
         return 0
 
     ms_step = ms / args.steps
-    value, steps_per_s = step_throughput(world, args.steps, ms)
-    e2e_value, e2e_steps_per_s = step_throughput(world, args.steps, ms_e2e)
+    # Replicas: every rank runs a whole step.  Sharded: the ranks share one.
+    copies = 1 if args.shard else world
+    value, steps_per_s = step_throughput(copies, args.steps, ms)
+    e2e_value, e2e_steps_per_s = step_throughput(copies, args.steps, ms_e2e)
     peak, peak_kind = measured_peaks()
-    per_rank_gbs = STEP_GEMV_BYTES / (ms_step * 1e-3) / 1e9
+    per_rank_gbs = STEP_GEMV_BYTES / (ms_step * 1e-3) / 1e9 / (world if args.shard else 1)
     roofline = {
         "bound": "hbm", "achieved": per_rank_gbs, "peak": peak, "unit": "GB/s",
         "frac": per_rank_gbs / peak, "traffic": None,
@@ -422,12 +483,13 @@ def run_ours(args, rank: int, world: int, dist):
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
+        "scaling": "strong" if args.shard else "weak", "vs_baseline": None,
         "dtype": "q4_0 x f16 (s32 block sums, f32 accumulate)", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "bytes_per_step": STEP_GEMV_BYTES,
+        "config": {"workload": WORKLOAD_SHARD if args.shard else WORKLOAD, "bytes_per_step": STEP_GEMV_BYTES,
                    "weight_bytes_per_step": STEP_WEIGHT_BYTES,
                    "l2": "inputs larger than L2 (11.9 GB of weights per step)",
-                   "parallelism": f"replicas x{world}", "seed": STEP_SEED},
+                   "parallelism": (f"row-sharded x{world} (NCCL all-gather after every GEMV)"
+                                   if args.shard else f"replicas x{world}"), "seed": STEP_SEED},
         "decode_steps_per_s": steps_per_s,
         "pct_of_8TBps_nominal": 100.0 * per_rank_gbs / NOMINAL_HBM_GBS,
         "roofline": roofline,
@@ -435,7 +497,9 @@ def run_ours(args, rank: int, world: int, dist):
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": 2 * HIDDEN,
                 "d2h_bytes_per_step": 2 * HIDDEN,
                 "steps_per_s": e2e_steps_per_s},
-        "gpu_launches": args.steps,      # one stack_kernel per step (and one 16-byte memset)
+        # one stack_kernel per step (and one 16-byte memset); sharded: per GEMV one
+        # kernel and one all-gather, and the final renorm
+        "gpu_launches": args.steps * ((8 * L + 1) if args.shard else 1),
         "clocks": clocks,
         "repack_s_per_step_weights": t_repack,
         "per_shape_m1": per_shape,
@@ -540,6 +604,8 @@ def main():
     ap.add_argument("--act", choices=["none", "swiglu"], default="none",
                     help="--case gemv: feed the GEMV SiLU(gate) * up of a 2K input (M = 1)")
     ap.add_argument("--layers", type=int, default=64, help="layers of the step (profiling only)")
+    ap.add_argument("--shard", action="store_true",
+                    help="row-shard every matrix over the ranks (one step shared by all GPUs)")
     args = ap.parse_args()
     if args.layers != 64:
         set_layers(args.layers)

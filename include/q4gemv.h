@@ -268,6 +268,51 @@ Q4GEMV_API int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_la
                      const void* x_in, void* x_out, void* trace_x,
                      void* trace_y, q4gemv_stream_t stream);
 
+/* ---- Row-sharded decode step over several GPUs (one process and one handle
+ * per GPU).  The pages run the model split by contiguous layer ranges across
+ * devices, passing the hidden state from one to the next (originshq.com page,
+ * section "The Architecture: Layers Distributed, Activations in Flight";
+ * taozi.news page, section "技术架构"); that pipelines tokens but does not
+ * speed up one.  Here every GEMV of the step is split by output rows over
+ * `world` GPUs and its output is all-gathered before the next GEMV, so one
+ * token's step divides its weight bytes over the GPUs.
+ *
+ * Rows of an N-row matrix held by rank `rank`: [*row0, *row0 + *rows), whole
+ * 32-row tiles, every rank holding *chunk = ceil(N / (32 world)) * 32 rows
+ * or fewer (the last ranks: the remainder, possibly 0).  Host-only; no
+ * device access.  Q4_EINVAL for N <= 0, world < 1 or rank outside
+ * [0, world). */
+Q4GEMV_API int q4gemv_shard_rows(int64_t N, int world, int rank, int64_t* row0, int64_t* rows,
+                      int64_t* chunk);
+
+/* An NCCL unique id (128 bytes, written to id) for q4gemv_comm_init: rank 0
+ * calls it and sends the bytes to the other ranks.  NCCL (libnccl.so.2) is
+ * loaded at run time; Q4_EUNSUPPORTED if it cannot be. */
+Q4GEMV_API int q4gemv_comm_unique_id(void* id);
+
+/* Binds the handle to rank `rank` of a `world`-GPU communicator created from
+ * the unique id (every rank calls it with the same id; collective, blocks
+ * until all ranks have joined).  Replaces an earlier communicator of the
+ * handle. */
+Q4GEMV_API int q4gemv_comm_init(q4gemv_t h, int world, int rank, const void* id);
+
+/* The decode step of q4gemv_run_stack, row-sharded: `layers` holds THIS
+ * rank's row slices (q4gemv_shard_rows of each matrix, packed as q4gemv_run
+ * matrices of `rows` rows; a slice of 0 rows may be NULL).  Per GEMV the rank
+ * computes its rows f16(s(v) * W_slice v) from the full previous output v
+ * (the M = 1 kernel; the scale as in q4gemv_run_stack), then an NCCL
+ * all-gather gives every rank the whole output; x_out = f16(s(x') x') on
+ * every rank.  x_in, x_out: device memory (hidden binary16), the same x_in on
+ * every rank.  Every rank must make the same calls in the same order.  The
+ * step is captured as one CUDA graph on the first call with these arguments
+ * (not inside the caller's capture) and replayed.  Results agree with
+ * q4gemv_run_stack within the GEMV tolerance (the row split changes the
+ * order of the partial sums, not the arithmetic).  Errors as
+ * q4gemv_run_stack; Q4_EINVAL without a communicator. */
+Q4GEMV_API int q4gemv_run_stack_sharded(q4gemv_t h, const q4gemv_layer* layers_local,
+                             int n_layers, int64_t hidden, int64_t qkv_n, int64_t ffn,
+                             const void* x_in, void* x_out, q4gemv_stream_t stream);
+
 /* Fixed limits of q4gemv_run_noalloc. */
 #define Q4GEMV_NOALLOC_MAX_N (1 << 22)                 /* rows */
 #define Q4GEMV_NOALLOC_SCRATCH_BYTES (2u << 20)        /* static device scratch */

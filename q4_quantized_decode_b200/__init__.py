@@ -57,6 +57,12 @@ def _load_library():
         "q4gemv_repack": ([vp, vp, vp, i64, i64, vp], ci),
         "q4gemv_run": ([vp, vp, vp, vp, ci, i64, i64, vp], ci),
         "q4gemv_run_swiglu": ([vp, vp, vp, vp, i64, i64, vp], ci),
+        "q4gemv_shard_rows": ([i64, ci, ci, ctypes.POINTER(i64), ctypes.POINTER(i64),
+                               ctypes.POINTER(i64)], ci),
+        "q4gemv_comm_unique_id": ([ctypes.c_char_p], ci),
+        "q4gemv_comm_init": ([vp, ci, ci, ctypes.c_char_p], ci),
+        "q4gemv_run_stack_sharded": ([vp, ctypes.POINTER(q4gemv_layer), ci, i64, i64, i64, vp, vp,
+                                      vp], ci),
         "q4gemv_run_stack": ([vp, ctypes.POINTER(q4gemv_layer), ci, i64, i64, i64,
                               vp, vp, vp, vp, vp], ci),
         "q4gemv_sync_status": ([vp, vp], ci),
@@ -139,6 +145,28 @@ def q4gemv_sync_status(h, stream) -> int:
 
 def q4gemv_set_fault(h, which: str) -> int:
     return _lib.q4gemv_set_fault(h, which.encode())
+
+
+def q4gemv_shard_rows(N: int, world: int, rank: int):
+    """(status, row0, rows, chunk) of rank's row slice of an N-row matrix."""
+    r0, n, c = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    st = _lib.q4gemv_shard_rows(N, world, rank, ctypes.byref(r0), ctypes.byref(n), ctypes.byref(c))
+    return st, r0.value, n.value, c.value
+
+
+def q4gemv_comm_unique_id():
+    """(status, 128-byte NCCL unique id)."""
+    buf = ctypes.create_string_buffer(128)
+    st = _lib.q4gemv_comm_unique_id(buf)
+    return st, buf.raw
+
+
+def q4gemv_comm_init(h, world: int, rank: int, uid: bytes) -> int:
+    return _lib.q4gemv_comm_init(h, world, rank, ctypes.create_string_buffer(uid, 128))
+
+
+def q4gemv_run_stack_sharded(h, layers, n_layers, hidden, qkv_n, ffn, x_in, x_out, stream) -> int:
+    return _lib.q4gemv_run_stack_sharded(h, layers, n_layers, hidden, qkv_n, ffn, x_in, x_out, stream)
 
 
 def q4gemv_run_noalloc(W, x, y, M, N, K, stream) -> int:
@@ -265,6 +293,24 @@ class Q4Gemv:
             arr[i] = q4gemv_layer(_ptr(a), _ptr(b), _ptr(c), _ptr(d))
         self._check(q4gemv_run_stack(self.h, arr, len(layers), hidden, qkv_n, ffn, _ptr(x_in),
                                      _ptr(x_out), _ptr(trace_x), _ptr(trace_y), _stream(stream)))
+        return x_out
+
+    def init_comm(self, world: int, rank: int, uid: bytes):
+        """Joins the `world`-GPU communicator of the row-sharded step as `rank`."""
+        self._check(q4gemv_comm_init(self.h, world, rank, uid))
+
+    def run_stack_sharded(self, layers_local, x_in, hidden: int, qkv_n: int, ffn: int, x_out=None,
+                          stream=None):
+        """layers_local: this rank's (qkv, o, gate_up, down) row slices (packed tensors, or
+        None for a slice of 0 rows)."""
+        import torch
+        if x_out is None:
+            x_out = torch.empty(hidden, dtype=torch.float16, device=x_in.device)
+        arr = (q4gemv_layer * len(layers_local))()
+        for i, (a, b, c, d) in enumerate(layers_local):
+            arr[i] = q4gemv_layer(_ptr(a), _ptr(b), _ptr(c), _ptr(d))
+        self._check(q4gemv_run_stack_sharded(self.h, arr, len(layers_local), hidden, qkv_n, ffn,
+                                             _ptr(x_in), _ptr(x_out), _stream(stream)))
         return x_out
 
     def sync_status(self, stream=None) -> int:

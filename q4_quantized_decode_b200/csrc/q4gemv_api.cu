@@ -2,11 +2,14 @@
 // workspace ownership, kernel selection and launch, and the CUDA-graph
 // decode-step runner.
 #include <cuda_runtime.h>
+#include <dlfcn.h>
+#include <nccl.h>   // types only: the functions are resolved at run time
 
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -109,6 +112,14 @@ struct q4gemv_ctx {
     uint8_t* ximg = nullptr;         // activation image of the tensor-core GEMM
     size_t ximg_bytes = 0;
     int64_t hio_elems = 0;           // per vector
+    // Row-sharded decode step (one rank of `world`).
+    ncclComm_t comm = nullptr;
+    int world = 1, rank = 0;
+    __half* sh_slice[4] = {nullptr, nullptr, nullptr, nullptr};    // this rank's output rows, per matrix type
+    __half* sh_gather[4] = {nullptr, nullptr, nullptr, nullptr};   // all ranks' rows, per matrix type
+    int64_t sh_chunk[4] = {0, 0, 0, 0};
+    cudaGraphExec_t sh_exec = nullptr;
+    StackKey sh_key;
     std::string last_error;
 };
 
@@ -506,6 +517,60 @@ bool q8_dp2a_fits(int M, int64_t K) {
            dp2a_smem(M, K, true) <= kMaxDynSmem;
 }
 
+// NCCL, loaded on first use (the library has no link-time dependency on it;
+// in a process that already uses NCCL the loaded copy is shared).
+struct NcclApi {
+    void* lib = nullptr;
+    ncclResult_t (*GetUniqueId)(ncclUniqueId*) = nullptr;
+    ncclResult_t (*CommInitRank)(ncclComm_t*, int, ncclUniqueId, int) = nullptr;
+    ncclResult_t (*AllGather)(const void*, void*, size_t, ncclDataType_t, ncclComm_t, cudaStream_t) = nullptr;
+    ncclResult_t (*CommDestroy)(ncclComm_t) = nullptr;
+    const char* (*GetErrorString)(ncclResult_t) = nullptr;
+};
+std::mutex g_nccl_mu;
+NcclApi g_nccl;
+
+bool nccl_load() {
+    std::lock_guard<std::mutex> lock(g_nccl_mu);
+    if (g_nccl.lib) return true;
+    void* lib = dlopen("libnccl.so.2", RTLD_NOW | RTLD_GLOBAL);
+    if (!lib) return false;
+    NcclApi a;
+    a.lib = lib;
+    a.GetUniqueId = reinterpret_cast<decltype(a.GetUniqueId)>(dlsym(lib, "ncclGetUniqueId"));
+    a.CommInitRank = reinterpret_cast<decltype(a.CommInitRank)>(dlsym(lib, "ncclCommInitRank"));
+    a.AllGather = reinterpret_cast<decltype(a.AllGather)>(dlsym(lib, "ncclAllGather"));
+    a.CommDestroy = reinterpret_cast<decltype(a.CommDestroy)>(dlsym(lib, "ncclCommDestroy"));
+    a.GetErrorString = reinterpret_cast<decltype(a.GetErrorString)>(dlsym(lib, "ncclGetErrorString"));
+    if (!a.GetUniqueId || !a.CommInitRank || !a.AllGather || !a.CommDestroy || !a.GetErrorString) {
+        dlclose(lib);
+        return false;
+    }
+    g_nccl = a;
+    return true;
+}
+
+// Frees the sharded step's communicator, buffers and graph.
+void shard_release(q4gemv_ctx* h) {
+    if (h->sh_exec) cudaGraphExecDestroy(h->sh_exec);
+    h->sh_exec = nullptr;
+    for (int t = 0; t < 4; ++t) {
+        cudaFree(h->sh_slice[t]);
+        cudaFree(h->sh_gather[t]);
+        h->sh_slice[t] = h->sh_gather[t] = nullptr;
+        h->sh_chunk[t] = 0;
+    }
+    if (h->comm && g_nccl.CommDestroy) g_nccl.CommDestroy(h->comm);
+    h->comm = nullptr;
+}
+
+// Rows per rank of an N-row matrix split over `world` ranks: whole 32-row
+// tiles, the same count for every rank (the all-gather sends equal pieces).
+int64_t shard_chunk(int64_t N, int world) {
+    const int64_t unit = 32 * (int64_t)world;
+    return (N + unit - 1) / unit * 32;
+}
+
 }  // namespace
 
 extern "C" {
@@ -650,6 +715,7 @@ int q4gemv_destroy(q4gemv_t h) {
     cudaFree(h->yacc);
     cudaFree(h->hio);
     cudaFree(h->ximg);
+    shard_release(h);
     delete h;
     return Q4_OK;
 }
@@ -1020,6 +1086,152 @@ int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64
     }
     Q4_CUDA(h, cudaGraphLaunch(h->exec, st));
     return finish_host_out(h, Q4_OK, host_out, x_out_user, x_out, hidden, st);
+}
+
+int q4gemv_shard_rows(int64_t N, int world, int rank, int64_t* row0, int64_t* rows, int64_t* chunk) {
+    if (N <= 0 || world < 1 || rank < 0 || rank >= world || !row0 || !rows) return Q4_EINVAL;
+    const int64_t c = shard_chunk(N, world);
+    const int64_t r0 = (int64_t)rank * c;
+    *row0 = r0 < N ? r0 : N;
+    *rows = N - r0 < 0 ? 0 : (N - r0 < c ? N - r0 : c);
+    if (chunk) *chunk = c;
+    return Q4_OK;
+}
+
+int q4gemv_comm_unique_id(void* id) {
+    if (!id) return Q4_EINVAL;
+    if (!nccl_load()) return Q4_EUNSUPPORTED;
+    ncclUniqueId u;
+    if (g_nccl.GetUniqueId(&u) != ncclSuccess) return Q4_ECUDA;
+    memcpy(id, &u, sizeof u);
+    return Q4_OK;
+}
+
+int q4gemv_comm_init(q4gemv_t h, int world, int rank, const void* id) {
+    if (!h || !id) return Q4_EINVAL;
+    if (world < 1 || rank < 0 || rank >= world) return fail(h, Q4_EINVAL, "comm_init: rank %d of %d", rank, world);
+    if (!nccl_load()) return fail(h, Q4_EUNSUPPORTED, "comm_init: libnccl.so.2 could not be loaded");
+    Q4_CUDA(h, cudaSetDevice(h->device));
+    Q4_CUDA(h, cudaDeviceSynchronize());
+    shard_release(h);
+    ncclUniqueId u;
+    memcpy(&u, id, sizeof u);
+    ncclComm_t c = nullptr;
+    const ncclResult_t r = g_nccl.CommInitRank(&c, world, u, rank);
+    if (r != ncclSuccess) return fail(h, Q4_ECUDA, "ncclCommInitRank: %s", g_nccl.GetErrorString(r));
+    h->comm = c;
+    h->world = world;
+    h->rank = rank;
+    return Q4_OK;
+}
+
+int q4gemv_run_stack_sharded(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64_t hidden,
+                             int64_t qkv_n, int64_t ffn, const void* x_in, void* x_out,
+                             q4gemv_stream_t stream) {
+    if (!h) return Q4_EINVAL;
+    if (!h->comm) return fail(h, Q4_EINVAL, "run_stack_sharded: no communicator (q4gemv_comm_init)");
+    if (!layers || !x_in || !x_out) return fail(h, Q4_EINVAL, "run_stack_sharded: null pointer");
+    if (n_layers < 1 || n_layers > 4096) return fail(h, Q4_ESHAPE, "run_stack_sharded: n_layers out of range");
+    if (qkv_n < hidden) return fail(h, Q4_ESHAPE, "run_stack_sharded: qkv_n < hidden");
+    const int64_t n_of[4] = {qkv_n, hidden, 2 * ffn, hidden};
+    const int64_t k_of[4] = {hidden, hidden, hidden, ffn};
+    for (int t = 0; t < 4; ++t) {
+        const int sc = check_shape(n_of[t], k_of[t]);
+        if (sc != Q4_OK) return fail(h, sc, "run_stack_sharded: invalid matrix shape");
+        if (!dp2a_fits(1, k_of[t])) return fail(h, Q4_EUNSUPPORTED, "run_stack_sharded: K too large");
+    }
+    if (is_host_pointer(x_in) || is_host_pointer(x_out))
+        return fail(h, Q4_EINVAL, "run_stack_sharded: x_in and x_out must be device memory");
+    if (!aligned16(x_in) || !aligned16(x_out)) return fail(h, Q4_EALIGN, "run_stack_sharded: misaligned vector");
+    int64_t rows[4], chunk[4];
+    for (int t = 0; t < 4; ++t) {
+        int64_t r0 = 0;
+        q4gemv_shard_rows(n_of[t], h->world, h->rank, &r0, &rows[t], &chunk[t]);
+    }
+    for (int l = 0; l < n_layers; ++l) {
+        const q4gemv_layer& L = layers[l];
+        const void* m[4] = {L.qkv, L.o, L.gate_up, L.down};
+        for (int t = 0; t < 4; ++t) {
+            if (rows[t] > 0 && !m[t]) return fail(h, Q4_EINVAL, "run_stack_sharded: null matrix in layer %d", l);
+            if (!aligned16(m[t])) return fail(h, Q4_EALIGN, "run_stack_sharded: misaligned matrix in layer %d", l);
+        }
+    }
+    Q4_CUDA(h, cudaSetDevice(h->device));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    Q4_CUDA(h, cudaStreamIsCapturing(st, &cs));
+    if (cs != cudaStreamCaptureStatusNone)
+        return fail(h, Q4_EUNSUPPORTED, "run_stack_sharded: not available inside a stream capture");
+    // Buffers: this rank's rows (zero past them) and the gathered vector, per
+    // matrix type.
+    for (int t = 0; t < 4; ++t) {
+        if (chunk[t] == h->sh_chunk[t] && h->sh_slice[t]) continue;
+        if (h->fault == kFaultAlloc) return fail(h, Q4_EFAULTINJ, "injected allocation failure");
+        Q4_CUDA(h, cudaStreamSynchronize(st));
+        if (h->sh_exec) {
+            cudaGraphExecDestroy(h->sh_exec);
+            h->sh_exec = nullptr;
+        }
+        cudaFree(h->sh_slice[t]);
+        cudaFree(h->sh_gather[t]);
+        h->sh_slice[t] = h->sh_gather[t] = nullptr;
+        h->sh_chunk[t] = 0;
+        if (cudaMalloc(&h->sh_slice[t], chunk[t] * sizeof(__half)) != cudaSuccess ||
+            cudaMalloc(&h->sh_gather[t], chunk[t] * h->world * sizeof(__half)) != cudaSuccess)
+            return fail(h, Q4_ENOMEM, "run_stack_sharded: buffer allocation failed");
+        Q4_CUDA(h, cudaMemset(h->sh_slice[t], 0, chunk[t] * sizeof(__half)));
+        h->sh_chunk[t] = chunk[t];
+    }
+    StackKey k;
+    k.layers.assign(layers, layers + n_layers);
+    k.hidden = hidden;
+    k.qkv_n = qkv_n;
+    k.ffn = ffn;
+    k.x_in = x_in;
+    k.x_out = x_out;
+    if (!h->sh_exec || !(h->sh_key == k)) {
+        if (h->fault == kFaultGraph) return fail(h, Q4_EFAULTINJ, "injected graph failure");
+        if (h->sh_exec) {
+            cudaGraphExecDestroy(h->sh_exec);
+            h->sh_exec = nullptr;
+        }
+        // Every rank enqueues the same sequence: per GEMV its rows (the
+        // M = 1 kernel on its row slice, input scaled to unit RMS), then the
+        // all-gather of every rank's rows; the step ends with the renorm.
+        Q4_CUDA(h, cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
+        int rc = Q4_OK;
+        for (int i = 0; i < 4 * n_layers && rc == Q4_OK; ++i) {
+            const int t = i % 4;
+            const q4gemv_layer& L = layers[i / 4];
+            const void* W = t == 0 ? L.qkv : t == 1 ? L.o : t == 2 ? L.gate_up : L.down;
+            const __half* xin = i == 0 ? static_cast<const __half*>(x_in) : h->sh_gather[(t + 3) % 4];
+            if (rows[t] > 0)
+                rc = launch_gemv(h, W, xin, h->sh_slice[t], 1, rows[t], k_of[t], i == 0 ? 0 : 1, nullptr,
+                                 h->cap, false);
+            if (rc == Q4_OK) {
+                const ncclResult_t r = g_nccl.AllGather(h->sh_slice[t], h->sh_gather[t], (size_t)chunk[t],
+                                                        ncclFloat16, h->comm, h->cap);
+                if (r != ncclSuccess) rc = fail(h, Q4_ECUDA, "ncclAllGather: %s", g_nccl.GetErrorString(r));
+            }
+        }
+        if (rc == Q4_OK) rc = launch_renorm(h, h->sh_gather[3], static_cast<__half*>(x_out), (int)hidden, h->cap, false);
+        cudaGraph_t graph = nullptr;
+        const cudaError_t ee = cudaStreamEndCapture(h->cap, &graph);
+        if (rc != Q4_OK) {
+            if (graph) cudaGraphDestroy(graph);
+            return rc;
+        }
+        if (ee != cudaSuccess) return cuda_fail(h, ee, "cudaStreamEndCapture");
+        const cudaError_t ei = cudaGraphInstantiate(&h->sh_exec, graph, 0);
+        cudaGraphDestroy(graph);
+        if (ei != cudaSuccess) {
+            h->sh_exec = nullptr;
+            return cuda_fail(h, ei, "cudaGraphInstantiate");
+        }
+        h->sh_key = k;
+    }
+    Q4_CUDA(h, cudaGraphLaunch(h->sh_exec, st));
+    return Q4_OK;
 }
 
 int q4gemv_sync_status(q4gemv_t h, q4gemv_stream_t stream) {
