@@ -193,20 +193,31 @@ def oracle_sample(min_seconds: float, threads: int):
     return done_bytes / elapsed / 1e9, f"{layers} full layer(s) of the step ({done_bytes / 1e6:.0f} MB), fp64 oracle", elapsed
 
 
-def oracle_rows_step(i: int, threads: int, frac: int = 64):
-    """One bounded reference step: GEMV (i mod 4) of layer (i/4 mod 64) on
-    every `frac`-th row."""
+def oracle_layer_step(i: int, threads: int):
+    """One reference step: all four GEMVs of layer i mod 64 of the workload,
+    whole matrices, fp64 oracle.  Returns (bytes, seconds)."""
     import oracle
-    l, t = (i // 4) % L, i % 4
-    N, K = DIMS[t]
-    sel = np.arange(0, N, frac)
-    rows = synth.q4_0_row_list(STEP_SEED, synth.weight_id(4 * l + t), K, sel) if len(sel) < 64 else \
-        synth.q4_0_matrix(STEP_SEED, synth.weight_id(4 * l + t), N, K)[sel]
-    x = synth.normal_f16(STEP_SEED, synth.act_id(0), K)
-    t0 = time.perf_counter()
-    oracle.q4_gemv(rows, K, x[None, :], threads=threads)
-    dt = time.perf_counter() - t0
-    return rows.size + 2 * K + 2 * len(sel), dt
+    l = i % L
+    x = synth.normal_f16(STEP_SEED, synth.act_id(0), max(HIDDEN, FFN))
+    done, dt = 0, 0.0
+    for t, (N, K) in enumerate(DIMS):
+        rows = synth.q4_0_matrix(STEP_SEED, synth.weight_id(4 * l + t), N, K)
+        t0 = time.perf_counter()
+        oracle.q4_gemv(rows, K, x[None, :K], threads=threads)
+        dt += time.perf_counter() - t0
+        done += gemv_bytes(N, K)
+    return done, dt
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def run_reference(args, rank: int):
@@ -214,15 +225,17 @@ def run_reference(args, rank: int):
     if rank != 0:
         return 0
     threads = os.cpu_count() or 1
-    for i in range(args.warmup):
-        oracle_rows_step(i, threads)
+    # Warm-up steps are short (one GEMV each): they only load the oracle.
+    for i in range(min(args.warmup, 1)):
+        oracle_layer_step(i, threads)
     tot_b, tot_t = 0, 0.0
     for i in range(args.steps):
-        b, dt = oracle_rows_step(args.warmup + i, threads)
+        b, dt = oracle_layer_step(i, threads)
         tot_b += b
         tot_t += dt
     gbs = tot_b / tot_t / 1e9
-    sample = "each step: one GEMV of the 27B-shaped step (cycling QKV, O, gate+up, down over the 64 layers) on every 64th row"
+    sample = ("each step: one whole layer of the 27B-shaped step (QKV, O, gate+up and down of "
+              "layer i mod 64, 186 MB of Q4_0), fp64 oracle; the step's GB/s")
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
@@ -349,6 +362,106 @@ def build_weights_sharded(eng, torch, q4, rank: int, world: int):
     return layers, t_repack
 
 
+def time_graph(torch, launch, n: int, reps: int = 5):
+    """Mean time (us) of launch(j), j < n, captured as one CUDA graph and
+    replayed `reps` times after a warm-up replay."""
+    launch(0)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for j in range(n):
+            launch(j)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / (reps * n)
+
+
+def extra_workloads(eng, torch, q4, layers):
+    """The benchmark's other configurations, each timed over matrices that
+    together exceed 4x L2 (the step's 64 distinct matrices of a shape, or
+    rotating copies): the 1024x1024 GEMV (also single-launch latency), M = 4
+    and 16 on both FFN shapes, Q8_0 at M = 1, the gated down GEMV, and the
+    prefill GEMM at the pages' two prompt lengths."""
+    peak, _ = measured_peaks()
+    tpeak, tkind = measured_tensor_peak()
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    out = {}
+
+    def hbm(us, nbytes, rows):
+        return {"us_per_call": us, "GB/s": nbytes / us / 1e3, "frac_of_hbm_peak": nbytes / us / 1e3 / peak,
+                "rows_per_s": rows / us * 1e6}
+
+    # config 0: 1024 x 1024, M = 1
+    N0 = K0 = 1024
+    seed0 = synth.workload_seed(0)
+    W0 = eng.repack(torch.from_numpy(synth.q4_0_matrix(seed0, synth.weight_id(0), N0, K0).reshape(-1)).cuda(), N0, K0)
+    R0 = -(-4 * l2 // W0.numel())
+    mats0 = [W0] + [W0.clone() for _ in range(R0 - 1)]
+    x0 = torch.from_numpy(synth.activations(seed0, 1, K0).view(np.float16)).cuda()
+    y0 = torch.empty(N0, dtype=torch.float16, device="cuda")
+    us0 = time_graph(torch, lambda j: eng.run(mats0[j], x0, N0, K0, out=y0), R0, reps=3)
+    lat = []
+    for j in range(30):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        eng.run(mats0[j % R0], x0, N0, K0, out=y0)
+        e1.record()
+        torch.cuda.synchronize()
+        lat.append(e0.elapsed_time(e1) * 1e3)
+    out["gemv_1024x1024_m1"] = dict(hbm(us0, gemv_bytes(N0, K0), N0),
+                                   single_launch_us_median=statistics.median(lat[5:]),
+                                   rotating_copies=R0)
+    del mats0
+
+    # config 3: M = 4 and 16 on the FFN shapes (the step's 64 matrices of each)
+    small = {}
+    for M in (4, 16):
+        for t in (2, 3):
+            N, K = DIMS[t]
+            x = torch.from_numpy(synth.activations(synth.workload_seed(3) + M, M, K).view(np.float16)).cuda()
+            y = torch.empty(M, N, dtype=torch.float16, device="cuda")
+            us = time_graph(torch, lambda j: eng.run(layers[j][t], x, N, K, out=y), L, reps=3)
+            nbytes = N * (K // 32) * 18 + 2 * M * (K + N)
+            small[f"M{M}_{SHAPE_NAMES[t]}"] = dict(hbm(us, nbytes, N), tflops=2.0 * M * N * K / us / 1e6)
+    out["small_m"] = small
+
+    # Q8_0 at M = 1 on the FFN shapes (rotating copies)
+    q8 = {}
+    for t in (2, 3):
+        N, K = DIMS[t]
+        Wq = eng.repack_q8_0(torch.from_numpy(synth.q8_0_matrix(synth.workload_seed(2), synth.weight_id(t), N, K)
+                                              .reshape(-1)).cuda(), N, K)
+        Rq = max(2, -(-4 * l2 // Wq.numel()))
+        mats = [Wq] + [Wq.clone() for _ in range(Rq - 1)]
+        x = torch.from_numpy(synth.activations(synth.workload_seed(2), 1, K).view(np.float16)).cuda()
+        y = torch.empty(N, dtype=torch.float16, device="cuda")
+        us = time_graph(torch, lambda j: eng.run_q8_0(mats[j], x, N, K, out=y), Rq, reps=3)
+        q8[SHAPE_NAMES[t]] = hbm(us, N * (K // 32) * 34 + 2 * (K + N), N)
+        del mats, Wq
+    out["q8_0_m1"] = q8
+
+    # the gated down GEMV: y = W_down (SiLU(gate) * up) from the 2*ffn gate+up output
+    N, K = DIMS[3]
+    gu = torch.from_numpy(synth.activations(synth.workload_seed(2) + 7, 1, 2 * K).view(np.float16)).cuda().reshape(-1)
+    y = torch.empty(N, dtype=torch.float16, device="cuda")
+    us = time_graph(torch, lambda j: eng.run_swiglu(layers[j][3], gu, N, K, out=y), L, reps=3)
+    out["gated_down_" + SHAPE_NAMES[3]] = hbm(us, N * (K // 32) * 18 + 4 * K + 2 * N, N)
+
+    # prefill GEMM at the pages' prompt lengths (86, 169)
+    for M in (86, 169):
+        out[f"prefill_gemm_m{M}"] = time_prefill(eng, torch, layers, M=M)
+    return out
+
+
 def run_ours(args, rank: int, world: int, dist):
     import torch
     import q4_quantized_decode_b200 as q4
@@ -440,7 +553,7 @@ def run_ours(args, rank: int, world: int, dist):
 
     extras = rank == 0 and not args.no_per_shape and not args.shard
     per_shape = time_shapes(eng, torch, layers) if extras else None
-    prefill = time_prefill(eng, torch, layers) if extras else None
+    others = extra_workloads(eng, torch, q4, layers) if extras else None
     if eng.sync_status() != q4.Q4_OK:
         raise RuntimeError("device status after timing")
 
@@ -478,8 +591,11 @@ def run_ours(args, rank: int, world: int, dist):
     if not args.no_cpu_baseline:
         threads = os.cpu_count() or 1
         cgbs, sample, secs = oracle_sample(args.cpu_seconds, threads)
+        c1, sample1, secs1 = oracle_sample(min(3.0, args.cpu_seconds), 1)
         cpu = {"value": cgbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
-               "sample": f"{sample}, {secs:.1f} s on {threads} host threads"}
+               "sample": f"{sample}, {secs:.1f} s on {threads} host threads",
+               "single_thread": {"value": c1, "unit": "GB/s", "sample": f"{sample1}, {secs1:.1f} s"},
+               "cpu_model": cpu_model()}
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -503,7 +619,7 @@ def run_ours(args, rank: int, world: int, dist):
         "clocks": clocks,
         "repack_s_per_step_weights": t_repack,
         "per_shape_m1": per_shape,
-        "prefill_gemm_m169": prefill,
+        "other_configs": others,
     }
     print(json.dumps(line), flush=True)
     return 0
