@@ -361,7 +361,12 @@ int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, in
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = mma_ring(nt8) + q4::gemv_mma_smem_bytes(nt8, Wf);
     cfg.stream = st;
-    cfg.numAttrs = 0;
+    // The weight stream starts before the wait for the previous kernel.
+    cudaLaunchAttribute pattr[1];
+    pattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pattr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pattr;
+    cfg.numAttrs = 1;
     cudaError_t e = nt8 == 1 ? cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_1, a)
                              : cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_2, a);
     if (e != cudaSuccess) return cuda_fail(h, e, "gemv (mma) launch");
@@ -758,7 +763,7 @@ int q4gemv_run(q4gemv_t h, const void* W, const void* x, void* y, int M, int64_t
                               K, st);
     if (dp2a_fits(M, K))
         return launch_gemv(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K,
-                           0, nullptr, st, false);
+                           0, nullptr, st, true);
     return launch_gemv_mma(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K,
                            st);
 }
@@ -773,7 +778,7 @@ int q4gemv_run_swiglu(q4gemv_t h, const void* W, const void* gate_up, void* y, i
                     (long long)K);
     Q4_CUDA(h, cudaSetDevice(h->device));
     return launch_gemv(h, W, static_cast<const __half*>(gate_up), static_cast<__half*>(y), 1, N, K,
-                       0, nullptr, static_cast<cudaStream_t>(stream), false, false, true);
+                       0, nullptr, static_cast<cudaStream_t>(stream), true, false, true);
 }
 
 size_t q4gemv_q8_0_gguf_bytes(int64_t N, int64_t K) {
@@ -828,7 +833,7 @@ int q4gemv_q8_0_run(q4gemv_t h, const void* W, const void* x, void* y, int M, in
     Q4_CUDA(h, cudaSetDevice(h->device));
     if (q8_dp2a_fits(M, K))
         return launch_gemv(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K, 0,
-                           nullptr, static_cast<cudaStream_t>(stream), false, true);
+                           nullptr, static_cast<cudaStream_t>(stream), true, true);
     return launch_gemm_tc(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K,
                           static_cast<cudaStream_t>(stream), true);
 }
