@@ -388,7 +388,7 @@ def extra_workloads(eng, torch, q4, layers):
     """The benchmark's other configurations, each timed over matrices that
     together exceed 4x L2 (the step's 64 distinct matrices of a shape, or
     rotating copies): the 1024x1024 GEMV (also single-launch latency), M = 4
-    and 16 on both FFN shapes, Q8_0 at M = 1, the gated down GEMV, and the
+    and 16 on both FFN shapes, Q8_0 at M = 1, 4, 16, the gated down GEMV, and the
     prefill GEMM at the pages' two prompt lengths."""
     peak, _ = measured_peaks()
     tpeak, tkind = measured_tensor_peak()
@@ -434,7 +434,7 @@ def extra_workloads(eng, torch, q4, layers):
             small[f"M{M}_{SHAPE_NAMES[t]}"] = dict(hbm(us, nbytes, N), tflops=2.0 * M * N * K / us / 1e6)
     out["small_m"] = small
 
-    # Q8_0 at M = 1 on the FFN shapes (rotating copies)
+    # Q8_0 at M = 1, 4, 16 on the FFN shapes (rotating copies)
     q8 = {}
     for t in (2, 3):
         N, K = DIMS[t]
@@ -442,12 +442,13 @@ def extra_workloads(eng, torch, q4, layers):
                                               .reshape(-1)).cuda(), N, K)
         Rq = max(2, -(-4 * l2 // Wq.numel()))
         mats = [Wq] + [Wq.clone() for _ in range(Rq - 1)]
-        x = torch.from_numpy(synth.activations(synth.workload_seed(2), 1, K).view(np.float16)).cuda()
-        y = torch.empty(N, dtype=torch.float16, device="cuda")
-        us = time_graph(torch, lambda j: eng.run_q8_0(mats[j], x, N, K, out=y), Rq, reps=3)
-        q8[SHAPE_NAMES[t]] = hbm(us, N * (K // 32) * 34 + 2 * (K + N), N)
+        for M in (1, 4, 16):
+            x = torch.from_numpy(synth.activations(synth.workload_seed(2) + M, M, K).view(np.float16)).cuda()
+            y = torch.empty(M, N, dtype=torch.float16, device="cuda")
+            us = time_graph(torch, lambda j: eng.run_q8_0(mats[j], x, N, K, out=y), Rq, reps=3)
+            q8[(f"M{M}_" if M > 1 else "") + SHAPE_NAMES[t]] = hbm(us, N * (K // 32) * 34 + 2 * M * (K + N), N)
         del mats, Wq
-    out["q8_0_m1"] = q8
+    out["q8_0"] = q8
 
     # the gated down GEMV: y = W_down (SiLU(gate) * up) from the 2*ffn gate+up output
     N, K = DIMS[3]

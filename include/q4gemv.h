@@ -211,7 +211,10 @@ Q4GEMV_API int q4gemv_q8_0_validate(int M, int64_t N, int64_t K, const void* W_p
  * q4gemv_run).  M <= 2 with M*K <= 36,864 (and the kernel's shared memory):
  * the activations are converted per 32-column block as for Q4_0 (exact for
  * the block maximum), each block's dot product with the 8-bit codes is an
- * exact integer, converted to fp32 once and scaled by d.  Otherwise the
+ * exact integer, converted to fp32 once and scaled by d.  M <= 16 otherwise:
+ * the mma.sync kernel of q4gemv_run's M = 3..16 path with Q8_0 segments (each
+ * signed code exact in binary16, exact per-block sums in fp32, d applied once
+ * per output and block; column panels for wide K).  M = 17..256: the
  * tcgen05 GEMM of q4gemv_run's M > 16 path runs with Q8_0 segments: each
  * weight q * d (up to 18 significant bits) is split exactly into two binary16
  * parts; scales |d| >= 512 overflow the split (non-finite outputs); its

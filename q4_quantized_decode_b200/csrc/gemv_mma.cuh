@@ -92,7 +92,7 @@ static __global__ void __launch_bounds__(256) panel_reduce_kernel(const float* _
 // A warp's ring over a panel: stage k holds C consecutive panel segments of
 // the warp's run [s0, s1), filled by one bulk copy per contiguous piece (a
 // stage that crosses a tile boundary of a narrower panel takes two or more).
-template <int R, int C>
+template <int R, int C, int SEG = kSegBytes>
 struct PanelRing {
     uint32_t stage0;
     uint64_t* bars;
@@ -102,7 +102,7 @@ struct PanelRing {
 
     __device__ void init(uint32_t ring_base, uint64_t* bar_base, int warp, const MmaArgs& a, int s0_,
                          int s1_) {
-        stage0 = ring_base + (uint32_t)warp * R * C * kSegBytes;
+        stage0 = ring_base + (uint32_t)warp * R * C * SEG;
         bars = bar_base + warp * R;
         W = a.W;
         s0 = s0_;
@@ -114,18 +114,17 @@ struct PanelRing {
         it = s0_ / KBv;
         ij = s0_ - it * KBv;
     }
-    __device__ uint32_t stage(int k) const { return stage0 + (uint32_t)k * C * kSegBytes; }
+    __device__ uint32_t stage(int k) const { return stage0 + (uint32_t)k * C * SEG; }
     // Lane 0 only, chunks in order.
     __device__ void issue(int ch) {
         const int k = ch % R;
         int n = min(C, nseg - ch * C);
-        mbar_arrive_expect_tx(bars + k, (uint32_t)n * kSegBytes);
+        mbar_arrive_expect_tx(bars + k, (uint32_t)n * SEG);
         uint32_t dst = stage(k);
         while (n > 0) {
             const int len = min(n, KBv - ij);
-            bulk_g2s_addr(dst, W + ((size_t)it * KB + p0 + ij) * kSegBytes, (uint32_t)len * kSegBytes,
-                          bars + k);
-            dst += (uint32_t)len * kSegBytes;
+            bulk_g2s_addr(dst, W + ((size_t)it * KB + p0 + ij) * SEG, (uint32_t)len * SEG, bars + k);
+            dst += (uint32_t)len * SEG;
             n -= len;
             ij += len;
             if (ij == KBv) {
@@ -190,14 +189,37 @@ __device__ __forceinline__ CodePairs unpack_pairs(uint32_t w) {
     return o;
 }
 
-template <int NT8, int WARPS, int R, int C>
+// Exact f16 pairs from two Q8_0 code words (signed bytes; lo: codes 4c..4c+3,
+// hi: codes 16+4c..): a byte with its sign bit flipped, placed in the
+// mantissa of f16 1024, is 1024 + q + 128; minus 1152 it is exactly q.  The
+// same k order as unpack_pairs.
+__device__ __forceinline__ CodePairs unpack_pairs_q8(uint32_t lo, uint32_t hi) {
+    CodePairs o;
+    asm("{\n\t.reg .b32 xl, xh, t0, t1, t2, t3;\n\t"
+        "xor.b32 xl, %4, 0x80808080;\n\t"
+        "xor.b32 xh, %5, 0x80808080;\n\t"
+        "prmt.b32 t0, xl, 0x64646464, 0x4240;\n\t"
+        "prmt.b32 t1, xl, 0x64646464, 0x4341;\n\t"
+        "prmt.b32 t2, xh, 0x64646464, 0x4240;\n\t"
+        "prmt.b32 t3, xh, 0x64646464, 0x4341;\n\t"
+        "sub.rn.f16x2 %0, t0, %6;\n\t"
+        "sub.rn.f16x2 %1, t1, %6;\n\t"
+        "sub.rn.f16x2 %2, t2, %6;\n\t"
+        "sub.rn.f16x2 %3, t3, %6;\n\t}"
+        : "=r"(o.p), "=r"(o.q), "=r"(o.r), "=r"(o.s)
+        : "r"(lo), "r"(hi), "r"(0x64806480u));
+    return o;
+}
+
+template <int NT8, int WARPS, int R, int C, bool Q8 = false>
 __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a_in) {
+    constexpr int SEG = SegFmt<Q8>::kBytes;
     const MmaArgs a = panel_view(a_in);
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[WARPS * R];
     constexpr int NT = WARPS * 32;
     const uint32_t smem_base = smem_addr(smem);
-    const uint32_t xsm = smem_base + (uint32_t)ring_bytes(WARPS, R, C);
+    const uint32_t xsm = smem_base + (uint32_t)ring_bytes(WARPS, R, C, SEG);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, c = lane & 3;
     const int gw = blockIdx.x * WARPS + warp;
@@ -215,7 +237,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
     const int b0 = (cs1 - cs0 >= KB) ? 0 : (cs0 % KB);
     const int vstride = mma_vstride(nblk);
 
-    PanelRing<R, C> ring;
+    PanelRing<R, C, SEG> ring;
     ring.init(smem_base, bars, warp, a, s0, s1);
     if (lane == 0) {
         for (int k = 0; k < R; ++k) mbar_init(bars + warp * R + k, 1);
@@ -313,8 +335,15 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
     const uint32_t x_lane = xsm + (uint32_t)g * vstride + (uint32_t)c * 16;
 
     auto segment = [&](uint32_t seg, int jbs) {
-        const uint4 w = lds128(seg + lane * 16);
-        const uint2 dd = lds64(seg + kSegSclOff + g * 8);
+        uint4 w, w2;
+        if constexpr (Q8) {
+            w = lds128(seg + lane * 32);        // rows g (lo, hi words), g+8 (lo, hi)
+            w2 = lds128(seg + lane * 32 + 16);  // rows g+16, g+24
+        } else {
+            w = lds128(seg + lane * 16);        // rows g, g+8, g+16, g+24
+            w2 = w;
+        }
+        const uint2 dd = lds64(seg + SegFmt<Q8>::kScl + g * 8);
         uint4 xv[NT8];
 #pragma unroll
         for (int nt = 0; nt < NT8; ++nt)
@@ -327,8 +356,14 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
         const uint32_t w1s[2] = {w.y, w.w};
 #pragma unroll
         for (int tt = 0; tt < 2; ++tt) {
-            const CodePairs u0 = unpack_pairs(w0s[tt]);   // row g (+16)
-            const CodePairs u1 = unpack_pairs(w1s[tt]);   // row g+8 (+16)
+            CodePairs u0, u1;
+            if constexpr (Q8) {
+                u0 = tt == 0 ? unpack_pairs_q8(w.x, w.y) : unpack_pairs_q8(w2.x, w2.y);    // row g (+16)
+                u1 = tt == 0 ? unpack_pairs_q8(w.z, w.w) : unpack_pairs_q8(w2.z, w2.w);    // row g+8 (+16)
+            } else {
+                u0 = unpack_pairs(w0s[tt]);   // row g (+16)
+                u1 = unpack_pairs(w1s[tt]);   // row g+8 (+16)
+            }
 #pragma unroll
             for (int nt = 0; nt < NT8; ++nt) {
                 float e0, e1, e2, e3;
@@ -352,7 +387,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
             // No tile ends inside this stage: its segments at constant
             // offsets, free to interleave.
 #pragma unroll
-            for (int j = 0; j < C; ++j) segment(st + j * kSegBytes, jb + j);
+            for (int j = 0; j < C; ++j) segment(st + j * SEG, jb + j);
             b += C;
             jb += C;
             if (jb == KB) jb = 0;
@@ -365,7 +400,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
                     jb = KB - b0;
                     if (jb >= KB) jb -= KB;
                 }
-                segment(st + j * kSegBytes, jb);
+                segment(st + j * SEG, jb);
                 ++b;
                 if (++jb == KB) jb = 0;
             }

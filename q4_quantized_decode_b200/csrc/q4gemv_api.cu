@@ -45,6 +45,10 @@ constexpr int kRq1 = 3, kCq1 = 3, kRq2 = 2, kCq2 = 3;
 #define Q4_Q8_KERNEL_2 q4::gemv_dp2a_kernel<2, kWarps, kRq2, kCq2, true>
 #define Q4_MMA_KERNEL_1 q4::gemv_mma_kernel<1, kWarps, kRm1, kCm1>
 #define Q4_MMA_KERNEL_2 q4::gemv_mma_kernel<2, kWarps, kRm2, kCm2>
+// The same for Q8_0 (1088-byte segments: stages of about the same bytes).
+constexpr int kRmq1 = 2, kCmq1 = 4, kRmq2 = 2, kCmq2 = 2;
+#define Q4_MMA_Q8_KERNEL_1 q4::gemv_mma_kernel<1, kWarps, kRmq1, kCmq1, true>
+#define Q4_MMA_Q8_KERNEL_2 q4::gemv_mma_kernel<2, kWarps, kRmq2, kCmq2, true>
 #define Q4_STACK_KERNEL q4::stack_kernel<kWarps, kR1, kC1>
 #define Q4_SWIGLU_KERNEL q4::gemv_swiglu_kernel<kWarps, kR1, kC1>
 // Largest input of a GEMV in the persistent step (its staging holds up to
@@ -257,13 +261,16 @@ int ensure_ws(q4gemv_ctx* h, int warps, cudaStream_t st) {
 }
 
 // Ring bytes of the tensor-core kernel (nt8 = 1: up to 8 vectors, 2: up to 16).
-size_t mma_ring(int nt8) {
+size_t mma_ring(int nt8, bool q8 = false) {
+    if (q8)
+        return nt8 == 1 ? q4::ring_bytes(kWarps, kRmq1, kCmq1, q4::kSegBytesQ8)
+                        : q4::ring_bytes(kWarps, kRmq2, kCmq2, q4::kSegBytesQ8);
     return nt8 == 1 ? q4::ring_bytes(kWarps, kRm1, kCm1) : q4::ring_bytes(kWarps, kRm2, kCm2);
 }
 
 // Largest block count one CTA may stage beside the ring.
-int mma_xcap(int nt8) {
-    const size_t ring = mma_ring(nt8);
+int mma_xcap(int nt8, bool q8 = false) {
+    const size_t ring = mma_ring(nt8, q8);
     int xcap = 1;
     while (ring + q4::gemv_mma_smem_bytes(nt8, xcap + 1) <= kMaxDynSmem) ++xcap;
     return xcap;
@@ -303,15 +310,16 @@ int ensure_cnt(q4gemv_ctx* h, int64_t n, cudaStream_t st) {
 // staging and keeps the staged slice (panel width × 8 or 16 vectors × 64 B)
 // at most half the weight bytes a CTA streams; P > 1 adds a reduce launch.
 int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M, int64_t N,
-                    int64_t K, cudaStream_t st) {
+                    int64_t K, cudaStream_t st, bool q8 = false) {
     if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
     const int nt8 = M <= 8 ? 1 : 2;
     const int KB = (int)(K / 32);
     const int T = (int)((N + 31) / 32);
-    const int xcap = mma_xcap(nt8);
+    const int xcap = mma_xcap(nt8, q8);
+    const int64_t seg = q8 ? q4::kSegBytesQ8 : q4::kSegBytes;
     int64_t P = (KB + xcap - 1) / xcap;
-    // staging per CTA <= half its weights: P >= 2 * 64 * vecs * sms / (576 * T)
-    const int64_t p_ratio = (2 * 64 * 8 * nt8 * (int64_t)h->sms + 576 * (int64_t)T - 1) / (576 * (int64_t)T);
+    // staging per CTA <= half its weights: P >= 2 * 64 * vecs * sms / (seg * T)
+    const int64_t p_ratio = (2 * 64 * 8 * nt8 * (int64_t)h->sms + seg * (int64_t)T - 1) / (seg * (int64_t)T);
     if (P < p_ratio) P = p_ratio;
     if (P > KB) P = KB;
     if (P > h->sms) P = h->sms;
@@ -359,7 +367,7 @@ int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, in
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)cpp, (unsigned)P);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = mma_ring(nt8) + q4::gemv_mma_smem_bytes(nt8, Wf);
+    cfg.dynamicSmemBytes = mma_ring(nt8, q8) + q4::gemv_mma_smem_bytes(nt8, Wf);
     cfg.stream = st;
     // The weight stream starts before the wait for the previous kernel.
     cudaLaunchAttribute pattr[1];
@@ -367,8 +375,11 @@ int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, in
     pattr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = pattr;
     cfg.numAttrs = 1;
-    cudaError_t e = nt8 == 1 ? cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_1, a)
-                             : cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_2, a);
+    cudaError_t e;
+    if (q8)
+        e = nt8 == 1 ? cudaLaunchKernelEx(&cfg, Q4_MMA_Q8_KERNEL_1, a) : cudaLaunchKernelEx(&cfg, Q4_MMA_Q8_KERNEL_2, a);
+    else
+        e = nt8 == 1 ? cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_1, a) : cudaLaunchKernelEx(&cfg, Q4_MMA_KERNEL_2, a);
     if (e != cudaSuccess) return cuda_fail(h, e, "gemv (mma) launch");
     if (P > 1) {
         const int64_t MN = (int64_t)M * N;
@@ -674,6 +685,7 @@ int q4gemv_create(q4gemv_t* out, int device) {
         if (set_smem_attr(Q4_DP2A_KERNEL_1) || set_smem_attr(Q4_DP2A_KERNEL_2) ||
             set_smem_attr(Q4_Q8_KERNEL_1) || set_smem_attr(Q4_Q8_KERNEL_2) ||
             set_smem_attr(Q4_MMA_KERNEL_1) || set_smem_attr(Q4_MMA_KERNEL_2) ||
+            set_smem_attr(Q4_MMA_Q8_KERNEL_1) || set_smem_attr(Q4_MMA_Q8_KERNEL_2) ||
             set_smem_attr(Q4_STACK_KERNEL) || set_smem_attr(Q4_SWIGLU_KERNEL) ||
             set_smem_attr(q4::gemm_tc_kernel<false>) ||
             set_smem_attr(q4::gemm_tc_kernel<true>) ||
@@ -834,6 +846,9 @@ int q4gemv_q8_0_run(q4gemv_t h, const void* W, const void* x, void* y, int M, in
     if (q8_dp2a_fits(M, K))
         return launch_gemv(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K, 0,
                            nullptr, static_cast<cudaStream_t>(stream), true, true);
+    if (M <= Q4GEMV_MAX_M_GEMV)
+        return launch_gemv_mma(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K,
+                               static_cast<cudaStream_t>(stream), true);
     return launch_gemm_tc(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K,
                           static_cast<cudaStream_t>(stream), true);
 }

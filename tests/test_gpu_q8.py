@@ -106,7 +106,8 @@ def test_q8_validate_limits(eng):
     assert q4.q4gemv_q8_0_validate(1, 32, 32, A + 8, A, A) == q4.Q4_EALIGN
 
 
-# ---------------------------------------------------------------- M >= 3: tensor-core GEMM
+# ---------------------------------------------------------------- M >= 3 (and wide K): tensor cores
+# (mma.sync kernel up to M = 16, the tcgen05 GEMM beyond)
 
 @pytest.mark.parametrize("N,K,M", [(256, 64, 3), (300, 96, 4), (520, 160, 16), (33, 1056, 17),
                                    (1024, 1024, 86), (5, 32, 256), (2048, 5120, 169),
@@ -129,8 +130,9 @@ def test_q8_gemm_full_shapes_sampled(eng, M, N, K):
     assert rel_err(np.ascontiguousarray(y[:, rows]), ref) <= TOL
 
 
-def test_q8_gemm_extreme_codes_and_deterministic(eng):
-    N, K, M = 300, 512, 40
+@pytest.mark.parametrize("M", [4, 16, 40])
+def test_q8_gemm_extreme_codes_and_deterministic(eng, M):
+    N, K = 300, 512
     g = synth.q8_0_matrix(15, synth.weight_id(2), N, K).reshape(N, K // 32, 34)
     g[:, :, 2:] = np.where(np.arange(32) % 3 == 0, 0x80, np.where(np.arange(32) % 3 == 1, 0x7F, 0xFF))
     g = g.reshape(N, -1)
