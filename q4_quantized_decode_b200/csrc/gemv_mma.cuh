@@ -144,8 +144,10 @@ struct PanelRing {
 __host__ __device__ constexpr int mma_vstride(int nblk) {
     return nblk * 64 + ((nblk & 1) ? 0 : 64);
 }
-__host__ __device__ constexpr size_t gemv_mma_smem_bytes(int nt8, int nblk) {
-    return (size_t)8 * nt8 * mma_vstride(nblk);
+// Only the M real vectors are staged: MMA columns past M read vector M - 1
+// (their outputs are never used).
+__host__ __device__ constexpr size_t gemv_mma_smem_bytes(int M, int nblk) {
+    return (size_t)M * mma_vstride(nblk);
 }
 
 // Position of element e of a 32-column block in the staged order: lane group
@@ -250,8 +252,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
     pdl_wait();
 
     // Stage the CTA's activation blocks with plain 16-byte loads (eight per
-    // round per thread), reordered into lane order; zero vectors pad M up to
-    // 8*NT8.
+    // round per thread), reordered into lane order (the M real vectors only).
     {
         const int nchunk = a.M * nblk * 4;
         for (int p0 = threadIdx.x; p0 < nchunk; p0 += 8 * NT) {
@@ -282,9 +283,6 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
                 }
             }
         }
-        const int zwords = (8 * NT8 - a.M) * vstride / 8;
-        for (int i = threadIdx.x; i < zwords; i += NT)
-            sts64(xsm + (uint32_t)a.M * vstride + (uint32_t)i * 8, make_uint2(0u, 0u));
         __syncthreads();
     }
 
@@ -332,7 +330,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
     int b = s0 - t_first * KB;                 // block of the next segment
     int jb = b - b0;                           // its staged slot
     if (jb < 0) jb += KB;
-    const uint32_t x_lane = xsm + (uint32_t)g * vstride + (uint32_t)c * 16;
+    // MMA column 8 nt + g reads vector min(8 nt + g, M - 1).
+    uint32_t x_lane[NT8];
+#pragma unroll
+    for (int nt = 0; nt < NT8; ++nt)
+        x_lane[nt] = xsm + (uint32_t)min(8 * nt + g, a.M - 1) * vstride + (uint32_t)c * 16;
 
     auto segment = [&](uint32_t seg, int jbs) {
         uint4 w, w2;
@@ -347,7 +349,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
         uint4 xv[NT8];
 #pragma unroll
         for (int nt = 0; nt < NT8; ++nt)
-            xv[nt] = lds128(x_lane + (uint32_t)(8 * nt) * vstride + (uint32_t)jbs * 64);
+            xv[nt] = lds128(x_lane[nt] + (uint32_t)jbs * 64);
         const float2 d01 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
         const float2 d23 = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
         const float dA[2] = {d01.x, d23.x};   // rows g, g+16

@@ -269,10 +269,10 @@ size_t mma_ring(int nt8, bool q8 = false) {
 }
 
 // Largest block count one CTA may stage beside the ring.
-int mma_xcap(int nt8, bool q8 = false) {
+int mma_xcap(int nt8, int M, bool q8 = false) {
     const size_t ring = mma_ring(nt8, q8);
     int xcap = 1;
-    while (ring + q4::gemv_mma_smem_bytes(nt8, xcap + 1) <= kMaxDynSmem) ++xcap;
+    while (ring + q4::gemv_mma_smem_bytes(M, xcap + 1) <= kMaxDynSmem) ++xcap;
     return xcap;
 }
 
@@ -315,11 +315,11 @@ int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, in
     const int nt8 = M <= 8 ? 1 : 2;
     const int KB = (int)(K / 32);
     const int T = (int)((N + 31) / 32);
-    const int xcap = mma_xcap(nt8, q8);
+    const int xcap = mma_xcap(nt8, M, q8);
     const int64_t seg = q8 ? q4::kSegBytesQ8 : q4::kSegBytes;
     int64_t P = (KB + xcap - 1) / xcap;
-    // staging per CTA <= half its weights: P >= 2 * 64 * vecs * sms / (seg * T)
-    const int64_t p_ratio = (2 * 64 * 8 * nt8 * (int64_t)h->sms + seg * (int64_t)T - 1) / (seg * (int64_t)T);
+    // staging per CTA <= half its weights: P >= 2 * 64 * M * sms / (seg * T)
+    const int64_t p_ratio = (2 * 64 * (int64_t)M * h->sms + seg * (int64_t)T - 1) / (seg * (int64_t)T);
     if (P < p_ratio) P = p_ratio;
     if (P > KB) P = KB;
     if (P > h->sms) P = h->sms;
@@ -367,7 +367,7 @@ int launch_gemv_mma(q4gemv_ctx* h, const void* W, const __half* x, __half* y, in
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)cpp, (unsigned)P);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = mma_ring(nt8, q8) + q4::gemv_mma_smem_bytes(nt8, Wf);
+    cfg.dynamicSmemBytes = mma_ring(nt8, q8) + q4::gemv_mma_smem_bytes(M, Wf);
     cfg.stream = st;
     // The weight stream starts before the wait for the previous kernel.
     cudaLaunchAttribute pattr[1];
