@@ -14,9 +14,11 @@
 
 namespace q4 {
 
-// SiLU(g) = g / (1 + e^-g) in fp32 (hardware exponential; +-0 for very
-// negative g, whose exponential overflows).
-__device__ __forceinline__ float silu_f32(float g) { return g / (1.f + __expf(-g)); }
+// SiLU(g) = g / (1 + e^-g) in fp32 with the hardware exponential and the
+// fast quotient (reciprocal approximation times g, within 2 ulp): every CTA
+// of the down GEMV converts all K entries, so the per-entry cost is on the
+// critical path.  +-0 for very negative g, whose exponential overflows.
+__device__ __forceinline__ float silu_f32(float g) { return __fdividef(g, 1.f + __expf(-g)); }
 
 // Gated staging for the M = 1 kernel, all threads of the CTA: thread t takes
 // the 16-byte chunks q = t, t + NT, ... of the gate half and the same chunks
