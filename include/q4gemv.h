@@ -147,6 +147,15 @@ Q4GEMV_API int q4gemv_repack(q4gemv_t h, const void* gguf, void* packed,
  * of P*M*N floats owned by the handle (preallocated for P*M*N <= 2^21; a
  * larger first call grows it, which synchronises the device and must not
  * happen during a stream capture).
+ * With the environment variable Q4GEMV_SMALL_M=tcs (read at create) that
+ * path runs on the tcgen05 tensor cores instead: kind::i8 MMAs, one per 128
+ * rows x 32 columns, the weights dequantised to 16 (q - 8) in tensor memory
+ * and the activations converted per block and vector to 15-bit integers X
+ * (|X| <= 2^14, the block maximum exact) split into two signed bytes; the
+ * int32 block sums are exact and scaled in fp32.  It keeps the same output
+ * contract (non-finite inputs give NaN outputs for their vector) and uses
+ * the same activation image buffer; it is slower than the mma.sync kernel on
+ * the measured shapes and is kept for comparison.
  * For M = 17..256 (prefill chunks) a dense-contraction path on the tcgen05
  * tensor cores runs instead: "dequantise the weight tile, then multiply" --
  * each weight (q - 8) * d is split exactly into two binary16 parts (the

@@ -12,7 +12,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libq4gemv.so")
 SOURCES = ["q4gemv_api.cu", "q4gemv_noalloc.cu"]
 HEADERS = ["device_common.cuh", "partition.cuh", "gemv_dp2a.cuh", "gemv_mma.cuh", "stack.cuh",
-           "gemm_tc.cuh", "gemv_swiglu.cuh"]
+           "gemm_tc.cuh", "gemv_swiglu.cuh", "gemv_tcs.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -18,6 +18,7 @@
 #include "gemm_tc.cuh"
 #include "gemv_mma.cuh"
 #include "gemv_swiglu.cuh"
+#include "gemv_tcs.cuh"
 #include "stack.cuh"
 
 namespace {
@@ -51,11 +52,17 @@ constexpr int kRmq1 = 2, kCmq1 = 4, kRmq2 = 2, kCmq2 = 2;
 #define Q4_MMA_Q8_KERNEL_2 q4::gemv_mma_kernel<2, kWarps, kRmq2, kCmq2, true>
 #define Q4_STACK_KERNEL q4::stack_kernel<kWarps, kR1, kC1>
 #define Q4_SWIGLU_KERNEL q4::gemv_swiglu_kernel<kWarps, kR1, kC1>
+static_assert(Q4GEMV_MAX_M_GEMV == 16, "the small-M tensor-core kernel reads 16 accumulator columns");
 // Largest input of a GEMV in the persistent step (its staging holds up to
 // kStackXChunks 16-byte chunks per thread).
 constexpr int kStackKmax = q4::kStackXChunks * 8 * kThreads;
 
 enum StackMode { kStackPersistent = 0, kStackKernels = 1 };
+// Kernel of the Q4_0 GEMVs with 3..16 vectors (and of M <= 2 with K beyond
+// the dp2a kernel's staging): the mma.sync kernel (default; the faster of the
+// two on every measured shape) or the tcgen05 kernel (Q4GEMV_SMALL_M = tcs,
+// read at create).
+enum SmallM { kSmallMma = 0, kSmallTcs = 1 };
 
 size_t dp2a_smem(int M, int64_t K, bool q8 = false) {
     if (q8)
@@ -104,6 +111,7 @@ struct q4gemv_ctx {
     cudaGraphExec_t exec = nullptr;
     StackKey key;
     int stack_mode = kStackPersistent;
+    int small_m = kSmallMma;
     q4::StackGemv* desc = nullptr;   // device descriptors of the persistent step
     int desc_cap = 0;
     StackKey desc_key;
@@ -414,6 +422,63 @@ int ensure_ximg(q4gemv_ctx* h, size_t bytes, cudaStream_t st) {
     return Q4_OK;
 }
 
+// Launch a Q4_0 GEMV with M <= 16 on the tcgen05 small-M kernel: the
+// activation image, then the GEMV over min(SMs, units) CTAs (units = 128-row
+// blocks x 32-column blocks, split flat) as its programmatic dependent.
+int launch_gemv_tcs(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M, int64_t N,
+                    int64_t K, cudaStream_t st) {
+    if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
+    const int KB = (int)(K / 32);
+    const int64_t T = (N + 31) / 32;
+    const int64_t RB = (T + 3) / 4;
+    const int64_t U = RB * KB;
+    if (U >= ((int64_t)1 << 31) - 1) return fail(h, Q4_EUNSUPPORTED, "small-M GEMV: too many units");
+    const int grid = (int)(U < h->sms ? U : h->sms);
+    const int V = q4::tcs_vecs(M);
+    // CTA partials: grid x 2 slots x 16 vectors x 128 rows (4 of the
+    // split-tile workspace's per-warp shares each).
+    int rc = ensure_ws(h, 4 * grid, st);
+    if (rc != Q4_OK) return rc;
+    rc = ensure_cnt(h, RB * q4::kTcsEp, st);
+    if (rc != Q4_OK) return rc;
+    rc = ensure_ximg(h, (size_t)KB * q4::tcs_img_blk(V), st);
+    if (rc != Q4_OK) return rc;
+    int64_t blocks = ((int64_t)KB * V + 255) / 256;
+    if (blocks > (int64_t)h->sms * 8) blocks = (int64_t)h->sms * 8;
+    q4::tcs_ximg_kernel<<<(unsigned)blocks, 256, 0, st>>>(x, h->ximg, M, (int)K, V, KB);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(h, e, "activation image launch");
+    q4::TcsArgs a;
+    a.W = static_cast<const uint8_t*>(W);
+    a.xi = h->ximg;
+    a.y = y;
+    a.ws = h->ws;
+    a.cnt = h->cnt;
+    a.err = h->err;
+    a.N = N;
+    a.KB = KB;
+    a.T = (int)T;
+    a.M = M;
+    a.sc = q4::make_split((int)U, grid);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(q4::kTcsThreads);
+    // One CTA per SM: two would fit beside each other and leave SMs idle.
+    size_t smem = (size_t)q4::tcs_smem_bytes(V);
+    if (smem < 116 * 1024) smem = 116 * 1024;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = V == 8 ? cudaLaunchKernelEx(&cfg, q4::gemv_tcs_kernel<8>, a)
+               : cudaLaunchKernelEx(&cfg, q4::gemv_tcs_kernel<16>, a);
+    if (e != cudaSuccess) return cuda_fail(h, e, "gemv (tcgen05 small-M) launch");
+    return Q4_OK;
+}
+
 // Launch the M = 17..256 product on the tcgen05 tensor cores: the activation
 // image, the GEMM over ceil(N/256) row tiles x P splits of the K steps (P as
 // large as keeps the grid within one wave of the SMs), and for P > 1 the
@@ -675,6 +740,8 @@ int q4gemv_create(q4gemv_t* out, int device) {
         }
         const char* mode = getenv("Q4GEMV_STACK_MODE");
         if (mode && !strcmp(mode, "kernels")) h->stack_mode = kStackKernels;
+        const char* sm = getenv("Q4GEMV_SMALL_M");
+        if (sm && !strcmp(sm, "tcs")) h->small_m = kSmallTcs;
     }
     if (rc == Q4_OK) {
         if (cudaMemset(h->cnt, 0, (size_t)kMaxTiles * sizeof(int)) != cudaSuccess ||
@@ -689,6 +756,7 @@ int q4gemv_create(q4gemv_t* out, int device) {
             set_smem_attr(Q4_STACK_KERNEL) || set_smem_attr(Q4_SWIGLU_KERNEL) ||
             set_smem_attr(q4::gemm_tc_kernel<false>) ||
             set_smem_attr(q4::gemm_tc_kernel<true>) ||
+            set_smem_attr(q4::gemv_tcs_kernel<8>) || set_smem_attr(q4::gemv_tcs_kernel<16>) ||
             0)
             rc = fail(h, Q4_ECUDA, "cudaFuncSetAttribute failed");
     }
@@ -776,6 +844,9 @@ int q4gemv_run(q4gemv_t h, const void* W, const void* x, void* y, int M, int64_t
     if (dp2a_fits(M, K))
         return launch_gemv(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K,
                            0, nullptr, st, true);
+    if (h->small_m == kSmallTcs)
+        return launch_gemv_tcs(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N,
+                               K, st);
     return launch_gemv_mma(h, W, static_cast<const __half*>(x), static_cast<__half*>(y), M, N, K,
                            st);
 }

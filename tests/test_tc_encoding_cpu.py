@@ -8,6 +8,17 @@ independently (cute/arch/mma_sm100_desc.hpp: UMMA::InstrDescriptor,
 UMMA::make_instr_desc, UMMA::SmemDescriptor).  A host program compiled with
 nvcc compares the two for every MMA width the kernel uses (N = 16..256) and
 for several start addresses.  Skipped when no CuTe header tree is installed.
+
+The tcgen05 small-M kernel's B descriptor (K-major, no swizzle, 32-byte rows
+in 8-row x 16-byte core matrices, the K-adjacent one 128 bytes on, the next
+8-row group 256 bytes on) is checked against CuTe's own reading of such a
+layout: UMMA::make_umma_desc<Major::K> (cute/atom/mma_traits_sm100.hpp)
+derives the leading and stride offsets from a CuTe layout written with
+exactly those strides, so a swap of the two offsets fails; its kind::i8
+instruction descriptor (signed 8-bit A and B, int32 accumulator) against
+UMMA::make_instr_desc<int8_t, int8_t, int32_t, ...>.  (On the host CuTe cannot read a shared-
+memory address -- it prints an error and uses 0 -- so the start address is
+compared at 0 there and field by field elsewhere.)
 """
 import importlib.util
 import os
@@ -23,9 +34,39 @@ PROGRAM = r"""
 #include <cstdio>
 #include <cute/arch/mma_sm100_desc.hpp>
 #include <cute/numeric/numeric_types.hpp>
+#include <cute/atom/mma_traits_sm100.hpp>
 #include "gemm_tc.cuh"
+#include "gemv_tcs.cuh"
 int main() {
+    using namespace cute;
     int bad = 0;
+    {
+        // The small-M kernel's B operand: rows of 32 signed bytes (K = 32);
+        // row-in-group stride 16 bytes, 8-row group stride 256; K: 16
+        // contiguous, the next chunk 128 bytes on.
+        auto mma_layout = make_layout(make_shape(make_shape(Int<8>{}, Int<4>{}), make_shape(Int<16>{}, Int<2>{})),
+                                      make_stride(make_stride(Int<16>{}, Int<256>{}), make_stride(Int<1>{}, Int<128>{})));
+        auto e = UMMA::make_umma_desc<UMMA::Major::K>(
+            make_tensor(make_smem_ptr(static_cast<int8_t*>(nullptr)), mma_layout));
+        if (e.desc_ != q4::tcs_sdesc(0u)) { printf("tcs sdesc layout\n"); ++bad; }
+        for (unsigned a : {0u, 128u, 1040u, 114688u, 229360u}) {
+            UMMA::SmemDescriptor s = e;
+            s.start_address_ = (uint16_t)(a >> 4);
+            if (s.desc_ != q4::tcs_sdesc(a)) { printf("tcs sdesc a=%u\n", a); ++bad; }
+        }
+        for (int r = 0; r < 32; ++r)
+            for (int k = 0; k < 2; ++k)
+                if ((int)q4::tcs_core_off(r, k) != (int)mma_layout(make_coord(make_coord(r % 8, r / 8), make_coord(0, k)))) {
+                    printf("tcs core offset r=%d k=%d\n", r, k);
+                    ++bad;
+                }
+        for (int n = 16; n <= 32; n += 16) {
+            auto d = cute::UMMA::make_instr_desc<int8_t, int8_t, int32_t, 128, 16,
+                                                 cute::UMMA::Major::K, cute::UMMA::Major::K>();
+            d.n_dim_ = n >> 3;
+            if (d.desc_ != q4::tcs_idesc_i8(n)) { printf("tcs idesc n=%d\n", n); ++bad; }
+        }
+    }
     for (int n = 16; n <= 256; n += 16) {
         auto d = cute::UMMA::make_instr_desc<cute::half_t, cute::half_t, float, 128, 0,
                                              cute::UMMA::Major::K, cute::UMMA::Major::K>();
