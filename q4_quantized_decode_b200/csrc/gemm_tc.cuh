@@ -73,10 +73,14 @@ __host__ __device__ constexpr uint32_t tc_load_stage_bytes(int Mp, bool q8 = fal
 // Dynamic shared memory of the kernel with L load stages: 1024 bytes of
 // alignment slack, the A buffers, the load stages, the barriers (2 per load
 // stage, 2 per A buffer, 1), the TMEM address word and the abort flag.
-__host__ __device__ constexpr uint32_t tc_smem_bytes(int Mp, int L, bool q8 = false) {
-    return 1024 + (uint32_t)(kTcABufs * kTcABytes) + (uint32_t)L * tc_load_stage_bytes(Mp, q8) +
+__host__ __device__ constexpr uint32_t tc_smem_bytes(int Mp, int L, bool q8 = false, bool at = false) {
+    return 1024 + (at ? 0u : (uint32_t)(kTcABufs * kTcABytes)) + (uint32_t)L * tc_load_stage_bytes(Mp, q8) +
            8u * (2 * L + 2 * kTcABufs + 1) + 16;
 }
+// With A in tensor memory (MMA width Mp <= 128): accumulators at columns
+// 128 acc, the two A buffers at 256 + 128 b (per accumulator 64 columns: the
+// main part's 64 K values, then the rest part's).
+constexpr int kTcAtMaxVec = 128;
 
 // Instruction descriptor of tcgen05.mma kind::f16: f16 A and B, both K-major,
 // fp32 accumulator, no negation or sparsity, shape m x n.
@@ -122,6 +126,28 @@ __device__ __forceinline__ void tc_mma_f16(uint32_t tmem_d, uint64_t adesc, uint
                  "setp.ne.b32 p, %4, 0;\n\t"
                  "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
                  :: "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc) : "memory");
+}
+// D (+)= A * B^T for one 16-column K slice with A in tensor memory (`tmem_a`:
+// lane = row, 8 columns = 16 f16 K values in order); `acc` = 0 overwrites D.
+__device__ __forceinline__ void tc_mma_f16_ta(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t acc) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+                 :: "r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(acc) : "memory");
+}
+// Eight registers into the tcgen05.st 16x256b fragment, two repetitions:
+// thread 4g + c writes TMEM lanes g (r0, r1, r4, r5) and g + 8 (r2, r3, r6,
+// r7) of the 16-lane group at `taddr`, 32-bit columns 2c, 2c + 1 (r0..r3)
+// and 8 + 2c, 9 + 2c (r4..r7).
+__device__ __forceinline__ void tc_st16x256b_x2(uint32_t taddr, uint2 a0, uint2 a1, uint2 b0, uint2 b1) {
+    asm volatile("tcgen05.st.sync.aligned.16x256b.x2.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 ::"r"(taddr), "r"(a0.x), "r"(a0.y), "r"(a1.x), "r"(a1.y), "r"(b0.x), "r"(b0.y),
+                   "r"(b1.x), "r"(b1.y)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 // Arrives once on `bar` when every MMA this thread issued so far has completed.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
@@ -208,15 +234,17 @@ __device__ __forceinline__ void tc_dequant_word_q8(uint32_t w, __half2 dd, uint2
     tc_split2(__hsub2(*reinterpret_cast<const __half2*>(&p23), k1152), dd, m.y, r.y);
 }
 
-template <bool Q8>
+// AT: the A tiles in tensor memory (Mp <= 128) instead of shared memory.
+template <bool Q8, bool AT = false>
 __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) {
     constexpr int SEG = tc_seg_bytes(Q8), SCL = Q8 ? 1024 : 512;
+    constexpr uint32_t kAccCols = AT ? (uint32_t)kTcAtMaxVec : (uint32_t)kTcAccCols;
     extern __shared__ uint8_t tc_smem_raw[];
     const int L = a.L;
     const uint32_t ld_bytes = tc_load_stage_bytes(a.Mp, Q8);
     const uint32_t raw0 = smem_addr(tc_smem_raw);
     const uint32_t base = (raw0 + 1023u) & ~1023u;               // swizzle needs 1024-byte tiles
-    const uint32_t ld0 = base + (uint32_t)(kTcABufs * kTcABytes);  // first load stage
+    const uint32_t ld0 = base + (AT ? 0u : (uint32_t)(kTcABufs * kTcABytes));  // first load stage
     uint8_t* gbar = tc_smem_raw + (ld0 - raw0) + (size_t)L * ld_bytes;
     uint64_t* full = reinterpret_cast<uint64_t*>(gbar);          // [L] copies landed
     uint64_t* lempty = full + L;                                 // [L] MMAs done with the stage
@@ -299,6 +327,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) 
                 tc_fence_after();
                 const uint32_t sA = base + (uint32_t)(b * kTcABytes);
                 const uint32_t sB = ld0 + (uint32_t)j * ld_bytes;
+                if constexpr (AT) {
+                    const uint32_t tA = tmem + 256u + (uint32_t)b * 128u;
+#pragma unroll
+                    for (int acc = 0; acc < kTcAcc; ++acc)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t bdesc = tc_sdesc_sw128(sB + (uint32_t)(32 * kk));
+                            const uint32_t ta = tA + (uint32_t)(acc * 64 + 8 * kk);
+                            tc_mma_f16_ta(tmem + (uint32_t)(acc * kAccCols), ta, bdesc, a.idesc,
+                                          (uint32_t)(i | kk));
+                            tc_mma_f16_ta(tmem + (uint32_t)(acc * kAccCols), ta + 32u, bdesc, a.idesc, 1u);
+                        }
+                } else
 #pragma unroll
                 for (int acc = 0; acc < kTcAcc; ++acc)
 #pragma unroll
@@ -323,6 +364,75 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) 
         // (g bits: lane bit 0, bit 3, bit 0 ^ bit 4; c: lane bits 1-2) makes
         // every quarter-warp's 16-byte loads and every half-warp's 8-byte
         // swizzled stores hit distinct banks ----
+        if constexpr (AT) {
+        // With A in tensor memory the thread is 4g + c (the tcgen05.st
+        // 16x256b fragment: TMEM lanes g and g + 8, columns 2c, 2c + 1 and
+        // 8 + 2c, 9 + 2c) and its 16 bytes are at 16 (4g + c): a warp's loads
+        // cover 512 contiguous bytes.  Columns 16h + 2c.. then hold K values
+        // 32h + 4c + e and columns 16h + 8 + 2c.. K values 32h + 16 + 4c + e:
+        // the natural K order, as in the activation image.
+        const int g = lane >> 2, c = lane & 3;
+        const int acc = warp >> 2;
+        const uint32_t trows = (uint32_t)(32 * (warp & 3)) << 16;
+        for (int i = 0; i < ns; ++i) {
+            const int j = i % L, b = i & 1;
+            const bool got = tc_wait(full + j, (uint32_t)((i / L) & 1), abort_flag) &&
+                             (i < kTcABufs ||
+                              tc_wait(aempty + b, (uint32_t)(((i >> 1) - 1) & 1), abort_flag));
+            if (!__all_sync(0xFFFFFFFFu, got)) {       // the warp leaves together
+                *abort_flag = 1;
+                set_device_error(a.err, kDevTimeout);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tA = tmem + trows + 256u + (uint32_t)b * 128u + (uint32_t)acc * 64u;
+            const uint32_t sraw = ld0 + (uint32_t)j * ld_bytes + bbytes + (uint32_t)(warp * 2 * SEG);
+            const int nb = min(2, a.KB - 2 * (k0 + i));
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t wv[Q8 ? 8 : 4];
+                uint2 sc = make_uint2(0, 0);
+                if (h < nb) {
+                    const uint32_t seg = sraw + (uint32_t)(h * SEG);
+                    if constexpr (Q8) {
+                        const uint4 u0 = lds128(seg + (uint32_t)(32 * lane));
+                        const uint4 u1 = lds128(seg + (uint32_t)(32 * lane + 16));
+                        wv[0] = u0.x; wv[1] = u0.y; wv[2] = u0.z; wv[3] = u0.w;
+                        wv[4] = u1.x; wv[5] = u1.y; wv[6] = u1.z; wv[7] = u1.w;
+                    } else {
+                        const uint4 u0 = lds128(seg + (uint32_t)(16 * lane));
+                        wv[0] = u0.x; wv[1] = u0.y; wv[2] = u0.z; wv[3] = u0.w;
+                    }
+                    sc = lds64(seg + (uint32_t)(SCL + 8 * g));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < (Q8 ? 8 : 4); ++e) wv[e] = 0;
+                }
+                const uint32_t sv[4] = {sc.x, sc.x >> 16, sc.y, sc.y >> 16};
+                uint2 lm[4], lr[4], hm[4], hr[4];            // rows g + 8ii
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii) {
+                    const __half2 dd = __half2half2(__ushort_as_half((unsigned short)(sv[ii] & 0xFFFFu)));
+                    if constexpr (Q8) {
+                        tc_dequant_word_q8(wv[2 * ii], dd, lm[ii], lr[ii]);
+                        tc_dequant_word_q8(wv[2 * ii + 1], dd, hm[ii], hr[ii]);
+                    } else {
+                        tc_dequant_word(wv[ii], dd, lm[ii], lr[ii], hm[ii], hr[ii]);
+                    }
+                    if (h >= nb) { lm[ii] = make_uint2(0, 0); lr[ii] = lm[ii]; hm[ii] = lm[ii]; hr[ii] = lm[ii]; }
+                }
+                const uint32_t col = tA + (uint32_t)(16 * h);
+                tc_st16x256b_x2(col, lm[0], lm[1], hm[0], hm[1]);                       // main, rows g, g + 8
+                tc_st16x256b_x2(col + 32u, lr[0], lr[1], hr[0], hr[1]);                 // rest
+                tc_st16x256b_x2(col + (16u << 16), lm[2], lm[3], hm[2], hm[3]);         // rows g + 16, g + 24
+                tc_st16x256b_x2(col + (16u << 16) + 32u, lr[2], lr[3], hr[2], hr[3]);
+            }
+            tc_wait_st();
+            tc_fence_before();            // tensor-memory writes -> the MMAs
+            __syncwarp();
+            if (lane == 0) mbar_arrive(aready + b);
+        }
+        } else {
         const int g = (lane & 1) | ((lane >> 2) & 2) | (((lane ^ (lane >> 4)) & 1) << 2);
         const int c = (lane >> 1) & 3;
         const int acc = warp >> 2;
@@ -393,13 +503,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) 
             if (lane == 0) mbar_arrive(aready + b);
         }
 
+        }
+
         // ---- epilogue: accumulator rows -> y (or the split's fp32 sums) ----
         // tcgen05.ld is warp-collective: the decision to read is made per warp.
+        const int acc = warp >> 2;
         const bool ok = __all_sync(0xFFFFFFFFu, tc_wait(accbar, 0u, abort_flag) && !*abort_flag);
         tc_fence_after();
         if (ok) {
             const int64_t n = (int64_t)blockIdx.x * kTcRows + acc * 128 + (warp & 3) * 32 + lane;
-            const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(acc * kTcAccCols);
+            const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(acc * kAccCols);
             for (int c0 = 0; c0 < a.Mp; c0 += 16) {
                 uint32_t v[16];
                 tc_ld16(taddr + (uint32_t)c0, v);

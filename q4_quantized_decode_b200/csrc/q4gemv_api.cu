@@ -495,14 +495,17 @@ int launch_gemm_tc(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int
     if (P > nk) P = nk;
     const int nkp = (int)((nk + P - 1) / P);
     P = (nk + nkp - 1) / nkp;                        // every split has steps
-    // Load stages: as many as fit beside the two A buffers (2..8; Q8_0 with
-    // more than 240 vectors fits one, which serialises copies and MMAs).
-    const size_t fixed = q4::tc_smem_bytes(Mp, 0, q8);
+    // Up to 128 vectors the A tiles live in tensor memory beside the
+    // accumulators (no shared-memory round trip); beyond, in shared memory.
+    const bool at = Mp <= q4::kTcAtMaxVec;
+    // Load stages: as many as fit beside the A buffers, if any (2..8; Q8_0
+    // with more than 240 vectors fits one, which serialises copies and MMAs).
+    const size_t fixed = q4::tc_smem_bytes(Mp, 0, q8, at);
     const size_t lsb = q4::tc_load_stage_bytes(Mp, q8) + 16;
     int L = (int)((kMaxDynSmem - fixed) / lsb);
     if (L > 8) L = 8;
     if (L < 1) L = 1;
-    size_t smem = q4::tc_smem_bytes(Mp, L, q8);
+    size_t smem = q4::tc_smem_bytes(Mp, L, q8, at);
     // One CTA per SM: each holds all 512 TMEM columns.
     if (smem < 116 * 1024) smem = 116 * 1024;
     int rc = ensure_ximg(h, (size_t)nk * Mp * 128, st);
@@ -543,8 +546,12 @@ int launch_gemm_tc(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int
     gattr[0].val.programmaticStreamSerializationAllowed = 1;
     gcfg.attrs = gattr;
     gcfg.numAttrs = 1;
-    e = q8 ? cudaLaunchKernelEx(&gcfg, q4::gemm_tc_kernel<true>, a)
-           : cudaLaunchKernelEx(&gcfg, q4::gemm_tc_kernel<false>, a);
+    if (at)
+        e = q8 ? cudaLaunchKernelEx(&gcfg, q4::gemm_tc_kernel<true, true>, a)
+               : cudaLaunchKernelEx(&gcfg, q4::gemm_tc_kernel<false, true>, a);
+    else
+        e = q8 ? cudaLaunchKernelEx(&gcfg, q4::gemm_tc_kernel<true>, a)
+               : cudaLaunchKernelEx(&gcfg, q4::gemm_tc_kernel<false>, a);
     if (e != cudaSuccess) return cuda_fail(h, e, "gemm (tcgen05) launch");
     if (P > 1) {
         const int64_t MN = (int64_t)M * N;
@@ -756,6 +763,8 @@ int q4gemv_create(q4gemv_t* out, int device) {
             set_smem_attr(Q4_STACK_KERNEL) || set_smem_attr(Q4_SWIGLU_KERNEL) ||
             set_smem_attr(q4::gemm_tc_kernel<false>) ||
             set_smem_attr(q4::gemm_tc_kernel<true>) ||
+            set_smem_attr(q4::gemm_tc_kernel<false, true>) ||
+            set_smem_attr(q4::gemm_tc_kernel<true, true>) ||
             set_smem_attr(q4::gemv_tcs_kernel<8>) || set_smem_attr(q4::gemv_tcs_kernel<16>) ||
             0)
             rc = fail(h, Q4_ECUDA, "cudaFuncSetAttribute failed");
