@@ -371,7 +371,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) 
         // cover 512 contiguous bytes.  Columns 16h + 2c.. then hold K values
         // 32h + 4c + e and columns 16h + 8 + 2c.. K values 32h + 16 + 4c + e:
         // the natural K order, as in the activation image.
-        const int g = lane >> 2, c = lane & 3;
+        const int g = lane >> 2;
         const int acc = warp >> 2;
         const uint32_t trows = (uint32_t)(32 * (warp & 3)) << 16;
         for (int i = 0; i < ns; ++i) {
