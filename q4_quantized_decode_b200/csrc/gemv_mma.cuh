@@ -373,10 +373,14 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_mma_kernel(const MmaArgs a
                           0.f, 0.f);
                 mma_16816(e0, e1, e2, e3, u0.r, u1.r, u0.s, u1.s, xv[nt].z, xv[nt].w, e0, e1, e2,
                           e3);
-                acc[tt][nt][0] = fmaf(e0, dA[tt], acc[tt][nt][0]);
-                acc[tt][nt][1] = fmaf(e1, dA[tt], acc[tt][nt][1]);
-                acc[tt][nt][2] = fmaf(e2, dB[tt], acc[tt][nt][2]);
-                acc[tt][nt][3] = fmaf(e3, dB[tt], acc[tt][nt][3]);
+                const float2 r01 = ffma2(make_float2(e0, e1), make_float2(dA[tt], dA[tt]),
+                                         make_float2(acc[tt][nt][0], acc[tt][nt][1]));
+                const float2 r23 = ffma2(make_float2(e2, e3), make_float2(dB[tt], dB[tt]),
+                                         make_float2(acc[tt][nt][2], acc[tt][nt][3]));
+                acc[tt][nt][0] = r01.x;
+                acc[tt][nt][1] = r01.y;
+                acc[tt][nt][2] = r23.x;
+                acc[tt][nt][3] = r23.y;
             }
         }
     };
