@@ -50,7 +50,8 @@ constexpr int kTcAcc = 2;                       // 128-row accumulators per CTA
 constexpr int kTcRows = 128 * kTcAcc;           // output rows per CTA
 constexpr int kTcTiles = kTcRows / 32;          // packed 32-row tiles per CTA
 constexpr int kTcDqWarps = 4 * kTcAcc;          // dequantise / epilogue warps
-constexpr int kTcThreads = 32 * (kTcDqWarps + 2);
+constexpr int kTcIssuers = 2;                   // MMA-issuing warps (alternate K steps)
+constexpr int kTcThreads = 32 * (kTcDqWarps + 1 + kTcIssuers);
 constexpr int kTcMaxVec = 256;                  // MMA N limit (vectors)
 constexpr int kTcAccCols = 256;                 // TMEM columns per accumulator
 constexpr int kTcTmemCols = kTcAcc * kTcAccCols;
@@ -166,6 +167,15 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
                  : "r"(taddr) : "memory");
 }
 
+__device__ __forceinline__ int ld_acquire_cta_shared(const int* p) {
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_cta_shared(int* p, int v) {
+    asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(p)), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_addr(bar)) : "memory");
 }
@@ -253,6 +263,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) 
     uint64_t* accbar = aempty + kTcABufs;
     uint32_t* tslot = reinterpret_cast<uint32_t*>(accbar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+    __shared__ int mma_turn_word;                                // next K step whose MMAs may be issued
+    int* mma_turn = &mma_turn_word;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = blockIdx.x * kTcTiles;                       // first packed tile
@@ -270,8 +282,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) 
             mbar_init(aready + b, kTcDqWarps);
             mbar_init(aempty + b, 1);
         }
-        mbar_init(accbar, 1);
+        mbar_init(accbar, kTcIssuers);
         *abort_flag = 0;
+        *mma_turn = 0;
         fence_barrier_init();
     }
     if (warp == 0) tc_alloc(tslot, kTcTmemCols);
@@ -313,13 +326,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) 
                 mbar_wait_bounded(full + j, (uint32_t)((last / L) & 1), 1u << 22);
             }
         }
-    } else if (warp == kTcDqWarps + 1) {
-        // ---- MMA issuer ----
+    } else if (warp > kTcDqWarps) {
+        // ---- MMA issuers: issuer q takes the K steps i with i % 2 == q.  It
+        // waits for its step's operands while the other issues, then for its
+        // turn (the MMAs enter the tensor pipe in step order, so the
+        // accumulation order is the step order and step 0's MMAs overwrite
+        // first); a tcgen05 fence before handing the turn on and after taking
+        // it orders the two threads' MMAs. ----
+        const int q = warp - (kTcDqWarps + 1);
         if (lane == 0) {
-            for (int i = 0; i < ns; ++i) {
+            for (int i = q; i < ns; i += kTcIssuers) {
                 const int j = i % L, b = i & 1;
-                if (!tc_wait(aready + b, (uint32_t)((i >> 1) & 1), abort_flag) ||
-                    !tc_wait(full + j, (uint32_t)((i / L) & 1), abort_flag)) {
+                bool got = tc_wait(aready + b, (uint32_t)((i >> 1) & 1), abort_flag) &&
+                           tc_wait(full + j, (uint32_t)((i / L) & 1), abort_flag);
+                for (uint32_t it = 0; got; ++it) {
+                    if (ld_acquire_cta_shared(mma_turn) == i) break;
+                    if (it >= (1u << 24) || ((it & 63) == 63 && *abort_flag)) got = false;
+                }
+                if (!got) {
                     *abort_flag = 1;
                     set_device_error(a.err, kDevTimeout);
                     break;
@@ -354,8 +378,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(const TcArgs a) 
                     }
                 tc_commit(lempty + j);
                 tc_commit(aempty + b);
+                tc_fence_before();
+                st_release_cta_shared(mma_turn, i + 1);
             }
-            tc_commit(accbar);        // also after an abort: tracks every MMA issued
+            tc_commit(accbar);        // also after an abort: tracks every MMA this thread issued
         }
     } else {
         // ---- dequantise: the thread with pair (g, c) takes the 16 bytes at
