@@ -18,9 +18,12 @@ its own activation stream); there is no data-path collective, only a barrier
 and a max-reduction of the timings.  Rank 0 prints one JSON line.
 
 --shard runs the row-sharded step instead (q4gemv_run_stack_sharded): each
-rank holds 1/N of every matrix's rows and the outputs are all-gathered over
-NCCL after every GEMV, so N GPUs share ONE decode step (strong scaling; the
-reported bytes are the model's once per step).
+rank holds 1/N of every matrix's rows and every GEMV's output reaches every
+rank before the next GEMV, so N GPUs share ONE decode step (strong scaling;
+the reported bytes are the model's once per step).  --exchange peer (the
+default) has each GEMV kernel store its rows into every rank's buffer over
+CUDA IPC peer memory and stamp them; --exchange nccl all-gathers them with
+NCCL after every GEMV instead.
 """
 from __future__ import annotations
 
@@ -63,7 +66,8 @@ WORKLOAD = ("27B-shaped decode step, M=1: 64 layers x (QKV 5120->7168, O 5120->5
 WORKLOAD_SHARD = ("27B-shaped decode step, M=1: 64 layers x (QKV 5120->7168, O 5120->5120, "
                   "gate+up 5120->34816, down 17408->5120) Q4_0 GEMVs with unit-RMS renorm between "
                   "matrices, every matrix row-sharded over the GPUs: per GEMV one kernel on each "
-                  "GPU's rows and an NCCL all-gather, replayed as one CUDA graph")
+                  "GPU's rows, every GPU getting all rows before the next GEMV, replayed as one CUDA "
+                  "graph")
 
 
 KERNEL_SOURCES = ["stack.cuh", "gemv_dp2a.cuh", "partition.cuh", "device_common.cuh"]
@@ -470,13 +474,24 @@ def run_ours(args, rank: int, world: int, dist):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     eng = q4.Q4Gemv(local)
-    if args.shard:
+    if args.shard and args.exchange == "nccl":
         # One communicator for the row-sharded step: rank 0's NCCL id, sent
         # to the others over the process group.
         uid = [q4.q4gemv_comm_unique_id()[1] if rank == 0 else None]
         if dist is not None and world > 1:
             dist.broadcast_object_list(uid, src=0)
         eng.init_comm(world, rank, uid[0])
+    elif args.shard:
+        # The peer exchange: every rank's buffer blob, gathered over the
+        # process group, then every peer's buffer mapped.
+        blob = eng.peer_export(world, rank, HIDDEN, QKV_N, FFN)
+        blobs = [None] * world
+        if dist is not None and world > 1:
+            dist.all_gather_object(blobs, blob)
+        else:
+            blobs = [blob]
+        eng.peer_open(blobs)
+    if args.shard:
         layers, t_repack = build_weights_sharded(eng, torch, q4, rank, world)
     else:
         layers, t_repack = build_weights(eng, torch, rank)
@@ -605,7 +620,10 @@ def run_ours(args, rank: int, world: int, dist):
         "config": {"workload": WORKLOAD_SHARD if args.shard else WORKLOAD, "bytes_per_step": STEP_GEMV_BYTES,
                    "weight_bytes_per_step": STEP_WEIGHT_BYTES,
                    "l2": "inputs larger than L2 (11.9 GB of weights per step)",
-                   "parallelism": (f"row-sharded x{world} (NCCL all-gather after every GEMV)"
+                   "parallelism": ((f"row-sharded x{world} (NCCL all-gather after every GEMV)"
+                                    if args.exchange == "nccl" else
+                                    f"row-sharded x{world} (GEMV kernels store their rows into every "
+                                    "rank's buffer over peer memory)")
                                    if args.shard else f"replicas x{world}"), "seed": STEP_SEED},
         "decode_steps_per_s": steps_per_s,
         "pct_of_8TBps_nominal": 100.0 * per_rank_gbs / NOMINAL_HBM_GBS,
@@ -614,9 +632,11 @@ def run_ours(args, rank: int, world: int, dist):
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": 2 * HIDDEN,
                 "d2h_bytes_per_step": 2 * HIDDEN,
                 "steps_per_s": e2e_steps_per_s},
-        # one stack_kernel per step (and one 16-byte memset); sharded: per GEMV one
-        # kernel and one all-gather, and the final renorm
-        "gpu_launches": args.steps * ((8 * L + 1) if args.shard else 1),
+        # one stack_kernel per step (and one 16-byte memset); sharded over NCCL: per
+        # GEMV one kernel and one all-gather, and the final renorm; over peer memory:
+        # per GEMV one kernel, the step-count update and the final unpack + renorm
+        "gpu_launches": args.steps * (((8 * L + 1) if args.exchange == "nccl" else (4 * L + 2))
+                                      if args.shard else 1),
         "clocks": clocks,
         "repack_s_per_step_weights": t_repack,
         "per_shape_m1": per_shape,
@@ -723,6 +743,8 @@ def main():
     ap.add_argument("--layers", type=int, default=64, help="layers of the step (profiling only)")
     ap.add_argument("--shard", action="store_true",
                     help="row-shard every matrix over the ranks (one step shared by all GPUs)")
+    ap.add_argument("--exchange", choices=["peer", "nccl"], default="peer",
+                    help="--shard: how each GEMV's rows reach every rank")
     args = ap.parse_args()
     if args.layers != 64:
         set_layers(args.layers)

@@ -308,19 +308,76 @@ Q4GEMV_API int q4gemv_comm_unique_id(void* id);
  * handle. */
 Q4GEMV_API int q4gemv_comm_init(q4gemv_t h, int world, int rank, const void* id);
 
+/* Peer-memory exchange for the row-sharded step: instead of an NCCL
+ * all-gather after every GEMV, each GEMV kernel stores its output rows
+ * directly into every rank's gather buffer (CUDA IPC mappings over NVLink /
+ * NVSwitch; plain stores, no multicast) and the next GEMV reads them there.
+ * Every entry of a gather buffer is one 32-bit word, the binary16 value in
+ * bits 0-15 and in bits 16-31 a stamp of the GEMV that wrote it: (steps run
+ * x GEMVs per step + the GEMV's index in the step) mod 2^16.  A reader polls
+ * (bounded) each word it needs until it carries the stamp it expects, so no
+ * fence, flag or collective separates the GEMVs, and a GEMV starts (its
+ * weights streaming) while the previous one ends.  The exchange buffer of a
+ * rank (zeroed once) holds, for the four matrix types of the step (QKV, O,
+ * gate+up, down), a gather buffer of world * chunk words (chunk from
+ * q4gemv_shard_rows, rank r's rows at r * chunk), then the rank's step
+ * count; offsets from q4gemv_peer_layout.
+ *
+ * Blob (Q4GEMV_PEER_BLOB_BYTES, little-endian): uint32 magic 0x51345045
+ * ("EP4Q"), uint32 version 1, int32 world, int32 rank, int64 hidden, qkv_n,
+ * ffn, uint64 buffer bytes, then the 64-byte cudaIpcMemHandle_t of the
+ * buffer, zero padding to the end. */
+#define Q4GEMV_PEER_BLOB_BYTES 128
+#define Q4GEMV_PEER_MAX_WORLD 8
+
+/* Byte offsets of the exchange buffer for these shapes: off[0..3] the gather
+ * buffers of QKV, O, gate+up and down outputs, off[4] the step count, off[5]
+ * the total size (six entries).  Host-only.  Q4_EINVAL for world outside
+ * [1, Q4GEMV_PEER_MAX_WORLD] or non-positive shapes. */
+Q4GEMV_API int q4gemv_peer_layout(int world, int64_t hidden, int64_t qkv_n, int64_t ffn,
+                                  int64_t* off);
+
+/* Checks `world` blobs (world * Q4GEMV_PEER_BLOB_BYTES bytes, rank order) for
+ * one exchange: magic and version, the same world, shapes and buffer size in
+ * all of them, blob r from rank r.  Host-only.  Q4_OK or Q4_EINVAL. */
+Q4GEMV_API int q4gemv_peer_check(const void* blobs, int world);
+
+/* Allocates (zeroed) this rank's exchange buffer for the step's shapes and
+ * writes its blob.  Every rank calls it, sends its blob to all ranks (any
+ * host channel) and then calls q4gemv_peer_open with all of them.  Replaces
+ * an earlier exchange of the handle (synchronises the device). */
+Q4GEMV_API int q4gemv_peer_export(q4gemv_t h, int world, int rank, int64_t hidden, int64_t qkv_n,
+                                  int64_t ffn, void* blob);
+
+/* Maps the other ranks' exchange buffers (cudaIpcOpenMemHandle) from the
+ * `world` blobs of q4gemv_peer_export, in rank order, after q4gemv_peer_check
+ * and a comparison with this handle's export.  From then on
+ * q4gemv_run_stack_sharded with the exported shapes uses the peer-memory
+ * exchange.  With world = 1 nothing is mapped (the rank's own buffer). */
+Q4GEMV_API int q4gemv_peer_open(q4gemv_t h, const void* blobs);
+
+/* Unmaps the peers' buffers and frees this rank's; every rank must stop
+ * using the exchange first (no step of any rank in flight). */
+Q4GEMV_API int q4gemv_peer_close(q4gemv_t h);
+
 /* The decode step of q4gemv_run_stack, row-sharded: `layers` holds THIS
  * rank's row slices (q4gemv_shard_rows of each matrix, packed as q4gemv_run
  * matrices of `rows` rows; a slice of 0 rows may be NULL).  Per GEMV the rank
  * computes its rows f16(s(v) * W_slice v) from the full previous output v
- * (the M = 1 kernel; the scale as in q4gemv_run_stack), then an NCCL
- * all-gather gives every rank the whole output; x_out = f16(s(x') x') on
- * every rank.  x_in, x_out: device memory (hidden binary16), the same x_in on
- * every rank.  Every rank must make the same calls in the same order.  The
- * step is captured as one CUDA graph on the first call with these arguments
- * (not inside the caller's capture) and replayed.  Results agree with
- * q4gemv_run_stack within the GEMV tolerance (the row split changes the
- * order of the partial sums, not the arithmetic).  Errors as
- * q4gemv_run_stack; Q4_EINVAL without a communicator. */
+ * (the M = 1 kernel; the scale as in q4gemv_run_stack), and every rank gets
+ * the whole output: through the peer-memory exchange when it is open for
+ * these shapes (stores by the GEMV kernel itself, above), else an NCCL
+ * all-gather; x_out = f16(s(x') x') on every rank.  x_in, x_out: device
+ * memory (hidden binary16), the same x_in on every rank.  Every rank must
+ * make the same calls in the same order.  The step is captured as one CUDA
+ * graph on the first call with these arguments (not inside the caller's
+ * capture) and replayed.  Results agree with q4gemv_run_stack within the
+ * GEMV tolerance (the row split changes the order of the partial sums, not
+ * the arithmetic) and are the same bits on both exchanges.  Errors as
+ * q4gemv_run_stack; Q4_EINVAL with neither a communicator nor an open
+ * exchange for these shapes; a peer whose rows never come makes the waiting
+ * GEMV report Q4_ETIMEOUT through q4gemv_sync_status (one time-out per step:
+ * later waits of the step give up at once). */
 Q4GEMV_API int q4gemv_run_stack_sharded(q4gemv_t h, const q4gemv_layer* layers_local,
                              int n_layers, int64_t hidden, int64_t qkv_n, int64_t ffn,
                              const void* x_in, void* x_out, q4gemv_stream_t stream);

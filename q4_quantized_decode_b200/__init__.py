@@ -63,6 +63,11 @@ def _load_library():
         "q4gemv_comm_init": ([vp, ci, ci, ctypes.c_char_p], ci),
         "q4gemv_run_stack_sharded": ([vp, ctypes.POINTER(q4gemv_layer), ci, i64, i64, i64, vp, vp,
                                       vp], ci),
+        "q4gemv_peer_layout": ([ci, i64, i64, i64, ctypes.POINTER(i64)], ci),
+        "q4gemv_peer_check": ([ctypes.c_char_p, ci], ci),
+        "q4gemv_peer_export": ([vp, ci, ci, i64, i64, i64, ctypes.c_char_p], ci),
+        "q4gemv_peer_open": ([vp, ctypes.c_char_p], ci),
+        "q4gemv_peer_close": ([vp], ci),
         "q4gemv_run_stack": ([vp, ctypes.POINTER(q4gemv_layer), ci, i64, i64, i64,
                               vp, vp, vp, vp, vp], ci),
         "q4gemv_sync_status": ([vp, vp], ci),
@@ -163,6 +168,36 @@ def q4gemv_comm_unique_id():
 
 def q4gemv_comm_init(h, world: int, rank: int, uid: bytes) -> int:
     return _lib.q4gemv_comm_init(h, world, rank, ctypes.create_string_buffer(uid, 128))
+
+
+PEER_BLOB_BYTES = 128
+PEER_MAX_WORLD = 8
+
+
+def q4gemv_peer_layout(world: int, hidden: int, qkv_n: int, ffn: int):
+    """(status, [6 byte offsets]) of the peer exchange buffer (see the header)."""
+    off = (ctypes.c_int64 * 6)()
+    st = _lib.q4gemv_peer_layout(world, hidden, qkv_n, ffn, off)
+    return st, list(off)
+
+
+def q4gemv_peer_check(blobs: bytes, world: int) -> int:
+    return _lib.q4gemv_peer_check(ctypes.create_string_buffer(blobs, len(blobs)), world)
+
+
+def q4gemv_peer_export(h, world: int, rank: int, hidden: int, qkv_n: int, ffn: int):
+    """(status, this rank's 128-byte exchange blob)."""
+    buf = ctypes.create_string_buffer(PEER_BLOB_BYTES)
+    st = _lib.q4gemv_peer_export(h, world, rank, hidden, qkv_n, ffn, buf)
+    return st, buf.raw
+
+
+def q4gemv_peer_open(h, blobs: bytes) -> int:
+    return _lib.q4gemv_peer_open(h, ctypes.create_string_buffer(blobs, len(blobs)))
+
+
+def q4gemv_peer_close(h) -> int:
+    return _lib.q4gemv_peer_close(h)
 
 
 def q4gemv_run_stack_sharded(h, layers, n_layers, hidden, qkv_n, ffn, x_in, x_out, stream) -> int:
@@ -298,6 +333,21 @@ class Q4Gemv:
     def init_comm(self, world: int, rank: int, uid: bytes):
         """Joins the `world`-GPU communicator of the row-sharded step as `rank`."""
         self._check(q4gemv_comm_init(self.h, world, rank, uid))
+
+    def peer_export(self, world: int, rank: int, hidden: int, qkv_n: int, ffn: int) -> bytes:
+        """Allocates this rank's exchange buffer for the peer-memory sharded step
+        and returns the blob every rank must receive (e.g. all_gather_object)."""
+        st, blob = q4gemv_peer_export(self.h, world, rank, hidden, qkv_n, ffn)
+        self._check(st)
+        return blob
+
+    def peer_open(self, blobs):
+        """Maps every rank's exchange buffer; `blobs`: the world's blobs in rank order.
+        run_stack_sharded then gathers over peer memory for these shapes."""
+        self._check(q4gemv_peer_open(self.h, b"".join(blobs)))
+
+    def peer_close(self):
+        self._check(q4gemv_peer_close(self.h))
 
     def run_stack_sharded(self, layers_local, x_in, hidden: int, qkv_n: int, ffn: int, x_out=None,
                           stream=None):

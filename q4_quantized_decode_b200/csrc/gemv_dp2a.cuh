@@ -47,6 +47,73 @@ struct SegFmt {
 };
 constexpr int kXChunksPerThread = 9; // activation staging: M*K <= 9 * 8 * threads
 
+// Row-sharded decode step over peer memory (M = 1).  Every entry of a
+// gathered vector is one 32-bit word: the binary16 value in the low half and
+// the stamp of the GEMV that wrote it in the high half.  A GEMV stores its
+// rows as such words straight into every rank's gather buffer; the next GEMV
+// polls the words it stages until each carries the stamp it expects.  A word
+// is written and read whole (single-copy atomic), so no fence, flag or
+// arrival count orders the exchange.  Stamps are (steps run x GEMVs per step
+// + GEMV index) mod 2^16: the word a reader finds is the one it expects or
+// the one written four GEMVs earlier into the same buffer, never equal.
+struct PeerArgs {
+    uint32_t* const* y;           // [n]: this rank's slice in rank p's gather buffer (rank p's memory)
+    const uint32_t* xw;           // wait: the gathered input words (this rank's memory)
+    const unsigned* seq;          // [0]: steps run including this one, [1]: the arrival-count epoch
+    int n;                        // ranks; 0: a plain GEMV
+    int g;                        // this GEMV's index in the step
+    int per_step;                 // GEMVs per step
+    int wait;                     // 1: the input is xw, stamped by GEMV g - 1
+    unsigned poll_limit;          // polls of one chunk before giving up
+    unsigned unreachable;         // test knob: 1 waits for a stamp no GEMV writes yet
+};
+
+__device__ __forceinline__ uint32_t peer_stamp(const unsigned* seq, int per_step, int g) {
+    return (seq[0] * (unsigned)per_step + (unsigned)g) & 0xFFFFu;
+}
+
+__device__ __forceinline__ void st_relaxed_sys_u32(uint32_t* p, uint32_t v) {
+    asm volatile("st.relaxed.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint4 ld_relaxed_sys_v4(const uint32_t* p) {
+    uint4 v;
+    asm volatile("ld.relaxed.sys.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+
+// The eight binary16 entries of two loaded word quads, and whether all
+// eight words carry `stamp`.
+__device__ __forceinline__ bool peer_words_ok(uint4 lo, uint4 hi, uint32_t stamp) {
+    const uint32_t s = stamp << 16;
+    return (((lo.x ^ s) | (lo.y ^ s) | (lo.z ^ s) | (lo.w ^ s) | (hi.x ^ s) | (hi.y ^ s) | (hi.z ^ s) |
+             (hi.w ^ s)) >> 16) == 0u;
+}
+__device__ __forceinline__ uint4 peer_words_f16(uint4 lo, uint4 hi) {
+    return make_uint4(__byte_perm(lo.x, lo.y, 0x5410), __byte_perm(lo.z, lo.w, 0x5410),
+                      __byte_perm(hi.x, hi.y, 0x5410), __byte_perm(hi.z, hi.w, 0x5410));
+}
+
+// Polls the chunk of eight words at w (first read: lo, hi) until all carry
+// `stamp`; bounded by poll_limit, and given up at once when an earlier wait
+// has already run out (the error word is set), so a lost peer costs one
+// time-out per step.  Returns the chunk's eight values.
+static __device__ __noinline__ uint4 peer_poll_chunk(const uint32_t* w, uint4 lo, uint4 hi, uint32_t stamp,
+                                              unsigned poll_limit, int* err) {
+    uint32_t it = 0;
+    while (!peer_words_ok(lo, hi, stamp)) {
+        if (++it > poll_limit || (!(it & 1023u) && *reinterpret_cast<volatile int*>(err) != 0)) {
+            set_device_error(err, kDevTimeout);
+            break;
+        }
+        lo = ld_relaxed_sys_v4(w);
+        hi = ld_relaxed_sys_v4(w + 4);
+    }
+    return peer_words_f16(lo, hi);
+}
+
 struct GemvArgs {
     const uint8_t* W;       // packed matrix (segments of 576 bytes)
     const __half* x;        // [M][K] activations (renorm: the previous f16 output, unscaled)
@@ -62,7 +129,27 @@ struct GemvArgs {
     int renorm;             // 1 (M == 1): the input is s * x[0:K], s its unit-RMS scale, applied
                             // to the outputs; 0: the input is x
     SplitConsts sc;         // make_split(S, G)
+    PeerArgs peer = {};     // n > 0: outputs stored into every rank's gather buffer (M = 1)
 };
+
+// One finished output: y, or with peers this rank's slice in every rank's
+// gather buffer as a stamped word (NVLink stores to the other GPUs).
+__device__ __forceinline__ void store_out(const GemvArgs& a, int m, int64_t row, __half v) {
+    if (a.peer.n > 0) {
+        const uint32_t w = (peer_stamp(a.peer.seq, a.peer.per_step, a.peer.g) << 16) |
+                           (uint32_t)__half_as_ushort(v);
+        for (int p = 0; p < a.peer.n; ++p) st_relaxed_sys_u32(a.peer.y[p] + row, w);
+    } else {
+        a.y[(size_t)m * a.N + row] = v;
+    }
+}
+
+// Step bookkeeping of the peer exchange (one thread): a new step -- the
+// stamps' step count and the arrival counts' epoch advance.
+static __global__ void peer_step_kernel(unsigned* seq) {
+    seq[0] = seq[0] + 1u;
+    seq[1] = seq[1] + 1u;
+}
 
 // Per-warp ring of R stages of C segments.
 __host__ __device__ constexpr size_t ring_bytes(int warps, int R, int C, int seg = kSegBytes) {
@@ -287,10 +374,36 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs
     const int tid = threadIdx.x;
     const int nq = M * a.K / 8;
     uint4 xr[QN];
+    if (M == 1 && a.peer.n > 0 && a.peer.wait) {
+        // stamped words of the previous GEMV, every rank's rows: all loads
+        // issued, then each chunk polled until it carries the stamp
+        const uint32_t stamp = (peer_stamp(a.peer.seq, a.peer.per_step, a.peer.g - 1) + a.peer.unreachable) & 0xFFFFu;
+        uint4 lo[QN], hi[QN];
 #pragma unroll
-    for (int i = 0; i < QN; ++i) {
-        const int q = tid + NT * i;
-        xr[i] = q < nq ? *reinterpret_cast<const uint4*>(a.x + (size_t)q * 8) : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < QN; ++i) {
+            const int q = tid + NT * i;
+            if (q < nq) {
+                lo[i] = ld_relaxed_sys_v4(a.peer.xw + (size_t)q * 8);
+                hi[i] = ld_relaxed_sys_v4(a.peer.xw + (size_t)q * 8 + 4);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < QN; ++i) {
+            const int q = tid + NT * i;
+            if (q >= nq) {
+                xr[i] = make_uint4(0, 0, 0, 0);
+            } else if (peer_words_ok(lo[i], hi[i], stamp)) {
+                xr[i] = peer_words_f16(lo[i], hi[i]);
+            } else {
+                xr[i] = peer_poll_chunk(a.peer.xw + (size_t)q * 8, lo[i], hi[i], stamp, a.peer.poll_limit, a.err);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < QN; ++i) {
+            const int q = tid + NT * i;
+            xr[i] = q < nq ? *reinterpret_cast<const uint4*>(a.x + (size_t)q * 8) : make_uint4(0, 0, 0, 0);
+        }
     }
 #pragma unroll
     for (int i = 0; i < QN; ++i) {
@@ -386,7 +499,7 @@ struct Dp2aConsumer {
             const float val = (c == 0) ? acc[m][0] : (c == 1) ? acc[m][1] : (c == 2) ? acc[m][2] : acc[m][3];
             if (whole) {
                 const __half yh = __float2half_rn(__fmul_rn(oscale, val));
-                if (row < a.N) a.y[(size_t)m * a.N + row] = yh;
+                if (row < a.N) store_out(a, m, row, yh);
                 if (M == 1 && t < qo.nb) quant_lane_store(__half2float(yh), t, qo.x, qo.rec, qo.sq);
             } else {
                 park[(sp.slot(t) * M + m) * 32 + r] = val;
@@ -544,7 +657,7 @@ struct Dp2aConsumer {
 #pragma unroll
                 for (int m = 0; m < M; ++m) {
                     const __half yh = __float2half_rn(__fmul_rn(oscale, sum[m]));
-                    if (row < a.N) a.y[(size_t)m * a.N + row] = yh;
+                    if (row < a.N) store_out(a, m, row, yh);
                     if (M == 1 && t < qo.nb) quant_lane_store(__half2float(yh), t, qo.x, qo.rec, qo.sq);
                 }
             } else {
@@ -573,6 +686,10 @@ __device__ __forceinline__ void combine_ctas_arrive(const GemvArgs& a, int t, in
     old = __shfl_sync(0xffffffffu, old, 0);
     __syncwarp();                       // order the lanes' reads after lane 0's acquire
     const int need = cl - cf + 1;
+    // With peers the counts run on across steps (a GEMV's slots are its
+    // own; nothing resets them): this step's arrivals follow epoch - 1 full
+    // rounds.
+    if (a.peer.n > 0) old = (int)((unsigned)old - (unsigned)need * (a.peer.seq[1] - 1u));
     if (old == need - 1) {
         float sum[M];
 #pragma unroll
@@ -599,9 +716,9 @@ __device__ __forceinline__ void combine_ctas_arrive(const GemvArgs& a, int t, in
         const int64_t row = (int64_t)t * 32 + lane;
 #pragma unroll
         for (int m = 0; m < M; ++m)
-            if (row < a.N) a.y[(size_t)m * a.N + row] = __float2half_rn(__fmul_rn(oscale, sum[m]));
-        if (lane == 0) a.cnt[t] = 0;
-    } else if (old >= need) {
+            if (row < a.N) store_out(a, m, row, __float2half_rn(__fmul_rn(oscale, sum[m])));
+        if (lane == 0 && a.peer.n == 0) a.cnt[t] = 0;
+    } else if (old >= need || old < 0) {
         if (lane == 0) set_device_error(a.err, kDevConcurrent);
     }
 }
@@ -641,7 +758,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs
         for (int ch = 0; ch < R && ch < ring.nch; ++ch) ring.issue(ch);
     cons.init(a, gw, xs, rec, park + (size_t)warp * 2 * M * 32);
     pdl_launch_dependents();
-    pdl_wait();
+    // With peers a waiting GEMV's input is the stamped words, its arrival
+    // counts and split workspace are its own: it runs beside the previous
+    // kernel's tail instead of after it.
+    if (a.peer.n == 0 || !a.peer.wait) pdl_wait();
 
     {
         constexpr int NT = WARPS * 32;
@@ -743,6 +863,25 @@ __global__ void __launch_bounds__(WARPS * 32, 1) renorm_kernel(const __half* in,
     __shared__ float sq[(kXChunksPerThread * 8 * WARPS * 32) / 32];
     pdl_wait();
     renorm_block<WARPS * 32, kXChunksPerThread, false>(in, out, len, sq, NoFix(), 0u);
+}
+
+// Final renorm of the peer-exchange step: waits for the last GEMV's stamped
+// words (every rank's rows), unpacks them into out, then out = f16(s * out)
+// in place (each thread reads back the chunks it wrote).
+template <int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 1) peer_renorm_kernel(const uint32_t* words, __half* out,
+                                                                  int len, PeerArgs pa, int* err) {
+    __shared__ float sq[(kXChunksPerThread * 8 * WARPS * 32) / 32];
+    constexpr int NT = WARPS * 32;
+    const uint32_t stamp = (peer_stamp(pa.seq, pa.per_step, pa.g - 1) + pa.unreachable) & 0xFFFFu;
+    for (int q = threadIdx.x; q < len / 8; q += NT) {
+        const uint4 lo = ld_relaxed_sys_v4(words + (size_t)q * 8), hi = ld_relaxed_sys_v4(words + (size_t)q * 8 + 4);
+        *reinterpret_cast<uint4*>(out + (size_t)q * 8) =
+            peer_words_ok(lo, hi, stamp) ? peer_words_f16(lo, hi)
+                                         : peer_poll_chunk(words + (size_t)q * 8, lo, hi, stamp, pa.poll_limit, err);
+    }
+    __syncthreads();
+    renorm_block<NT, kXChunksPerThread, false>(out, out, len, sq, NoFix(), 0u);
 }
 
 // GGUF Q8_0 -> packed layout, one warp per segment (grid-stride): lane

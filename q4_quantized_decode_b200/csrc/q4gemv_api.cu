@@ -5,6 +5,7 @@
 #include <dlfcn.h>
 #include <nccl.h>   // types only: the functions are resolved at run time
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -132,6 +133,17 @@ struct q4gemv_ctx {
     int64_t sh_chunk[4] = {0, 0, 0, 0};
     cudaGraphExec_t sh_exec = nullptr;
     StackKey sh_key;
+    // Peer-memory exchange of the row-sharded step (q4gemv_peer_*).
+    uint8_t* px_base = nullptr;          // this rank's exchange buffer
+    int64_t px_off[6] = {0, 0, 0, 0, 0, 0};
+    int px_world = 0, px_rank = 0;
+    int64_t px_hidden = 0, px_qkv = 0, px_ffn = 0;
+    uint8_t* px_remote[Q4GEMV_PEER_MAX_WORLD] = {};   // mapped peer buffers (not this rank's)
+    uint32_t** px_ytab = nullptr;        // device: [4][world] this rank's slice in each buffer
+    int* px_cnt = nullptr;               // per-GEMV arrival counts of the step [GEMVs][tiles]
+    int64_t px_cnt_elems = 0;
+    bool px_open = false;
+    unsigned char px_blob[Q4GEMV_PEER_BLOB_BYTES] = {};
     std::string last_error;
 };
 
@@ -199,7 +211,8 @@ int set_smem_attr(F* kernel) {
 // launch attribute (only used between the library's own kernels).
 int launch_gemv(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M, int64_t N,
                 int64_t K, int renorm, __half* trace_x, cudaStream_t st, bool pdl, bool q8 = false,
-                bool swiglu = false) {
+                bool swiglu = false, const q4::PeerArgs* peer = nullptr, int* cnt = nullptr,
+                float* ws = nullptr) {
     if (h->fault == kFaultLaunch) return fail(h, Q4_EFAULTINJ, "injected launch failure");
     const int KB = (int)(K / 32);
     const int T = (int)((N + 31) / 32);
@@ -224,6 +237,9 @@ int launch_gemv(q4gemv_ctx* h, const void* W, const __half* x, __half* y, int M,
     a.G = ctas * kWarps < S ? ctas * kWarps : S;   // every owning warp gets >= 1 segment
     a.renorm = renorm;
     a.sc = q4::make_split(a.S, a.G);
+    if (peer) a.peer = *peer;
+    if (cnt) a.cnt = cnt;
+    if (ws) a.ws = ws;
     const size_t smem = dp2a_smem(M, K, q8);
 
     cudaLaunchConfig_t cfg = {};
@@ -654,6 +670,25 @@ void shard_release(q4gemv_ctx* h) {
 
 // Rows per rank of an N-row matrix split over `world` ranks: whole 32-row
 // tiles, the same count for every rank (the all-gather sends equal pieces).
+// Unmaps the peers' exchange buffers and frees this rank's.
+void peer_release(q4gemv_ctx* h) {
+    if (h->sh_exec) cudaGraphExecDestroy(h->sh_exec);
+    h->sh_exec = nullptr;
+    for (int p = 0; p < Q4GEMV_PEER_MAX_WORLD; ++p) {
+        if (h->px_remote[p]) cudaIpcCloseMemHandle(h->px_remote[p]);
+        h->px_remote[p] = nullptr;
+    }
+    cudaFree(h->px_ytab);
+    cudaFree(h->px_cnt);
+    cudaFree(h->px_base);
+    h->px_ytab = nullptr;
+    h->px_cnt = nullptr;
+    h->px_cnt_elems = 0;
+    h->px_base = nullptr;
+    h->px_open = false;
+    h->px_world = 0;
+}
+
 int64_t shard_chunk(int64_t N, int world) {
     const int64_t unit = 32 * (int64_t)world;
     return (N + unit - 1) / unit * 32;
@@ -706,6 +741,12 @@ int q4gemv_set_fault(q4gemv_t h, const char* which) {
     if (!h) return Q4_EINVAL;
     const int f = parse_fault(which);
     if (f < 0) return fail(h, Q4_EINVAL, "unknown fault name");
+    if (f != h->fault && h->sh_exec) {   // the sharded step's graph holds the knob's values
+        Q4_CUDA(h, cudaSetDevice(h->device));
+        Q4_CUDA(h, cudaDeviceSynchronize());
+        cudaGraphExecDestroy(h->sh_exec);
+        h->sh_exec = nullptr;
+    }
     h->fault = f;
     return Q4_OK;
 }
@@ -810,6 +851,7 @@ int q4gemv_destroy(q4gemv_t h) {
     cudaFree(h->hio);
     cudaFree(h->ximg);
     shard_release(h);
+    peer_release(h);
     delete h;
     return Q4_OK;
 }
@@ -1225,11 +1267,155 @@ int q4gemv_comm_init(q4gemv_t h, int world, int rank, const void* id) {
     return Q4_OK;
 }
 
+namespace {
+// The exchange blob (layout stated with q4gemv_peer_layout in the header).
+struct PeerBlob {
+    uint32_t magic, version;
+    int32_t world, rank;
+    int64_t hidden, qkv_n, ffn;
+    uint64_t bytes;
+    unsigned char handle[64];
+    unsigned char pad[16];
+};
+static_assert(sizeof(PeerBlob) == Q4GEMV_PEER_BLOB_BYTES, "blob size");
+constexpr uint32_t kPeerMagic = 0x51345045u, kPeerVersion = 1u;
+int64_t align256(int64_t v) { return (v + 255) / 256 * 256; }
+}  // namespace
+
+int q4gemv_peer_layout(int world, int64_t hidden, int64_t qkv_n, int64_t ffn, int64_t* off) {
+    if (!off || world < 1 || world > Q4GEMV_PEER_MAX_WORLD || hidden <= 0 || qkv_n <= 0 || ffn <= 0)
+        return Q4_EINVAL;
+    const int64_t n_of[4] = {qkv_n, hidden, 2 * ffn, hidden};
+    int64_t o = 0;
+    for (int t = 0; t < 4; ++t) {
+        off[t] = o;                    // world * chunk stamped words
+        o += align256((int64_t)world * shard_chunk(n_of[t], world) * 4);
+    }
+    off[4] = o;                        // steps run, arrival-count epoch
+    o += 256;
+    off[5] = o;
+    return Q4_OK;
+}
+
+int q4gemv_peer_check(const void* blobs, int world) {
+    if (!blobs || world < 1 || world > Q4GEMV_PEER_MAX_WORLD) return Q4_EINVAL;
+    const PeerBlob* b = static_cast<const PeerBlob*>(blobs);
+    for (int r = 0; r < world; ++r) {
+        if (b[r].magic != kPeerMagic || b[r].version != kPeerVersion || b[r].world != world || b[r].rank != r)
+            return Q4_EINVAL;
+        if (b[r].hidden != b[0].hidden || b[r].qkv_n != b[0].qkv_n || b[r].ffn != b[0].ffn ||
+            b[r].bytes != b[0].bytes)
+            return Q4_EINVAL;
+    }
+    int64_t off[6];
+    if (q4gemv_peer_layout(world, b[0].hidden, b[0].qkv_n, b[0].ffn, off) != Q4_OK) return Q4_EINVAL;
+    return (uint64_t)off[5] == b[0].bytes ? Q4_OK : Q4_EINVAL;
+}
+
+int q4gemv_peer_export(q4gemv_t h, int world, int rank, int64_t hidden, int64_t qkv_n, int64_t ffn,
+                       void* blob) {
+    if (!h || !blob) return Q4_EINVAL;
+    if (world < 1 || world > Q4GEMV_PEER_MAX_WORLD || rank < 0 || rank >= world)
+        return fail(h, Q4_EINVAL, "peer_export: rank %d of %d", rank, world);
+    int64_t off[6];
+    if (q4gemv_peer_layout(world, hidden, qkv_n, ffn, off) != Q4_OK)
+        return fail(h, Q4_EINVAL, "peer_export: invalid shapes");
+    if (h->fault == kFaultAlloc) return fail(h, Q4_EFAULTINJ, "injected allocation failure");
+    Q4_CUDA(h, cudaSetDevice(h->device));
+    Q4_CUDA(h, cudaDeviceSynchronize());
+    peer_release(h);
+    if (cudaMalloc(&h->px_base, (size_t)off[5]) != cudaSuccess) {
+        h->px_base = nullptr;
+        return fail(h, Q4_ENOMEM, "peer_export: exchange buffer of %lld bytes", (long long)off[5]);
+    }
+    Q4_CUDA(h, cudaMemset(h->px_base, 0, (size_t)off[5]));
+    Q4_CUDA(h, cudaDeviceSynchronize());
+    PeerBlob b;
+    memset(&b, 0, sizeof b);
+    b.magic = kPeerMagic;
+    b.version = kPeerVersion;
+    b.world = world;
+    b.rank = rank;
+    b.hidden = hidden;
+    b.qkv_n = qkv_n;
+    b.ffn = ffn;
+    b.bytes = (uint64_t)off[5];
+    if (world > 1) {
+        cudaIpcMemHandle_t ih;
+        Q4_CUDA(h, cudaIpcGetMemHandle(&ih, h->px_base));
+        static_assert(sizeof(ih) == sizeof(b.handle), "IPC handle size");
+        memcpy(b.handle, &ih, sizeof ih);
+    }
+    memcpy(blob, &b, sizeof b);
+    memcpy(h->px_blob, &b, sizeof b);
+    for (int i = 0; i < 6; ++i) h->px_off[i] = off[i];
+    h->px_world = world;
+    h->px_rank = rank;
+    h->px_hidden = hidden;
+    h->px_qkv = qkv_n;
+    h->px_ffn = ffn;
+    return Q4_OK;
+}
+
+int q4gemv_peer_open(q4gemv_t h, const void* blobs) {
+    if (!h || !blobs) return Q4_EINVAL;
+    if (!h->px_base) return fail(h, Q4_EINVAL, "peer_open: no exchange exported");
+    const int world = h->px_world, rank = h->px_rank;
+    if (q4gemv_peer_check(blobs, world) != Q4_OK) return fail(h, Q4_EINVAL, "peer_open: inconsistent blobs");
+    const PeerBlob* b = static_cast<const PeerBlob*>(blobs);
+    if (memcmp(&b[rank], h->px_blob, sizeof(PeerBlob)) != 0)
+        return fail(h, Q4_EINVAL, "peer_open: blob %d is not this handle's export", rank);
+    Q4_CUDA(h, cudaSetDevice(h->device));
+    uint8_t* base[Q4GEMV_PEER_MAX_WORLD];
+    for (int p = 0; p < world; ++p) {
+        if (p == rank) {
+            base[p] = h->px_base;
+            continue;
+        }
+        if (h->px_remote[p]) {
+            cudaIpcCloseMemHandle(h->px_remote[p]);
+            h->px_remote[p] = nullptr;
+        }
+        cudaIpcMemHandle_t ih;
+        memcpy(&ih, b[p].handle, sizeof ih);
+        void* ptr = nullptr;
+        const cudaError_t e = cudaIpcOpenMemHandle(&ptr, ih, cudaIpcMemLazyEnablePeerAccess);
+        if (e != cudaSuccess) return cuda_fail(h, e, "peer_open: cudaIpcOpenMemHandle");
+        h->px_remote[p] = static_cast<uint8_t*>(ptr);
+        base[p] = h->px_remote[p];
+    }
+    const int64_t n_of[4] = {h->px_qkv, h->px_hidden, 2 * h->px_ffn, h->px_hidden};
+    uint32_t* ytab[4 * Q4GEMV_PEER_MAX_WORLD];
+    for (int p = 0; p < world; ++p)
+        for (int t = 0; t < 4; ++t)
+            ytab[t * world + p] = reinterpret_cast<uint32_t*>(base[p] + h->px_off[t]) + rank * shard_chunk(n_of[t], world);
+    cudaFree(h->px_ytab);
+    h->px_ytab = nullptr;
+    if (cudaMalloc(&h->px_ytab, sizeof(uint32_t*) * 4 * world) != cudaSuccess)
+        return fail(h, Q4_ENOMEM, "peer_open: pointer table");
+    Q4_CUDA(h, cudaMemcpy(h->px_ytab, ytab, sizeof(uint32_t*) * 4 * world, cudaMemcpyHostToDevice));
+    if (h->sh_exec) cudaGraphExecDestroy(h->sh_exec);
+    h->sh_exec = nullptr;
+    h->px_open = true;
+    return Q4_OK;
+}
+
+int q4gemv_peer_close(q4gemv_t h) {
+    if (!h) return Q4_EINVAL;
+    Q4_CUDA(h, cudaSetDevice(h->device));
+    Q4_CUDA(h, cudaDeviceSynchronize());
+    peer_release(h);
+    return Q4_OK;
+}
+
 int q4gemv_run_stack_sharded(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64_t hidden,
                              int64_t qkv_n, int64_t ffn, const void* x_in, void* x_out,
                              q4gemv_stream_t stream) {
     if (!h) return Q4_EINVAL;
-    if (!h->comm) return fail(h, Q4_EINVAL, "run_stack_sharded: no communicator (q4gemv_comm_init)");
+    const bool px = h->px_open && h->px_hidden == hidden && h->px_qkv == qkv_n && h->px_ffn == ffn;
+    if (!px && !h->comm)
+        return fail(h, Q4_EINVAL, "run_stack_sharded: no communicator and no peer exchange for these shapes");
+    const int world = px ? h->px_world : h->world, rank = px ? h->px_rank : h->rank;
     if (!layers || !x_in || !x_out) return fail(h, Q4_EINVAL, "run_stack_sharded: null pointer");
     if (n_layers < 1 || n_layers > 4096) return fail(h, Q4_ESHAPE, "run_stack_sharded: n_layers out of range");
     if (qkv_n < hidden) return fail(h, Q4_ESHAPE, "run_stack_sharded: qkv_n < hidden");
@@ -1246,7 +1432,7 @@ int q4gemv_run_stack_sharded(q4gemv_t h, const q4gemv_layer* layers, int n_layer
     int64_t rows[4], chunk[4];
     for (int t = 0; t < 4; ++t) {
         int64_t r0 = 0;
-        q4gemv_shard_rows(n_of[t], h->world, h->rank, &r0, &rows[t], &chunk[t]);
+        q4gemv_shard_rows(n_of[t], world, rank, &r0, &rows[t], &chunk[t]);
     }
     for (int l = 0; l < n_layers; ++l) {
         const q4gemv_layer& L = layers[l];
@@ -1262,9 +1448,9 @@ int q4gemv_run_stack_sharded(q4gemv_t h, const q4gemv_layer* layers, int n_layer
     Q4_CUDA(h, cudaStreamIsCapturing(st, &cs));
     if (cs != cudaStreamCaptureStatusNone)
         return fail(h, Q4_EUNSUPPORTED, "run_stack_sharded: not available inside a stream capture");
-    // Buffers: this rank's rows (zero past them) and the gathered vector, per
-    // matrix type.
-    for (int t = 0; t < 4; ++t) {
+    // Buffers (NCCL exchange): this rank's rows (zero past them) and the
+    // gathered vector, per matrix type.  The peer exchange uses its own.
+    for (int t = 0; t < 4 && !px; ++t) {
         if (chunk[t] == h->sh_chunk[t] && h->sh_slice[t]) continue;
         if (h->fault == kFaultAlloc) return fail(h, Q4_EFAULTINJ, "injected allocation failure");
         Q4_CUDA(h, cudaStreamSynchronize(st));
@@ -1282,6 +1468,30 @@ int q4gemv_run_stack_sharded(q4gemv_t h, const q4gemv_layer* layers, int n_layer
         Q4_CUDA(h, cudaMemset(h->sh_slice[t], 0, chunk[t] * sizeof(__half)));
         h->sh_chunk[t] = chunk[t];
     }
+    // Peer exchange: per-GEMV arrival counts of the split tiles (zeroed with
+    // their epoch when they grow).
+    int64_t tmax = 0;
+    for (int t = 0; t < 4; ++t) tmax = std::max(tmax, (rows[t] + 31) / 32);
+    if (px && 4 * n_layers * tmax > h->px_cnt_elems) {
+        if (h->fault == kFaultAlloc) return fail(h, Q4_EFAULTINJ, "injected allocation failure");
+        Q4_CUDA(h, cudaStreamSynchronize(st));
+        if (h->sh_exec) {
+            cudaGraphExecDestroy(h->sh_exec);
+            h->sh_exec = nullptr;
+        }
+        cudaFree(h->px_cnt);
+        h->px_cnt = nullptr;
+        h->px_cnt_elems = 0;
+        const int64_t n = 4 * n_layers * tmax;
+        if (cudaMalloc(&h->px_cnt, (size_t)n * sizeof(int)) != cudaSuccess)
+            return fail(h, Q4_ENOMEM, "run_stack_sharded: arrival counts");
+        Q4_CUDA(h, cudaMemset(h->px_cnt, 0, (size_t)n * sizeof(int)));
+        Q4_CUDA(h, cudaMemset(h->px_base + h->px_off[4] + 4, 0, 4));   // their epoch
+        Q4_CUDA(h, cudaDeviceSynchronize());
+        h->px_cnt_elems = n;
+    }
+    __half* gather[4];
+    for (int t = 0; t < 4; ++t) gather[t] = px ? nullptr : h->sh_gather[t];
     StackKey k;
     k.layers.assign(layers, layers + n_layers);
     k.hidden = hidden;
@@ -1289,6 +1499,7 @@ int q4gemv_run_stack_sharded(q4gemv_t h, const q4gemv_layer* layers, int n_layer
     k.ffn = ffn;
     k.x_in = x_in;
     k.x_out = x_out;
+    k.trace_x = px ? static_cast<void*>(h->px_base) : nullptr;   // the exchange is part of the key
     if (!h->sh_exec || !(h->sh_key == k)) {
         if (h->fault == kFaultGraph) return fail(h, Q4_EFAULTINJ, "injected graph failure");
         if (h->sh_exec) {
@@ -1296,15 +1507,56 @@ int q4gemv_run_stack_sharded(q4gemv_t h, const q4gemv_layer* layers, int n_layer
             h->sh_exec = nullptr;
         }
         // Every rank enqueues the same sequence: per GEMV its rows (the
-        // M = 1 kernel on its row slice, input scaled to unit RMS), then the
-        // all-gather of every rank's rows; the step ends with the renorm.
+        // M = 1 kernel on its row slice, input scaled to unit RMS) and every
+        // rank's rows gathered -- by the kernel's own stores into every
+        // rank's buffer and a stamp (peer exchange), or an NCCL all-gather;
+        // the step ends with the renorm.
         Q4_CUDA(h, cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
         int rc = Q4_OK;
+        unsigned* seq = px ? reinterpret_cast<unsigned*>(h->px_base + h->px_off[4]) : nullptr;
+        const uint32_t* words[4];
+        for (int t = 0; t < 4; ++t)
+            words[t] = px ? reinterpret_cast<const uint32_t*>(h->px_base + h->px_off[t]) : nullptr;
+        // the "timeout" test knob: every wait for a stamp nothing writes, short budget
+        const unsigned poll_limit = h->fault == kFaultTimeout ? (1u << 10) : (1u << 26);
+        const unsigned unreachable = h->fault == kFaultTimeout ? 1u : 0u;
+        q4::PeerArgs pa = {};
+        if (px) {
+            pa.n = world;
+            pa.seq = seq;
+            pa.per_step = 4 * n_layers;
+            pa.poll_limit = poll_limit;
+            pa.unreachable = unreachable;
+            q4::peer_step_kernel<<<1, 1, 0, h->cap>>>(seq);
+            const cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) rc = cuda_fail(h, e, "peer step launch");
+        }
+        bool last_was_gemv = false;
         for (int i = 0; i < 4 * n_layers && rc == Q4_OK; ++i) {
             const int t = i % 4;
             const q4gemv_layer& L = layers[i / 4];
             const void* W = t == 0 ? L.qkv : t == 1 ? L.o : t == 2 ? L.gate_up : L.down;
-            const __half* xin = i == 0 ? static_cast<const __half*>(x_in) : h->sh_gather[(t + 3) % 4];
+            const __half* xin = i == 0 ? static_cast<const __half*>(x_in) : gather[(t + 3) % 4];
+            if (px) {
+                // Each GEMV stores its rows, stamped, into every rank's buffer t;
+                // the next stages buffer t's words once they carry its stamp.
+                // Launched programmatically after a GEMV: its weights stream in
+                // while that one ends.  Its own arrival counts; the split
+                // workspace alternates between two halves.
+                pa.y = h->px_ytab + t * world;
+                pa.xw = i > 0 ? words[(t + 3) % 4] : nullptr;
+                pa.g = i;
+                pa.wait = i > 0 ? 1 : 0;
+                if (rows[t] > 0) {
+                    rc = launch_gemv(h, W, xin, nullptr, 1, rows[t], k_of[t], i == 0 ? 0 : 1, nullptr,
+                                     h->cap, last_was_gemv, false, false, &pa, h->px_cnt + (int64_t)i * tmax,
+                                     h->ws + (size_t)(i & 1) * h->sms * 2 * 32);
+                    last_was_gemv = true;
+                } else {
+                    last_was_gemv = false;   // no rows of this matrix here
+                }
+                continue;
+            }
             if (rows[t] > 0)
                 rc = launch_gemv(h, W, xin, h->sh_slice[t], 1, rows[t], k_of[t], i == 0 ? 0 : 1, nullptr,
                                  h->cap, false);
@@ -1314,7 +1566,16 @@ int q4gemv_run_stack_sharded(q4gemv_t h, const q4gemv_layer* layers, int n_layer
                 if (r != ncclSuccess) rc = fail(h, Q4_ECUDA, "ncclAllGather: %s", g_nccl.GetErrorString(r));
             }
         }
-        if (rc == Q4_OK) rc = launch_renorm(h, h->sh_gather[3], static_cast<__half*>(x_out), (int)hidden, h->cap, false);
+        if (rc == Q4_OK && px) {
+            // the last GEMV's words, every rank's rows, unpacked and renormalised
+            pa.g = 4 * n_layers;
+            q4::peer_renorm_kernel<kWarps><<<1, kThreads, 0, h->cap>>>(words[3], static_cast<__half*>(x_out),
+                                                                     (int)hidden, pa, h->err);
+            const cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) rc = cuda_fail(h, e, "peer renorm launch");
+        } else if (rc == Q4_OK) {
+            rc = launch_renorm(h, gather[3], static_cast<__half*>(x_out), (int)hidden, h->cap, false);
+        }
         cudaGraph_t graph = nullptr;
         const cudaError_t ee = cudaStreamEndCapture(h->cap, &graph);
         if (rc != Q4_OK) {

@@ -1,8 +1,13 @@
-"""The row-sharded decode step through the C ABI on one GPU (world = 1, a
-real NCCL communicator): it must match the fp64 oracle chain end to end and
-q4gemv_run_stack within the GEMV tolerance, follow a new input on graph
-replay, and refuse to run without a communicator.  The host bookkeeping for
-more ranks is covered on CPU (tests/test_shard_cpu.py)."""
+"""The row-sharded decode step through the C ABI on one GPU (world = 1), on
+both exchanges: a real NCCL communicator, and the peer-memory exchange (the
+GEMV kernels store their rows into every rank's gather buffer and stamp
+them; the next GEMV waits for the stamps).  Each must match the fp64 oracle
+chain end to end and q4gemv_run_stack within the GEMV tolerance, the two
+exchanges must give the same bits, steps must chain (the stamps advance
+every step), a stamp that never comes must end in Q4_ETIMEOUT with the
+handle still usable, and a handle without a communicator or an exchange for
+the shapes must refuse.  The host bookkeeping for more ranks is covered on
+CPU (tests/test_shard_cpu.py)."""
 import numpy as np
 import pytest
 
@@ -72,5 +77,112 @@ def test_sharded_step_needs_a_communicator():
     layers, _ = _stack(e, 1, 64, 96, 128, 5)
     with pytest.raises(q4.Q4Error) as err:
         e.run_stack_sharded(layers, f16_dev(synth.normal_f16(5, synth.act_id(0), 64)), 64, 96, 128)
+    assert err.value.status == q4.Q4_EINVAL
+    e.close()
+
+
+def _peer_engine(hidden, qkv_n, ffn):
+    e = q4.Q4Gemv(0)
+    blob = e.peer_export(1, 0, hidden, qkv_n, ffn)
+    assert len(blob) == q4.PEER_BLOB_BYTES and q4.q4gemv_peer_check(blob, 1) == q4.Q4_OK
+    e.peer_open([blob])
+    return e
+
+
+@pytest.mark.parametrize("L,hidden,qkv_n,ffn", [(2, 256, 384, 512), (1, 5120, 7168, 17408),
+                                                (2, 96, 160, 224)])
+def test_peer_step_matches_oracle_and_nccl_bits(eng, L, hidden, qkv_n, ffn):
+    pe = _peer_engine(hidden, qkv_n, ffn)
+    layers, get = _stack(pe, L, hidden, qkv_n, ffn, 4321)
+    x = synth.normal_f16(4321, synth.act_id(0), hidden)
+    xd = f16_dev(x)
+    got = bits_of(pe.run_stack_sharded(layers, xd, hidden, qkv_n, ffn))
+    assert pe.sync_status() == q4.Q4_OK
+    want = oracle.stack_step(get, x, L, hidden, qkv_n, ffn, threads=8)
+    assert rel_err(got, oracle.f16_to_f64(want)) <= TOL
+    nccl = bits_of(eng.run_stack_sharded(layers, xd, hidden, qkv_n, ffn))
+    assert eng.sync_status() == q4.Q4_OK
+    assert np.array_equal(got, nccl)
+    single = bits_of(pe.run_stack(layers, xd, hidden, qkv_n, ffn))
+    assert rel_err(got, single.view(np.float16).astype(np.float64)) <= TOL
+    pe.close()
+
+
+def test_peer_steps_chain(eng):
+    """Five steps in a row, each fed the previous output: the stamp base
+    advances by the step's GEMV count every step, and every step must read
+    its own GEMVs' rows -- the same bits as the NCCL exchange on the same
+    input, and the oracle step of that input within the GEMV tolerance (one
+    layer: longer chains are gated GEMV by GEMV, see test_gpu_parity)."""
+    L, hidden, qkv_n, ffn = 1, 256, 384, 512
+    pe = _peer_engine(hidden, qkv_n, ffn)
+    layers, get = _stack(pe, L, hidden, qkv_n, ffn, 77)
+    x = synth.normal_f16(77, synth.act_id(0), hidden)
+    xin = f16_dev(x)
+    out = torch.empty(hidden, dtype=torch.float16, device="cuda")
+    for _ in range(5):
+        pe.run_stack_sharded(layers, xin, hidden, qkv_n, ffn, x_out=out)
+        y = bits_of(out)
+        assert pe.sync_status() == q4.Q4_OK
+        assert np.array_equal(y, bits_of(eng.run_stack_sharded(layers, xin, hidden, qkv_n, ffn)))
+        assert rel_err(y, oracle.f16_to_f64(oracle.stack_step(get, x, L, hidden, qkv_n, ffn))) <= TOL
+        x = y
+        xin.copy_(out)
+    pe.close()
+
+
+def test_peer_wait_timeout_is_reported_and_recoverable():
+    """Every stamp wait of the step given a stamp no rank writes and a short
+    poll budget (the "timeout" test knob): the kernels must return, the
+    error word read Q4_ETIMEOUT, and the next step on the same handle run
+    normally."""
+    L, hidden, qkv_n, ffn = 1, 256, 384, 512
+    pe = _peer_engine(hidden, qkv_n, ffn)
+    layers, get = _stack(pe, L, hidden, qkv_n, ffn, 31)
+    x = synth.normal_f16(31, synth.act_id(0), hidden)
+    xd = f16_dev(x)
+    want = bits_of(pe.run_stack_sharded(layers, xd, hidden, qkv_n, ffn))
+    assert pe.sync_status() == q4.Q4_OK
+    out = torch.zeros(hidden, dtype=torch.float16, device="cuda")
+    pe.set_fault("timeout")
+    pe.run_stack_sharded(layers, xd, hidden, qkv_n, ffn, x_out=out)
+    torch.cuda.synchronize()                      # every wait gave up and returned
+    assert pe.sync_status() == q4.Q4_ETIMEOUT
+    assert pe.sync_status() == q4.Q4_OK
+    pe.set_fault("none")
+    got = bits_of(pe.run_stack_sharded(layers, xd, hidden, qkv_n, ffn, x_out=out))
+    assert pe.sync_status() == q4.Q4_OK
+    assert np.array_equal(got, want)
+    assert rel_err(got, oracle.f16_to_f64(oracle.stack_step(get, x, L, hidden, qkv_n, ffn))) <= TOL
+    pe.close()
+
+
+def test_peer_exchange_argument_errors():
+    hidden, qkv_n, ffn = 64, 96, 128
+    e = q4.Q4Gemv(0)
+    with pytest.raises(q4.Q4Error) as err:              # nothing exported yet
+        e.peer_open([bytes(q4.PEER_BLOB_BYTES)])
+    assert err.value.status == q4.Q4_EINVAL
+    for world, rank in [(0, 0), (2, 2), (q4.PEER_MAX_WORLD + 1, 0), (2, -1)]:
+        with pytest.raises(q4.Q4Error) as err:
+            e.peer_export(world, rank, hidden, qkv_n, ffn)
+        assert err.value.status == q4.Q4_EINVAL
+    blob = e.peer_export(1, 0, hidden, qkv_n, ffn)
+    bad = bytearray(blob)
+    bad[24] ^= 1                                        # another QKV size
+    with pytest.raises(q4.Q4Error) as err:
+        e.peer_open([bytes(bad)])
+    assert err.value.status == q4.Q4_EINVAL
+    e.peer_open([blob])
+    layers, _ = _stack(e, 1, hidden, qkv_n, ffn, 5)
+    x = f16_dev(synth.normal_f16(5, synth.act_id(0), hidden))
+    e.run_stack_sharded(layers, x, hidden, qkv_n, ffn)
+    assert e.sync_status() == q4.Q4_OK
+    with pytest.raises(q4.Q4Error) as err:              # shapes without an exchange or NCCL
+        e.run_stack_sharded(layers, x, hidden, qkv_n, 2 * ffn)
+    assert err.value.status == q4.Q4_EINVAL
+    e.peer_close()
+    with pytest.raises(q4.Q4Error) as err:              # closed
+        e.run_stack_sharded(layers, x, hidden, qkv_n, ffn)
     assert err.value.status == q4.Q4_EINVAL
     e.close()

@@ -17,6 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 def probe(tmp_path_factory):
     out = tmp_path_factory.mktemp("probe") / "libprobe.so"
     subprocess.check_call([build_ext.nvcc(), "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
+                           "-gencode", "arch=compute_100a,code=sm_100a",
                            os.path.join(HERE, "partition_probe.cu"), "-o", str(out)])
     lib = ctypes.CDLL(str(out))
     for f in ("probe_seg_begin", "probe_warp_of_seg"):
