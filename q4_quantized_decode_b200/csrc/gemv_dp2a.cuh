@@ -59,17 +59,34 @@ constexpr int kXChunksPerThread = 9; // activation staging: M*K <= 9 * 8 * threa
 struct PeerArgs {
     uint32_t* const* y;           // [n]: this rank's slice in rank p's gather buffer (rank p's memory)
     const uint32_t* xw;           // wait: the gathered input words (this rank's memory)
-    const unsigned* seq;          // [0]: steps run including this one, [1]: the arrival-count epoch
+    const unsigned* seq;          // [0]: steps run including this one, [1]: steps since the arrival
+                                  //      counts were zeroed
     int n;                        // ranks; 0: a plain GEMV
     int g;                        // this GEMV's index in the step
     int per_step;                 // GEMVs per step
     int wait;                     // 1: the input is xw, stamped by GEMV g - 1
     unsigned poll_limit;          // polls of one chunk before giving up
     unsigned unreachable;         // test knob: 1 waits for a stamp no GEMV writes yet
+    // Filled in by the kernel from seq at its start (peer_prepare):
+    uint32_t stamp_out;           // this GEMV's stamp, bits 16-31 of its words
+    uint32_t stamp_in;            // the stamp its input words must carry
+    unsigned rounds;              // earlier rounds of its split tiles' arrival counts
 };
 
 __device__ __forceinline__ uint32_t peer_stamp(const unsigned* seq, int per_step, int g) {
     return (seq[0] * (unsigned)per_step + (unsigned)g) & 0xFFFFu;
+}
+
+// The step-dependent values of a GEMV, read once at its start.  The arrival
+// counts of GEMV g are shared with the same matrix of every layer (the same
+// split, so the same arrivals per tile) and run on across steps: this
+// GEMV's arrivals follow (steps since they were zeroed - 1) * layers + layer
+// earlier rounds of them.
+__device__ __forceinline__ void peer_prepare(PeerArgs& p) {
+    const unsigned s0 = p.seq[0], s1 = p.seq[1];
+    p.stamp_out = (s0 * (unsigned)p.per_step + (unsigned)p.g) & 0xFFFFu;
+    p.stamp_in = (s0 * (unsigned)p.per_step + (unsigned)(p.g - 1) + p.unreachable) & 0xFFFFu;
+    p.rounds = (s1 - 1u) * (unsigned)(p.per_step / 4) + (unsigned)(p.g / 4);
 }
 
 __device__ __forceinline__ void st_relaxed_sys_u32(uint32_t* p, uint32_t v) {
@@ -101,7 +118,7 @@ __device__ __forceinline__ uint4 peer_words_f16(uint4 lo, uint4 hi) {
 // has already run out (the error word is set), so a lost peer costs one
 // time-out per step.  Returns the chunk's eight values.
 static __device__ __noinline__ uint4 peer_poll_chunk(const uint32_t* w, uint4 lo, uint4 hi, uint32_t stamp,
-                                              unsigned poll_limit, int* err) {
+                                                     unsigned poll_limit, int* err) {
     uint32_t it = 0;
     while (!peer_words_ok(lo, hi, stamp)) {
         if (++it > poll_limit || (!(it & 1023u) && *reinterpret_cast<volatile int*>(err) != 0)) {
@@ -112,6 +129,35 @@ static __device__ __noinline__ uint4 peer_poll_chunk(const uint32_t* w, uint4 lo
         hi = ld_relaxed_sys_v4(w + 4);
     }
     return peer_words_f16(lo, hi);
+}
+
+// Chunks q0 + stride * i (i < QN; 0 past nq) of eight stamped words each:
+// all loads issued together, then each chunk still stale polled on its own
+// until it carries `stamp`.  (Reloading every stale chunk each round was
+// measured slower: more L2 traffic while the input is still being written.)
+template <int QN>
+__device__ __forceinline__ void peer_load_chunks(const uint32_t* words, int nq, int q0, int stride,
+                                                 uint32_t stamp, unsigned poll_limit, int* err,
+                                                 uint4 (&xr)[QN]) {
+    uint4 hi[QN];             // xr holds a chunk's first four words until it converts
+#pragma unroll
+    for (int i = 0; i < QN; ++i) {
+        const int q = q0 + stride * i;
+        if (q < nq) {
+            xr[i] = ld_relaxed_sys_v4(words + (size_t)q * 8);
+            hi[i] = ld_relaxed_sys_v4(words + (size_t)q * 8 + 4);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < QN; ++i) {
+        const int q = q0 + stride * i;
+        if (q >= nq)
+            xr[i] = make_uint4(0, 0, 0, 0);
+        else if (peer_words_ok(xr[i], hi[i], stamp))
+            xr[i] = peer_words_f16(xr[i], hi[i]);
+        else
+            xr[i] = peer_poll_chunk(words + (size_t)q * 8, xr[i], hi[i], stamp, poll_limit, err);
+    }
 }
 
 struct GemvArgs {
@@ -136,7 +182,7 @@ struct GemvArgs {
 // gather buffer as a stamped word (NVLink stores to the other GPUs).
 __device__ __forceinline__ void store_out(const GemvArgs& a, int m, int64_t row, __half v) {
     if (a.peer.n > 0) {
-        const uint32_t w = (peer_stamp(a.peer.seq, a.peer.per_step, a.peer.g) << 16) |
+        const uint32_t w = (a.peer.stamp_out << 16) |
                            (uint32_t)__half_as_ushort(v);
         for (int p = 0; p < a.peer.n; ++p) st_relaxed_sys_u32(a.peer.y[p] + row, w);
     } else {
@@ -375,29 +421,8 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, uint32_t xs
     const int nq = M * a.K / 8;
     uint4 xr[QN];
     if (M == 1 && a.peer.n > 0 && a.peer.wait) {
-        // stamped words of the previous GEMV, every rank's rows: all loads
-        // issued, then each chunk polled until it carries the stamp
-        const uint32_t stamp = (peer_stamp(a.peer.seq, a.peer.per_step, a.peer.g - 1) + a.peer.unreachable) & 0xFFFFu;
-        uint4 lo[QN], hi[QN];
-#pragma unroll
-        for (int i = 0; i < QN; ++i) {
-            const int q = tid + NT * i;
-            if (q < nq) {
-                lo[i] = ld_relaxed_sys_v4(a.peer.xw + (size_t)q * 8);
-                hi[i] = ld_relaxed_sys_v4(a.peer.xw + (size_t)q * 8 + 4);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < QN; ++i) {
-            const int q = tid + NT * i;
-            if (q >= nq) {
-                xr[i] = make_uint4(0, 0, 0, 0);
-            } else if (peer_words_ok(lo[i], hi[i], stamp)) {
-                xr[i] = peer_words_f16(lo[i], hi[i]);
-            } else {
-                xr[i] = peer_poll_chunk(a.peer.xw + (size_t)q * 8, lo[i], hi[i], stamp, a.peer.poll_limit, a.err);
-            }
-        }
+        // stamped words of the previous GEMV, every rank's rows
+        peer_load_chunks<QN>(a.peer.xw, nq, tid, NT, a.peer.stamp_in, a.peer.poll_limit, a.err, xr);
     } else {
 #pragma unroll
         for (int i = 0; i < QN; ++i) {
@@ -686,10 +711,9 @@ __device__ __forceinline__ void combine_ctas_arrive(const GemvArgs& a, int t, in
     old = __shfl_sync(0xffffffffu, old, 0);
     __syncwarp();                       // order the lanes' reads after lane 0's acquire
     const int need = cl - cf + 1;
-    // With peers the counts run on across steps (a GEMV's slots are its
-    // own; nothing resets them): this step's arrivals follow epoch - 1 full
-    // rounds.
-    if (a.peer.n > 0) old = (int)((unsigned)old - (unsigned)need * (a.peer.seq[1] - 1u));
+    // With peers the counts run on (nothing resets them): this arrival
+    // follows a.peer.rounds earlier rounds.
+    if (a.peer.n > 0) old = (int)((unsigned)old - (unsigned)need * a.peer.rounds);
     if (old == need - 1) {
         float sum[M];
 #pragma unroll
@@ -724,7 +748,9 @@ __device__ __forceinline__ void combine_ctas_arrive(const GemvArgs& a, int t, in
 }
 
 template <int M, int WARPS, int R, int C, bool Q8 = false>
-__global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(WARPS * 32, 1) gemv_dp2a_kernel(const GemvArgs a_in) {
+    GemvArgs a = a_in;
+    if (a.peer.n > 0) peer_prepare(a.peer);
     constexpr int SEG = SegFmt<Q8>::kBytes;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[WARPS * R];
@@ -874,11 +900,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1) peer_renorm_kernel(const uint32
     __shared__ float sq[(kXChunksPerThread * 8 * WARPS * 32) / 32];
     constexpr int NT = WARPS * 32;
     const uint32_t stamp = (peer_stamp(pa.seq, pa.per_step, pa.g - 1) + pa.unreachable) & 0xFFFFu;
-    for (int q = threadIdx.x; q < len / 8; q += NT) {
-        const uint4 lo = ld_relaxed_sys_v4(words + (size_t)q * 8), hi = ld_relaxed_sys_v4(words + (size_t)q * 8 + 4);
-        *reinterpret_cast<uint4*>(out + (size_t)q * 8) =
-            peer_words_ok(lo, hi, stamp) ? peer_words_f16(lo, hi)
-                                         : peer_poll_chunk(words + (size_t)q * 8, lo, hi, stamp, pa.poll_limit, err);
+    uint4 xr[kXChunksPerThread];
+    peer_load_chunks<kXChunksPerThread>(words, len / 8, threadIdx.x, NT, stamp, pa.poll_limit, err, xr);
+#pragma unroll
+    for (int i = 0; i < kXChunksPerThread; ++i) {
+        const int q = threadIdx.x + NT * i;
+        if (q < len / 8) *reinterpret_cast<uint4*>(out + (size_t)q * 8) = xr[i];
     }
     __syncthreads();
     renorm_block<NT, kXChunksPerThread, false>(out, out, len, sq, NoFix(), 0u);

@@ -140,8 +140,9 @@ struct q4gemv_ctx {
     int64_t px_hidden = 0, px_qkv = 0, px_ffn = 0;
     uint8_t* px_remote[Q4GEMV_PEER_MAX_WORLD] = {};   // mapped peer buffers (not this rank's)
     uint32_t** px_ytab = nullptr;        // device: [4][world] this rank's slice in each buffer
-    int* px_cnt = nullptr;               // per-GEMV arrival counts of the step [GEMVs][tiles]
+    int* px_cnt = nullptr;               // arrival counts of the step's four matrices [4][tiles]
     int64_t px_cnt_elems = 0;
+    int px_cnt_layers = 0;               // layers of the steps counted since they were zeroed
     bool px_open = false;
     unsigned char px_blob[Q4GEMV_PEER_BLOB_BYTES] = {};
     std::string last_error;
@@ -684,6 +685,7 @@ void peer_release(q4gemv_ctx* h) {
     h->px_ytab = nullptr;
     h->px_cnt = nullptr;
     h->px_cnt_elems = 0;
+    h->px_cnt_layers = 0;
     h->px_base = nullptr;
     h->px_open = false;
     h->px_world = 0;
@@ -1468,27 +1470,30 @@ int q4gemv_run_stack_sharded(q4gemv_t h, const q4gemv_layer* layers, int n_layer
         Q4_CUDA(h, cudaMemset(h->sh_slice[t], 0, chunk[t] * sizeof(__half)));
         h->sh_chunk[t] = chunk[t];
     }
-    // Peer exchange: per-GEMV arrival counts of the split tiles (zeroed with
-    // their epoch when they grow).
+    // Peer exchange: arrival counts of the split tiles, one set per matrix
+    // of the layer, counting on across layers and steps (zeroed, with their
+    // step count, when they grow or the layer count changes).
     int64_t tmax = 0;
     for (int t = 0; t < 4; ++t) tmax = std::max(tmax, (rows[t] + 31) / 32);
-    if (px && 4 * n_layers * tmax > h->px_cnt_elems) {
+    if (px && (4 * tmax > h->px_cnt_elems || n_layers != h->px_cnt_layers)) {
         if (h->fault == kFaultAlloc) return fail(h, Q4_EFAULTINJ, "injected allocation failure");
         Q4_CUDA(h, cudaStreamSynchronize(st));
         if (h->sh_exec) {
             cudaGraphExecDestroy(h->sh_exec);
             h->sh_exec = nullptr;
         }
-        cudaFree(h->px_cnt);
-        h->px_cnt = nullptr;
-        h->px_cnt_elems = 0;
-        const int64_t n = 4 * n_layers * tmax;
-        if (cudaMalloc(&h->px_cnt, (size_t)n * sizeof(int)) != cudaSuccess)
-            return fail(h, Q4_ENOMEM, "run_stack_sharded: arrival counts");
-        Q4_CUDA(h, cudaMemset(h->px_cnt, 0, (size_t)n * sizeof(int)));
-        Q4_CUDA(h, cudaMemset(h->px_base + h->px_off[4] + 4, 0, 4));   // their epoch
+        if (4 * tmax > h->px_cnt_elems) {
+            cudaFree(h->px_cnt);
+            h->px_cnt = nullptr;
+            h->px_cnt_elems = 0;
+            if (cudaMalloc(&h->px_cnt, (size_t)(4 * tmax) * sizeof(int)) != cudaSuccess)
+                return fail(h, Q4_ENOMEM, "run_stack_sharded: arrival counts");
+            h->px_cnt_elems = 4 * tmax;
+        }
+        Q4_CUDA(h, cudaMemset(h->px_cnt, 0, (size_t)h->px_cnt_elems * sizeof(int)));
+        Q4_CUDA(h, cudaMemset(h->px_base + h->px_off[4] + 4, 0, 4));   // their step count
         Q4_CUDA(h, cudaDeviceSynchronize());
-        h->px_cnt_elems = n;
+        h->px_cnt_layers = n_layers;
     }
     __half* gather[4];
     for (int t = 0; t < 4; ++t) gather[t] = px ? nullptr : h->sh_gather[t];
@@ -1541,15 +1546,15 @@ int q4gemv_run_stack_sharded(q4gemv_t h, const q4gemv_layer* layers, int n_layer
                 // Each GEMV stores its rows, stamped, into every rank's buffer t;
                 // the next stages buffer t's words once they carry its stamp.
                 // Launched programmatically after a GEMV: its weights stream in
-                // while that one ends.  Its own arrival counts; the split
-                // workspace alternates between two halves.
+                // while that one ends.  Arrival counts per matrix of the layer;
+                // the split workspace alternates between two halves.
                 pa.y = h->px_ytab + t * world;
                 pa.xw = i > 0 ? words[(t + 3) % 4] : nullptr;
                 pa.g = i;
                 pa.wait = i > 0 ? 1 : 0;
                 if (rows[t] > 0) {
                     rc = launch_gemv(h, W, xin, nullptr, 1, rows[t], k_of[t], i == 0 ? 0 : 1, nullptr,
-                                     h->cap, last_was_gemv, false, false, &pa, h->px_cnt + (int64_t)i * tmax,
+                                     h->cap, last_was_gemv, false, false, &pa, h->px_cnt + (int64_t)t * tmax,
                                      h->ws + (size_t)(i & 1) * h->sms * 2 * 32);
                     last_was_gemv = true;
                 } else {

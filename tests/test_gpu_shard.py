@@ -131,6 +131,27 @@ def test_peer_steps_chain(eng):
     pe.close()
 
 
+def test_peer_layer_count_change():
+    """The split tiles' arrival counts run on across layers and steps with
+    the layer count in their arithmetic: a step of another depth on the same
+    exchange (counts zeroed, graph recaptured) must still be right, and so
+    must the first depth again."""
+    hidden, qkv_n, ffn = 256, 384, 512
+    pe = _peer_engine(hidden, qkv_n, ffn)
+    layers, get = _stack(pe, 3, hidden, qkv_n, ffn, 55)
+    x = synth.normal_f16(55, synth.act_id(0), hidden)
+    xd = f16_dev(x)
+    for L in (1, 3, 1, 1):
+        y = bits_of(pe.run_stack_sharded(layers[:L], xd, hidden, qkv_n, ffn))
+        assert pe.sync_status() == q4.Q4_OK
+        single = bits_of(pe.run_stack(layers[:L], xd, hidden, qkv_n, ffn))
+        assert pe.sync_status() == q4.Q4_OK
+        assert rel_err(y, single.view(np.float16).astype(np.float64)) <= TOL
+        if L == 1:
+            assert rel_err(y, oracle.f16_to_f64(oracle.stack_step(get, x, L, hidden, qkv_n, ffn))) <= TOL
+    pe.close()
+
+
 def test_peer_wait_timeout_is_reported_and_recoverable():
     """Every stamp wait of the step given a stamp no rank writes and a short
     poll budget (the "timeout" test knob): the kernels must return, the
