@@ -587,14 +587,18 @@ def run_ours(args, rank: int, world: int, dist):
     roofline = {
         "bound": "hbm", "achieved": per_rank_gbs, "peak": peak, "unit": "GB/s",
         "frac": per_rank_gbs / peak, "traffic": None,
-        "kernel": "q4::stack_kernel<16,3,6> (one persistent launch per step, all 4L GEMVs and "
-                  "the final renorm; duration = step time, which also holds the 16-byte "
-                  "barrier-word reset before each launch)",
+        "kernel": ("q4::gemv_dp2a_kernel<1,16,3,6> (per rank: one launch per GEMV on its rows, "
+                   "4L per step in one graph, plus the step-count update and the final renorm; "
+                   "duration = step time; bytes = this rank's share of the step)"
+                   if args.shard else
+                   "q4::stack_kernel<16,3,6> (one persistent launch per step, all 4L GEMVs and "
+                   "the final renorm; duration = step time, which also holds the 16-byte "
+                   "barrier-word reset before each launch)"),
         "peak_source": f"{peak_kind} hbm_gbs (copy) in MEASURED_PEAKS.json",
         "frac_of_nominal_8TBps": per_rank_gbs / NOMINAL_HBM_GBS,
     }
     traffic = os.path.join(ROOT, "profiles", "traffic_per_launch.json")
-    if os.path.exists(traffic) and L == 64:
+    if os.path.exists(traffic) and L == 64 and not args.shard:
         with open(traffic) as f:
             tr = json.load(f)
         # Counters taken on another version of the kernel's source do not count.
