@@ -574,6 +574,12 @@ def run_ours(args, rank: int, world: int, dist):
         raise RuntimeError("device status after timing")
 
     ms, ms_e2e = max_over_ranks(dist, [ms, ms_e2e], device=dev)
+    # Every rank's steps are complete (synchronised before the reduction):
+    # no rank stores into another's exchange buffer any more, and the step
+    # graphs (which may hold NCCL calls) go before the process group.
+    torch.cuda.synchronize()
+    barrier()
+    eng.close()
     if rank != 0:
         return 0
 
