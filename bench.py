@@ -24,6 +24,12 @@ the reported bytes are the model's once per step).  --exchange peer (the
 default) has each GEMV kernel store its rows into every rank's buffer over
 CUDA IPC peer memory and stamp them; --exchange nccl all-gathers them with
 NCCL after every GEMV instead.
+
+--pipeline runs the pages' own multi-device split for comparison: contiguous
+layer ranges, one per rank, the f16 hidden state sent from GPU to GPU (NCCL
+send/recv) and from the last back to the first for the next token.  For one
+autoregressive stream the ranges run one after another, so N GPUs hold 1/N
+of the weights each but do not shorten the step.
 """
 from __future__ import annotations
 
@@ -68,6 +74,11 @@ WORKLOAD_SHARD = ("27B-shaped decode step, M=1: 64 layers x (QKV 5120->7168, O 5
                   "matrices, every matrix row-sharded over the GPUs: per GEMV one kernel on each "
                   "GPU's rows, every GPU getting all rows before the next GEMV, replayed as one CUDA "
                   "graph")
+WORKLOAD_PIPE = ("27B-shaped decode step, M=1: 64 layers x (QKV 5120->7168, O 5120->5120, "
+                 "gate+up 5120->34816, down 17408->5120) Q4_0 GEMVs with unit-RMS renorm between "
+                 "matrices, split into contiguous layer ranges over the GPUs: one persistent kernel "
+                 "per GPU and token, the f16 hidden state sent to the next GPU after each range and "
+                 "back to the first for the next token (one autoregressive stream)")
 
 
 KERNEL_SOURCES = ["stack.cuh", "gemv_dp2a.cuh", "partition.cuh", "device_common.cuh"]
@@ -255,14 +266,22 @@ def run_reference(args, rank: int):
 
 # ------------------------------------------------------------------ GPU arm
 
-def build_weights(eng, torch, rank: int):
-    """Packed weights of the 64-layer step: generated on the host (seeded),
-    copied to the device, repacked by the library's repack kernel."""
+def layer_range(world: int, rank: int, n_layers: int):
+    """Contiguous layers [l0, l1) of `rank` in the layer-range pipeline: the
+    pages' split of the model over devices, ranks in order, sizes within
+    one layer of each other."""
+    return rank * n_layers // world, (rank + 1) * n_layers // world
+
+
+def build_weights(eng, torch, rank: int, l0: int = 0, l1: int = None):
+    """Packed weights of layers [l0, l1) of the 64-layer step (all by
+    default): generated on the host (seeded), copied to the device,
+    repacked by the library's repack kernel."""
     layers = []
     host = {t: np.empty((N, (K // 32) * 18), dtype=np.uint8) for t, (N, K) in enumerate(DIMS)}
     staging = torch.empty(max(h.size for h in host.values()), dtype=torch.uint8, device="cuda")
     t_repack = 0.0
-    for l in range(L):
+    for l in range(l0, L if l1 is None else l1):
         mats = []
         for t, (N, K) in enumerate(DIMS):
             synth.q4_0_matrix(STEP_SEED, synth.weight_id(4 * l + t), N, K, out=host[t])
@@ -493,23 +512,51 @@ def run_ours(args, rank: int, world: int, dist):
         eng.peer_open(blobs)
     if args.shard:
         layers, t_repack = build_weights_sharded(eng, torch, q4, rank, world)
+    elif args.pipeline:
+        layers, t_repack = build_weights(eng, torch, rank, *layer_range(world, rank, L))
     else:
         layers, t_repack = build_weights(eng, torch, rank)
-    act = 0 if args.shard else rank          # the sharded ranks share one step's input
+    one_step = args.shard or args.pipeline   # the ranks share one step (and its input)
+    act = 0 if one_step else rank
     x_host = torch.from_numpy(synth.normal_f16(STEP_SEED, synth.act_id(act), HIDDEN).view(np.float16)).pin_memory()
     out_host = torch.empty(HIDDEN, dtype=torch.float16).pin_memory()
     x_in = x_host.to(dev)
     x_out = torch.empty(HIDDEN, dtype=torch.float16, device=dev)
     stream = torch.cuda.current_stream()
 
+    def pipeline_step(copy_in=None, copy_out=None):
+        # One token of one decode stream through the layer-range pipeline:
+        # rank r runs its layers on the hidden state from rank r - 1 and
+        # sends its output on; the last rank's output is the next token's
+        # input on rank 0 (autoregressive, so the stages cannot overlap).
+        if world > 1 and rank > 0:
+            dist.recv(x_in, src=rank - 1)
+        elif copy_in is not None:
+            x_in.copy_(copy_in, non_blocking=True)
+        eng.run_stack(layers, x_in, HIDDEN, QKV_N, FFN, x_out=x_out)
+        if world > 1:
+            dist.send(x_out, dst=(rank + 1) % world)
+            if rank == 0:
+                dist.recv(x_in, src=world - 1)
+        else:
+            x_in.copy_(x_out)
+        if copy_out is not None and rank == 0:
+            copy_out.copy_(x_in, non_blocking=True)
+
     def step():
-        if args.shard:
+        if args.pipeline:
+            pipeline_step()
+        elif args.shard:
             eng.run_stack_sharded(layers, x_in, HIDDEN, QKV_N, FFN, x_out=x_out)
         else:
             eng.run_stack(layers, x_in, HIDDEN, QKV_N, FFN, x_out=x_out)
 
     def step_e2e():
-        if args.shard:
+        if args.pipeline:
+            # the token's input from pinned host memory on rank 0, the next
+            # input back to it
+            pipeline_step(copy_in=x_host if rank == 0 else None, copy_out=out_host)
+        elif args.shard:
             # the sharded call takes device vectors: the copies from and to
             # pinned host memory are made around it, every step
             x_in.copy_(x_host, non_blocking=True)
@@ -567,7 +614,7 @@ def run_ours(args, rank: int, world: int, dist):
     barrier()
     ms_e2e = f0.elapsed_time(f1)
 
-    extras = rank == 0 and not args.no_per_shape and not args.shard
+    extras = rank == 0 and not args.no_per_shape and not one_step
     per_shape = time_shapes(eng, torch, layers) if extras else None
     others = extra_workloads(eng, torch, q4, layers) if extras else None
     if eng.sync_status() != q4.Q4_OK:
@@ -584,12 +631,13 @@ def run_ours(args, rank: int, world: int, dist):
         return 0
 
     ms_step = ms / args.steps
-    # Replicas: every rank runs a whole step.  Sharded: the ranks share one.
-    copies = 1 if args.shard else world
+    # Replicas: every rank runs a whole step.  Sharded or pipelined: the ranks
+    # share one.
+    copies = 1 if one_step else world
     value, steps_per_s = step_throughput(copies, args.steps, ms)
     e2e_value, e2e_steps_per_s = step_throughput(copies, args.steps, ms_e2e)
     peak, peak_kind = measured_peaks()
-    per_rank_gbs = STEP_GEMV_BYTES / (ms_step * 1e-3) / 1e9 / (world if args.shard else 1)
+    per_rank_gbs = STEP_GEMV_BYTES / (ms_step * 1e-3) / 1e9 / (world if one_step else 1)
     roofline = {
         "bound": "hbm", "achieved": per_rank_gbs, "peak": peak, "unit": "GB/s",
         "frac": per_rank_gbs / peak, "traffic": None,
@@ -597,6 +645,9 @@ def run_ours(args, rank: int, world: int, dist):
                    "4L per step in one graph, plus the step-count update and the final renorm; "
                    "duration = step time; bytes = this rank's share of the step)"
                    if args.shard else
+                   "q4::stack_kernel<16,3,6> (per rank: one persistent launch per token over its "
+                   "layer range; duration = step time, all ranks in turn; bytes = this rank's share)"
+                   if args.pipeline else
                    "q4::stack_kernel<16,3,6> (one persistent launch per step, all 4L GEMVs and "
                    "the final renorm; duration = step time, which also holds the 16-byte "
                    "barrier-word reset before each launch)"),
@@ -604,7 +655,7 @@ def run_ours(args, rank: int, world: int, dist):
         "frac_of_nominal_8TBps": per_rank_gbs / NOMINAL_HBM_GBS,
     }
     traffic = os.path.join(ROOT, "profiles", "traffic_per_launch.json")
-    if os.path.exists(traffic) and L == 64 and not args.shard:
+    if os.path.exists(traffic) and L == 64 and not one_step:
         with open(traffic) as f:
             tr = json.load(f)
         # Counters taken on another version of the kernel's source do not count.
@@ -625,16 +676,19 @@ def run_ours(args, rank: int, world: int, dist):
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "strong" if args.shard else "weak", "vs_baseline": None,
+        "scaling": "strong" if one_step else "weak", "vs_baseline": None,
         "dtype": "q4_0 x f16 (s32 block sums, f32 accumulate)", "data": "synthetic",
-        "config": {"workload": WORKLOAD_SHARD if args.shard else WORKLOAD, "bytes_per_step": STEP_GEMV_BYTES,
+        "config": {"workload": WORKLOAD_SHARD if args.shard else WORKLOAD_PIPE if args.pipeline else WORKLOAD,
+                   "bytes_per_step": STEP_GEMV_BYTES,
                    "weight_bytes_per_step": STEP_WEIGHT_BYTES,
                    "l2": "inputs larger than L2 (11.9 GB of weights per step)",
                    "parallelism": ((f"row-sharded x{world} (NCCL all-gather after every GEMV)"
                                     if args.exchange == "nccl" else
                                     f"row-sharded x{world} (GEMV kernels store their rows into every "
                                     "rank's buffer over peer memory)")
-                                   if args.shard else f"replicas x{world}"), "seed": STEP_SEED},
+                                   if args.shard else
+                                   f"layer-range pipeline x{world} (hidden state sent between GPUs)"
+                                   if args.pipeline else f"replicas x{world}"), "seed": STEP_SEED},
         "decode_steps_per_s": steps_per_s,
         "pct_of_8TBps_nominal": 100.0 * per_rank_gbs / NOMINAL_HBM_GBS,
         "roofline": roofline,
@@ -644,7 +698,8 @@ def run_ours(args, rank: int, world: int, dist):
                 "steps_per_s": e2e_steps_per_s},
         # one stack_kernel per step (and one 16-byte memset); sharded over NCCL: per
         # GEMV one kernel and one all-gather, and the final renorm; over peer memory:
-        # per GEMV one kernel, the step-count update and the final unpack + renorm
+        # per GEMV one kernel, the step-count update and the final unpack + renorm;
+        # pipelined: one stack_kernel per GPU (this rank's count)
         "gpu_launches": args.steps * (((8 * L + 1) if args.exchange == "nccl" else (4 * L + 2))
                                       if args.shard else 1),
         "clocks": clocks,
@@ -755,7 +810,12 @@ def main():
                     help="row-shard every matrix over the ranks (one step shared by all GPUs)")
     ap.add_argument("--exchange", choices=["peer", "nccl"], default="peer",
                     help="--shard: how each GEMV's rows reach every rank")
+    ap.add_argument("--pipeline", action="store_true",
+                    help="split the layers into contiguous ranges over the ranks, the hidden state "
+                         "passed from GPU to GPU (the pages' multi-device design; one stream)")
     args = ap.parse_args()
+    if args.shard and args.pipeline:
+        ap.error("--shard and --pipeline are two ways to split one step: pick one")
     if args.layers != 64:
         set_layers(args.layers)
     if args.warmup < 3:
