@@ -8,6 +8,8 @@ every step), a stamp that never comes must end in Q4_ETIMEOUT with the
 handle still usable, and a handle without a communicator or an exchange for
 the shapes must refuse.  The host bookkeeping for more ranks is covered on
 CPU (tests/test_shard_cpu.py)."""
+import os
+
 import numpy as np
 import pytest
 
@@ -105,10 +107,27 @@ def test_peer_step_matches_oracle_and_nccl_bits(eng, L, hidden, qkv_n, ffn):
     nccl = bits_of(eng.run_stack_sharded(layers, xd, hidden, qkv_n, ffn))
     assert eng.sync_status() == q4.Q4_OK
     assert np.array_equal(got, nccl)
-    # at world 1 the row split is the whole matrix: the single-GPU step's
-    # kernels, split and combine order, so its bits
+    # at world 1 the row split is the whole matrix: the per-GEMV kernels of
+    # the single-GPU step (same kernel, split and combine order), so their
+    # bits; the persistent step splits small shapes over more warps, so it
+    # agrees within the tolerance (and bit for bit at full width)
+    old = os.environ.get("Q4GEMV_STACK_MODE")
+    os.environ["Q4GEMV_STACK_MODE"] = "kernels"
+    try:
+        ek = q4.Q4Gemv(0)
+    finally:
+        if old is None:
+            os.environ.pop("Q4GEMV_STACK_MODE", None)
+        else:
+            os.environ["Q4GEMV_STACK_MODE"] = old
+    kern = bits_of(ek.run_stack(layers, xd, hidden, qkv_n, ffn))
+    assert ek.sync_status() == q4.Q4_OK
+    ek.close()
+    assert np.array_equal(got, kern)
     single = bits_of(pe.run_stack(layers, xd, hidden, qkv_n, ffn))
-    assert np.array_equal(got, single)
+    assert rel_err(got, single.view(np.float16).astype(np.float64)) <= TOL
+    if hidden == 5120:
+        assert np.array_equal(got, single)
     pe.close()
 
 
