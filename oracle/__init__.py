@@ -228,7 +228,7 @@ def unit_rms_scale(v: np.ndarray) -> float:
 
 
 def stack_step(get_rows, x_in: np.ndarray, n_layers: int, hidden: int,
-               qkv_n: int, ffn: int, threads: int = 1, record=None):
+               qkv_n: int, ffn: int, threads: int = 1, record=None, gated: bool = False):
     """The renormalised 64-layer-style chain of GEMVs (one decode step, M=1).
 
     Layer l, with matrices QKV (qkv_n x hidden), O (hidden x hidden),
@@ -244,19 +244,34 @@ def stack_step(get_rows, x_in: np.ndarray, n_layers: int, hidden: int,
     layer l.  ``record(i, x_f16, s, y_f64)`` is called for each GEMV
     i = 4l + t when given (x_f16: the unscaled input, s its scale, y_f64 the
     output before rounding).
+
+    ``gated``: the FFN with its activation -- the down GEMV's input is
+    u = SiLU(gate) * up of the whole f16 gate+up output (``swiglu``: gate
+    half first, fp64, never rounded), scaled to unit RMS like every input of
+    the chain: x' = f16(s(u) (down u)), s(u) = 1/sqrt(mean(u^2)) in fp64 (0
+    for u = 0).  ``record`` then gets the 2*ffn-entry gate+up vector as the
+    down GEMV's input.
     """
     dims = [(qkv_n, hidden), (hidden, hidden), (2 * ffn, hidden), (hidden, ffn)]
     x = np.ascontiguousarray(x_in, dtype=np.uint16)
     s = 1.0
     for l in range(n_layers):
         for t, (N, K) in enumerate(dims):
-            assert x.size == K
-            with np.errstate(invalid="ignore"):          # 0 * inf of a non-finite row is NaN
-                y = s * q4_gemv(get_rows(l, t), K, x.reshape(1, K), threads=threads)[0]
+            if gated and t == 3:
+                assert x.size == 2 * K
+                u = swiglu(x.reshape(1, 2 * K))[0]
+                ms = float(np.mean(u * u))
+                s = 1.0 / np.sqrt(ms) if ms > 0 else 0.0
+                with np.errstate(invalid="ignore"):
+                    y = s * q4_gemv_f64(get_rows(l, t), K, u.reshape(1, K), threads=threads)[0]
+            else:
+                assert x.size == K
+                with np.errstate(invalid="ignore"):      # 0 * inf of a non-finite row is NaN
+                    y = s * q4_gemv(get_rows(l, t), K, x.reshape(1, K), threads=threads)[0]
             if record is not None:
                 record(4 * l + t, x, s, y)
             yh = f64_to_f16(y)
-            keep = {0: hidden, 1: hidden, 2: ffn, 3: hidden}[t]
+            keep = {0: hidden, 1: hidden, 2: 2 * ffn if gated else ffn, 3: hidden}[t]
             x = np.ascontiguousarray(yh[:keep])
             s = unit_rms_scale(x)
     return renorm(x)

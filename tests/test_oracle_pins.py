@@ -364,3 +364,73 @@ def test_stack_chain_closed_form():
     x = RNG.choice([-1.0, 1.0], hidden)
     out = oracle.stack_step(lambda l, t: mats[(l, t)], f16_bits(x), L, hidden, qkv_n, ffn)
     assert np.array_equal(f16_values(out), perm_stack_expected(x, maps))
+
+
+def make_gated_perm_stack(L, hidden, qkv_n, ffn):
+    """Signed selections for every matrix, the up half of gate+up too."""
+    mats, maps = {}, []
+    for l in range(L):
+        p_qkv = RNG.permutation(hidden); s_qkv = RNG.choice([-1, 1], hidden)
+        p_o = RNG.permutation(hidden); s_o = RNG.choice([-1, 1], hidden)
+        p_g = RNG.integers(0, hidden, ffn); s_g = RNG.choice([-1, 1], ffn)
+        p_u = RNG.integers(0, hidden, ffn); s_u = RNG.choice([-1, 1], ffn)
+        p_dn = RNG.choice(ffn, hidden, replace=False); s_dn = RNG.choice([-1, 1], hidden)
+        mats[(l, 0)] = signed_selection(qkv_n, hidden, np.concatenate([p_qkv, np.zeros(qkv_n - hidden, int)]),
+                                        np.concatenate([s_qkv, np.ones(qkv_n - hidden, int)]), junk_from=hidden)
+        mats[(l, 1)] = signed_selection(hidden, hidden, p_o, s_o)
+        mats[(l, 2)] = signed_selection(2 * ffn, hidden, np.concatenate([p_g, p_u]), np.concatenate([s_g, s_u]))
+        mats[(l, 3)] = signed_selection(hidden, ffn, p_dn, s_dn)
+        maps.append((p_qkv, s_qkv, p_o, s_o, p_g, s_g, p_u, s_u, p_dn, s_dn))
+    return mats, maps
+
+
+def test_gated_stack_chain_closed_form():
+    """The gated chain on signed selections (row n of every matrix is
+    +-2^-5 e_p(n)): each GEMV's output is f16(s * 2^-5 * sign * v[p]) for its
+    input v and the input's unit-RMS scale s (1 for the step's own input),
+    and the gated down GEMV's input is u = g/(1 + e^-g) * up of the f16
+    gate and up halves, scaled by 1/sqrt(mean(u^2)).  Written here with
+    numpy's exponential and sums, the oracle's with the C library's; f16
+    rounding only where the chain rounds."""
+    L, hidden, qkv_n, ffn = 2, 64, 96, 128
+    mats, maps = make_gated_perm_stack(L, hidden, qkv_n, ffn)
+    x = RNG.choice([-1.0, 1.0], hidden)
+    out = oracle.stack_step(lambda l, t: mats[(l, t)], f16_bits(x), L, hidden, qkv_n, ffn, gated=True)
+
+    def f16(v):
+        return v.astype(np.float16).astype(np.float64)
+
+    def scale(v):
+        return 1.0 / np.sqrt(np.mean(v * v))
+
+    v, s = x.copy(), 1.0
+    for (p_qkv, s_qkv, p_o, s_o, p_g, s_g, p_u, s_u, p_dn, s_dn) in maps:
+        a = f16(s * 2.0 ** -5 * s_qkv * v[p_qkv])         # QKV rows past hidden unused
+        b = f16(scale(a) * 2.0 ** -5 * s_o * a[p_o])
+        sb = scale(b)
+        g = f16(sb * 2.0 ** -5 * s_g * b[p_g])
+        up = f16(sb * 2.0 ** -5 * s_u * b[p_u])
+        u = g / (1.0 + np.exp(-g)) * up
+        v = f16(scale(u) * 2.0 ** -5 * s_dn * u[p_dn])
+        s = scale(v)
+    want = f16(s * v)
+    assert np.array_equal(f16_values(out), want)
+
+
+def test_gated_stack_differs_from_the_plain_chain_only_in_down():
+    """gated=True changes the down GEMV's input and nothing before it: the
+    first three GEMVs of each layer see the same inputs as in the plain
+    chain (one layer), and the down input recorded is the whole gate+up
+    output."""
+    L, hidden, qkv_n, ffn = 1, 64, 96, 128
+    mats, _ = make_gated_perm_stack(L, hidden, qkv_n, ffn)
+    x = f16_bits(RNG.choice([-1.0, 1.0], hidden))
+    rec_p, rec_g = {}, {}
+    oracle.stack_step(lambda l, t: mats[(l, t)], x, L, hidden, qkv_n, ffn,
+                      record=lambda i, xf, s, y: rec_p.setdefault(i, xf.copy()))
+    oracle.stack_step(lambda l, t: mats[(l, t)], x, L, hidden, qkv_n, ffn, gated=True,
+                      record=lambda i, xf, s, y: rec_g.setdefault(i, xf.copy()))
+    for i in range(3):
+        assert np.array_equal(rec_p[i], rec_g[i])
+    assert rec_g[3].size == 2 * ffn and rec_p[3].size == ffn
+    assert np.array_equal(rec_g[3][:ffn], rec_p[3])
