@@ -74,6 +74,10 @@ WORKLOAD_SHARD = ("27B-shaped decode step, M=1: 64 layers x (QKV 5120->7168, O 5
                   "matrices, every matrix row-sharded over the GPUs: per GEMV one kernel on each "
                   "GPU's rows, every GPU getting all rows before the next GEMV, replayed as one CUDA "
                   "graph")
+WORKLOAD_GATED = ("27B-shaped decode step, M=1: 64 layers x (QKV 5120->7168, O 5120->5120, "
+                  "gate+up 5120->34816, down 17408->5120) Q4_0 GEMVs with unit-RMS renorm between "
+                  "matrices, each down GEMV fed SiLU(gate) * up of the gate+up output (computed in "
+                  "its staging), one persistent kernel launch per step")
 WORKLOAD_PIPE = ("27B-shaped decode step, M=1: 64 layers x (QKV 5120->7168, O 5120->5120, "
                  "gate+up 5120->34816, down 17408->5120) Q4_0 GEMVs with unit-RMS renorm between "
                  "matrices, split into contiguous layer ranges over the GPUs: one persistent kernel "
@@ -548,6 +552,8 @@ def run_ours(args, rank: int, world: int, dist):
             pipeline_step()
         elif args.shard:
             eng.run_stack_sharded(layers, x_in, HIDDEN, QKV_N, FFN, x_out=x_out)
+        elif args.gated:
+            eng.run_stack_gated(layers, x_in, HIDDEN, QKV_N, FFN, x_out=x_out)
         else:
             eng.run_stack(layers, x_in, HIDDEN, QKV_N, FFN, x_out=x_out)
 
@@ -562,6 +568,8 @@ def run_ours(args, rank: int, world: int, dist):
             x_in.copy_(x_host, non_blocking=True)
             eng.run_stack_sharded(layers, x_in, HIDDEN, QKV_N, FFN, x_out=x_out)
             out_host.copy_(x_out, non_blocking=True)
+        elif args.gated:
+            eng.run_stack_gated(layers, x_host, HIDDEN, QKV_N, FFN, x_out=out_host)
         else:
             eng.run_stack(layers, x_host, HIDDEN, QKV_N, FFN, x_out=out_host)
 
@@ -648,6 +656,8 @@ def run_ours(args, rank: int, world: int, dist):
                    "q4::stack_kernel<16,3,6> (per rank: one persistent launch per token over its "
                    "layer range; duration = step time, all ranks in turn; bytes = this rank's share)"
                    if args.pipeline else
+                   "q4::stack_kernel<16,3,6,true> (gated: one persistent launch per step)"
+                   if args.gated else
                    "q4::stack_kernel<16,3,6> (one persistent launch per step, all 4L GEMVs and "
                    "the final renorm; duration = step time, which also holds the 16-byte "
                    "barrier-word reset before each launch)"),
@@ -655,7 +665,7 @@ def run_ours(args, rank: int, world: int, dist):
         "frac_of_nominal_8TBps": per_rank_gbs / NOMINAL_HBM_GBS,
     }
     traffic = os.path.join(ROOT, "profiles", "traffic_per_launch.json")
-    if os.path.exists(traffic) and L == 64 and not one_step:
+    if os.path.exists(traffic) and L == 64 and not one_step and not args.gated:
         with open(traffic) as f:
             tr = json.load(f)
         # Counters taken on another version of the kernel's source do not count.
@@ -678,7 +688,8 @@ def run_ours(args, rank: int, world: int, dist):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "strong" if one_step else "weak", "vs_baseline": None,
         "dtype": "q4_0 x f16 (s32 block sums, f32 accumulate)", "data": "synthetic",
-        "config": {"workload": WORKLOAD_SHARD if args.shard else WORKLOAD_PIPE if args.pipeline else WORKLOAD,
+        "config": {"workload": WORKLOAD_SHARD if args.shard else WORKLOAD_PIPE if args.pipeline else
+                   WORKLOAD_GATED if args.gated else WORKLOAD,
                    "bytes_per_step": STEP_GEMV_BYTES,
                    "weight_bytes_per_step": STEP_WEIGHT_BYTES,
                    "l2": "inputs larger than L2 (11.9 GB of weights per step)",
@@ -810,12 +821,16 @@ def main():
                     help="row-shard every matrix over the ranks (one step shared by all GPUs)")
     ap.add_argument("--exchange", choices=["peer", "nccl"], default="peer",
                     help="--shard: how each GEMV's rows reach every rank")
+    ap.add_argument("--gated", action="store_true",
+                    help="the step with each down GEMV fed SiLU(gate) * up (q4gemv_run_stack_gated)")
     ap.add_argument("--pipeline", action="store_true",
                     help="split the layers into contiguous ranges over the ranks, the hidden state "
                          "passed from GPU to GPU (the pages' multi-device design; one stream)")
     args = ap.parse_args()
     if args.shard and args.pipeline:
         ap.error("--shard and --pipeline are two ways to split one step: pick one")
+    if args.gated and (args.shard or args.pipeline):
+        ap.error("--gated runs on one GPU per step (replicas)")
     if args.layers != 64:
         set_layers(args.layers)
     if args.warmup < 3:

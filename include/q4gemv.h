@@ -280,6 +280,19 @@ Q4GEMV_API int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_la
                      const void* x_in, void* x_out, void* trace_x,
                      void* trace_y, q4gemv_stream_t stream);
 
+/* The decode step of q4gemv_run_stack with the feed-forward block's
+ * activation: each layer's down GEMV takes u = SiLU(gate) * up of the whole
+ * gate+up output (gate = rows [0, ffn), up = rows [ffn, 2 ffn); the pages
+ * name the model family but not its activation -- taozi.news page, section
+ * 支持模型与限制 -- so this is the common gated form, as in
+ * q4gemv_run_swiglu), computed in fp32 inside the down GEMV's staging and
+ * never written, and scaled to unit RMS like every input of the chain:
+ * x' = f16(s(u) (down u)), s(u) = 1/sqrt(mean(u^2)).  Everything else,
+ * arguments, modes and errors as q4gemv_run_stack (no traces). */
+Q4GEMV_API int q4gemv_run_stack_gated(q4gemv_t h, const q4gemv_layer* layers, int n_layers,
+                                      int64_t hidden, int64_t qkv_n, int64_t ffn,
+                                      const void* x_in, void* x_out, q4gemv_stream_t stream);
+
 /* ---- Row-sharded decode step over several GPUs (one process and one handle
  * per GPU).  The pages run the model split by contiguous layer ranges across
  * devices, passing the hidden state from one to the next (originshq.com page,

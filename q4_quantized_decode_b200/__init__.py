@@ -70,6 +70,8 @@ def _load_library():
         "q4gemv_peer_close": ([vp], ci),
         "q4gemv_run_stack": ([vp, ctypes.POINTER(q4gemv_layer), ci, i64, i64, i64,
                               vp, vp, vp, vp, vp], ci),
+        "q4gemv_run_stack_gated": ([vp, ctypes.POINTER(q4gemv_layer), ci, i64, i64, i64,
+                                    vp, vp, vp], ci),
         "q4gemv_sync_status": ([vp, vp], ci),
         "q4gemv_strerror": ([ci], ctypes.c_char_p),
         "q4gemv_last_error": ([vp], ctypes.c_char_p),
@@ -142,6 +144,10 @@ def q4gemv_run_stack(h, layers, n_layers, hidden, qkv_n, ffn, x_in, x_out,
                      trace_x, trace_y, stream) -> int:
     return _lib.q4gemv_run_stack(h, layers, n_layers, hidden, qkv_n, ffn, x_in, x_out,
                                  trace_x, trace_y, stream)
+
+
+def q4gemv_run_stack_gated(h, layers, n_layers, hidden, qkv_n, ffn, x_in, x_out, stream) -> int:
+    return _lib.q4gemv_run_stack_gated(h, layers, n_layers, hidden, qkv_n, ffn, x_in, x_out, stream)
 
 
 def q4gemv_sync_status(h, stream) -> int:
@@ -328,6 +334,18 @@ class Q4Gemv:
             arr[i] = q4gemv_layer(_ptr(a), _ptr(b), _ptr(c), _ptr(d))
         self._check(q4gemv_run_stack(self.h, arr, len(layers), hidden, qkv_n, ffn, _ptr(x_in),
                                      _ptr(x_out), _ptr(trace_x), _ptr(trace_y), _stream(stream)))
+        return x_out
+
+    def run_stack_gated(self, layers, x_in, hidden: int, qkv_n: int, ffn: int, x_out=None, stream=None):
+        """The step with each down GEMV fed SiLU(gate) * up (see the header)."""
+        import torch
+        if x_out is None:
+            x_out = torch.empty(hidden, dtype=torch.float16, device=x_in.device)
+        arr = (q4gemv_layer * len(layers))()
+        for i, (a, b, c, d) in enumerate(layers):
+            arr[i] = q4gemv_layer(_ptr(a), _ptr(b), _ptr(c), _ptr(d))
+        self._check(q4gemv_run_stack_gated(self.h, arr, len(layers), hidden, qkv_n, ffn, _ptr(x_in),
+                                           _ptr(x_out), _stream(stream)))
         return x_out
 
     def init_comm(self, world: int, rank: int, uid: bytes):

@@ -59,7 +59,9 @@ __device__ __forceinline__ void stage_swiglu(const GemvArgs& a, uint32_t xs, uin
     __syncthreads();
 }
 
-// gemv_dp2a_kernel<1> with the gated staging (no renormalisation).
+// gemv_dp2a_kernel<1> with the gated staging; with a.renorm the outputs are
+// scaled by the unit-RMS scale of u (the gated step's down GEMV), else not
+// (q4gemv_run_swiglu).
 template <int WARPS, int R, int C>
 __global__ void __launch_bounds__(WARPS * 32, 1) gemv_swiglu_kernel(const GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -99,6 +101,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_swiglu_kernel(const GemvAr
         else if (nq <= 5 * NT) stage_swiglu<NT, 5>(a, xs, rec, sq);
         else stage_swiglu<NT, kXChunksPerThread>(a, xs, rec, sq);
     }
+    if (a.renorm) cons.oscale = unit_rms_scale(sq, a.KB, a.K);
 
     for (int ch = 0; ch < ring.nch; ++ch) {
         if (!ring.wait(ch)) set_device_error(a.err, kDevTimeout);   // data then unreliable

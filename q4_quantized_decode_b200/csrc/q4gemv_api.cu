@@ -52,6 +52,7 @@ constexpr int kRmq1 = 2, kCmq1 = 4, kRmq2 = 2, kCmq2 = 2;
 #define Q4_MMA_Q8_KERNEL_1 q4::gemv_mma_kernel<1, kWarps, kRmq1, kCmq1, true>
 #define Q4_MMA_Q8_KERNEL_2 q4::gemv_mma_kernel<2, kWarps, kRmq2, kCmq2, true>
 #define Q4_STACK_KERNEL q4::stack_kernel<kWarps, kR1, kC1>
+#define Q4_STACK_KERNEL_GATED q4::stack_kernel<kWarps, kR1, kC1, true>
 #define Q4_SWIGLU_KERNEL q4::gemv_swiglu_kernel<kWarps, kR1, kC1>
 static_assert(Q4GEMV_MAX_M_GEMV == 16, "the small-M tensor-core kernel reads 16 accumulator columns");
 // Largest input of a GEMV in the persistent step (its staging holds up to
@@ -82,6 +83,7 @@ struct StackKey {
     void* x_out = nullptr;
     void* trace_x = nullptr;
     void* trace_y = nullptr;
+    bool gated = false;
     bool operator==(const StackKey& o) const {
         if (layers.size() != o.layers.size()) return false;
         for (size_t i = 0; i < layers.size(); ++i) {
@@ -91,7 +93,7 @@ struct StackKey {
                 return false;
         }
         return hidden == o.hidden && qkv_n == o.qkv_n && ffn == o.ffn && x_in == o.x_in &&
-               x_out == o.x_out && trace_x == o.trace_x && trace_y == o.trace_y;
+               x_out == o.x_out && trace_x == o.trace_x && trace_y == o.trace_y && gated == o.gated;
     }
 };
 
@@ -119,6 +121,7 @@ struct q4gemv_ctx {
     bool desc_valid = false;
     int* sync = nullptr;             // grid barrier words of the persistent step
     uint8_t* xq = nullptr;           // pre-quantised inputs of the persistent step (two halves)
+    uint4* gscr = nullptr;           // gated persistent step: per-CTA combined shared tiles
     float* yacc = nullptr;           // fp32 panel sums of wide tensor-core GEMVs
     size_t yacc_floats = 0;
     __half* hio = nullptr;           // device copies of host x_in / x_out of run_stack
@@ -803,7 +806,8 @@ int q4gemv_create(q4gemv_t* out, int device) {
             set_smem_attr(Q4_Q8_KERNEL_1) || set_smem_attr(Q4_Q8_KERNEL_2) ||
             set_smem_attr(Q4_MMA_KERNEL_1) || set_smem_attr(Q4_MMA_KERNEL_2) ||
             set_smem_attr(Q4_MMA_Q8_KERNEL_1) || set_smem_attr(Q4_MMA_Q8_KERNEL_2) ||
-            set_smem_attr(Q4_STACK_KERNEL) || set_smem_attr(Q4_SWIGLU_KERNEL) ||
+            set_smem_attr(Q4_STACK_KERNEL) || set_smem_attr(Q4_STACK_KERNEL_GATED) ||
+            set_smem_attr(Q4_SWIGLU_KERNEL) ||
             set_smem_attr(q4::gemm_tc_kernel<false>) ||
             set_smem_attr(q4::gemm_tc_kernel<true>) ||
             set_smem_attr(q4::gemm_tc_kernel<false, true>) ||
@@ -852,6 +856,7 @@ int q4gemv_destroy(q4gemv_t h) {
     cudaFree(h->yacc);
     cudaFree(h->hio);
     cudaFree(h->ximg);
+    cudaFree(h->gscr);
     shard_release(h);
     peer_release(h);
     delete h;
@@ -1012,8 +1017,9 @@ int enqueue_stack(q4gemv_ctx* h, const StackKey& k, cudaStream_t st) {
         __half* yout = k.trace_y ? static_cast<__half*>(k.trace_y) + (size_t)i * nmax : buf[t];
         __half* tx = k.trace_x ? static_cast<__half*>(k.trace_x) + (size_t)i * kmax : nullptr;
         const __half* xin = (i == 0) ? static_cast<const __half*>(k.x_in) : prev;
+        const bool gated = k.gated && t == 3;   // SiLU(gate) * up of the 2K gate+up outputs
         const int rc = launch_gemv(h, W, xin, yout, 1, n_of[t], k_of[t], i == 0 ? 0 : 1, tx, st,
-                                   i != 0);
+                                   i != 0, false, gated);
         if (rc != Q4_OK) return rc;
         prev = yout;
     }
@@ -1047,6 +1053,7 @@ void build_descriptors(q4gemv_ctx* h, const StackKey& k, std::vector<q4::StackGe
         d.K = (int)k_of[t];
         d.renorm = i == 0 ? 0 : 1;
         d.fill_y = k.trace_y ? 1 : 0;
+        d.gated = k.gated && t == 3 ? 1 : 0;
         const int S = (int)((n_of[t] + 31) / 32 * (k_of[t] / 32));
         const int gmax = h->sms * kWarps;
         d.sc = q4::make_split(S, gmax < S ? gmax : S);
@@ -1075,6 +1082,7 @@ int enqueue_stack_persistent(q4gemv_ctx* h, const StackKey& k, cudaStream_t st) 
     // that no arrival count satisfies.
     sa.poll_limit = h->fault == kFaultTimeout ? (1u << 10) : (1u << 26);
     sa.unreachable = h->fault == kFaultTimeout ? 1 : 0;
+    sa.gscr = h->gscr;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(h->sms);
     cfg.blockDim = dim3(kThreads);
@@ -1085,16 +1093,18 @@ int enqueue_stack_persistent(q4gemv_ctx* h, const StackKey& k, cudaStream_t st) 
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, Q4_STACK_KERNEL, sa, (int)kmax);
+    const cudaError_t e = k.gated ? cudaLaunchKernelEx(&cfg, Q4_STACK_KERNEL_GATED, sa, (int)kmax)
+                                  : cudaLaunchKernelEx(&cfg, Q4_STACK_KERNEL, sa, (int)kmax);
     if (e != cudaSuccess) return cuda_fail(h, e, "decode-step launch");
     return Q4_OK;
 }
 
 }  // namespace
 
-int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64_t hidden,
-                     int64_t qkv_n, int64_t ffn, const void* x_in, void* x_out, void* trace_x,
-                     void* trace_y, q4gemv_stream_t stream) {
+namespace {
+int run_stack_impl(q4gemv_ctx* h, const q4gemv_layer* layers, int n_layers, int64_t hidden,
+                   int64_t qkv_n, int64_t ffn, const void* x_in, void* x_out, void* trace_x,
+                   void* trace_y, q4gemv_stream_t stream, bool gated) {
     if (!h) return Q4_EINVAL;
     if (!layers || !x_in || !x_out) return fail(h, Q4_EINVAL, "run_stack: null pointer");
     if (n_layers < 1 || n_layers > 4096) return fail(h, Q4_ESHAPE, "run_stack: n_layers out of range");
@@ -1155,6 +1165,7 @@ int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64
     k.x_out = x_out;
     k.trace_x = trace_x;
     k.trace_y = trace_y;
+    k.gated = gated;
 
     // Intermediate buffers (outside any capture: allocation is not captured).
     const size_t need = (size_t)((qkv_n + 7) / 8 * 8 + (hidden + 7) / 8 * 8 +
@@ -1177,11 +1188,19 @@ int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64
 
     const int64_t kmax_step = hidden > ffn ? hidden : ffn;
     if (h->stack_mode == kStackPersistent && kmax_step <= (int64_t)kStackKmax &&
-        q4::stack_smem_bytes((int)kmax_step, kWarps, kR1, kC1) <= kMaxDynSmem) {
+        q4::stack_smem_bytes((int)kmax_step, kWarps, kR1, kC1) <= kMaxDynSmem &&
+        (!gated || h->sms <= q4::kStackMaxCtas)) {
         if (!h->desc_valid || !(h->desc_key == k)) {
             if (cs != cudaStreamCaptureStatusNone)
                 return fail(h, Q4_EUNSUPPORTED,
                             "run_stack: first call with these arguments must happen outside stream capture");
+            if (gated && !h->gscr) {
+                if (h->fault == kFaultAlloc) return fail(h, Q4_EFAULTINJ, "injected allocation failure");
+                if (cudaMalloc(&h->gscr, (size_t)h->sms * q4::kStackMaxCtas * 4 * sizeof(uint4)) != cudaSuccess) {
+                    h->gscr = nullptr;
+                    return fail(h, Q4_ENOMEM, "run_stack: gated scratch allocation failed");
+                }
+            }
             std::vector<q4::StackGemv> desc;
             build_descriptors(h, k, desc);
             if ((int)desc.size() > h->desc_cap) {
@@ -1230,6 +1249,21 @@ int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64
     }
     Q4_CUDA(h, cudaGraphLaunch(h->exec, st));
     return finish_host_out(h, Q4_OK, host_out, x_out_user, x_out, hidden, st);
+}
+}  // namespace
+
+int q4gemv_run_stack(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64_t hidden,
+                     int64_t qkv_n, int64_t ffn, const void* x_in, void* x_out, void* trace_x,
+                     void* trace_y, q4gemv_stream_t stream) {
+    return run_stack_impl(h, layers, n_layers, hidden, qkv_n, ffn, x_in, x_out, trace_x, trace_y, stream,
+                          false);
+}
+
+int q4gemv_run_stack_gated(q4gemv_t h, const q4gemv_layer* layers, int n_layers, int64_t hidden,
+                           int64_t qkv_n, int64_t ffn, const void* x_in, void* x_out,
+                           q4gemv_stream_t stream) {
+    return run_stack_impl(h, layers, n_layers, hidden, qkv_n, ffn, x_in, x_out, nullptr, nullptr, stream,
+                          true);
 }
 
 int q4gemv_shard_rows(int64_t N, int world, int rank, int64_t* row0, int64_t* rows, int64_t* chunk) {

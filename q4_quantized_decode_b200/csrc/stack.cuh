@@ -17,6 +17,7 @@
 #pragma once
 
 #include "gemv_dp2a.cuh"
+#include "gemv_swiglu.cuh"
 
 namespace q4 {
 
@@ -28,6 +29,7 @@ struct StackGemv {
     int N, K;
     int renorm;           // 1: input = unit-RMS scale * previous output[0:K]; 0: input = x_in
     int fill_y;           // 1: also write y of tiles shared by CTAs (y is traced)
+    int gated;            // 1: input = SiLU(gate) * up of the previous 2K outputs, scaled to unit RMS
     SplitConsts sc;       // split of its segments over the grid's warps
 };
 
@@ -46,6 +48,7 @@ struct StackArgs {
     int* sync;            // [0] grid arrivals, [1] abort flag; zero at launch
     uint32_t poll_limit;  // polls of a grid wait before it gives up
     int unreachable;      // test knob: the first grid wait asks for one arrival too many
+    uint4* gscr;          // gated steps: per CTA, the combined shared tiles [kStackMaxCtas][4] (16 B each)
 };
 
 // Outputs of the previous GEMV in tiles shared by several CTAs exist only as
@@ -201,6 +204,67 @@ __device__ __forceinline__ void stage_prequant(const StackArgs& sa, int i, int K
     __syncthreads();
 }
 
+// Largest grid of the gated step (its per-CTA scratch holds one combined
+// chunk per CTA boundary and chunk).
+constexpr int kStackMaxCtas = 256;
+
+// Staging of a gated GEMV i (the down GEMV of the FFN with its activation):
+// its K-entry input is u = SiLU(gate) * up of GEMV i-1's 2K outputs (gate
+// half first), computed in fp32 and converted per block as any input; the
+// step's pre-converted hand-off is not used (u needs both halves, which
+// different CTAs finish).  Two passes: the tiles of GEMV i-1 shared by CTAs
+// are combined (CTA partials in CTA order, scaled, rounded: the values the
+// plain staging would use) into this CTA's scratch, one 16-byte chunk per
+// CTA boundary and chunk; then every thread loads its chunks of both halves
+// -- from y for tiles one CTA finished, from the scratch for shared ones --
+// and converts SiLU(g) * up.  QN: chunks of u per thread (K <= QN * 8 * NT).
+template <int WARPS, int NT, int QN>
+__device__ __forceinline__ void stage_gated(const StackArgs& sa, int K, const SplitFix<WARPS>& fx,
+                                            const __half* y_prev, uint32_t xs, uint32_t rec, float* sq) {
+    uint4* scr = sa.gscr + (size_t)blockIdx.x * kStackMaxCtas * 4;
+    const int nb = (fx.sc.G + WARPS - 1) / WARPS;
+    const int total = (nb - 1) * 4;
+    for (int p = threadIdx.x; p < total; p += NT) {
+        const int t = shared_tile_of_boundary((p >> 2) + 1, fx.KB, fx.sc, WARPS);
+        if (t >= 0) scr[p] = fx.combine(t, p >> 2, p & 3);   // slot: first contributor, chunk
+    }
+    __syncthreads();
+    const int nq = K / 8;
+    auto chunk = [&](int c) -> uint4 {                       // chunk c of GEMV i-1's output
+        const int t = c >> 2;
+        const int cf = warp_of_seg(t * fx.KB, fx.sc) / WARPS;
+        const int cl = warp_of_seg(t * fx.KB + fx.KB - 1, fx.sc) / WARPS;
+        return cf == cl ? __ldcg(reinterpret_cast<const uint4*>(y_prev) + c) : scr[cf * 4 + (c & 3)];
+    };
+    uint4 gr[QN], ur[QN];
+#pragma unroll
+    for (int r = 0; r < QN; ++r) {
+        const int q = (int)threadIdx.x + NT * r;
+        gr[r] = q < nq ? chunk(q) : make_uint4(0, 0, 0, 0);
+        ur[r] = q < nq ? chunk(q + nq) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int r = 0; r < QN; ++r) {
+        const int q = (int)threadIdx.x + NT * r;
+        const __half2* gh = reinterpret_cast<const __half2*>(&gr[r]);
+        const __half2* uh = reinterpret_cast<const __half2*>(&ur[r]);
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 g2 = __half22float2(gh[e]);
+            const float2 u2 = __half22float2(uh[e]);
+            v[2 * e] = silu_f32(g2.x) * u2.x;
+            v[2 * e + 1] = silu_f32(g2.y) * u2.y;
+        }
+        const ChunkQ o = quant_chunk(v);                    // all lanes (shuffles inside a block)
+        if (q < nq) {
+            store_chunk_smem(o, xs, rec, q >> 2, q & 3);
+            if ((q & 3) == 0) sq[q >> 2] = o.sq;
+        }
+    }
+    __syncthreads();
+}
+
 // The view of GEMV i that the per-warp consumer and the staging work on.
 __device__ __forceinline__ GemvArgs stack_view(const StackArgs& sa, int i) {
     const StackGemv d = sa.gemv[i];
@@ -336,7 +400,7 @@ __device__ __forceinline__ bool grid_wait(int* sync, int target, int* err, int* 
     return *flag_smem != 0;
 }
 
-template <int WARPS, int R, int C>
+template <int WARPS, int R, int C, bool GATED = false>
 __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa, int kmax) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[WARPS * R];
@@ -374,6 +438,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa
 
     bool ok = true;
     float s_prev = 1.f;                   // output scale of GEMV i-1
+    int xphases = 0;                      // phases of the copy barrier completed
     for (int i = 0; i < sa.n_gemv && ok; ++i) {
         GemvArgs a = stack_view(sa, i);
         a.ws = sa.ws + (size_t)(i & 1) * sa.ws_half;
@@ -381,7 +446,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa
         // barrier.  Finished output blocks go out pre-quantised for GEMV i+1.
         Dp2aConsumer<1> cons;
         cons.init(a, gw, xs, rec, park + (size_t)warp * 2 * 32);
-        if (i + 1 < sa.n_gemv) {
+        if (i + 1 < sa.n_gemv && !(GATED && sa.gemv[i + 1].gated)) {
             uint8_t* ob = sa.xq + (size_t)((i + 1) & 1) * sa.xq_half;
             cons.qo.x = reinterpret_cast<int16_t*>(ob);
             cons.qo.rec = reinterpret_cast<uint2*>(ob + (size_t)sa.kmax * 2);
@@ -405,7 +470,15 @@ __global__ void __launch_bounds__(WARPS * 32, 1) stack_kernel(const StackArgs sa
             fix.fill_y = pd.fill_y ? pd.y : nullptr;
             fix.fill_n = pd.N;
             fix.fill_all = false;
-            stage_prequant<WARPS, NT>(sa, i, a.K, fix, xs, rec, sq, &xbar, (uint32_t)((i - 1) & 1));
+            if (GATED && sa.gemv[i].gated) {
+                if (a.K <= 2 * NT * 8) stage_gated<WARPS, NT, 2>(sa, a.K, fix, pd.y, xs, rec, sq);
+                else stage_gated<WARPS, NT, kStackXChunks>(sa, a.K, fix, pd.y, xs, rec, sq);
+            } else {
+                // the copy barrier completes one phase per pre-converted staging
+                const uint32_t parity = GATED ? (uint32_t)(xphases & 1) : (uint32_t)((i - 1) & 1);
+                stage_prequant<WARPS, NT>(sa, i, a.K, fix, xs, rec, sq, &xbar, parity);
+                ++xphases;
+            }
             cons.oscale = unit_rms_scale(sq, a.KB, a.K);
         }
         const int nseg = cons.sp.s1 - cons.sp.s0;
