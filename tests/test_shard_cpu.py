@@ -12,10 +12,12 @@ entries -- the bookkeeping the GPU path uses.
 
 For the peer-memory exchange: q4gemv_peer_layout's offsets, q4gemv_peer_check
 on hand-built blobs (each kind of mismatch refused), and the exchange's
-protocol -- rows stored into every rank's buffer, stamps base + g + 1, waits
-for base + g, the base advanced every step, compared modulo 2^32 -- run by
-two processes over shared memory with the oracle standing in for the
-kernels, reproducing the unsharded oracle chain over three steps."""
+protocol -- every row stored into every rank's buffer as a word carrying a
+16-bit stamp (steps run x GEMVs per step + GEMV index), each reader polling
+the words it needs for the previous GEMV's stamp, across the 16-bit wrap --
+run by two or three processes over shared memory with the oracle standing
+in for the kernels, reproducing the unsharded oracle chain over three
+steps."""
 import os
 import sys
 
@@ -261,15 +263,19 @@ def _peer_worker(rank, world, port, shm_names, out, steps):
         dist.destroy_process_group()
 
 
-def test_peer_exchange_two_ranks_chains_the_unsharded_oracle():
-    """Two ranks (spawned processes, gloo for the blob exchange) run three
-    chained steps through the peer-exchange bookkeeping; every step on every
-    rank must equal the unsharded oracle step of the previous output bit for
-    bit, the step count starting where the 16-bit stamps wrap inside the
-    first step."""
+@pytest.mark.parametrize("world", [2, 3])
+def test_peer_exchange_ranks_chain_the_unsharded_oracle(world):
+    """Two or three ranks (spawned processes, gloo for the blob exchange)
+    run three chained steps through the peer-exchange bookkeeping; every
+    step on every rank must equal the unsharded oracle step of the previous
+    output bit for bit, the step count starting where the 16-bit stamps wrap
+    inside the first step.  With three ranks the last holds no rows of the
+    128-row matrices (64 + 64 + 0) and writes nothing for them."""
     import torch.multiprocessing as mp
     from multiprocessing import shared_memory
-    world, steps = 2, 3
+    steps = 3
+    if world == 3:
+        assert q4.q4gemv_shard_rows(HIDDEN, 3, 2)[2] == 0
     st, off = q4.q4gemv_peer_layout(world, HIDDEN, QKV_N, FFN)
     shms = [shared_memory.SharedMemory(create=True, size=off[5]) for _ in range(world)]
     try:
@@ -279,7 +285,7 @@ def test_peer_exchange_two_ranks_chains_the_unsharded_oracle():
             np.frombuffer(m.buf, dtype=np.uint32, count=2, offset=off[4])[:] = [8190, 0]
         ctx = mp.get_context("spawn")
         q = ctx.Queue()
-        port = 29700 + os.getpid() % 1000
+        port = 29700 + 10 * world + os.getpid() % 1000
         procs = [ctx.Process(target=_peer_worker, args=(r, world, port, [m.name for m in shms], q, steps))
                  for r in range(world)]
         for p in procs:
