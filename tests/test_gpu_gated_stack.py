@@ -114,3 +114,31 @@ def test_gated_and_plain_steps_alternate_on_one_handle():
         assert rel_err(bits_of(eng.run_stack_gated(layers, xd, hidden, qkv_n, ffn)), wg) <= TOL
     assert eng.sync_status() == q4.Q4_OK
     eng.close()
+
+
+def test_gated_step_host_vectors_and_errors():
+    """Host (pinned) input and output vectors, staged inside the call, give
+    the device-vector result; null and misaligned arguments are refused."""
+    L, hidden, qkv_n, ffn = 1, 128, 192, 256
+    eng = q4.Q4Gemv(0)
+    layers, _ = _stack(eng, L, hidden, qkv_n, ffn, 1010)
+    x = synth.normal_f16(1010, synth.act_id(0), hidden)
+    dev = bits_of(eng.run_stack_gated(layers, f16_dev(x), hidden, qkv_n, ffn))
+    xh = torch.from_numpy(x.view(np.float16).copy()).pin_memory()
+    oh = torch.empty(hidden, dtype=torch.float16).pin_memory()
+    eng.run_stack_gated(layers, xh, hidden, qkv_n, ffn, x_out=oh)
+    torch.cuda.synchronize()
+    assert eng.sync_status() == q4.Q4_OK
+    assert np.array_equal(oh.view(torch.int16).numpy().view(np.uint16), dev)
+    arr = (q4.q4gemv_layer * 1)()
+    arr[0] = q4.q4gemv_layer(None, None, None, None)
+    out = torch.empty(hidden, dtype=torch.float16, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    xd = f16_dev(x)
+    assert q4.q4gemv_run_stack_gated(eng.h, arr, 1, hidden, qkv_n, ffn, xd.data_ptr(), out.data_ptr(),
+                                     st) == q4.Q4_EINVAL
+    a, b, c, d = layers[0]
+    arr[0] = q4.q4gemv_layer(a.data_ptr(), b.data_ptr() + 8, c.data_ptr(), d.data_ptr())
+    assert q4.q4gemv_run_stack_gated(eng.h, arr, 1, hidden, qkv_n, ffn, xd.data_ptr(), out.data_ptr(),
+                                     st) == q4.Q4_EALIGN
+    eng.close()
